@@ -1,0 +1,432 @@
+"""Benchmark of the GDN token mixer on B200: prefill T=4096 and decode B=64.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl gdn|reference]
+
+One step = one gdn_prefill over a Qwen3.8-shaped layer (B=1, T=4096, 16 key /
+48 value heads x 128, chunk 64, bf16 inputs, zero initial state), which runs
+every prefill stage of the mixer.  The decode entry point (64 sequences, one
+token each, fresh bf16 inputs per step, states ~N(0, 0.02)) is timed over
+1000 consecutive steps in the same run and reported under "decode".
+
+Inputs are synthetic (seeded numpy draws) and resident in HBM before timing.
+Between timed prefill steps the inputs rotate over 3 sets (~540 MB, > 4x L2)
+so no step reads its inputs from L2; the decode state alone is 201 MB.
+Times are CUDA events on the launching stream; the dominant kernel's average
+launch time comes from the library's own per-launch events.  Under torchrun
+every rank runs its own replica (no data-path collective) and the slowest
+rank's time is reported.  ``--impl reference`` times the float64 CPU oracle
+on a bounded sample of the same workload on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_attention_recurrence_deltanet_b200 import inputs as gi  # noqa: E402
+
+METRIC = "GDN tokens/s (prefill T=4096, decode B=64) and % of HBM/tensor roofline"
+PREFILL_WORKLOAD = "prefill_t4096"
+DECODE_WORKLOAD = "decode_b64"
+DECODE_STEPS = 1000
+ROTATE = 3
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sus=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# ------------------------------------------------------------------ algorithmic traffic
+
+
+def prefill_bytes(geo, lengths, zero_state: bool) -> int:
+    """Bytes the prefill must move at minimum: every token's qkv, z, a, b in
+    and o out (io dtype), each sequence's fp32 state written (and read unless
+    it starts at zero), its conv history read and written, and the
+    parameters read once."""
+    io = geo.io_bytes
+    T = int(sum(lengths))
+    per_tok = (geo.conv_dim + geo.value_dim + 2 * geo.num_v_heads + geo.value_dim) * io
+    state = geo.num_v_heads * geo.head_v_dim * geo.head_k_dim * 4
+    hist = (geo.conv_width - 1) * geo.conv_dim * io
+    params = (geo.conv_dim * geo.conv_width + 2 * geo.num_v_heads + geo.head_v_dim) * 4
+    n = len(lengths)
+    return T * per_tok + n * state * (1 if zero_state else 2) + n * 2 * hist + params
+
+
+def decode_bytes(geo, num_seqs: int) -> int:
+    io = geo.io_bytes
+    per_seq = (geo.conv_dim + geo.value_dim + 2 * geo.num_v_heads + geo.value_dim) * io \
+        + 2 * geo.num_v_heads * geo.head_v_dim * geo.head_k_dim * 4 + 2 * (geo.conv_width - 1) * geo.conv_dim * io
+    params = (geo.conv_dim * geo.conv_width + 2 * geo.num_v_heads + geo.head_v_dim) * 4
+    return num_seqs * per_seq + params
+
+
+def source_hash(*names) -> str:
+    h = hashlib.sha256()
+    for n in names:
+        h.update(open(os.path.join(ROOT, "linear_attention_recurrence_deltanet_b200", "csrc", n), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str, src_hash: str):
+    """dram bytes per launch from a committed ncu summary, if it was taken on
+    the current source of the kernel; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(kernel)
+    if not d or d.get("source_hash") != src_hash:
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks
+
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons through NVML while
+    active (reading only; no setting is changed)."""
+
+    NAMES = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+             0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+             0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, torch_device: int):
+        self.ok = False
+        self.samples = []
+        self.active = False
+        try:
+            import pynvml as nv
+            import torch
+            nv.nvmlInit()
+            props = torch.cuda.get_device_properties(torch_device)
+            h = None
+            bus = getattr(props, "pci_bus_id", None)
+            if bus is not None:
+                try:
+                    pci = "%08x:%02x:%02x.0" % (getattr(props, "pci_domain_id", 0), bus, getattr(props, "pci_device_id", 0))
+                    h = nv.nvmlDeviceGetHandleByPciBusId(pci.encode())
+                except Exception:
+                    h = None
+            if h is None:
+                h = nv.nvmlDeviceGetHandleByIndex(torch_device)
+            self.nv, self.h = nv, h
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report no clocks
+            self.err = str(e)
+        self._stop = threading.Event()
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def _reasons(self):
+        nv = self.nv
+        f = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        return f(self.h)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            if self.active:
+                try:
+                    self.samples.append((nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM), self._reasons(),
+                                         nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0))
+                except Exception:
+                    pass
+            time.sleep(0.005)
+
+    def summary(self):
+        if not self.ok:
+            return None
+        self._stop.set()
+        s = self.samples
+        if not s:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mask = 0
+        for _, r, _ in s:
+            mask |= r
+        reasons = sorted(n for b, n in self.NAMES.items() if mask & b and b != 0x1)
+        return {"sm_mhz": statistics.median(x[0] for x in s), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(s), "power_w_max": round(max(x[2] for x in s), 1), "source": "nvml"}
+
+
+# ------------------------------------------------------------------ oracle timing
+
+
+def time_oracle(inp, tokens: int):
+    """Wall time of the float64 oracle over the first `tokens` tokens of a
+    single-sequence problem (all heads, all host cores)."""
+    import oracle
+    sl = slice(0, tokens)
+    params = (inp.conv_w, inp.A_log, inp.dt_bias, inp.norm_w)
+    t0 = time.perf_counter()
+    oracle.prefill(inp.geo, params, inp.f32("qkv")[sl], inp.f32("z")[sl], inp.f32("a")[sl], inp.f32("b")[sl],
+                   [0, tokens], inp.f32("conv_state"), inp.state)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(inp, budget_s=8.0):
+    import oracle
+    cores = oracle.default_threads()
+    probe = 128
+    dt = time_oracle(inp, probe)
+    tokens = int(min(inp.total_tokens, max(probe, budget_s / max(dt, 1e-6) * probe)))
+    dt = time_oracle(inp, tokens)
+    return {"value": round(tokens / dt, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"float64 oracle, first {tokens} of the 4096 prefill tokens, all 48 value heads, "
+                      f"{cores} threads, {dt:.2f} s wall"}
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return 0
+    w = gi.WORKLOADS[PREFILL_WORKLOAD]
+    inp = gi.workload_inputs(PREFILL_WORKLOAD)
+    import oracle
+    cores = oracle.default_threads()
+    # size each step so the whole run stays near a minute
+    probe = time_oracle(inp, 64) / 64
+    per_step = 60.0 / max(1, args.steps + args.warmup)
+    tokens = int(max(16, min(inp.total_tokens, per_step / max(probe, 1e-9))))
+    for _ in range(args.warmup):
+        time_oracle(inp, tokens)
+    t = 0.0
+    for _ in range(args.steps):
+        t += time_oracle(inp, tokens)
+    value = tokens * args.steps / t
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1000 * t / args.steps, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "GDN prefill, B=1, T=4096, 16 key / 48 value heads x 128, chunk 64, bf16 inputs",
+                       "global_batch": 1, "seq_len": 4096, "chunk": w["chunks"][0], "parallelism": "none (CPU)"},
+            "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"first {tokens} tokens of the 4096-token prefill per step, all heads"},
+            "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+
+
+def run_gdn(args, rank, world, local_rank):
+    import torch
+    import linear_attention_recurrence_deltanet_b200 as gdn
+    from linear_attention_recurrence_deltanet_b200.device import io_tensor
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
+    stream = torch.cuda.current_stream()
+    pk = peaks()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---------------- prefill workload (B=1, T=4096)
+    w = gi.WORKLOADS[PREFILL_WORKLOAD]
+    inp = gi.workload_inputs(PREFILL_WORKLOAD)
+    geo, C = inp.geo, w["chunks"][0]
+    cfg = gdn.make_config(geo)
+    T = inp.total_tokens
+    params = tuple(torch.from_numpy(np.ascontiguousarray(p)).cuda() for p in (inp.conv_w, inp.A_log, inp.dt_bias,
+                                                                               inp.norm_w))
+    cu_h = np.ascontiguousarray(inp.cu_seqlens, np.int32)
+    cu_d = torch.from_numpy(cu_h).cuda()
+    sets = []
+    base = [io_tensor(x) for x in (inp.qkv, inp.z, inp.a, inp.b)]
+    for r in range(ROTATE):
+        sets.append(dict(qkv=base[0].clone(), z=base[1].clone(), a=base[2].clone(), b=base[3].clone(),
+                         o=torch.empty((T, geo.value_dim), dtype=torch.bfloat16, device="cuda"),
+                         conv=io_tensor(inp.conv_state), state=torch.zeros((1, geo.num_v_heads, 128, 128),
+                                                                           dtype=torch.float32, device="cuda")))
+    del base
+    ws = torch.empty(gdn.prefill_workspace_size(cfg, T, 1, C) + 256, dtype=torch.uint8, device="cuda")
+    flags = gdn.ZERO_INIT_STATE | (gdn.PREFILL_RECURRENT if args.recurrent else 0)
+
+    def prefill(i):
+        s = sets[i % ROTATE]
+        gdn.prefill(cfg, params, s["qkv"], s["z"], s["a"], s["b"], cu_d, cu_h, C, flags, s["conv"], s["state"],
+                    s["o"], ws, stream=stream)
+
+    clocks = ClockSampler(local_rank)
+    for i in range(args.warmup):
+        prefill(i)
+    barrier()
+    gdn.profiler_reset()
+    gdn.profiler_enable(True)
+    gdn.launch_count_reset()
+    clocks.active = True
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(args.steps):
+        prefill(i)
+    ev1.record(stream)
+    barrier()
+    clocks.active = False
+    launches = gdn.launch_count()
+    gdn.profiler_enable(False)
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1))
+    kid = gdn.K.PREFILL_RECURRENT if args.recurrent else None
+    per_kernel = {gdn.kernel_name(k): gdn.profiler_read(k) for k in range(gdn.K.COUNT)}
+    if kid is None:  # the dominant prefill kernel is whichever mixer kernel ran
+        kid = max((gdn.K.PREFILL_CHUNKED, gdn.K.PREFILL_RECURRENT), key=lambda k: per_kernel[gdn.kernel_name(k)][1])
+    kname = gdn.kernel_name(kid)
+    n_launch, k_ms = per_kernel[kname]
+    k_avg_ms = max_over_ranks(k_ms / max(1, n_launch))
+    ms_per_step = ms_total / args.steps
+    value = world * T * args.steps / (ms_total / 1000.0)
+    pbytes = prefill_bytes(geo, [T], zero_state=True)
+    src = source_hash("prefill_recurrent.cu" if kid == gdn.K.PREFILL_RECURRENT else "prefill_chunked.cu")
+    roof_p = {"bound": "hbm", "achieved": round(pbytes / (k_avg_ms / 1000.0) / 1e9, 1), "peak": pk["hbm"],
+              "unit": "GB/s", "frac": round(pbytes / (k_avg_ms / 1000.0) / 1e9 / pk["hbm"], 4),
+              "traffic": measured_traffic(kname + ":" + PREFILL_WORKLOAD, src), "kernel": kname,
+              "kernel_ms": round(k_avg_ms, 5), "algorithmic_bytes": pbytes, "peak_source": pk["src"]}
+    kernel_share = {k: {"launches": v[0], "ms": round(v[1], 3)} for k, v in per_kernel.items() if v[0]}
+
+    # ---------------- end to end: pinned host inputs -> device -> prefill -> host output
+    e2e_steps = max(3, min(args.steps, 20))
+    pin = {k: sets[0][k].cpu().pin_memory() for k in ("qkv", "z", "a", "b")}
+    o_host = torch.empty_like(sets[0]["o"], device="cpu").pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = o_host.numel() * o_host.element_size()
+
+    def e2e_step():
+        s = sets[0]
+        for k in ("qkv", "z", "a", "b"):
+            s[k].copy_(pin[k], non_blocking=True)
+        gdn.prefill(cfg, params, s["qkv"], s["z"], s["a"], s["b"], cu_d, cu_h, C, flags, s["conv"], s["state"],
+                    s["o"], ws, stream=stream)
+        o_host.copy_(s["o"], non_blocking=True)
+
+    e2e_step()
+    barrier()
+    ev0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    ev1.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1)) / e2e_steps
+    e2e = {"value": round(world * T / (e2e_ms / 1000.0), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4), "steps": e2e_steps}
+    del sets, pin
+    torch.cuda.empty_cache()
+
+    # ---------------- decode workload (64 sequences, 1000 steps)
+    wd = gi.WORKLOADS[DECODE_WORKLOAD]
+    gd, seed, N = wd["geo"], wd["seed"], 64
+    dparams = tuple(torch.from_numpy(np.ascontiguousarray(p)).cuda() for p in gi.make_params(gd, seed))
+    conv0, st0 = gi.make_initial_state(gd, N, seed, zero=False)
+    conv = io_tensor(conv0)
+    st = torch.from_numpy(st0).cuda()
+    dsteps = args.decode_steps
+    toks = [gi.make_decode_step_tokens(gd, N, seed, s) for s in range(dsteps)]
+    dq = torch.stack([io_tensor(t[0]) for t in toks])
+    dz = torch.stack([io_tensor(t[1]) for t in toks])
+    da = torch.stack([io_tensor(t[2]) for t in toks])
+    db = torch.stack([io_tensor(t[3]) for t in toks])
+    del toks
+    do = torch.empty((N, gd.value_dim), dtype=torch.bfloat16, device="cuda")
+    for s in range(min(20, dsteps)):  # warm-up on the first steps' inputs, then restart from the initial state
+        gdn.decode_step(cfg, dparams, dq[s], dz[s], da[s], db[s], N, conv, st, do, stream=stream)
+    conv.copy_(io_tensor(conv0))
+    st.copy_(torch.from_numpy(st0))
+    barrier()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(dsteps + 1)]
+    gdn.profiler_reset()
+    gdn.profiler_enable(True)
+    clocks.active = True
+    evs[0].record(stream)
+    for s in range(dsteps):
+        gdn.decode_step(cfg, dparams, dq[s], dz[s], da[s], db[s], N, conv, st, do, stream=stream)
+        evs[s + 1].record(stream)
+    barrier()
+    clocks.active = False
+    gdn.profiler_enable(False)
+    step_ms = [evs[s].elapsed_time(evs[s + 1]) for s in range(dsteps)]
+    dn, dms = gdn.profiler_read(gdn.K.DECODE)
+    d_kernel_ms = max_over_ranks(dms / max(1, dn))
+    d_mean = max_over_ranks(sum(step_ms) / dsteps)
+    dbytes = decode_bytes(gd, N)
+    roof_d = {"bound": "hbm", "achieved": round(dbytes / (d_kernel_ms / 1000.0) / 1e9, 1), "peak": pk["hbm"],
+              "unit": "GB/s", "frac": round(dbytes / (d_kernel_ms / 1000.0) / 1e9 / pk["hbm"], 4),
+              "traffic": measured_traffic("decode:" + DECODE_WORKLOAD, source_hash("decode.cu")), "kernel": "decode",
+              "kernel_ms": round(d_kernel_ms, 5), "algorithmic_bytes": dbytes, "peak_source": pk["src"]}
+    decode = {"value": round(world * N / (d_mean / 1000.0), 1), "unit": "tokens/s", "ms_per_step": round(d_mean, 5),
+              "median_ms": round(statistics.median(step_ms), 5), "steps": dsteps, "num_seqs": N, "roofline": roof_d,
+              "workload": "GDN decode, 64 sequences x 1 token, 16 key / 48 value heads x 128, bf16 inputs, "
+                          "fp32 states ~N(0,0.02), fresh inputs every step"}
+
+    clk = clocks.summary()
+    cpu = cpu_baseline(inp) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "GDN prefill, B=1, T=4096, 16 key / 48 value heads x 128, chunk 64, bf16 inputs, "
+                                   "fp32 state from zero", "global_batch": world, "seq_len": T, "chunk": C,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": f"inputs rotate over {ROTATE} sets (> 4x L2) between steps"},
+            "roofline": roof_p, "decode": decode, "e2e": e2e, "gpu_launches": launches,
+            "kernels": kernel_share, "clocks": clk, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["gdn", "reference"], default="gdn")
+    ap.add_argument("--decode-steps", type=int, default=DECODE_STEPS)
+    ap.add_argument("--recurrent", action="store_true", help="time the token-recurrent prefill kernel")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+    return run_gdn(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

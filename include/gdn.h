@@ -1,0 +1,225 @@
+/*
+ * gdn.h -- C ABI of libgdn.so, the Gated DeltaNet (GDN) token mixer on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The mixer is the one the reference pages build for Qwen3.8's hybrid
+ * 3-GDN + 1-attention layers: "causal depthwise Conv1D, Gated DeltaNet
+ * recurrence, and recurrent-state cache", with "separately tuned GDN prefill
+ * and single-step decode behind one semantic interface" (DS4Server issue
+ * #88, "Add a performance-parity Qwen3.8-27B Q4 and Q8 text backend on
+ * Metal", section Scope), in the "16-key/48-value-head GDN geometry,
+ * convolution width 4, fp32 recurrent state, sigmoid output gate, and exact
+ * L2-normalization epsilon placement" with "zero-centered norms" (DS4Server
+ * issue #95, "Implement the Qwen3.8 Flash Next Rust and Metal text core",
+ * section Implementation).
+ *
+ * Per token t and value head h (key head kh = h / (Hv/Hk)):
+ *   u      = SiLU(causal depthwise conv, width W, over the raw q/k/v channels)
+ *   q^     = q_scale * q / sqrt(sum q^2 + l2_eps),  k^ = k / sqrt(sum k^2 + l2_eps)
+ *   g      = -exp(A_log[h]) * softplus(a + dt_bias[h]),  alpha = exp(g),  beta = sigmoid(b)
+ *   S      = alpha*S + beta * k^ (v - alpha * S^T k^)^T      (S is d_k x d_v, fp32)
+ *   o      = S^T q^
+ *   out_j  = o_j / sqrt(mean(o^2) + norm_eps) * (1 + norm_w[j]) * sigmoid(z_j)
+ *
+ * Conventions shared by every entry point
+ *   - Memory: every pointer is device memory owned by the caller unless a
+ *     parameter says otherwise; the library never allocates device memory.
+ *     Tensors are dense row-major and 16-byte aligned (a and b: aligned to
+ *     their element size).
+ *   - Streams: every call is asynchronous on the caller's stream and
+ *     stream-ordered; nothing blocks the host except where stated.
+ *   - Validation: every argument is checked on the host before anything is
+ *     launched.  On any error no kernel runs and no buffer is written
+ *     ("fail before unsafe or partial execution", issue #95 implementation
+ *     comment); the message is available from gdn_last_error().
+ *   - Layouts (N sequences, T_tot packed tokens, C_conv = 2*Hk*d_k + Hv*d_v):
+ *       qkv        [T_tot, C_conv]   io dtype; channels q (Hk*d_k), k (Hk*d_k), v (Hv*d_v),
+ *                                    each head's slice contiguous
+ *       z          [T_tot, Hv*d_v]   io dtype
+ *       a, b       [T_tot, Hv]       io dtype
+ *       o          [T_tot, Hv*d_v]   io dtype (written)
+ *       conv_state [N, W-1, C_conv]  io dtype; the last W-1 raw inputs, oldest first
+ *       state      [N, Hv, d_v, d_k] fp32; element [n,h,j,i] = S[i][j] (S transposed)
+ *       conv_w     [C_conv, W] fp32; tap W-1 multiplies the current token
+ *       A_log, dt_bias [Hv] fp32;  norm_w [d_v] fp32 (applied as 1 + w)
+ *   - Supported geometry: Hv % Hk == 0, d_k == d_v in {32, 64, 128}, W == 4,
+ *     io dtype fp32 or bf16.  Anything else returns GDN_E_UNSUPPORTED.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GDN_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+typedef struct CUstream_st* gdn_stream_t; /* a cudaStream_t; NULL = the legacy default stream */
+
+typedef enum {
+  GDN_OK = 0,
+  GDN_E_INVAL = -1,          /* bad pointer, size, alignment or cu_seqlens */
+  GDN_E_UNSUPPORTED = -2,    /* geometry or dtype this build does not run */
+  GDN_E_WORKSPACE = -3,      /* workspace missing or smaller than gdn_prefill_workspace_size() */
+  GDN_E_CUDA = -4,           /* a CUDA runtime call failed; see gdn_last_error() */
+  GDN_E_BLOB_FORMAT = -5,    /* state blob: bad magic, size or layout id */
+  GDN_E_BLOB_VERSION = -6,   /* state blob: unknown format version */
+  GDN_E_BLOB_GEOMETRY = -7,  /* state blob: saved under another geometry or dtype */
+  GDN_E_BLOB_CHECKSUM = -8,  /* state blob: payload does not match its checksum */
+  GDN_E_DEVICE = -9          /* no usable CUDA device, or not an sm_100 device */
+} gdn_status;
+
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
+
+typedef struct {
+  int32_t num_k_heads; /* Hk */
+  int32_t num_v_heads; /* Hv; value heads G*kh .. G*kh+G-1 (G = Hv/Hk) share key head kh */
+  int32_t head_k_dim;  /* d_k */
+  int32_t head_v_dim;  /* d_v */
+  int32_t conv_width;  /* W */
+  float l2_eps;        /* inside the square root of the L2 norm's sum of squares */
+  float norm_eps;      /* inside the square root of the output RMSNorm's mean square */
+  float q_scale;       /* factor on the normalised query (1.0 for the plain rule) */
+  int32_t io_dtype;    /* gdn_dtype of qkv, z, a, b, o and conv_state */
+} gdn_config;
+
+typedef struct {
+  const float* conv_w;  /* [C_conv, W] */
+  const float* A_log;   /* [Hv] */
+  const float* dt_bias; /* [Hv] */
+  const float* norm_w;  /* [d_v] */
+} gdn_params;
+
+/* flags of gdn_prefill */
+#define GDN_ZERO_INIT_STATE 0x1u /* ignore the incoming recurrent state: start from S = 0 */
+#define GDN_ZERO_INIT_CONV 0x2u  /* ignore the incoming conv history: treat it as zeros */
+#define GDN_PREFILL_RECURRENT 0x4u /* run the token-recurrent fp32 kernel instead of the chunked one */
+
+/* --------------------------------------------------------------------------
+ * Causal depthwise Conv1D + SiLU over the q/k/v channels (issue #88, Scope:
+ * "causal depthwise Conv1D"; width 4 per issue #95, Implementation).
+ *
+ * gdn_conv_prefill: y[t, c] = SiLU(sum_j conv_w[c, j] * x~[t - (W-1) + j, c])
+ * where x~ is the sequence's inputs preceded by its conv_state.  cu_seqlens
+ * [N+1] int32 gives the packed sequence boundaries (cu[0] = 0, non-decreasing,
+ * cu[N] = T_tot); the device and host copies must hold the same values (the
+ * host copy is validated and sizes the launch).  conv_state is read, then
+ * replaced by the last W-1 raw inputs of each sequence (bit-exact copies).
+ * y [T_tot, C_conv] in the io dtype.  Length-0 sequences are allowed.
+ */
+GDN_API gdn_status gdn_conv_prefill(const gdn_config* cfg, const void* x, const float* conv_w,
+                            const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host, int32_t num_seqs,
+                            void* conv_state, void* y, gdn_stream_t stream);
+
+/* gdn_conv_step: the same for one token per sequence.  x and y are [N, C_conv]. */
+GDN_API gdn_status gdn_conv_step(const gdn_config* cfg, const void* x, const float* conv_w, int32_t num_seqs,
+                         void* conv_state, void* y, gdn_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * Chunked prefill over packed variable-length sequences ("separately tuned
+ * GDN prefill", issue #88, Scope; "prefill/decode equivalence across chunk
+ * sizes", issue #95, Verification).
+ *
+ * Workspace: caller-provided device scratch of at least the size that
+ * gdn_prefill_workspace_size() returns for the same (cfg, total_tokens,
+ * num_seqs, chunk_size); 256-byte aligned.
+ */
+GDN_API gdn_status gdn_prefill_workspace_size(const gdn_config* cfg, int64_t total_tokens, int32_t num_seqs,
+                                      int32_t chunk_size, size_t* bytes);
+
+/* gdn_prefill: runs the whole mixer over every token of every sequence.
+ *   chunk_size: 16, 32, 64 or 128 (tokens per chunk of the chunkwise form;
+ *               chunks restart at each sequence start).
+ *   flags:      GDN_ZERO_INIT_STATE / GDN_ZERO_INIT_CONV / GDN_PREFILL_RECURRENT.
+ *   conv_state and state are read and updated in place; o is written.
+ * The chunked kernel runs when io dtype is bf16 and d_k = d_v = 128; every
+ * other supported case (and GDN_PREFILL_RECURRENT) runs the token-recurrent
+ * fp32 kernel.  Both compute in fp32 with an fp32 state. */
+GDN_API gdn_status gdn_prefill(const gdn_config* cfg, const gdn_params* params, const void* qkv, const void* z,
+                       const void* a, const void* b, const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host,
+                       int32_t num_seqs, int32_t chunk_size, uint32_t flags, void* conv_state, float* state,
+                       void* o, void* workspace, size_t workspace_bytes, gdn_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * Single-step decode ("single-step decode", issue #88, Scope): every one of
+ * num_seqs sequences advances by one token.  qkv [N, C_conv], z [N, Hv*d_v],
+ * a, b [N, Hv], o [N, Hv*d_v].  One fused kernel: conv step, L2 norms, gates,
+ * rank-1 state update, readout, RMSNorm and output gate; each state is read
+ * and written once.  conv_state and state are updated in place. */
+GDN_API gdn_status gdn_decode_step(const gdn_config* cfg, const gdn_params* params, const void* qkv, const void* z,
+                           const void* a, const void* b, int32_t num_seqs, void* conv_state, float* state, void* o,
+                           gdn_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * Versioned state checkpoint of one sequence ("Persist every GDN convolution
+ * and recurrent component in session checkpoints with versioned validation",
+ * issue #95, Implementation; "identical ... BF16 convolution bytes, and fp32
+ * recurrent bytes after checkpoint/resume", implementation comment).
+ *
+ * Blob = 128-byte header {magic "GDNSTATE", format version, geometry, io
+ * dtype, state dtype, layout id, payload bytes, 64-bit checksum} followed by
+ * the sequence's conv history bytes ([W-1, C_conv], io dtype) and recurrent
+ * state bytes ([Hv, d_v, d_k], fp32), copied unchanged.
+ *
+ * blob may be host or device memory (detected).  With a host blob the call
+ * synchronises the stream before returning (save) or before validating
+ * (restore); with a device blob it synchronises once to read the header and
+ * checksum.  Restore checks every header field and the checksum before it
+ * writes anything; on a mismatch it returns the matching GDN_E_BLOB_* code and
+ * leaves conv_state and state untouched.
+ */
+GDN_API gdn_status gdn_state_blob_size(const gdn_config* cfg, size_t* bytes);
+GDN_API gdn_status gdn_state_save(const gdn_config* cfg, const void* conv_state, const float* state, int32_t seq,
+                          void* blob, size_t blob_bytes, gdn_stream_t stream);
+GDN_API gdn_status gdn_state_restore(const gdn_config* cfg, const void* blob, size_t blob_bytes, int32_t seq,
+                             void* conv_state, float* state, gdn_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * Diagnostics and measurement.
+ *
+ * gdn_get_device_status: reads and clears the device status word, which a
+ * kernel sets (never traps) when an internal wait reaches its iteration limit
+ * or a debug bounds check fails.  0 = clean.  Synchronises the stream.
+ * gdn_last_error: message of the calling thread's last failed call.
+ * gdn_launch_count: kernels this library has launched since load or reset.
+ * gdn_profiler_*: when enabled, every launch is bracketed by CUDA events on
+ * its own stream; gdn_profiler_read synchronises those events and returns the
+ * launch count and summed device time of one kernel id (see gdn_kernel_name).
+ */
+GDN_API gdn_status gdn_get_device_status(int32_t* code, gdn_stream_t stream);
+GDN_API const char* gdn_last_error(void);
+GDN_API int32_t gdn_abi_version(void);
+GDN_API int64_t gdn_launch_count(void);
+GDN_API void gdn_launch_count_reset(void);
+
+typedef enum {
+  GDN_K_CONV_PREFILL = 0,
+  GDN_K_CONV_STEP = 1,
+  GDN_K_CONV_HISTORY = 2,
+  GDN_K_SCHEDULE = 3,
+  GDN_K_PREFILL_RECURRENT = 4,
+  GDN_K_PREFILL_CHUNKED = 5,
+  GDN_K_DECODE = 6,
+  GDN_K_STATE_CHECKSUM = 7,
+  GDN_K_COUNT = 8
+} gdn_kernel_id;
+
+GDN_API const char* gdn_kernel_name(int32_t kernel_id);
+GDN_API gdn_status gdn_profiler_enable(int32_t enable);
+GDN_API gdn_status gdn_profiler_reset(void);
+GDN_API gdn_status gdn_profiler_read(int32_t kernel_id, int64_t* launches, double* total_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

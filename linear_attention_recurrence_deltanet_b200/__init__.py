@@ -1,0 +1,242 @@
+"""Python binding of libgdn.so, the Gated DeltaNet token mixer for B200.
+
+Argument marshalling only: every function here hands device pointers of
+torch tensors, sizes and the current CUDA stream to one C entry point of
+``libgdn.so`` (declared in ``include/gdn.h``) and raises ``GdnError`` on a
+non-zero status.  There is no fallback: if the library is missing or was not
+built, the first call raises.  Build it with
+``python -m linear_attention_recurrence_deltanet_b200.build``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+
+__all__ = [
+    "GdnError", "Config", "Params", "lib", "make_config", "conv_prefill", "conv_step", "prefill_workspace_size",
+    "prefill", "decode_step", "state_blob_size", "state_save", "state_restore", "device_status", "last_error",
+    "abi_version", "launch_count", "launch_count_reset", "profiler_enable", "profiler_reset", "profiler_read",
+    "kernel_name", "EXPORTS", "ZERO_INIT_STATE", "ZERO_INIT_CONV", "PREFILL_RECURRENT", "K",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
+
+ZERO_INIT_STATE = 0x1
+ZERO_INIT_CONV = 0x2
+PREFILL_RECURRENT = 0x4
+
+F32, BF16 = 0, 1
+
+STATUS = {0: "GDN_OK", -1: "GDN_E_INVAL", -2: "GDN_E_UNSUPPORTED", -3: "GDN_E_WORKSPACE", -4: "GDN_E_CUDA",
+          -5: "GDN_E_BLOB_FORMAT", -6: "GDN_E_BLOB_VERSION", -7: "GDN_E_BLOB_GEOMETRY", -8: "GDN_E_BLOB_CHECKSUM",
+          -9: "GDN_E_DEVICE"}
+
+
+class K:
+    """Kernel ids of the profiler (gdn_kernel_id)."""
+    CONV_PREFILL, CONV_STEP, CONV_HISTORY, SCHEDULE, PREFILL_RECURRENT, PREFILL_CHUNKED, DECODE, STATE_CHECKSUM = \
+        range(8)
+    COUNT = 8
+
+
+# Every symbol include/gdn.h declares.
+EXPORTS = [
+    "gdn_conv_prefill", "gdn_conv_step", "gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode_step",
+    "gdn_state_blob_size", "gdn_state_save", "gdn_state_restore", "gdn_get_device_status", "gdn_last_error",
+    "gdn_abi_version", "gdn_launch_count", "gdn_launch_count_reset", "gdn_kernel_name", "gdn_profiler_enable",
+    "gdn_profiler_reset", "gdn_profiler_read",
+]
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+        self.name = STATUS.get(status, str(status))
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("num_k_heads", ctypes.c_int32), ("num_v_heads", ctypes.c_int32), ("head_k_dim", ctypes.c_int32),
+                ("head_v_dim", ctypes.c_int32), ("conv_width", ctypes.c_int32), ("l2_eps", ctypes.c_float),
+                ("norm_eps", ctypes.c_float), ("q_scale", ctypes.c_float), ("io_dtype", ctypes.c_int32)]
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("conv_w", ctypes.c_void_p), ("A_log", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p),
+                ("norm_w", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libgdn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m linear_attention_recurrence_deltanet_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I32, I64, U32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_size_t
+        sig = {
+            "gdn_conv_prefill": [P, P, P, P, P, I32, P, P, P],
+            "gdn_conv_step": [P, P, P, I32, P, P, P],
+            "gdn_prefill_workspace_size": [P, I64, I32, I32, P],
+            "gdn_prefill": [P, P, P, P, P, P, P, P, I32, I32, U32, P, P, P, P, SZ, P],
+            "gdn_decode_step": [P, P, P, P, P, P, I32, P, P, P, P],
+            "gdn_state_blob_size": [P, P],
+            "gdn_state_save": [P, P, P, I32, P, SZ, P],
+            "gdn_state_restore": [P, P, SZ, I32, P, P, P],
+            "gdn_get_device_status": [P, P],
+            "gdn_profiler_enable": [I32],
+            "gdn_profiler_reset": [],
+            "gdn_profiler_read": [I32, P, P],
+        }
+        for name, args in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = I32
+        L.gdn_last_error.restype = ctypes.c_char_p
+        L.gdn_kernel_name.restype = ctypes.c_char_p
+        L.gdn_kernel_name.argtypes = [I32]
+        L.gdn_abi_version.restype = I32
+        L.gdn_launch_count.restype = I64
+        L.gdn_launch_count_reset.restype = None
+        _lib = L
+    return _lib
+
+
+def last_error() -> str:
+    return lib().gdn_last_error().decode()
+
+
+def _check(rc: int):
+    if rc != 0:
+        raise GdnError(rc, last_error())
+
+
+def make_config(geo) -> Config:
+    """Config from an ``inputs.Geometry`` (or any object with the same fields)."""
+    return Config(geo.num_k_heads, geo.num_v_heads, geo.head_k_dim, geo.head_v_dim, geo.conv_width, geo.l2_eps,
+                  geo.norm_eps, geo.q_scale, BF16 if geo.io_dtype == "bf16" else F32)
+
+
+def _p(t) -> Optional[int]:
+    """Data pointer of a torch tensor / numpy array (None passes NULL)."""
+    if t is None:
+        return None
+    if isinstance(t, np.ndarray):
+        return t.ctypes.data
+    return t.data_ptr()
+
+
+def _stream(stream=None) -> Optional[int]:
+    if stream is not None:
+        return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _host_cu(cu_host) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(cu_host), dtype=np.int32)
+
+
+def _params(conv_w, A_log, dt_bias, norm_w) -> Params:
+    return Params(_p(conv_w), _p(A_log), _p(dt_bias), _p(norm_w))
+
+
+def conv_prefill(cfg, x, conv_w, cu_dev, cu_host, conv_state, y, stream=None):
+    cu_h = _host_cu(cu_host)
+    _check(lib().gdn_conv_prefill(ctypes.byref(cfg), _p(x), _p(conv_w), _p(cu_dev), cu_h.ctypes.data,
+                                  cu_h.size - 1, _p(conv_state), _p(y), _stream(stream)))
+
+
+def conv_step(cfg, x, conv_w, num_seqs, conv_state, y, stream=None):
+    _check(lib().gdn_conv_step(ctypes.byref(cfg), _p(x), _p(conv_w), num_seqs, _p(conv_state), _p(y),
+                               _stream(stream)))
+
+
+def prefill_workspace_size(cfg, total_tokens: int, num_seqs: int, chunk_size: int) -> int:
+    out = ctypes.c_size_t()
+    _check(lib().gdn_prefill_workspace_size(ctypes.byref(cfg), total_tokens, num_seqs, chunk_size,
+                                            ctypes.byref(out)))
+    return out.value
+
+
+def prefill(cfg, params, qkv, z, a, b, cu_dev, cu_host, chunk_size, flags, conv_state, state, o, workspace,
+            workspace_bytes=None, stream=None):
+    """gdn_prefill.  params = (conv_w, A_log, dt_bias, norm_w) device tensors."""
+    cu_h = _host_cu(cu_host)
+    prm = _params(*params)
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().gdn_prefill(ctypes.byref(cfg), ctypes.byref(prm), _p(qkv), _p(z), _p(a), _p(b), _p(cu_dev),
+                             cu_h.ctypes.data, cu_h.size - 1, chunk_size, flags, _p(conv_state), _p(state), _p(o),
+                             _p(workspace), workspace_bytes, _stream(stream)))
+
+
+def decode_step(cfg, params, qkv, z, a, b, num_seqs, conv_state, state, o, stream=None):
+    prm = _params(*params)
+    _check(lib().gdn_decode_step(ctypes.byref(cfg), ctypes.byref(prm), _p(qkv), _p(z), _p(a), _p(b), num_seqs,
+                                 _p(conv_state), _p(state), _p(o), _stream(stream)))
+
+
+def state_blob_size(cfg) -> int:
+    out = ctypes.c_size_t()
+    _check(lib().gdn_state_blob_size(ctypes.byref(cfg), ctypes.byref(out)))
+    return out.value
+
+
+def _nbytes(t) -> int:
+    return t.nbytes if isinstance(t, np.ndarray) else t.numel() * t.element_size()
+
+
+def state_save(cfg, conv_state, state, seq, blob, stream=None):
+    _check(lib().gdn_state_save(ctypes.byref(cfg), _p(conv_state), _p(state), seq, _p(blob), _nbytes(blob),
+                                _stream(stream)))
+
+
+def state_restore(cfg, blob, seq, conv_state, state, stream=None):
+    _check(lib().gdn_state_restore(ctypes.byref(cfg), _p(blob), _nbytes(blob), seq, _p(conv_state), _p(state),
+                                   _stream(stream)))
+
+
+def device_status(stream=None) -> int:
+    code = ctypes.c_int32()
+    _check(lib().gdn_get_device_status(ctypes.byref(code), _stream(stream)))
+    return code.value
+
+
+def abi_version() -> int:
+    return lib().gdn_abi_version()
+
+
+def launch_count() -> int:
+    return lib().gdn_launch_count()
+
+
+def launch_count_reset():
+    lib().gdn_launch_count_reset()
+
+
+def kernel_name(kid: int) -> str:
+    return lib().gdn_kernel_name(kid).decode()
+
+
+def profiler_enable(on: bool = True):
+    _check(lib().gdn_profiler_enable(1 if on else 0))
+
+
+def profiler_reset():
+    _check(lib().gdn_profiler_reset())
+
+
+def profiler_read(kid: int):
+    """(launches, total device ms) of one kernel id since the last reset."""
+    n, ms = ctypes.c_int64(), ctypes.c_double()
+    _check(lib().gdn_profiler_read(kid, ctypes.byref(n), ctypes.byref(ms)))
+    return n.value, ms.value

@@ -1,0 +1,213 @@
+// Single-step GDN decode: one fused, HBM-bound kernel ("single-step decode",
+// DS4Server issue #88, section Scope; fp32 recurrent state, sigmoid output
+// gate, exact L2 epsilon placement: issue #95, section Implementation).
+//
+// One CTA per (sequence n, key head kh).  It owns the conv channels of q and k
+// of key head kh and of v for the G value heads that share it, so the rolling
+// conv history is read and rewritten by exactly one CTA (no race on the
+// shared q/k channels).  Per value head the state is stored transposed,
+// state[n,h,j,:] = column j of S (d_k contiguous floats), and the rank-1
+// update decomposes into independent rows:
+//   kappa_j = k^ . r_j,  rho_j = q^ . r_j              (r_j = old row j)
+//   delta_j = beta * (v_j - alpha * kappa_j)
+//   r_j'    = alpha * r_j + delta_j * k^               (written back once)
+//   o_j     = q^ . r_j' = alpha * rho_j + delta_j * (q^ . k^)
+// so every state byte crosses HBM exactly once in each direction.  Eight
+// lanes share a row (16-byte loads, 3 shuffle steps for the two dots); each
+// warp keeps two row groups of loads in flight.
+#include "../../include/gdn.h"
+#include "internal.h"
+
+namespace gdn {
+namespace {
+
+constexpr int kDecThreads = 256;
+constexpr int kDecWarps = kDecThreads / 32;
+constexpr int kUnroll = 2;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kDecThreads, 2)
+    decode_kernel(Dims d, const float* __restrict__ conv_w, const float* __restrict__ A_log,
+                  const float* __restrict__ dt_bias, const float* __restrict__ norm_w, const T* __restrict__ qkv,
+                  const T* __restrict__ z, const T* __restrict__ a, const T* __restrict__ b, T* __restrict__ hist,
+                  float* __restrict__ state, T* __restrict__ o) {
+  constexpr int F4 = D / 32;  // float4s of a row held by one lane (8 lanes per row)
+  extern __shared__ float smem[];
+  const int G = d.G;
+  const int nch = (2 + G) * D;
+  float* u = smem;                 // [q (D) | k (D) | v of the G heads (G*D)] after conv + SiLU
+  float* osm = u + nch;            // [G*D] o before the output norm
+  float* gate = osm + G * D;       // alpha[G], beta[G]
+  __shared__ float red[3];         // q scale, k scale, q^.k^
+
+  const int n = blockIdx.x / d.Hk;
+  const int kh = blockIdx.x - n * d.Hk;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t C = d.C;
+  const int h0 = G * kh;  // first value head of this key head
+
+  // ---- conv step + SiLU for the owned channels; rotate the history
+  for (int idx = tid; idx < nch; idx += kDecThreads) {
+    const int64_t c = idx < D ? (int64_t)kh * D + idx
+                              : (idx < 2 * D ? (int64_t)d.Hk * D + (int64_t)kh * D + (idx - D)
+                                             : 2LL * d.Hk * D + (int64_t)h0 * D + (idx - 2 * D));
+    T* hp = hist + (int64_t)n * 3 * C + c;
+    const T h0v = hp[0], h1v = hp[C], h2v = hp[2 * C];
+    const T xv = qkv[(int64_t)n * C + c];
+    const float4 w = __ldg(reinterpret_cast<const float4*>(conv_w + c * 4));
+    const float y = w.x * to_f(h0v) + w.y * to_f(h1v) + w.z * to_f(h2v) + w.w * to_f(xv);
+    u[idx] = silu_f(y);
+    hp[0] = h1v;
+    hp[C] = h2v;
+    hp[2 * C] = xv;
+  }
+  if (tid < G) {
+    const int h = h0 + tid;
+    float g, al, be;
+    gates_f(ldg_f(a + (int64_t)n * d.Hv + h), dt_bias[h], A_log[h], ldg_f(b + (int64_t)n * d.Hv + h), g, al, be);
+    gate[tid] = al;
+    gate[G + tid] = be;
+  }
+  __syncthreads();
+
+  // ---- L2 norms of q and k (epsilon inside the square root of the sum)
+  if (warp == 0) {
+    float sq = 0.f, sk = 0.f, sqk = 0.f;
+    for (int i = lane; i < D; i += 32) {
+      const float qv = u[i], kv = u[D + i];
+      sq += qv * qv;
+      sk += kv * kv;
+      sqk += qv * kv;
+    }
+    sq = warp_sum(sq);
+    sk = warp_sum(sk);
+    sqk = warp_sum(sqk);
+    if (lane == 0) {
+      const float rq = d.q_scale * rsqrtf(sq + d.l2_eps), rk = rsqrtf(sk + d.l2_eps);
+      red[0] = rq;
+      red[1] = rk;
+      red[2] = rq * rk * sqk;
+    }
+  }
+  __syncthreads();
+
+  // ---- stream the G states of this key head, row by row
+  const int l8 = lane & 7, grp = lane >> 3;
+  float kq[F4][4], qq[F4][4];
+  {
+    const float rq = red[0], rk = red[1];
+#pragma unroll
+    for (int m = 0; m < F4; ++m)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        qq[m][e] = u[4 * (l8 + 8 * m) + e] * rq;
+        kq[m][e] = u[D + 4 * (l8 + 8 * m) + e] * rk;
+      }
+  }
+  const float qk = red[2];
+  const int rows = G * D;
+  const int groups = rows / 4;
+  float* st = state + ((int64_t)n * d.Hv + h0) * D * D;  // the G heads' rows are contiguous
+  for (int base = warp; base < groups; base += kDecWarps * kUnroll) {
+    float4 r[kUnroll][F4];
+#pragma unroll
+    for (int x = 0; x < kUnroll; ++x) {
+      const int g4 = base + x * kDecWarps;
+      if (g4 < groups) {
+        const float4* p = reinterpret_cast<const float4*>(st + (int64_t)(g4 * 4 + grp) * D);
+#pragma unroll
+        for (int m = 0; m < F4; ++m) r[x][m] = __ldcs(p + l8 + 8 * m);
+      }
+    }
+#pragma unroll
+    for (int x = 0; x < kUnroll; ++x) {
+      const int g4 = base + x * kDecWarps;
+      if (g4 < groups) {  // warp-uniform
+        const int row = g4 * 4 + grp;
+        float kap = 0.f, rho = 0.f;
+#pragma unroll
+        for (int m = 0; m < F4; ++m) {
+          kap += kq[m][0] * r[x][m].x + kq[m][1] * r[x][m].y + kq[m][2] * r[x][m].z + kq[m][3] * r[x][m].w;
+          rho += qq[m][0] * r[x][m].x + qq[m][1] * r[x][m].y + qq[m][2] * r[x][m].z + qq[m][3] * r[x][m].w;
+        }
+#pragma unroll
+        for (int off = 1; off < 8; off <<= 1) {
+          kap += __shfl_xor_sync(0xffffffffu, kap, off);
+          rho += __shfl_xor_sync(0xffffffffu, rho, off);
+        }
+        const int hh = row / D;
+        const float al = gate[hh], be = gate[G + hh];
+        const float delta = be * (u[2 * D + row] - al * kap);
+        float4* p = reinterpret_cast<float4*>(st + (int64_t)row * D);
+#pragma unroll
+        for (int m = 0; m < F4; ++m) {
+          float4 w4;
+          w4.x = al * r[x][m].x + delta * kq[m][0];
+          w4.y = al * r[x][m].y + delta * kq[m][1];
+          w4.z = al * r[x][m].z + delta * kq[m][2];
+          w4.w = al * r[x][m].w + delta * kq[m][3];
+          __stcs(p + l8 + 8 * m, w4);
+        }
+        if (l8 == 0) osm[row] = al * rho + delta * qk;
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- zero-centred RMSNorm over d_v, times sigmoid(z); one rounding to io dtype
+  for (int hh = warp; hh < G; hh += kDecWarps) {
+    float ss = 0.f;
+    for (int j = lane; j < D; j += 32) ss += osm[hh * D + j] * osm[hh * D + j];
+    ss = warp_sum(ss);
+    const float r = rsqrtf(ss / D + d.norm_eps);
+    const int64_t off = ((int64_t)n * d.Hv + h0 + hh) * D;
+    for (int j = lane; j < D; j += 32) {
+      const float zz = ldg_f(z + off + j);
+      o[off + j] = from_f<T>(osm[hh * D + j] * r * (1.0f + norm_w[j]) * sigmoid_f(zz));
+    }
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch_t(const Dims& d, const float* conv_w, const float* A_log, const float* dt_bias,
+                     const float* norm_w, const void* qkv, const void* z, const void* a, const void* b, int32_t N,
+                     void* hist, float* state, void* o, cudaStream_t stream) {
+  const size_t smem = (size_t)((2 + d.G) * D + d.G * D + 2 * d.G) * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  LaunchScope scope(GDN_K_DECODE, stream);
+  decode_kernel<T, D><<<(unsigned)((int64_t)N * d.Hk), kDecThreads, smem, stream>>>(
+      d, conv_w, A_log, dt_bias, norm_w, (const T*)qkv, (const T*)z, (const T*)a, (const T*)b, (T*)hist, state,
+      (T*)o);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode_step(const Dims& d, bool bf16, const float* conv_w, const float* A_log,
+                               const float* dt_bias, const float* norm_w, const void* qkv, const void* z,
+                               const void* a, const void* b, int32_t N, void* conv_state, float* state, void* o,
+                               cudaStream_t stream) {
+  if (N <= 0) return cudaSuccess;
+#define GDN_DEC(T, D) \
+  return launch_t<T, D>(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, N, conv_state, state, o, stream)
+  if (bf16) {
+    switch (d.dk) {
+      case 32: GDN_DEC(__nv_bfloat16, 32);
+      case 64: GDN_DEC(__nv_bfloat16, 64);
+      default: GDN_DEC(__nv_bfloat16, 128);
+    }
+  } else {
+    switch (d.dk) {
+      case 32: GDN_DEC(float, 32);
+      case 64: GDN_DEC(float, 64);
+      default: GDN_DEC(float, 128);
+    }
+  }
+#undef GDN_DEC
+}
+
+}  // namespace gdn

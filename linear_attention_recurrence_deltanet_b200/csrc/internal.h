@@ -1,0 +1,56 @@
+// Host-side launchers of the GDN kernels.  Each returns cudaSuccess or the
+// launch error; arguments are validated by the C-ABI layer (api.cu) first.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace gdn {
+
+// Launch bracket used by every launcher: counts the launch and, when the
+// profiler is on, records CUDA events around it on `stream`.
+struct LaunchScope {
+  LaunchScope(int kernel_id, cudaStream_t stream);
+  ~LaunchScope();
+  int id;
+  cudaStream_t stream;
+  void* token;
+};
+
+// conv.cu
+cudaError_t launch_conv_prefill(const Dims& d, bool bf16, const void* x, const float* conv_w, const int32_t* cu,
+                                int32_t num_seqs, int32_t max_len, const void* conv_state, void* y,
+                                cudaStream_t stream);
+cudaError_t launch_conv_history(const Dims& d, bool bf16, const void* x, const int32_t* cu, int32_t num_seqs,
+                                bool zero_history, void* conv_state, cudaStream_t stream);
+cudaError_t launch_conv_step(const Dims& d, bool bf16, const void* x, const float* conv_w, int32_t num_seqs,
+                             void* conv_state, void* y, cudaStream_t stream);
+
+// schedule.cu -- varlen schedule: longest-first sequence order and the chunk map.
+struct ScheduleLayout {
+  size_t order_off, chunk_off_off, chunk_map_off, total_bytes;
+};
+ScheduleLayout schedule_layout(int32_t num_seqs, int64_t total_chunks);
+cudaError_t launch_schedule(const int32_t* cu, int32_t num_seqs, int32_t chunk_size, int64_t total_chunks,
+                            void* workspace, cudaStream_t stream);
+
+// decode.cu
+cudaError_t launch_decode_step(const Dims& d, bool bf16, const float* conv_w, const float* A_log,
+                               const float* dt_bias, const float* norm_w, const void* qkv, const void* z,
+                               const void* a, const void* b, int32_t num_seqs, void* conv_state, float* state,
+                               void* o, cudaStream_t stream);
+
+// prefill_recurrent.cu
+cudaError_t launch_prefill_recurrent(const Dims& d, bool bf16, const float* conv_w, const float* A_log,
+                                     const float* dt_bias, const float* norm_w, const void* qkv, const void* z,
+                                     const void* a, const void* b, const int32_t* cu, const int32_t* seq_order,
+                                     int32_t num_seqs, bool zero_state, bool zero_conv, const void* conv_state,
+                                     float* state, void* o, cudaStream_t stream);
+
+// checksum.cu
+cudaError_t launch_checksum(const void* payload, size_t bytes, unsigned long long* out, cudaStream_t stream);
+uint64_t host_checksum(const void* payload, size_t bytes);
+
+}  // namespace gdn

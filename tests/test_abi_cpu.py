@@ -1,0 +1,210 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and rejects bad arguments and bad state blobs on the host
+before touching any buffer."""
+
+import ctypes
+import os
+import re
+import struct
+
+import numpy as np
+import pytest
+
+import linear_attention_recurrence_deltanet_b200 as gdn
+from linear_attention_recurrence_deltanet_b200 import inputs as gi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from linear_attention_recurrence_deltanet_b200 import build
+    build.build()
+    yield
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "gdn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    L = gdn.lib()
+    declared = header_functions()
+    assert len(declared) >= 17
+    for name in declared:
+        assert hasattr(L, name), name
+    assert sorted(gdn.EXPORTS) == declared
+
+
+def test_abi_version_and_names():
+    assert gdn.abi_version() == 1
+    assert gdn.kernel_name(gdn.K.DECODE) == "decode"
+    assert gdn.kernel_name(99) == "unknown"
+
+
+def qwen_cfg(**kw):
+    return gdn.make_config(gi.Geometry(**kw))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(num_k_heads=16, num_v_heads=40), "GDN_E_INVAL"),       # Hv not a multiple of Hk
+    (dict(head_k_dim=96, head_v_dim=96), "GDN_E_UNSUPPORTED"),
+    (dict(head_k_dim=128, head_v_dim=64), "GDN_E_UNSUPPORTED"),
+    (dict(conv_width=3), "GDN_E_UNSUPPORTED"),
+    (dict(l2_eps=-1.0), "GDN_E_INVAL"),
+])
+def test_bad_config_rejected(kw, status):
+    with pytest.raises(gdn.GdnError) as e:
+        gdn.prefill_workspace_size(qwen_cfg(**kw), 4096, 1, 64)
+    assert e.value.name == status
+
+
+def test_workspace_size_and_bad_chunk():
+    cfg = qwen_cfg()
+    small = gdn.prefill_workspace_size(cfg, 4096, 1, 64)
+    big = gdn.prefill_workspace_size(cfg, 65536, 16, 16)
+    assert 0 < small < big
+    with pytest.raises(gdn.GdnError) as e:
+        gdn.prefill_workspace_size(cfg, 4096, 1, 48)
+    assert e.value.name == "GDN_E_INVAL"
+
+
+class FakeTensor:
+    """Host buffer with a data_ptr(), standing in for device memory in calls
+    that must fail during validation (nothing may be written)."""
+
+    def __init__(self, nbytes, fill=0x5A):
+        self.buf = np.full(nbytes + 64, fill, np.uint8)
+        off = (-self.buf.ctypes.data) % 64
+        self.view = self.buf[off:off + nbytes]
+
+    def data_ptr(self):
+        return self.view.ctypes.data
+
+    def numel(self):
+        return self.view.size
+
+    def element_size(self):
+        return 1
+
+
+def test_prefill_validation_rejects_before_launch():
+    geo = gi.Geometry()
+    cfg = gdn.make_config(geo)
+    T = 8
+    t = {k: FakeTensor(n) for k, n in dict(qkv=T * geo.conv_dim * 2, z=T * geo.value_dim * 2, a=T * 96, b=T * 96,
+                                           o=T * geo.value_dim * 2, conv=3 * geo.conv_dim * 2,
+                                           state=geo.num_v_heads * 128 * 128 * 4, ws=1 << 16).items()}
+    params = tuple(FakeTensor(n) for n in (geo.conv_dim * 16, 192, 192, 512))
+    cu_dev = FakeTensor(8)
+    snapshot = {k: v.view.copy() for k, v in t.items()}
+
+    def call(cu_host, chunk=64, flags=0, ws=t["ws"], wsb=None):
+        gdn.prefill(cfg, params, t["qkv"], t["z"], t["a"], t["b"], cu_dev, cu_host, chunk, flags, t["conv"],
+                    t["state"], t["o"], ws, workspace_bytes=wsb, stream=0)
+
+    cases = [
+        (dict(cu_host=[1, 8]), "GDN_E_INVAL"),            # cu[0] != 0
+        (dict(cu_host=[0, 8, 4]), "GDN_E_INVAL"),         # decreasing
+        (dict(cu_host=[0, 8], chunk=100), "GDN_E_INVAL"),
+        (dict(cu_host=[0, 8], flags=0x80), "GDN_E_INVAL"),
+        (dict(cu_host=[0, 8], wsb=16), "GDN_E_WORKSPACE"),
+    ]
+    for kw, status in cases:
+        with pytest.raises(gdn.GdnError) as e:
+            call(**kw)
+        assert e.value.name == status, (kw, e.value)
+    # misaligned output pointer
+    class Off(FakeTensor):
+        def data_ptr(self):
+            return self.view.ctypes.data + 2
+    bad_o = Off(T * geo.value_dim * 2 + 16)
+    with pytest.raises(gdn.GdnError) as e:
+        gdn.prefill(cfg, params, t["qkv"], t["z"], t["a"], t["b"], cu_dev, [0, 8], 64, 0, t["conv"], t["state"],
+                    bad_o, t["ws"], stream=0)
+    assert e.value.name == "GDN_E_INVAL" and "aligned" in str(e.value)
+    for k, v in t.items():
+        assert np.array_equal(v.view, snapshot[k]), k
+
+
+# ---------------------------------------------------------------- state blobs (host memory)
+
+MAGIC = b"GDNSTATE"
+
+
+def mix64(z):
+    M = (1 << 64) - 1
+    z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & M
+    z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & M
+    return z ^ (z >> 31)
+
+
+def checksum(payload: bytes) -> int:
+    w = np.frombuffer(payload, dtype="<u8")
+    M = (1 << 64) - 1
+    s = 0
+    for i, x in enumerate(w.tolist()):
+        s = (s + mix64((x + (i + 1) * 0x9E3779B97F4A7C15) & M)) & M
+    return s
+
+
+def make_blob(geo, version=1, io_dtype=None, layout=1, corrupt_payload=False, hk=None):
+    cb = 3 * geo.conv_dim * geo.io_bytes
+    sb = geo.num_v_heads * geo.head_v_dim * geo.head_k_dim * 4
+    rng = np.random.default_rng(0)
+    payload = rng.integers(0, 256, cb + sb, dtype=np.uint8).tobytes()
+    io = (1 if geo.io_dtype == "bf16" else 0) if io_dtype is None else io_dtype
+    hdr = struct.pack("<8sII8iQQQ", MAGIC, version, 128, hk or geo.num_k_heads, geo.num_v_heads, geo.head_k_dim,
+                      geo.head_v_dim, geo.conv_width, io, 0, layout, cb, sb, checksum(payload))
+    hdr = hdr + bytes(128 - len(hdr))
+    if corrupt_payload:
+        payload = payload[:100] + bytes([payload[100] ^ 1]) + payload[101:]
+    return np.frombuffer(hdr + payload, np.uint8).copy()
+
+
+def test_blob_size_matches_layout():
+    geo = gi.Geometry(num_k_heads=2, num_v_heads=4, head_k_dim=32, head_v_dim=32)
+    assert gdn.state_blob_size(gdn.make_config(geo)) == 128 + 3 * geo.conv_dim * 2 + 4 * 32 * 32 * 4
+
+
+@pytest.mark.parametrize("mut,status", [
+    (lambda b: b.__setitem__(0, ord("X")), "GDN_E_BLOB_FORMAT"),
+    (None, "GDN_E_BLOB_VERSION"),
+    (None, "GDN_E_BLOB_GEOMETRY"),
+    (None, "GDN_E_BLOB_CHECKSUM"),
+    (None, "GDN_E_BLOB_FORMAT_LAYOUT"),
+    (None, "GDN_E_BLOB_GEOMETRY_DTYPE"),
+])
+def test_corrupt_host_blob_rejected_without_writes(mut, status):
+    geo = gi.Geometry(num_k_heads=2, num_v_heads=4, head_k_dim=32, head_v_dim=32)
+    cfg = gdn.make_config(geo)
+    if status == "GDN_E_BLOB_VERSION":
+        blob = make_blob(geo, version=2)
+    elif status == "GDN_E_BLOB_GEOMETRY":
+        blob = make_blob(geo, hk=1)
+    elif status == "GDN_E_BLOB_CHECKSUM":
+        blob = make_blob(geo, corrupt_payload=True)
+    elif status == "GDN_E_BLOB_FORMAT_LAYOUT":
+        blob, status = make_blob(geo, layout=7), "GDN_E_BLOB_FORMAT"
+    elif status == "GDN_E_BLOB_GEOMETRY_DTYPE":
+        blob, status = make_blob(geo, io_dtype=0), "GDN_E_BLOB_GEOMETRY"
+    else:
+        blob = make_blob(geo)
+        mut(blob)
+    conv = FakeTensor(3 * geo.conv_dim * 2)
+    st = FakeTensor(4 * 32 * 32 * 4)
+    c0, s0 = conv.view.copy(), st.view.copy()
+    with pytest.raises(gdn.GdnError) as e:
+        gdn.state_restore(cfg, blob, 0, conv, st, stream=0)
+    assert e.value.name == status, e.value
+    assert np.array_equal(conv.view, c0) and np.array_equal(st.view, s0)
+
+
+def test_truncated_blob_rejected():
+    geo = gi.Geometry(num_k_heads=2, num_v_heads=4, head_k_dim=32, head_v_dim=32)
+    blob = make_blob(geo)[:-8]
+    with pytest.raises(gdn.GdnError) as e:
+        gdn.state_restore(gdn.make_config(geo), blob, 0, FakeTensor(4096), FakeTensor(65536), stream=0)
+    assert e.value.name == "GDN_E_BLOB_FORMAT"

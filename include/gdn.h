@@ -149,6 +149,32 @@ GDN_API gdn_status gdn_prefill(const gdn_config* cfg, const gdn_params* params, 
                        int32_t num_seqs, int32_t chunk_size, uint32_t flags, void* conv_state, float* state,
                        void* o, void* workspace, size_t workspace_bytes, gdn_stream_t stream);
 
+/* gdn_prefill_noalloc: gdn_prefill for callers that cannot provide scratch
+ * device memory -- for example a host runtime whose device memory is owned by
+ * another allocator (a framework's caching allocator, a serving engine's
+ * pre-reserved pool) with no way to borrow from it, or latency-critical code
+ * that must not call cudaMalloc/cudaFree because they can synchronise the
+ * device.  The reference pages have no counterpart to this entry point.
+ *
+ * Same arguments and results as gdn_prefill, minus the workspace: the scratch
+ * is a fixed array of GDN_NOALLOC_SCRATCH_BYTES inside the library's device
+ * memory, present on every GPU that loads the library until the process
+ * exits.  The call allocates nothing.  A problem whose gdn_prefill workspace
+ * would exceed that size is rejected with GDN_E_WORKSPACE before anything
+ * runs.  The first call on a device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * Every call on a device shares the one array, which keeps whatever the last
+ * call left in it (nothing in it needs to start at zero: every kernel writes
+ * the scratch it later reads), so calls whose executions overlap on the GPU --
+ * for example on two streams -- race with each other and must be ordered by
+ * the caller. */
+#define GDN_NOALLOC_SCRATCH_BYTES (4u << 20)
+GDN_API gdn_status gdn_prefill_noalloc(const gdn_config* cfg, const gdn_params* params, const void* qkv,
+                                       const void* z, const void* a, const void* b, const int32_t* cu_seqlens_dev,
+                                       const int32_t* cu_seqlens_host, int32_t num_seqs, int32_t chunk_size,
+                                       uint32_t flags, void* conv_state, float* state, void* o,
+                                       gdn_stream_t stream);
+
 /* --------------------------------------------------------------------------
  * Single-step decode ("single-step decode", issue #88, Scope): every one of
  * num_seqs sequences advances by one token.  qkv [N, C_conv], z [N, Hv*d_v],

@@ -18,7 +18,7 @@ import numpy as np
 
 __all__ = [
     "GdnError", "Config", "Params", "lib", "make_config", "conv_prefill", "conv_step", "prefill_workspace_size",
-    "prefill", "decode_step", "state_blob_size", "state_save", "state_restore", "device_status", "last_error",
+    "prefill", "prefill_noalloc", "decode_step", "state_blob_size", "state_save", "state_restore", "device_status", "last_error",
     "abi_version", "launch_count", "launch_count_reset", "profiler_enable", "profiler_reset", "profiler_read",
     "kernel_name", "EXPORTS", "ZERO_INIT_STATE", "ZERO_INIT_CONV", "PREFILL_RECURRENT", "K",
 ]
@@ -48,7 +48,7 @@ EXPORTS = [
     "gdn_conv_prefill", "gdn_conv_step", "gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode_step",
     "gdn_state_blob_size", "gdn_state_save", "gdn_state_restore", "gdn_get_device_status", "gdn_last_error",
     "gdn_abi_version", "gdn_launch_count", "gdn_launch_count_reset", "gdn_kernel_name", "gdn_profiler_enable",
-    "gdn_profiler_reset", "gdn_profiler_read",
+    "gdn_profiler_reset", "gdn_profiler_read", "gdn_prefill_noalloc",
 ]
 
 
@@ -87,6 +87,7 @@ def lib():
             "gdn_conv_step": [P, P, P, I32, P, P, P],
             "gdn_prefill_workspace_size": [P, I64, I32, I32, P],
             "gdn_prefill": [P, P, P, P, P, P, P, P, I32, I32, U32, P, P, P, P, SZ, P],
+            "gdn_prefill_noalloc": [P, P, P, P, P, P, P, P, I32, I32, U32, P, P, P, P],
             "gdn_decode_step": [P, P, P, P, P, P, I32, P, P, P, P],
             "gdn_state_blob_size": [P, P],
             "gdn_state_save": [P, P, P, I32, P, SZ, P],
@@ -177,6 +178,18 @@ def prefill(cfg, params, qkv, z, a, b, cu_dev, cu_host, chunk_size, flags, conv_
     _check(lib().gdn_prefill(ctypes.byref(cfg), ctypes.byref(prm), _p(qkv), _p(z), _p(a), _p(b), _p(cu_dev),
                              cu_h.ctypes.data, cu_h.size - 1, chunk_size, flags, _p(conv_state), _p(state), _p(o),
                              _p(workspace), workspace_bytes, _stream(stream)))
+
+
+def prefill_noalloc(cfg, params, qkv, z, a, b, cu_dev, cu_host, chunk_size, flags, conv_state, state, o,
+                    stream=None):
+    """gdn_prefill_noalloc: gdn_prefill with the library's built-in scratch
+    instead of a caller workspace (for callers that cannot allocate device
+    memory); calls that overlap on the GPU share that scratch and race."""
+    cu_h = _host_cu(cu_host)
+    prm = _params(*params)
+    _check(lib().gdn_prefill_noalloc(ctypes.byref(cfg), ctypes.byref(prm), _p(qkv), _p(z), _p(a), _p(b), _p(cu_dev),
+                                     cu_h.ctypes.data, cu_h.size - 1, chunk_size, flags, _p(conv_state), _p(state),
+                                     _p(o), _stream(stream)))
 
 
 def decode_step(cfg, params, qkv, z, a, b, num_seqs, conv_state, state, o, stream=None):

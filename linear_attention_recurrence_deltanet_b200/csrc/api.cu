@@ -239,6 +239,8 @@ bool is_device_ptr(const void* p) {
 
 // ------------------------------------------------------------------ LaunchScope
 namespace gdn {
+void set_error_message(const char* msg) { g_err = msg; }
+
 LaunchScope::LaunchScope(int kernel_id, cudaStream_t s) : id(kernel_id), stream(s), token(nullptr) {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (g_prof.on) {

@@ -49,6 +49,9 @@ cudaError_t launch_prefill_recurrent(const Dims& d, bool bf16, const float* conv
                                      int32_t num_seqs, bool zero_state, bool zero_conv, const void* conv_state,
                                      float* state, void* o, cudaStream_t stream);
 
+// api.cu: records a message for gdn_last_error() on the calling thread.
+void set_error_message(const char* msg);
+
 // checksum.cu
 cudaError_t launch_checksum(const void* payload, size_t bytes, unsigned long long* out, cudaStream_t stream);
 uint64_t host_checksum(const void* payload, size_t bytes);

@@ -395,7 +395,8 @@ gdn_status gdn_prefill(const gdn_config* cfg, const gdn_params* params, const vo
   if (workspace_bytes < need || (need > 0 && !workspace))
     return fail(GDN_E_WORKSPACE, "workspace of %zu bytes at %p, need %zu", workspace_bytes, workspace, need);
   if (((uintptr_t)workspace & 255u) != 0) return fail(GDN_E_WORKSPACE, "workspace is not 256-byte aligned");
-  if ((s = check_device()) != GDN_OK) return s;
+  int dev = 0;
+  if ((s = check_device(&dev)) != GDN_OK) return s;
   if (total == 0) return GDN_OK;  // every sequence empty: nothing changes
 
   cudaStream_t st = (cudaStream_t)stream;
@@ -410,7 +411,12 @@ gdn_status gdn_prefill(const gdn_config* cfg, const gdn_params* params, const vo
     e = gdn::launch_schedule(cu_seqlens_dev, num_seqs, chunk_size, chunks, workspace, st);
     order = (const int32_t*)((const char*)workspace + L.order_off);
   }
-  if (e == cudaSuccess)
+  const bool chunked = !(flags & GDN_PREFILL_RECURRENT) && gdn::prefill_chunked_supported(d, bf16, chunk_size);
+  if (e == cudaSuccess && chunked)
+    e = gdn::launch_prefill_chunked(d, params->conv_w, params->A_log, params->dt_bias, params->norm_w, qkv, z, a, b,
+                                    cu_seqlens_dev, order, num_seqs, total, zero_state, zero_conv, conv_state, state,
+                                    o, g_status_ptr[dev], st);
+  else if (e == cudaSuccess)
     e = gdn::launch_prefill_recurrent(d, bf16, params->conv_w, params->A_log, params->dt_bias, params->norm_w, qkv,
                                       z, a, b, cu_seqlens_dev, order, num_seqs, zero_state, zero_conv, conv_state,
                                       state, o, st);

@@ -49,6 +49,14 @@ cudaError_t launch_prefill_recurrent(const Dims& d, bool bf16, const float* conv
                                      int32_t num_seqs, bool zero_state, bool zero_conv, const void* conv_state,
                                      float* state, void* o, cudaStream_t stream);
 
+// prefill_chunked.cu (tcgen05; bf16 io, d_k = d_v = 128, chunk 64)
+bool prefill_chunked_supported(const Dims& d, bool bf16, int chunk_size);
+cudaError_t launch_prefill_chunked(const Dims& d, const float* conv_w, const float* A_log, const float* dt_bias,
+                                   const float* norm_w, const void* qkv, const void* z, const void* a, const void* b,
+                                   const int32_t* cu, const int32_t* order, int32_t N, int64_t total_tokens,
+                                   bool zero_state, bool zero_conv, const void* conv_state, float* state, void* o,
+                                   int32_t* status, cudaStream_t stream);
+
 // api.cu: records a message for gdn_last_error() on the calling thread.
 void set_error_message(const char* msg);
 

@@ -1,0 +1,154 @@
+// sm_100a primitives: tcgen05 MMA / TMEM, TMA tensor loads, mbarriers, and
+// the shared-memory operand layouts the MMAs read.
+//
+// Operand layouts (fp16 elements, 128-byte swizzle; every tile base is
+// 1024-byte aligned):
+//   K-major tile of R rows x K (K a multiple of 64): K-blocks of 64 elements
+//     are stored one after another (R*128 bytes each); inside a block, 8-row
+//     groups are 1024 bytes apart, rows 128 bytes apart, and the 16-byte
+//     chunk index is XORed with (row % 8).
+//     Descriptor: LBO 16 B (unused), SBO 1024 B; an MMA step of K=16 starts
+//     32 bytes further inside the block.
+//   MN-major tile of K rows x N (N contiguous, N a multiple of 64): N-blocks
+//     of 64 elements, each holding K/8 groups of 8 rows x 128 bytes (1024 B),
+//     same 16-byte-chunk swizzle with (k % 8).
+//     Descriptor: LBO = stride between N-blocks = (K/8)*1024 B, SBO 1024 B;
+//     an MMA step of K=16 starts 2048 bytes further.
+// Accumulators (fp32 in TMEM): M=128 puts row r in lane r; M=64 puts row r in
+// lane (r % 16) + 32*(r / 16).  Column c of the accumulator is TMEM column
+// base + c.  Warp w may only touch lanes 32*(w % 4) .. 32*(w % 4) + 31.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace gdn {
+namespace tc {
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+// byte offset of element (row, k) in a K-major SW128 tile with `rows` rows
+__host__ __device__ __forceinline__ uint32_t kmaj(int rows, int row, int k) {
+  return (uint32_t)((k >> 6) * (rows * 128) + (row >> 3) * 1024 + (row & 7) * 128 + ((((k & 63) >> 3) ^ (row & 7)) << 4) +
+                    (k & 7) * 2);
+}
+// byte offset of the 16-byte chunk holding elements (row, k..k+7), k % 8 == 0
+__host__ __device__ __forceinline__ uint32_t kmaj_chunk(int rows, int row, int k) {
+  return (uint32_t)((k >> 6) * (rows * 128) + (row >> 3) * 1024 + (row & 7) * 128 + ((((k & 63) >> 3) ^ (row & 7)) << 4));
+}
+// byte offset of element (k, n) in an MN-major SW128 tile with K rows
+__host__ __device__ __forceinline__ uint32_t mnmaj(int K, int k, int n) {
+  return (uint32_t)((n >> 6) * ((K >> 3) * 1024) + (k >> 3) * 1024 + (k & 7) * 128 + ((((n & 63) >> 3) ^ (k & 7)) << 4) +
+                    (n & 7) * 2);
+}
+__host__ __device__ __forceinline__ uint32_t mnmaj_chunk(int K, int k, int n) {
+  return (uint32_t)((n >> 6) * ((K >> 3) * 1024) + (k >> 3) * 1024 + (k & 7) * 128 + ((((n & 63) >> 3) ^ (k & 7)) << 4));
+}
+
+// shared-memory matrix descriptor: SW128, version 1
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr & 0x3FFFF) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
+}
+// descriptor of MMA step s (K = 16 elements per step) of a K-major tile with `rows` rows
+__device__ __forceinline__ uint64_t desc_kmaj(uint32_t base, int rows, int s) {
+  const int k0 = s * 16;
+  return sdesc(base + (k0 >> 6) * (rows * 128) + (k0 & 63) * 2, 16, 1024);
+}
+// descriptor of MMA step s of an MN-major tile with K rows
+__device__ __forceinline__ uint64_t desc_mnmaj(uint32_t base, int K, int s) {
+  return sdesc(base + s * 2048, (K >> 3) * 1024, 1024);
+}
+
+// instruction descriptor, kind::f16: fp16 A and B, fp32 accumulator
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+          d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void mma_commit(uint64_t* mbar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(mbar))
+               : "memory");
+}
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// generic-proxy shared-memory writes -> visible to the tensor core (async proxy)
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's lane
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
+      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ---------------------------------------------------------------- mbarriers
+__device__ __forceinline__ void mbar_init(uint64_t* m, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(m)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_init_fence() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* m, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(m)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* m, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(m)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Wait for phase `parity` of `m`, for at most `limit_ns`; false on timeout.
+__device__ __forceinline__ bool mbar_wait(uint64_t* m, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(m, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(m, parity)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// ---------------------------------------------------------------- TMA
+// 2D tiled load of the box at (x = inner coordinate, y = row) into shared memory,
+// completing `bytes` on mbarrier m (no multicast).
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* m) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"((uint64_t)map), "r"(x), "r"(y), "r"(smem_u32(m))
+      : "memory");
+}
+
+}  // namespace tc
+}  // namespace gdn

@@ -389,3 +389,31 @@ def test_launch_count_and_profiler():
         assert ms >= 0
     assert total == n
     assert gdn.device_status() == 0
+
+
+# ------------------------------------------------------------------ chunked tensor-core prefill
+
+
+@pytest.mark.parametrize("zero_init", [True, False])
+def test_chunked_partial_chunks_match_oracle(zero_init):
+    # lengths around chunk boundaries (64): partial first/last chunks, exact multiples, short sequences
+    geo = gi.Geometry(num_k_heads=2, num_v_heads=6, head_k_dim=128, head_v_dim=128)
+    lengths = [1, 63, 64, 65, 127, 128, 129, 200, 2, 3]
+    inp = gi.make_prefill_inputs(geo, lengths, seed=31, zero_init=zero_init)
+    o_ref, st_ref, hist_ref = oracle.prefill_inputs(inp)
+    _, o, st, hist = run_gpu_prefill(inp, 64)
+    eo, es = compare_prefill(inp, o, st, o_ref, st_ref, TOL_O_BF16, TOL_S_BF16)
+    print(f"chunked partial chunks: o {eo:.2e} state {es:.2e}")
+    assert np.array_equal(hist, ref_hist_bits(inp, hist_ref))
+
+
+def test_chunked_matches_recurrent_kernel():
+    geo = gi.Geometry(num_k_heads=4, num_v_heads=12, head_k_dim=128, head_v_dim=128)
+    inp = gi.make_prefill_inputs(geo, [300, 64, 1, 517], seed=32, zero_init=False)
+    _, o1, st1, h1 = run_gpu_prefill(inp, 64)
+    _, o2, st2, h2 = run_gpu_prefill(inp, 64, RECURRENT)
+    for n in range(inp.num_seqs):
+        sl = slice(inp.cu_seqlens[n], inp.cu_seqlens[n + 1])
+        assert maxrel(o1[sl], o2[sl], 2 * U_BF16) <= TOL_O_BF16
+        assert maxrel(st1[n], st2[n]) <= TOL_S_BF16
+    assert np.array_equal(h1, h2)

@@ -63,12 +63,14 @@ constexpr int OFF_KQL = OFF_TA;                // [k^ lo ; q^ lo] 128x128 K-majo
 constexpr int OFF_DB = OFF_PA + 16384;         // Delta                   MN-major K=64 x N=128
 constexpr int OFF_SB = OFF_DB + 16384;         // S (fp16)                MN-major K=128 x N=128
 constexpr int OFF_MISC = OFF_SB + 32768;
-constexpr int kMiscFloats = 64 * 6 + 8;
+constexpr int kMiscFloats = 64 * 6 + 8 + 128;  // gates, row sums, gamma_C, norm weights
 constexpr int kSmemBytes = OFF_MISC + kMiscFloats * 4 + 1024;  // + base alignment slack
-constexpr int LDS = 65;                         // fp32 solve scratch row stride (aliases RAW)
+constexpr int LDS = 68;                         // fp32 solve scratch row stride (aliases RAW; 16-byte rows)
+constexpr int kOStride = 132;                   // fp32 O staging row stride (aliases RAW after the z tile)
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t COL_D1 = 0;     // [K;Q]K^T           64 columns
+constexpr uint32_t COL_S = 128;    // the fp32 state S   128 columns (row i = d_k index, column j)
 constexpr uint32_t COL_W = 256;    // W (M2), later K~^T Delta (M5)
 constexpr uint32_t COL_U = 384;    // U -> [Delta ; O]
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait, then report and stop
@@ -109,7 +111,7 @@ __device__ __forceinline__ void sync_tc() {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    prefill_chunked_kernel(const __grid_constant__ CUtensorMap tm_qkv, Dims d, const float* __restrict__ conv_w,
+    prefill_chunked_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_z, Dims d, const float* __restrict__ conv_w,
                            const float* __restrict__ A_log, const float* __restrict__ dt_bias,
                            const float* __restrict__ norm_w, const __nv_bfloat16* __restrict__ z,
                            const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
@@ -118,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                            __nv_bfloat16* __restrict__ o, int32_t* status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  __shared__ uint64_t mb_tma, mb_mma;
+  __shared__ uint64_t mb_tma, mb_mma, mb_z;
   __shared__ uint32_t tslot;
   __shared__ int abort_flag;
 
@@ -140,6 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* s_ekd = misc + 192;   // e^{gamma_C - gamma_r}
   float* s_rms = misc + 256;   // [2][64] partial sums of squares of the O rows
   float* s_gC = misc + 384;    // gamma_C
+  float* s_nw = misc + 392;    // 1 + norm_w
   float* Am = reinterpret_cast<float*>(sm + OFF_RAW);   // solve scratch, aliases the raw tiles
   float* Tm = Am + 64 * LDS;
   float* Ym = Tm + 64 * LDS;
@@ -147,28 +150,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     mbar_init(&mb_tma, 1);
     mbar_init(&mb_mma, 1);
+    mbar_init(&mb_z, 1);
     mbar_init_fence();
     abort_flag = 0;
   }
   if (warp == 0) tmem_alloc(&tslot, kTmemCols);
 
-  // recurrent state: thread owns row si of S (d_k index) and columns [64 hc, 64 hc + 64)
+  if (tid < kD) s_nw[tid] = 1.0f + norm_w[tid];
+  // recurrent state (fp32, in TMEM): thread owns row si of S (d_k index), columns [64 hc, 64 hc + 64)
   const int si = 32 * (warp & 3) + lane, hc = warp >> 2;
   const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-  float S[64];
   float* gst = state + ((int64_t)n * d.Hv + h) * kD * kD;  // stored [j][i]
-#pragma unroll
-  for (int jj = 0; jj < 64; ++jj) S[jj] = zero_state ? 0.f : gst[(int64_t)(64 * hc + jj) * kD + si];
-#pragma unroll
-  for (int m = 0; m < 8; ++m) st16h(sm + OFF_SB + mnmaj_chunk(kD, si, 64 * hc + 8 * m), S + 8 * m);
-  fence_async_smem();
   sync_tc();
   const uint32_t tbase = tslot;
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    float S[32];
+#pragma unroll
+    for (int jj = 0; jj < 32; ++jj) S[jj] = zero_state ? 0.f : gst[(int64_t)(64 * hc + 32 * hh + jj) * kD + si];
+    tmem_st32(tbase + lane_base + COL_S + 64 * hc + 32 * hh, S);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) st16h(sm + OFF_SB + mnmaj_chunk(kD, si, 64 * hc + 32 * hh + 8 * m), S + 8 * m);
+  }
+  fence_async_smem();
+  sync_tc();
 
   const float negA = -expf(A_log[h]);
   const float dtb = dt_bias[h];
   const int nchunks = (len + kC - 1) / kC;
-  uint32_t ph_tma = 0, ph_mma = 0;
+  uint32_t ph_tma = 0, ph_mma = 0, ph_z = 0;
   const int64_t q_col = (int64_t)kh * kD, k_col = (int64_t)d.Hk * kD + q_col, v_col = 2LL * d.Hk * kD + (int64_t)h * kD;
 
   for (int c = 0; c < nchunks; ++c) {
@@ -246,60 +256,77 @@ __global__ void __launch_bounds__(kThreads, 1)
       const unsigned char* rk = sm + OFF_RAW + (2 + half) * kRawBox;
       const unsigned char* rv = sm + OFF_RAW + (4 + half) * kRawBox;
 #pragma unroll 1
-      for (int rr = 0; rr < 8; ++rr) {
-        const int r = 8 * warp + rr;
-        float yq[4] = {0.f, 0.f, 0.f, 0.f}, yk[4] = {0.f, 0.f, 0.f, 0.f}, yv[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int rp = 0; rp < 4; ++rp) {  // two rows per pass for instruction-level parallelism
+        const int r0 = 8 * warp + 2 * rp;
+        float yq[2][4], yk[2][4], yv[2][4];
 #pragma unroll
-        for (int tap = 0; tap < 4; ++tap) {
+        for (int x = 0; x < 2; ++x)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) yq[x][e] = yk[x][e] = yv[x][e] = 0.f;
+#pragma unroll
+        for (int rowi = 0; rowi < 5; ++rowi) {  // raw rows r0 .. r0+4 feed the taps of both rows
           float xq[4], xk[4], xv[4];
-          const int off = raw_off(r + tap, cc);
+          const int off = raw_off(r0 + rowi, cc);
           ld4bf(rq + off, xq);
           ld4bf(rk + off, xk);
           ld4bf(rv + off, xv);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            yq[e] += wq[e][tap] * xq[e];
-            yk[e] += wk[e][tap] * xk[e];
-            yv[e] += wv[e][tap] * xv[e];
+          for (int x = 0; x < 2; ++x) {
+            const int tap = rowi - x;
+            if (tap >= 0 && tap < 4) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                yq[x][e] += wq[e][tap] * xq[e];
+                yk[x][e] += wk[e][tap] * xk[e];
+                yv[x][e] += wv[e][tap] * xv[e];
+              }
+            }
           }
         }
-        float sq = 0.f, sk = 0.f;
+        float sq[2] = {0.f, 0.f}, sk[2] = {0.f, 0.f};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          yq[e] = silu_fast(yq[e]);
-          yk[e] = silu_fast(yk[e]);
-          yv[e] = silu_fast(yv[e]);
-          sq += yq[e] * yq[e];
-          sk += yk[e] * yk[e];
-        }
-        sq = warp_sum(sq);
-        sk = warp_sum(sk);
-        const bool valid = r < L;
-        const float rqs = d.q_scale * rsqrtf(sq + d.l2_eps);
-        const float rks = valid ? rsqrtf(sk + d.l2_eps) : 0.f;
-        const float be = s_beta[r], eg = s_eg[r], ekd = s_ekd[r];
-        float qh[4], kk[4], vv[4];
+        for (int x = 0; x < 2; ++x)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          qh[e] = yq[e] * rqs;
-          kk[e] = yk[e] * rks;
-          vv[e] = valid ? yv[e] : 0.f;
-        }
-        const int k4 = 4 * lane;
-        st8(sm + OFF_KQ + kmaj(128, r, k4), kk[0], kk[1], kk[2], kk[3]);
-        st8(sm + OFF_KQ + kmaj(128, 64 + r, k4), qh[0], qh[1], qh[2], qh[3]);
-        float kl[4], ql[4];
+          for (int e = 0; e < 4; ++e) {
+            yq[x][e] = silu_fast(yq[x][e]);
+            yk[x][e] = silu_fast(yk[x][e]);
+            yv[x][e] = silu_fast(yv[x][e]);
+            sq[x] += yq[x][e] * yq[x][e];
+            sk[x] += yk[x][e] * yk[x][e];
+          }
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          kl[e] = kk[e] - __half2float(__float2half_rn(kk[e]));
-          ql[e] = qh[e] - __half2float(__float2half_rn(qh[e]));
+        for (int off = 16; off > 0; off >>= 1) {
+          sq[0] += __shfl_xor_sync(0xffffffffu, sq[0], off);
+          sq[1] += __shfl_xor_sync(0xffffffffu, sq[1], off);
+          sk[0] += __shfl_xor_sync(0xffffffffu, sk[0], off);
+          sk[1] += __shfl_xor_sync(0xffffffffu, sk[1], off);
         }
-        st8(sm + OFF_KQL + kmaj(128, r, k4), kl[0], kl[1], kl[2], kl[3]);
-        st8(sm + OFF_KQL + kmaj(128, 64 + r, k4), ql[0], ql[1], ql[2], ql[3]);
-        const float bg = be * eg;
-        st8(sm + OFF_X + mnmaj(kC, r, k4), bg * kk[0], bg * kk[1], bg * kk[2], bg * kk[3]);
-        st8(sm + OFF_X + mnmaj(kC, r, 128 + k4), be * vv[0], be * vv[1], be * vv[2], be * vv[3]);
-        st8(sm + OFF_KD + mnmaj(kC, r, k4), ekd * kk[0], ekd * kk[1], ekd * kk[2], ekd * kk[3]);
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          const int r = r0 + x;
+          const bool valid = r < L;
+          const float rqs = d.q_scale * rsqrtf(sq[x] + d.l2_eps);
+          const float rks = valid ? rsqrtf(sk[x] + d.l2_eps) : 0.f;
+          const float be = s_beta[r], eg = s_eg[r], ekd = s_ekd[r];
+          float qh[4], kk[4], vv[4], kl[4], ql[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            qh[e] = yq[x][e] * rqs;
+            kk[e] = yk[x][e] * rks;
+            vv[e] = valid ? yv[x][e] : 0.f;
+            kl[e] = kk[e] - __half2float(__float2half_rn(kk[e]));
+            ql[e] = qh[e] - __half2float(__float2half_rn(qh[e]));
+          }
+          const int k4 = 4 * lane;
+          st8(sm + OFF_KQ + kmaj(128, r, k4), kk[0], kk[1], kk[2], kk[3]);
+          st8(sm + OFF_KQ + kmaj(128, 64 + r, k4), qh[0], qh[1], qh[2], qh[3]);
+          st8(sm + OFF_KQL + kmaj(128, r, k4), kl[0], kl[1], kl[2], kl[3]);
+          st8(sm + OFF_KQL + kmaj(128, 64 + r, k4), ql[0], ql[1], ql[2], ql[3]);
+          const float bg = be * eg;
+          st8(sm + OFF_X + mnmaj(kC, r, k4), bg * kk[0], bg * kk[1], bg * kk[2], bg * kk[3]);
+          st8(sm + OFF_X + mnmaj(kC, r, 128 + k4), be * vv[0], be * vv[1], be * vv[2], be * vv[3]);
+          st8(sm + OFF_KD + mnmaj(kC, r, k4), ekd * kk[0], ekd * kk[1], ekd * kk[2], ekd * kk[3]);
+        }
       }
     }
     fence_async_smem();
@@ -334,9 +361,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (row < 64) {  // A_rj = beta_r e^{gamma_r - gamma_j} (k_r . k_j), j < r
         const float br = s_beta[row], gr = s_gam[row];
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const int j = 32 * hc + jj;
-          Am[row * LDS + j] = (j < row) ? br * __expf(gr - s_gam[j]) * v[jj] : 0.f;
+        for (int m = 0; m < 8; ++m) {
+          float a4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = 32 * hc + 4 * m + e;
+            a4[e] = (j < row) ? br * __expf(gr - s_gam[j]) * v[4 * m + e] : 0.f;
+          }
+          *reinterpret_cast<float4*>(Am + row * LDS + 32 * hc + 4 * m) = make_float4(a4[0], a4[1], a4[2], a4[3]);
         }
       } else {  // P_rj = e^{gamma_r - gamma_j} (q_r . k_j), j <= r
         const int r = row - 64;
@@ -354,40 +386,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncthreads();
-    if (tid < 64) {  // diagonal 16x16 blocks by forward substitution: column c16 of block bb
+    // T = (I + A)^-1 in 16x16 blocks.  Diagonal blocks T_bb = (I + A_bb)^-1 by
+    // right-looking forward substitution (one column per thread: each new
+    // entry updates the running sums of the rows below it, so the dependent
+    // chain is one FMA per row).
+    if (tid < 64) {
       const int bb = tid >> 4, c16 = tid & 15;
-      float t[16];
+      const float* Ab = Am + (16 * bb) * LDS + 16 * bb;
+      float acc[16], t[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) t[i] = (i == c16) ? 1.f : 0.f;
+      for (int i = 0; i < 16; ++i) acc[i] = 0.f;
 #pragma unroll
-      for (int i = 1; i < 16; ++i) {
-        float s = 0.f;
+      for (int k = 0; k < 16; ++k) {
+        t[k] = (k < c16) ? 0.f : (k == c16 ? 1.f : -acc[k]);
 #pragma unroll
-        for (int k = 0; k < i; ++k) s += Am[(16 * bb + i) * LDS + 16 * bb + k] * t[k];
-        if (i > c16) t[i] = -s;
+        for (int i = k + 1; i < 16; ++i) acc[i] += Ab[i * LDS + k] * t[k];
       }
 #pragma unroll
       for (int i = 0; i < 16; ++i) Tm[(16 * bb + i) * LDS + 16 * bb + c16] = t[i];
     }
     __syncthreads();
-    for (int dl = 1; dl < 4; ++dl) {  // off-diagonal blocks T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj
-      const int npairs = 4 - dl;
-      for (int e = tid; e < npairs * 256; e += kThreads) {
-        const int bj = e >> 8, bi = bj + dl, p = (e >> 4) & 15, q = e & 15;
-        float s = 0.f;
+    // At_ij = T_ii A_ij for the six blocks below the diagonal (into Ym); each work
+    // item is one row p and four columns q..q+3 of one block (float4 along q)
+    for (int e = tid; e < 6 * 64; e += kThreads) {
+      const int pr = e >> 6, p = (e >> 2) & 15, q = 4 * (e & 3);
+      // pairs pr = 0..5: (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
+      const int bi = pr == 0 ? 1 : (pr < 3 ? 2 : 3), bj = pr == 0 ? 0 : (pr < 3 ? pr - 1 : pr - 3);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int kk = 0; kk < 16; ++kk) {
+        const float t = Tm[(16 * bi + p) * LDS + 16 * bi + kk];
+        const float4 a4 = *reinterpret_cast<const float4*>(Am + (16 * bi + kk) * LDS + 16 * bj + q);
+        acc.x += t * a4.x; acc.y += t * a4.y; acc.z += t * a4.z; acc.w += t * a4.w;
+      }
+      *reinterpret_cast<float4*>(Ym + (16 * bi + p) * LDS + 16 * bj + q) = acc;
+    }
+    __syncthreads();
+    // off-diagonal blocks by distance: T_ij = -sum_{k=j}^{i-1} At_ik T_kj
+    for (int dl = 1; dl < 4; ++dl) {
+      for (int e = tid; e < (4 - dl) * 64; e += kThreads) {
+        const int bj = e >> 6, bi = bj + dl, p = (e >> 2) & 15, q = 4 * (e & 3);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int bk = bj; bk < bi; ++bk) {
 #pragma unroll
-          for (int kk = 0; kk < 16; ++kk) s += Am[(16 * bi + p) * LDS + 16 * bk + kk] * Tm[(16 * bk + kk) * LDS + 16 * bj + q];
+          for (int kk = 0; kk < 16; ++kk) {
+            const float y = Ym[(16 * bi + p) * LDS + 16 * bk + kk];
+            const float4 t4 = *reinterpret_cast<const float4*>(Tm + (16 * bk + kk) * LDS + 16 * bj + q);
+            acc.x += y * t4.x; acc.y += y * t4.y; acc.z += y * t4.z; acc.w += y * t4.w;
+          }
         }
-        Ym[(16 * bi + p) * LDS + 16 * bj + q] = s;
-      }
-      __syncthreads();
-      for (int e = tid; e < npairs * 256; e += kThreads) {
-        const int bj = e >> 8, bi = bj + dl, p = (e >> 4) & 15, q = e & 15;
-        float s = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < 16; ++kk) s += Tm[(16 * bi + p) * LDS + 16 * bi + kk] * Ym[(16 * bi + kk) * LDS + 16 * bj + q];
-        Tm[(16 * bi + p) * LDS + 16 * bj + q] = -s;
+        *reinterpret_cast<float4*>(Tm + (16 * bi + p) * LDS + 16 * bj + q) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
       }
       __syncthreads();
     }
@@ -395,7 +443,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int r = tid >> 2, j0 = 16 * (tid & 3);
       float tv[16];
 #pragma unroll
-      for (int jj = 0; jj < 16; ++jj) tv[jj] = (j0 + jj <= r) ? Tm[r * LDS + j0 + jj] : 0.f;
+      for (int m = 0; m < 4; ++m) {
+        const float4 t4 = *reinterpret_cast<const float4*>(Tm + r * LDS + j0 + 4 * m);
+        tv[4 * m] = t4.x; tv[4 * m + 1] = t4.y; tv[4 * m + 2] = t4.z; tv[4 * m + 3] = t4.w;
+      }
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) tv[jj] = (j0 + jj <= r) ? tv[jj] : 0.f;
       st16h(sm + OFF_TA + kmaj_chunk(128, r, j0), tv);
       st16h(sm + OFF_TA + kmaj_chunk(128, r, j0 + 8), tv + 8);
     }
@@ -403,6 +456,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     sync_tc();
 
     // ------------------------------------------------------------ M2: [T;0] [beta e^g K | beta V]
+    if (tid == 0) {  // z rows of this chunk, for the output gate (into the now idle raw-tile space)
+      mbar_expect_tx(&mb_z, 2 * 64 * 64 * 2);
+      tma_load_2d(sm + OFF_RAW, &tm_z, h * kD, (int)t0, &mb_z);
+      tma_load_2d(sm + OFF_RAW + 8192, &tm_z, h * kD + 64, (int)t0, &mb_z);
+    }
     if (tid == 0) {
       const uint32_t ta = smem_u32(sm + OFF_TA), x = smem_u32(sm + OFF_X);
       constexpr uint32_t id = idesc_f16(128, 256, false, true);
@@ -489,49 +547,60 @@ __global__ void __launch_bounds__(kThreads, 1)
       float v[32];
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
+        float S[32];
         tmem_ld32(tbase + lane_base + COL_W + 64 * hc + 32 * hh, v);
+        tmem_ld32(tbase + lane_base + COL_S + 64 * hc + 32 * hh, S);
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) S[32 * hh + jj] = egC * S[32 * hh + jj] + v[jj];
+        for (int jj = 0; jj < 32; ++jj) S[jj] = egC * S[jj] + v[jj];
+        tmem_st32(tbase + lane_base + COL_S + 64 * hc + 32 * hh, S);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) st16h(sm + OFF_SB + mnmaj_chunk(kD, si, 64 * hc + 32 * hh + 8 * m), S + 8 * m);
       }
-#pragma unroll
-      for (int m = 0; m < 8; ++m) st16h(sm + OFF_SB + mnmaj_chunk(kD, si, 64 * hc + 8 * m), S + 8 * m);
-      if (si >= 64) {
+      if (si >= 64) {  // O rows: fp32 to shared memory (after the z tile) and row sums of squares
+        const int r = si - 64;
+        float* orow = reinterpret_cast<float*>(sm + OFF_RAW + 16384) + r * kOStride + 64 * hc;
         float ss = 0.f;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           tmem_ld32(tbase + lane_base + COL_U + 64 * hc + 32 * hh, v);
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) ss += v[jj] * v[jj];
+#pragma unroll
+          for (int m = 0; m < 8; ++m)
+            *reinterpret_cast<float4*>(orow + 32 * hh + 4 * m) = make_float4(v[4 * m], v[4 * m + 1], v[4 * m + 2], v[4 * m + 3]);
         }
-        s_rms[64 * hc + (si - 64)] = ss;
+        s_rms[64 * hc + r] = ss;
       }
     }
+    if (!mbar_wait(&mb_z, ph_z, kWaitNs)) abort_flag = 1;
+    ph_z ^= 1;
     __syncthreads();
-    if (si >= 64) {
-      const int r = si - 64;
-      const float rinv = rsqrtf((s_rms[r] + s_rms[64 + r]) * (1.0f / kD) + d.norm_eps);
-      float v[32];
+    {  // zero-centred RMSNorm over d_v, times sigmoid(z): row r = tid / 4, columns [32 q4, 32 q4 + 32)
+      const int r = tid >> 2, q4 = tid & 3;
+      if (r < L) {
+        const float rinv = rsqrtf((s_rms[r] + s_rms[64 + r]) * (1.0f / kD) + d.norm_eps);
+        const float* orow = reinterpret_cast<const float*>(sm + OFF_RAW + 16384) + r * kOStride + 32 * q4;
+        const unsigned char* zbox = sm + OFF_RAW + (q4 >> 1) * 8192;
+        const int64_t off = (t0 + r) * HvD + (int64_t)h * kD + 32 * q4;
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        tmem_ld32(tbase + lane_base + COL_U + 64 * hc + 32 * hh, v);
-        if (r < L) {
-          const int64_t off = (t0 + r) * HvD + (int64_t)h * kD + 64 * hc + 32 * hh;
+        for (int m = 0; m < 4; ++m) {
+          const int zc = 32 * (q4 & 1) + 8 * m;  // column inside the 64-column z box
+          const uint4 zr = *reinterpret_cast<const uint4*>(zbox + r * 128 + ((((zc >> 3) ^ (r & 7))) << 4));
+          const float4 oa = *reinterpret_cast<const float4*>(orow + 8 * m);
+          const float4 ob = *reinterpret_cast<const float4*>(orow + 8 * m + 4);
+          const float ov[8] = {oa.x, oa.y, oa.z, oa.w, ob.x, ob.y, ob.z, ob.w};
+          const uint32_t zw[4] = {zr.x, zr.y, zr.z, zr.w};
+          uint32_t ow[4];
 #pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const uint4 zr = __ldg(reinterpret_cast<const uint4*>(z + off + 8 * m));
-            const uint32_t zw[4] = {zr.x, zr.y, zr.z, zr.w};
-            uint32_t ow[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int j = 64 * hc + 32 * hh + 8 * m + 2 * e;
-              const float z0 = __uint_as_float(zw[e] << 16), z1 = __uint_as_float(zw[e] & 0xffff0000u);
-              const float o0 = v[8 * m + 2 * e] * rinv * (1.0f + norm_w[j]) * sigmoid_f(z0);
-              const float o1 = v[8 * m + 2 * e + 1] * rinv * (1.0f + norm_w[j + 1]) * sigmoid_f(z1);
-              __nv_bfloat162 pr = __floats2bfloat162_rn(o0, o1);
-              ow[e] = *reinterpret_cast<uint32_t*>(&pr);
-            }
-            *reinterpret_cast<uint4*>(o + off + 8 * m) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+          for (int e = 0; e < 4; ++e) {
+            const int j = 32 * q4 + 8 * m + 2 * e;
+            const float z0 = __uint_as_float(zw[e] << 16), z1 = __uint_as_float(zw[e] & 0xffff0000u);
+            const float o0 = ov[2 * e] * rinv * s_nw[j] * __fdividef(1.0f, 1.0f + __expf(-z0));
+            const float o1 = ov[2 * e + 1] * rinv * s_nw[j + 1] * __fdividef(1.0f, 1.0f + __expf(-z1));
+            __nv_bfloat162 pr = __floats2bfloat162_rn(o0, o1);
+            ow[e] = *reinterpret_cast<uint32_t*>(&pr);
           }
+          *reinterpret_cast<uint4*>(o + off + 8 * m) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
         }
       }
     }
@@ -543,7 +612,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) set_status(status, kStatusWaitTimeout);
   } else {
 #pragma unroll
-    for (int jj = 0; jj < 64; ++jj) gst[(int64_t)(64 * hc + jj) * kD + si] = S[jj];
+    for (int hh = 0; hh < 2; ++hh) {
+      float S[32];
+      tmem_ld32(tbase + lane_base + COL_S + 64 * hc + 32 * hh, S);
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) gst[(int64_t)(64 * hc + 32 * hh + jj) * kD + si] = S[jj];
+    }
   }
   sync_tc();
   if (warp == 0) tmem_dealloc(tbase, kTmemCols);
@@ -584,12 +658,18 @@ cudaError_t launch_prefill_chunked(const Dims& d, const float* conv_w, const flo
   if (N <= 0 || total_tokens <= 0) return cudaSuccess;
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
-  CUtensorMap tm;
+  CUtensorMap tm, tmz;
+  const cuuint64_t zdim[2] = {(cuuint64_t)d.Hv * kD, (cuuint64_t)total_tokens};
+  const cuuint64_t zstride[1] = {(cuuint64_t)d.Hv * kD * 2};
+  const cuuint32_t zbox[2] = {64, 64};
   const cuuint64_t gdim[2] = {(cuuint64_t)d.C, (cuuint64_t)total_tokens};
   const cuuint64_t gstride[1] = {(cuuint64_t)d.C * 2};
   const cuuint32_t box[2] = {64, (cuuint32_t)kRawRows};
   const cuuint32_t estr[2] = {1, 1};
   if (enc(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(qkv), gdim, gstride, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+      enc(&tmz, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(z), zdim, zstride, zbox, estr,
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
@@ -598,7 +678,7 @@ cudaError_t launch_prefill_chunked(const Dims& d, const float* conv_w, const flo
   if (e != cudaSuccess) return e;
   LaunchScope scope(GDN_K_PREFILL_CHUNKED, stream);
   prefill_chunked_kernel<<<(unsigned)((int64_t)N * d.Hv), kThreads, kSmemBytes, stream>>>(
-      tm, d, conv_w, A_log, dt_bias, norm_w, (const __nv_bfloat16*)z, (const __nv_bfloat16*)a,
+      tm, tmz, d, conv_w, A_log, dt_bias, norm_w, (const __nv_bfloat16*)z, (const __nv_bfloat16*)a,
       (const __nv_bfloat16*)b, cu, order, zero_state, zero_conv, (const __nv_bfloat16*)conv_state, state,
       (__nv_bfloat16*)o, status);
   return cudaGetLastError();

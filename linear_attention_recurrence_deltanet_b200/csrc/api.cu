@@ -438,10 +438,11 @@ gdn_status gdn_decode_step(const gdn_config* cfg, const gdn_params* params, cons
       (s = check_ptr(conv_state, "conv_state")) != GDN_OK || (s = check_ptr(state, "state")) != GDN_OK ||
       (s = check_ptr(o, "o")) != GDN_OK)
     return s;
-  if ((s = check_device()) != GDN_OK) return s;
+  int dev = 0;
+  if ((s = check_device(&dev)) != GDN_OK) return s;
   cudaError_t e = gdn::launch_decode_step(d, cfg->io_dtype == GDN_BF16, params->conv_w, params->A_log,
                                           params->dt_bias, params->norm_w, qkv, z, a, b, num_seqs, conv_state,
-                                          state, o, (cudaStream_t)stream);
+                                          state, o, g_status_ptr[dev], (cudaStream_t)stream);
   return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_decode_step launch");
 }
 

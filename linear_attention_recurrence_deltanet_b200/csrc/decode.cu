@@ -17,6 +17,7 @@
 // warp keeps two row groups of loads in flight.
 #include "../../include/gdn.h"
 #include "internal.h"
+#include "tc.cuh"
 
 namespace gdn {
 namespace {
@@ -168,6 +169,199 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   }
 }
 
+// d_k = d_v = 128: the state rows stream through a 4-stage shared-memory ring
+// fed by 1D bulk copies (cp.async.bulk), so the bytes in flight no longer
+// depend on registers.  128 threads and ~21 KB of shared memory per CTA let 8
+// CTAs share an SM, so the whole B=64 grid (1024 CTAs) is resident in one
+// wave; the first stages are requested before the conv/norm prologue runs.
+constexpr int kBulkThreads = 128;
+constexpr int kBulkRows = 8;     // state rows per stage (4 KB)
+constexpr int kBulkStages = 4;
+constexpr uint64_t kBulkWaitNs = 2000000000ull;
+
+template <typename T>
+__global__ void __launch_bounds__(kBulkThreads, 8)
+    decode_bulk_kernel(Dims d, const float* __restrict__ conv_w, const float* __restrict__ A_log,
+                       const float* __restrict__ dt_bias, const float* __restrict__ norm_w,
+                       const T* __restrict__ qkv, const T* __restrict__ z, const T* __restrict__ a,
+                       const T* __restrict__ b, T* __restrict__ hist, float* __restrict__ state, T* __restrict__ o,
+                       int32_t* status) {
+  constexpr int D = 128;
+  constexpr int kStageFloats = kBulkRows * D;
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  float* ring = reinterpret_cast<float*>(smem_raw);          // kBulkStages x 8 rows x 128
+  const int G = d.G;
+  float* u = ring + kBulkStages * kStageFloats;               // [q (D) | k (D) | v of G heads]
+  float* osm = u + (2 + G) * D;                               // [G*D]
+  float* gate = osm + G * D;                                  // alpha[G], beta[G]
+  __shared__ uint64_t full[kBulkStages], empty[kBulkStages];
+  __shared__ float red[3];
+  __shared__ int abort_flag;
+
+  const int n = blockIdx.x / d.Hk;
+  const int kh = blockIdx.x - n * d.Hk;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t C = d.C;
+  const int h0 = G * kh;
+  const int nst = G * D / kBulkRows;
+  float* st = state + ((int64_t)n * d.Hv + h0) * D * D;   // the G heads' rows are contiguous
+
+  if (tid == 0) {
+    for (int s = 0; s < kBulkStages; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], kBulkThreads / 32);
+    }
+    tc::mbar_init_fence();
+    abort_flag = 0;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    for (int s = 0; s < kBulkStages && s < nst; ++s) {
+      tc::mbar_expect_tx(&full[s], kStageFloats * 4);
+      tc::bulk_load(ring + s * kStageFloats, st + (int64_t)s * kStageFloats, kStageFloats * 4, &full[s]);
+    }
+  }
+
+  // ---- conv step + SiLU for the owned channels; rotate the history
+  const int nch = (2 + G) * D;
+  for (int idx = tid; idx < nch; idx += kBulkThreads) {
+    const int64_t c = idx < D ? (int64_t)kh * D + idx
+                              : (idx < 2 * D ? (int64_t)d.Hk * D + (int64_t)kh * D + (idx - D)
+                                             : 2LL * d.Hk * D + (int64_t)h0 * D + (idx - 2 * D));
+    T* hp = hist + (int64_t)n * 3 * C + c;
+    const T h0v = hp[0], h1v = hp[C], h2v = hp[2 * C];
+    const T xv = qkv[(int64_t)n * C + c];
+    const float4 w = __ldg(reinterpret_cast<const float4*>(conv_w + c * 4));
+    const float y = w.x * to_f(h0v) + w.y * to_f(h1v) + w.z * to_f(h2v) + w.w * to_f(xv);
+    u[idx] = silu_f(y);
+    hp[0] = h1v;
+    hp[C] = h2v;
+    hp[2 * C] = xv;
+  }
+  if (tid < G) {
+    const int h = h0 + tid;
+    float g, al, be;
+    gates_f(ldg_f(a + (int64_t)n * d.Hv + h), dt_bias[h], A_log[h], ldg_f(b + (int64_t)n * d.Hv + h), g, al, be);
+    gate[tid] = al;
+    gate[G + tid] = be;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float sq = 0.f, sk = 0.f, sqk = 0.f;
+    for (int i = lane; i < D; i += 32) {
+      const float qv = u[i], kv = u[D + i];
+      sq += qv * qv;
+      sk += kv * kv;
+      sqk += qv * kv;
+    }
+    sq = warp_sum(sq);
+    sk = warp_sum(sk);
+    sqk = warp_sum(sqk);
+    if (lane == 0) {
+      const float rq = d.q_scale * rsqrtf(sq + d.l2_eps), rk = rsqrtf(sk + d.l2_eps);
+      red[0] = rq;
+      red[1] = rk;
+      red[2] = rq * rk * sqk;
+    }
+  }
+  __syncthreads();
+
+  // ---- stream the rows: 16 lanes per row, 2 rows per warp, 8 rows per stage
+  const int l16 = lane & 15, hr = lane >> 4;
+  float4 kq[2], qq[2];
+  {
+    const float rq = red[0], rk = red[1];
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const int i0 = 4 * l16 + 64 * m;
+      qq[m] = make_float4(u[i0] * rq, u[i0 + 1] * rq, u[i0 + 2] * rq, u[i0 + 3] * rq);
+      kq[m] = make_float4(u[D + i0] * rk, u[D + i0 + 1] * rk, u[D + i0 + 2] * rk, u[D + i0 + 3] * rk);
+    }
+  }
+  const float qk = red[2];
+  for (int s = 0; s < nst; ++s) {
+    const int slot = s % kBulkStages;
+    const uint32_t par = (uint32_t)(s / kBulkStages) & 1u;
+    if (!tc::mbar_wait(&full[slot], par, kBulkWaitNs)) abort_flag = 1;
+    if (!abort_flag) {
+      const int lrow = 2 * warp + hr;
+      const int row = s * kBulkRows + lrow;
+      const float* src = ring + slot * kStageFloats + lrow * D;
+      float4 r[2];
+      r[0] = *reinterpret_cast<const float4*>(src + 4 * l16);
+      r[1] = *reinterpret_cast<const float4*>(src + 64 + 4 * l16);
+      float kap = 0.f, rho = 0.f;
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        kap += kq[m].x * r[m].x + kq[m].y * r[m].y + kq[m].z * r[m].z + kq[m].w * r[m].w;
+        rho += qq[m].x * r[m].x + qq[m].y * r[m].y + qq[m].z * r[m].z + qq[m].w * r[m].w;
+      }
+#pragma unroll
+      for (int off = 1; off < 16; off <<= 1) {
+        kap += __shfl_xor_sync(0xffffffffu, kap, off);
+        rho += __shfl_xor_sync(0xffffffffu, rho, off);
+      }
+      const int hh = row / D;
+      const float al = gate[hh], be = gate[G + hh];
+      const float delta = be * (u[2 * D + row] - al * kap);
+      float4* dst = reinterpret_cast<float4*>(st + (int64_t)row * D);
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        float4 w4;
+        w4.x = al * r[m].x + delta * kq[m].x;
+        w4.y = al * r[m].y + delta * kq[m].y;
+        w4.z = al * r[m].z + delta * kq[m].z;
+        w4.w = al * r[m].w + delta * kq[m].w;
+        __stcs(dst + l16 + 16 * m, w4);
+      }
+      if (l16 == 0) osm[row] = al * rho + delta * qk;
+    }
+    __syncwarp();
+    if (lane == 0) tc::mbar_arrive(&empty[slot]);
+    if (tid == 0 && s + kBulkStages < nst) {  // refill this slot once every warp has read it
+      if (!tc::mbar_wait(&empty[slot], par, kBulkWaitNs)) abort_flag = 1;
+      tc::fence_async_smem();
+      tc::mbar_expect_tx(&full[slot], kStageFloats * 4);
+      tc::bulk_load(ring + slot * kStageFloats, st + (int64_t)(s + kBulkStages) * kStageFloats, kStageFloats * 4,
+                    &full[slot]);
+    }
+  }
+  __syncthreads();
+  if (abort_flag) {
+    if (tid == 0) set_status(status, kStatusWaitTimeout);
+    return;
+  }
+
+  // ---- zero-centred RMSNorm over d_v, times sigmoid(z); one rounding to io dtype
+  for (int hh = warp; hh < G; hh += kBulkThreads / 32) {
+    float ss = 0.f;
+    for (int j = lane; j < D; j += 32) ss += osm[hh * D + j] * osm[hh * D + j];
+    ss = warp_sum(ss);
+    const float rr = rsqrtf(ss / D + d.norm_eps);
+    const int64_t off = ((int64_t)n * d.Hv + h0 + hh) * D;
+    for (int j = lane; j < D; j += 32) {
+      const float zz = ldg_f(z + off + j);
+      o[off + j] = from_f<T>(osm[hh * D + j] * rr * (1.0f + norm_w[j]) * sigmoid_f(zz));
+    }
+  }
+}
+
+template <typename T>
+cudaError_t launch_bulk(const Dims& d, const float* conv_w, const float* A_log, const float* dt_bias,
+                        const float* norm_w, const void* qkv, const void* z, const void* a, const void* b, int32_t N,
+                        void* hist, float* state, void* o, int32_t* status, cudaStream_t stream) {
+  const size_t smem = (size_t)(kBulkStages * kBulkRows * 128 + (2 + d.G) * 128 + d.G * 128 + 2 * d.G) * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(decode_bulk_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  LaunchScope scope(GDN_K_DECODE, stream);
+  decode_bulk_kernel<T><<<(unsigned)((int64_t)N * d.Hk), kBulkThreads, smem, stream>>>(
+      d, conv_w, A_log, dt_bias, norm_w, (const T*)qkv, (const T*)z, (const T*)a, (const T*)b, (T*)hist, state,
+      (T*)o, status);
+  return cudaGetLastError();
+}
+
 template <typename T, int D>
 cudaError_t launch_t(const Dims& d, const float* conv_w, const float* A_log, const float* dt_bias,
                      const float* norm_w, const void* qkv, const void* z, const void* a, const void* b, int32_t N,
@@ -190,8 +384,14 @@ cudaError_t launch_t(const Dims& d, const float* conv_w, const float* A_log, con
 cudaError_t launch_decode_step(const Dims& d, bool bf16, const float* conv_w, const float* A_log,
                                const float* dt_bias, const float* norm_w, const void* qkv, const void* z,
                                const void* a, const void* b, int32_t N, void* conv_state, float* state, void* o,
-                               cudaStream_t stream) {
+                               int32_t* status, cudaStream_t stream) {
   if (N <= 0) return cudaSuccess;
+  if (d.dk == 128) {
+    return bf16 ? launch_bulk<__nv_bfloat16>(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, N, conv_state, state, o,
+                                             status, stream)
+                : launch_bulk<float>(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, N, conv_state, state, o, status,
+                                     stream);
+  }
 #define GDN_DEC(T, D) \
   return launch_t<T, D>(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, N, conv_state, state, o, stream)
   if (bf16) {

@@ -40,7 +40,7 @@ cudaError_t launch_schedule(const int32_t* cu, int32_t num_seqs, int32_t chunk_s
 cudaError_t launch_decode_step(const Dims& d, bool bf16, const float* conv_w, const float* A_log,
                                const float* dt_bias, const float* norm_w, const void* qkv, const void* z,
                                const void* a, const void* b, int32_t num_seqs, void* conv_state, float* state,
-                               void* o, cudaStream_t stream);
+                               void* o, int32_t* status, cudaStream_t stream);
 
 // prefill_recurrent.cu
 cudaError_t launch_prefill_recurrent(const Dims& d, bool bf16, const float* conv_w, const float* A_log,

@@ -156,7 +156,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* m, uint32_t parity, uint64_t
   }
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* m) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(m)) : "memory");
+}
+
 // ---------------------------------------------------------------- TMA
+// 1D bulk copy global -> shared (both 16-byte aligned, size a multiple of 16),
+// completing `bytes` on mbarrier m.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* m) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"((uint64_t)src), "r"(bytes), "r"(smem_u32(m))
+               : "memory");
+}
+
 // 2D tiled load of the box at (x = inner coordinate, y = row) into shared memory,
 // completing `bytes` on mbarrier m (no multicast).
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* m) {

@@ -66,7 +66,6 @@ constexpr int OFF_MISC = OFF_SB + 32768;
 constexpr int kMiscFloats = 64 * 6 + 8 + 128;  // gates, row sums, gamma_C, norm weights
 constexpr int kSmemBytes = OFF_MISC + kMiscFloats * 4 + 1024;  // + base alignment slack
 constexpr int LDS = 68;                         // fp32 solve scratch row stride (aliases RAW; 16-byte rows)
-constexpr int kOStride = 132;                   // fp32 O staging row stride (aliases RAW after the z tile)
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t COL_D1 = 0;     // [K;Q]K^T           64 columns
@@ -181,19 +180,42 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t ph_tma = 0, ph_mma = 0, ph_z = 0;
   const int64_t q_col = (int64_t)kh * kD, k_col = (int64_t)d.Hk * kD + q_col, v_col = 2LL * d.Hk * kD + (int64_t)h * kD;
 
+  // The raw tiles and the a/b gate inputs of chunk c+1 are requested while
+  // chunk c is still in its MMA phases (the raw-tile space is idle by then).
+  auto issue_raw = [&](int cc) {
+    const int64_t tt = seq0 + (int64_t)cc * kC;
+    mbar_expect_tx(&mb_tma, 6 * kRawBoxBytes);
+#pragma unroll
+    for (int bx = 0; bx < 6; ++bx) {
+      const int64_t col = (bx < 2 ? q_col : bx < 4 ? k_col : v_col) + (bx & 1) * 64;
+      tma_load_2d(sm + OFF_RAW + bx * kRawBox, &tm_qkv, (int)col, (int)(tt - kHalo), &mb_tma);
+    }
+  };
+  // gate inputs of the next chunk (warp 0), kept as raw bf16 bits so that the
+  // loads are not waited for until the chunk that uses them
+  unsigned short pa[2] = {0, 0}, pb[2] = {0, 0};
+  const unsigned short* a16 = reinterpret_cast<const unsigned short*>(a);
+  const unsigned short* b16 = reinterpret_cast<const unsigned short*>(b);
+  auto load_gates = [&](int cc) {
+    const int64_t tt = seq0 + (int64_t)cc * kC;
+    const int LL = min(kC, len - cc * kC);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int r = 2 * lane + e;
+      if (r < LL) {
+        pa[e] = __ldg(a16 + (tt + r) * d.Hv + h);
+        pb[e] = __ldg(b16 + (tt + r) * d.Hv + h);
+      }
+    }
+  };
+  if (tid == 0) issue_raw(0);
+  if (warp == 0) load_gates(0);
+
   for (int c = 0; c < nchunks; ++c) {
     const int64_t t0 = seq0 + (int64_t)c * kC;
     const int L = min(kC, len - c * kC);
 
     // ------------------------------------------------------------ P0: raw tiles, gates
-    if (tid == 0) {
-      mbar_expect_tx(&mb_tma, 6 * kRawBoxBytes);
-#pragma unroll
-      for (int bx = 0; bx < 6; ++bx) {
-        const int64_t col = (bx < 2 ? q_col : bx < 4 ? k_col : v_col) + (bx & 1) * 64;
-        tma_load_2d(sm + OFF_RAW + bx * kRawBox, &tm_qkv, (int)col, (int)(t0 - kHalo), &mb_tma);
-      }
-    }
     if (warp == 0) {  // gates of rows 2*lane, 2*lane+1; inclusive scan of g
       float g2[2], be2[2];
 #pragma unroll
@@ -202,9 +224,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         g2[e] = 0.f;
         be2[e] = 0.f;
         if (r < L) {
-          const int64_t t = t0 + r;
-          g2[e] = negA * softplus_f(__bfloat162float(a[t * d.Hv + h]) + dtb);
-          be2[e] = 1.0f / (1.0f + expf(-__bfloat162float(b[t * d.Hv + h])));
+          g2[e] = negA * softplus_f(__uint_as_float((uint32_t)pa[e] << 16) + dtb);
+          be2[e] = 1.0f / (1.0f + expf(-__uint_as_float((uint32_t)pb[e] << 16)));
         }
       }
       float incl = g2[0] + g2[1];
@@ -456,10 +477,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     sync_tc();
 
     // ------------------------------------------------------------ M2: [T;0] [beta e^g K | beta V]
-    if (tid == 0) {  // z rows of this chunk, for the output gate (into the now idle raw-tile space)
-      mbar_expect_tx(&mb_z, 2 * 64 * 64 * 2);
-      tma_load_2d(sm + OFF_RAW, &tm_z, h * kD, (int)t0, &mb_z);
-      tma_load_2d(sm + OFF_RAW + 8192, &tm_z, h * kD + 64, (int)t0, &mb_z);
+    if (c + 1 < nchunks) {  // the raw-tile space is idle from here on: fetch the next chunk
+      if (tid == 0) issue_raw(c + 1);
+      if (warp == 0) load_gates(c + 1);
     }
     if (tid == 0) {
       const uint32_t ta = smem_u32(sm + OFF_TA), x = smem_u32(sm + OFF_X);
@@ -473,6 +493,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_after();
 
     // ------------------------------------------------------------ P2: [-W ; diag(e^gamma) Q]
+    if (tid == 0) {  // z rows of this chunk, for the output gate (into the X tile, idle after M2)
+      mbar_expect_tx(&mb_z, 2 * 64 * 64 * 2);
+      tma_load_2d(sm + OFF_X, &tm_z, h * kD, (int)t0, &mb_z);
+      tma_load_2d(sm + OFF_X + 8192, &tm_z, h * kD + 64, (int)t0, &mb_z);
+    }
     if (si < 64) {
       float v[32];
 #pragma unroll
@@ -556,9 +581,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int m = 0; m < 4; ++m) st16h(sm + OFF_SB + mnmaj_chunk(kD, si, 64 * hc + 32 * hh + 8 * m), S + 8 * m);
       }
-      if (si >= 64) {  // O rows: fp32 to shared memory (after the z tile) and row sums of squares
+      if (si >= 64) {  // O rows: fp32 into the [-W;Qg] tile (idle after M3), row sums of squares
         const int r = si - 64;
-        float* orow = reinterpret_cast<float*>(sm + OFF_RAW + 16384) + r * kOStride + 64 * hc;
+        float* orow = reinterpret_cast<float*>(sm + OFF_KQ) + r * kD;
         float ss = 0.f;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
@@ -566,8 +591,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) ss += v[jj] * v[jj];
 #pragma unroll
-          for (int m = 0; m < 8; ++m)
-            *reinterpret_cast<float4*>(orow + 32 * hh + 4 * m) = make_float4(v[4 * m], v[4 * m + 1], v[4 * m + 2], v[4 * m + 3]);
+          for (int m = 0; m < 8; ++m) {  // float4 slot c4 stored at c4 ^ (r % 8): conflict-free rows
+            const int c4 = 16 * hc + 8 * hh + m;
+            *reinterpret_cast<float4*>(orow + 4 * (c4 ^ (r & 7))) =
+                make_float4(v[4 * m], v[4 * m + 1], v[4 * m + 2], v[4 * m + 3]);
+          }
         }
         s_rms[64 * hc + r] = ss;
       }
@@ -579,15 +607,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int r = tid >> 2, q4 = tid & 3;
       if (r < L) {
         const float rinv = rsqrtf((s_rms[r] + s_rms[64 + r]) * (1.0f / kD) + d.norm_eps);
-        const float* orow = reinterpret_cast<const float*>(sm + OFF_RAW + 16384) + r * kOStride + 32 * q4;
-        const unsigned char* zbox = sm + OFF_RAW + (q4 >> 1) * 8192;
+        const float* orow = reinterpret_cast<const float*>(sm + OFF_KQ) + r * kD;
+        const unsigned char* zbox = sm + OFF_X + (q4 >> 1) * 8192;
         const int64_t off = (t0 + r) * HvD + (int64_t)h * kD + 32 * q4;
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
           const int zc = 32 * (q4 & 1) + 8 * m;  // column inside the 64-column z box
           const uint4 zr = *reinterpret_cast<const uint4*>(zbox + r * 128 + ((((zc >> 3) ^ (r & 7))) << 4));
-          const float4 oa = *reinterpret_cast<const float4*>(orow + 8 * m);
-          const float4 ob = *reinterpret_cast<const float4*>(orow + 8 * m + 4);
+          const int c4 = 8 * q4 + 2 * m;
+          const float4 oa = *reinterpret_cast<const float4*>(orow + 4 * (c4 ^ (r & 7)));
+          const float4 ob = *reinterpret_cast<const float4*>(orow + 4 * ((c4 + 1) ^ (r & 7)));
           const float ov[8] = {oa.x, oa.y, oa.z, oa.w, ob.x, ob.y, ob.z, ob.w};
           const uint32_t zw[4] = {zr.x, zr.y, zr.z, zr.w};
           uint32_t ow[4];

@@ -170,6 +170,36 @@ class ClockSampler:
                 "samples": len(s), "power_w_max": round(max(x[2] for x in s), 1), "source": "nvml"}
 
 
+# ------------------------------------------------------------------ ranks
+
+
+def rank_ops(dist, device):
+    """(barrier, max_over_ranks) for one process per GPU; with dist None, a
+    single process.  The barrier also synchronises the local device."""
+    import torch
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        if device.type == "cuda":
+            torch.cuda.synchronize(device)
+
+    def max_over_ranks(x: float) -> float:
+        if dist is None:
+            return float(x)
+        t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    return barrier, max_over_ranks
+
+
+def whole_job_rate(world: int, units_per_rank_step: float, steps: int, max_ms: float) -> float:
+    """Units per second of the whole job: every rank processes the same units
+    per step (weak scaling) and the slowest rank's time counts."""
+    return world * units_per_rank_step * steps / (max_ms / 1000.0)
+
+
 # ------------------------------------------------------------------ oracle timing
 
 
@@ -241,18 +271,7 @@ def run_gdn(args, rank, world, local_rank):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
     stream = torch.cuda.current_stream()
     pk = peaks()
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-        torch.cuda.synchronize()
-
-    def max_over_ranks(x: float) -> float:
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier, max_over_ranks = rank_ops(dist, torch.device("cuda", local_rank))
 
     # ---------------- prefill workload (B=1, T=4096)
     w = gi.WORKLOADS[PREFILL_WORKLOAD]
@@ -306,7 +325,7 @@ def run_gdn(args, rank, world, local_rank):
     n_launch, k_ms = per_kernel[kname]
     k_avg_ms = max_over_ranks(k_ms / max(1, n_launch))
     ms_per_step = ms_total / args.steps
-    value = world * T * args.steps / (ms_total / 1000.0)
+    value = whole_job_rate(world, T, args.steps, ms_total)
     pbytes = prefill_bytes(geo, [T], zero_state=True)
     src = source_hash("prefill_recurrent.cu" if kid == gdn.K.PREFILL_RECURRENT else "prefill_chunked.cu")
     roof_p = {"bound": "hbm", "achieved": round(pbytes / (k_avg_ms / 1000.0) / 1e9, 1), "peak": pk["hbm"],
@@ -338,7 +357,7 @@ def run_gdn(args, rank, world, local_rank):
     ev1.record(stream)
     barrier()
     e2e_ms = max_over_ranks(ev0.elapsed_time(ev1)) / e2e_steps
-    e2e = {"value": round(world * T / (e2e_ms / 1000.0), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+    e2e = {"value": round(whole_job_rate(world, T, 1, e2e_ms), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4), "steps": e2e_steps}
     del sets, pin
     torch.cuda.empty_cache()
@@ -383,7 +402,7 @@ def run_gdn(args, rank, world, local_rank):
               "unit": "GB/s", "frac": round(dbytes / (d_kernel_ms / 1000.0) / 1e9 / pk["hbm"], 4),
               "traffic": measured_traffic("decode:" + DECODE_WORKLOAD, source_hash("decode.cu")), "kernel": "decode",
               "kernel_ms": round(d_kernel_ms, 5), "algorithmic_bytes": dbytes, "peak_source": pk["src"]}
-    decode = {"value": round(world * N / (d_mean / 1000.0), 1), "unit": "tokens/s", "ms_per_step": round(d_mean, 5),
+    decode = {"value": round(whole_job_rate(world, N, 1, d_mean), 1), "unit": "tokens/s", "ms_per_step": round(d_mean, 5),
               "median_ms": round(statistics.median(step_ms), 5), "steps": dsteps, "num_seqs": N, "roofline": roof_d,
               "workload": "GDN decode, 64 sequences x 1 token, 16 key / 48 value heads x 128, bf16 inputs, "
                           "fp32 states ~N(0,0.02), fresh inputs every step"}

@@ -246,6 +246,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       s_ekd[2 * lane + 1] = expf(gC - gam1);
       if (lane == 0) *s_gC = gC;
     }
+    // conv weights of this lane's 12 channels, requested before waiting for the raw tiles
+    float wq[4][4], wk[4][4], wv[4][4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float4 x = __ldg(reinterpret_cast<const float4*>(conv_w + (q_col + 4 * lane + e) * 4));
+      const float4 y = __ldg(reinterpret_cast<const float4*>(conv_w + (k_col + 4 * lane + e) * 4));
+      const float4 zz = __ldg(reinterpret_cast<const float4*>(conv_w + (v_col + 4 * lane + e) * 4));
+      wq[e][0] = x.x; wq[e][1] = x.y; wq[e][2] = x.z; wq[e][3] = x.w;
+      wk[e][0] = y.x; wk[e][1] = y.y; wk[e][2] = y.z; wk[e][3] = y.w;
+      wv[e][0] = zz.x; wv[e][1] = zz.y; wv[e][2] = zz.z; wv[e][3] = zz.w;
+    }
     if (!mbar_wait(&mb_tma, ph_tma, kWaitNs)) abort_flag = 1;
     ph_tma ^= 1;
     if (c == 0) {  // rows before the sequence start come from the conv history
@@ -263,36 +274,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     {
       const int cc = (4 * lane) & 63;  // channel inside the lane's 64-channel box
       const int half = lane >> 4;
-      float wq[4][4], wk[4][4], wv[4][4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float4 x = __ldg(reinterpret_cast<const float4*>(conv_w + (q_col + 4 * lane + e) * 4));
-        const float4 y = __ldg(reinterpret_cast<const float4*>(conv_w + (k_col + 4 * lane + e) * 4));
-        const float4 zz = __ldg(reinterpret_cast<const float4*>(conv_w + (v_col + 4 * lane + e) * 4));
-        wq[e][0] = x.x; wq[e][1] = x.y; wq[e][2] = x.z; wq[e][3] = x.w;
-        wk[e][0] = y.x; wk[e][1] = y.y; wk[e][2] = y.z; wk[e][3] = y.w;
-        wv[e][0] = zz.x; wv[e][1] = zz.y; wv[e][2] = zz.z; wv[e][3] = zz.w;
-      }
       const unsigned char* rq = sm + OFF_RAW + (0 + half) * kRawBox;
       const unsigned char* rk = sm + OFF_RAW + (2 + half) * kRawBox;
       const unsigned char* rv = sm + OFF_RAW + (4 + half) * kRawBox;
 #pragma unroll 1
-      for (int rp = 0; rp < 4; ++rp) {  // two rows per pass for instruction-level parallelism
-        const int r0 = 8 * warp + 2 * rp;
-        float yq[2][4], yk[2][4], yv[2][4];
+      for (int rp = 0; rp < 2; ++rp) {  // four rows per pass for instruction-level parallelism
+        const int r0 = 8 * warp + 4 * rp;
+        float yq[4][4], yk[4][4], yv[4][4];
 #pragma unroll
-        for (int x = 0; x < 2; ++x)
+        for (int x = 0; x < 4; ++x)
 #pragma unroll
           for (int e = 0; e < 4; ++e) yq[x][e] = yk[x][e] = yv[x][e] = 0.f;
 #pragma unroll
-        for (int rowi = 0; rowi < 5; ++rowi) {  // raw rows r0 .. r0+4 feed the taps of both rows
+        for (int rowi = 0; rowi < 7; ++rowi) {  // raw rows r0 .. r0+6 feed the taps of the four rows
           float xq[4], xk[4], xv[4];
           const int off = raw_off(r0 + rowi, cc);
           ld4bf(rq + off, xq);
           ld4bf(rk + off, xk);
           ld4bf(rv + off, xv);
 #pragma unroll
-          for (int x = 0; x < 2; ++x) {
+          for (int x = 0; x < 4; ++x) {
             const int tap = rowi - x;
             if (tap >= 0 && tap < 4) {
 #pragma unroll
@@ -304,9 +305,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        float sq[2] = {0.f, 0.f}, sk[2] = {0.f, 0.f};
+        float sq[4] = {0.f, 0.f, 0.f, 0.f}, sk[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int x = 0; x < 2; ++x)
+        for (int x = 0; x < 4; ++x)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             yq[x][e] = silu_fast(yq[x][e]);
@@ -317,13 +318,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
-          sq[0] += __shfl_xor_sync(0xffffffffu, sq[0], off);
-          sq[1] += __shfl_xor_sync(0xffffffffu, sq[1], off);
-          sk[0] += __shfl_xor_sync(0xffffffffu, sk[0], off);
-          sk[1] += __shfl_xor_sync(0xffffffffu, sk[1], off);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            sq[x] += __shfl_xor_sync(0xffffffffu, sq[x], off);
+            sk[x] += __shfl_xor_sync(0xffffffffu, sk[x], off);
+          }
         }
 #pragma unroll
-        for (int x = 0; x < 2; ++x) {
+        for (int x = 0; x < 4; ++x) {
           const int r = r0 + x;
           const bool valid = r < L;
           const float rqs = d.q_scale * rsqrtf(sq[x] + d.l2_eps);

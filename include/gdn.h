@@ -186,6 +186,34 @@ GDN_API gdn_status gdn_decode_step(const gdn_config* cfg, const gdn_params* para
                            gdn_stream_t stream);
 
 /* --------------------------------------------------------------------------
+ * Multi-token decode for draft-and-verify rounds ("MTP candidate generation,
+ * verification, cache updates, rollback, accepted tokens", issue #89,
+ * Correctness gates; the K=2 draft-and-verify round of the Qwen3.8-27B FP8
+ * Core AI model card, What is fused).  Each of num_seqs sequences takes
+ * num_tokens (K, 1..GDN_MAX_DRAFT_TOKENS) consecutive tokens in one pass over
+ * its state: qkv [N, K, C_conv], z [N, K, Hv*d_v], a, b [N, K, Hv],
+ * o [N, K, Hv*d_v], token-major inside a sequence.  Token t is computed
+ * exactly as the t-th of K gdn_decode_step calls would compute it -- the same
+ * operations in the same order, so the results agree bit for bit.
+ *
+ *   commit == 0 (verify): o receives all K tokens' outputs; conv_state and
+ *     state are read but not written, so a rejected draft needs no rollback.
+ *     accept must be NULL.
+ *   commit != 0: sequence n applies its first accept[n] tokens (accept is a
+ *     device array of num_seqs counts, clamped to [0, K]; NULL means K) to
+ *     conv_state and state, and writes o for those tokens only.  Committing
+ *     a tokens equals a gdn_decode_step calls with those tokens.
+ *
+ * A verify followed by a commit of the accepted prefix reads each state twice
+ * and writes it once; that is the rollback-free form of the round.  Only
+ * d_k = d_v = 128 runs here; other geometries return GDN_E_UNSUPPORTED. */
+#define GDN_MAX_DRAFT_TOKENS 4
+GDN_API gdn_status gdn_decode_multi(const gdn_config* cfg, const gdn_params* params, const void* qkv, const void* z,
+                                    const void* a, const void* b, int32_t num_seqs, int32_t num_tokens,
+                                    int32_t commit, const int32_t* accept_dev, void* conv_state, float* state,
+                                    void* o, gdn_stream_t stream);
+
+/* --------------------------------------------------------------------------
  * Versioned state checkpoint of one sequence ("Persist every GDN convolution
  * and recurrent component in session checkpoints with versioned validation",
  * issue #95, Implementation; "identical ... BF16 convolution bytes, and fp32

@@ -18,9 +18,9 @@ import numpy as np
 
 __all__ = [
     "GdnError", "Config", "Params", "lib", "make_config", "conv_prefill", "conv_step", "prefill_workspace_size",
-    "prefill", "prefill_noalloc", "decode_step", "state_blob_size", "state_save", "state_restore", "device_status", "last_error",
+    "prefill", "prefill_noalloc", "decode_step", "decode_multi", "state_blob_size", "state_save", "state_restore", "device_status", "last_error",
     "abi_version", "launch_count", "launch_count_reset", "profiler_enable", "profiler_reset", "profiler_read",
-    "kernel_name", "EXPORTS", "ZERO_INIT_STATE", "ZERO_INIT_CONV", "PREFILL_RECURRENT", "K",
+    "kernel_name", "EXPORTS", "ZERO_INIT_STATE", "ZERO_INIT_CONV", "PREFILL_RECURRENT", "K", "MAX_DRAFT_TOKENS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
@@ -28,6 +28,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
 ZERO_INIT_STATE = 0x1
 ZERO_INIT_CONV = 0x2
 PREFILL_RECURRENT = 0x4
+MAX_DRAFT_TOKENS = 4
 
 F32, BF16 = 0, 1
 
@@ -48,7 +49,7 @@ EXPORTS = [
     "gdn_conv_prefill", "gdn_conv_step", "gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode_step",
     "gdn_state_blob_size", "gdn_state_save", "gdn_state_restore", "gdn_get_device_status", "gdn_last_error",
     "gdn_abi_version", "gdn_launch_count", "gdn_launch_count_reset", "gdn_kernel_name", "gdn_profiler_enable",
-    "gdn_profiler_reset", "gdn_profiler_read", "gdn_prefill_noalloc",
+    "gdn_profiler_reset", "gdn_profiler_read", "gdn_prefill_noalloc", "gdn_decode_multi",
 ]
 
 
@@ -89,6 +90,7 @@ def lib():
             "gdn_prefill": [P, P, P, P, P, P, P, P, I32, I32, U32, P, P, P, P, SZ, P],
             "gdn_prefill_noalloc": [P, P, P, P, P, P, P, P, I32, I32, U32, P, P, P, P],
             "gdn_decode_step": [P, P, P, P, P, P, I32, P, P, P, P],
+            "gdn_decode_multi": [P, P, P, P, P, P, I32, I32, I32, P, P, P, P, P],
             "gdn_state_blob_size": [P, P],
             "gdn_state_save": [P, P, P, I32, P, SZ, P],
             "gdn_state_restore": [P, P, SZ, I32, P, P, P],
@@ -196,6 +198,17 @@ def decode_step(cfg, params, qkv, z, a, b, num_seqs, conv_state, state, o, strea
     prm = _params(*params)
     _check(lib().gdn_decode_step(ctypes.byref(cfg), ctypes.byref(prm), _p(qkv), _p(z), _p(a), _p(b), num_seqs,
                                  _p(conv_state), _p(state), _p(o), _stream(stream)))
+
+
+def decode_multi(cfg, params, qkv, z, a, b, num_seqs, num_tokens, commit, accept, conv_state, state, o,
+                 stream=None):
+    """gdn_decode_multi: num_tokens draft tokens per sequence in one pass.
+    commit=False verifies (outputs only, caches untouched, accept None);
+    commit=True applies accept[n] tokens (device int32, None = all)."""
+    prm = _params(*params)
+    _check(lib().gdn_decode_multi(ctypes.byref(cfg), ctypes.byref(prm), _p(qkv), _p(z), _p(a), _p(b), num_seqs,
+                                  num_tokens, 1 if commit else 0, _p(accept),
+                                  _p(conv_state), _p(state), _p(o), _stream(stream)))
 
 
 def state_blob_size(cfg) -> int:

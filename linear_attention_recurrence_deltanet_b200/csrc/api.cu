@@ -446,6 +446,36 @@ gdn_status gdn_decode_step(const gdn_config* cfg, const gdn_params* params, cons
   return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_decode_step launch");
 }
 
+gdn_status gdn_decode_multi(const gdn_config* cfg, const gdn_params* params, const void* qkv, const void* z,
+                            const void* a, const void* b, int32_t num_seqs, int32_t num_tokens, int32_t commit,
+                            const int32_t* accept_dev, void* conv_state, float* state, void* o,
+                            gdn_stream_t stream) {
+  gdn::Dims d;
+  gdn_status s;
+  if ((s = check_cfg(cfg, &d)) != GDN_OK) return s;
+  if ((s = check_params(params)) != GDN_OK) return s;
+  if (num_seqs <= 0 || (int64_t)num_seqs * d.Hk > 0x7fffffffLL)
+    return fail(GDN_E_INVAL, "num_seqs %d out of range", num_seqs);
+  if (num_tokens < 1 || num_tokens > GDN_MAX_DRAFT_TOKENS)
+    return fail(GDN_E_INVAL, "num_tokens %d outside [1, %d]", num_tokens, GDN_MAX_DRAFT_TOKENS);
+  if (!commit && accept_dev) return fail(GDN_E_INVAL, "accept must be NULL when commit == 0");
+  if (d.dk != 128 || d.dv != 128)
+    return fail(GDN_E_UNSUPPORTED, "gdn_decode_multi runs d_k = d_v = 128 only (got %d, %d)", d.dk, d.dv);
+  if ((s = check_ptr(qkv, "qkv")) != GDN_OK || (s = check_ptr(z, "z")) != GDN_OK ||
+      (s = check_gate_ptr(a, "a", cfg)) != GDN_OK || (s = check_gate_ptr(b, "b", cfg)) != GDN_OK ||
+      (s = check_ptr(conv_state, "conv_state")) != GDN_OK || (s = check_ptr(state, "state")) != GDN_OK ||
+      (s = check_ptr(o, "o")) != GDN_OK)
+    return s;
+  if (accept_dev && ((uintptr_t)accept_dev & 3u)) return fail(GDN_E_INVAL, "accept is not 4-byte aligned");
+  int dev = 0;
+  if ((s = check_device(&dev)) != GDN_OK) return s;
+  cudaError_t e = gdn::launch_decode_multi(d, cfg->io_dtype == GDN_BF16, params->conv_w, params->A_log,
+                                           params->dt_bias, params->norm_w, qkv, z, a, b, num_seqs, num_tokens,
+                                           accept_dev, commit ? 1 : 0, conv_state, state, o, g_status_ptr[dev],
+                                           (cudaStream_t)stream);
+  return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_decode_multi launch");
+}
+
 gdn_status gdn_state_blob_size(const gdn_config* cfg, size_t* bytes) {
   gdn::Dims d;
   gdn_status s;

@@ -42,6 +42,13 @@ cudaError_t launch_decode_step(const Dims& d, bool bf16, const float* conv_w, co
                                const void* a, const void* b, int32_t num_seqs, void* conv_state, float* state,
                                void* o, int32_t* status, cudaStream_t stream);
 
+// multi-token decode (draft-and-verify), d = 128: verify (write_state 0) or commit
+cudaError_t launch_decode_multi(const Dims& d, bool bf16, const float* conv_w, const float* A_log,
+                                const float* dt_bias, const float* norm_w, const void* qkv, const void* z,
+                                const void* a, const void* b, int32_t num_seqs, int32_t num_tokens,
+                                const int32_t* accept, int write_state, void* conv_state, float* state, void* o,
+                                int32_t* status, cudaStream_t stream);
+
 // prefill_recurrent.cu
 cudaError_t launch_prefill_recurrent(const Dims& d, bool bf16, const float* conv_w, const float* A_log,
                                      const float* dt_bias, const float* norm_w, const void* qkv, const void* z,

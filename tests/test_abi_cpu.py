@@ -129,6 +129,39 @@ def test_prefill_validation_rejects_before_launch():
         assert np.array_equal(v.view, snapshot[k]), k
 
 
+def test_decode_multi_validation_rejects_before_launch():
+    """Draft counts outside 1..4, an accept array on a verify call and head
+    dims other than 128 are refused on the host, with every buffer intact."""
+    def bufs(geo, N, K):
+        t = dict(qkv=FakeTensor(N * K * geo.conv_dim * 2), z=FakeTensor(N * K * geo.value_dim * 2),
+                 a=FakeTensor(N * K * geo.num_v_heads * 2), b=FakeTensor(N * K * geo.num_v_heads * 2),
+                 conv=FakeTensor(N * 3 * geo.conv_dim * 2), acc=FakeTensor(4 * N),
+                 state=FakeTensor(N * geo.num_v_heads * geo.head_v_dim * geo.head_k_dim * 4),
+                 o=FakeTensor(N * K * geo.value_dim * 2))
+        params = tuple(FakeTensor(n) for n in (geo.conv_dim * 16, 4 * geo.num_v_heads, 4 * geo.num_v_heads,
+                                               4 * geo.head_v_dim))
+        return t, params
+
+    geo = gi.Geometry(num_k_heads=2, num_v_heads=6)
+    t, params = bufs(geo, 2, 2)
+    snap = {k: v.view.copy() for k, v in t.items()}
+    cfg = gdn.make_config(geo)
+    for K, commit, acc, N, status in [(0, True, None, 2, "GDN_E_INVAL"), (5, True, None, 2, "GDN_E_INVAL"),
+                                      (2, False, t["acc"], 2, "GDN_E_INVAL"), (2, True, None, 0, "GDN_E_INVAL")]:
+        with pytest.raises(gdn.GdnError) as e:
+            gdn.decode_multi(cfg, params, t["qkv"], t["z"], t["a"], t["b"], N, K, commit, acc, t["conv"],
+                             t["state"], t["o"], stream=0)
+        assert e.value.name == status, (K, commit, N)
+    geo64 = gi.Geometry(num_k_heads=2, num_v_heads=4, head_k_dim=64, head_v_dim=64)
+    t64, params64 = bufs(geo64, 2, 2)
+    with pytest.raises(gdn.GdnError) as e:
+        gdn.decode_multi(gdn.make_config(geo64), params64, t64["qkv"], t64["z"], t64["a"], t64["b"], 2, 2, True,
+                         None, t64["conv"], t64["state"], t64["o"], stream=0)
+    assert e.value.name == "GDN_E_UNSUPPORTED"
+    for k, v in t.items():
+        assert np.array_equal(v.view, snap[k]), k
+
+
 # ---------------------------------------------------------------- state blobs (host memory)
 
 MAGIC = b"GDNSTATE"

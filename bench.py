@@ -6,7 +6,9 @@ One step = one gdn_prefill over a Qwen3.8-shaped layer (B=1, T=4096, 16 key /
 48 value heads x 128, chunk 64, bf16 inputs, zero initial state), which runs
 every prefill stage of the mixer.  The decode entry point (64 sequences, one
 token each, fresh bf16 inputs per step, states ~N(0, 0.02)) is timed over
-1000 consecutive steps in the same run and reported under "decode".
+1000 consecutive steps in the same run and reported under "decode"; K=2
+draft-and-verify rounds (a verify pass, then a commit of a seeded accepted
+prefix) on the same sequences are reported under "draft_verify".
 
 Inputs are synthetic (seeded numpy draws) and resident in HBM before timing.
 Between timed prefill steps the inputs rotate over 3 sets (~540 MB, > 4x L2)
@@ -42,6 +44,7 @@ PREFILL_WORKLOAD = "prefill_t4096"
 DECODE_WORKLOAD = "decode_b64"
 DECODE_STEPS = 1000
 ROTATE = 3
+DRAFT_ROUNDS = 200
 
 
 def peaks():
@@ -407,6 +410,60 @@ def run_gdn(args, rank, world, local_rank):
               "workload": "GDN decode, 64 sequences x 1 token, 16 key / 48 value heads x 128, bf16 inputs, "
                           "fp32 states ~N(0,0.02), fresh inputs every step"}
 
+    # ---------------- K=2 draft-and-verify rounds on the same sequences: a verify pass over both tokens, then a
+    # commit of each sequence's accepted prefix (1 or 2 tokens, seeded); accepted tokens/s is the rate
+    K = 2
+    rounds = max(1, min(DRAFT_ROUNDS, dsteps // K))
+    mq, mz, ma, mb = (x[:rounds * K].view(rounds, K, *x.shape[1:]).transpose(1, 2).contiguous()
+                      for x in (dq, dz, da, db))
+    del dq, dz, da, db
+    acc_h = np.random.default_rng([seed, 7]).integers(1, K + 1, size=(rounds, N)).astype(np.int32)
+    acc = torch.from_numpy(acc_h).cuda()
+    mo = torch.empty((N, K, gd.value_dim), dtype=torch.bfloat16, device="cuda")
+
+    def draft_round(r):
+        gdn.decode_multi(cfg, dparams, mq[r], mz[r], ma[r], mb[r], N, K, False, None, conv, st, mo, stream=stream)
+        vev[r].record(stream)
+        gdn.decode_multi(cfg, dparams, mq[r], mz[r], ma[r], mb[r], N, K, True, acc[r], conv, st, mo, stream=stream)
+        cev[r + 1].record(stream)
+
+    vev = [torch.cuda.Event(enable_timing=True) for _ in range(rounds)]
+    cev = [torch.cuda.Event(enable_timing=True) for _ in range(rounds + 1)]
+    for r in range(min(3, rounds)):
+        draft_round(r)
+    conv.copy_(io_tensor(conv0))
+    st.copy_(torch.from_numpy(st0))
+    barrier()
+    clocks.active = True
+    cev[0].record(stream)
+    for r in range(rounds):
+        draft_round(r)
+    barrier()
+    clocks.active = False
+    v_ms = max_over_ranks(sum(cev[r].elapsed_time(vev[r]) for r in range(rounds)) / rounds)
+    c_ms = max_over_ranks(sum(vev[r].elapsed_time(cev[r + 1]) for r in range(rounds)) / rounds)
+    r_ms = max_over_ranks(cev[0].elapsed_time(cev[rounds]) / rounds)
+    state_b = N * gd.num_v_heads * gd.head_v_dim * gd.head_k_dim * 4
+    tok_in = N * K * (gd.conv_dim + gd.value_dim + 2 * gd.num_v_heads) * gd.io_bytes
+    hist_b = N * (gd.conv_width - 1) * gd.conv_dim * gd.io_bytes
+    prm_b = (gd.conv_dim * gd.conv_width + 2 * gd.num_v_heads + gd.head_v_dim) * 4
+    v_bytes = state_b + tok_in + hist_b + prm_b + N * K * gd.value_dim * gd.io_bytes
+    c_bytes = 2 * state_b + tok_in + 2 * hist_b + prm_b + int(acc_h.mean() * N) * gd.value_dim * gd.io_bytes
+
+    def roof(b, ms, name):
+        return {"bound": "hbm", "achieved": round(b / (ms / 1000.0) / 1e9, 1), "peak": pk["hbm"], "unit": "GB/s",
+                "frac": round(b / (ms / 1000.0) / 1e9 / pk["hbm"], 4), "traffic": None, "kernel": name,
+                "kernel_ms": round(ms, 5), "algorithmic_bytes": int(b), "peak_source": pk["src"]}
+
+    draft = {"value": round(whole_job_rate(world, float(acc_h.sum()) / rounds, 1, r_ms), 1),
+             "unit": "accepted tokens/s", "ms_per_round": round(r_ms, 5), "rounds": rounds, "draft_tokens": K,
+             "mean_accepted": round(float(acc_h.mean()), 4), "verify": roof(v_bytes, v_ms, "decode (verify, K=2)"),
+             "commit": roof(c_bytes, c_ms, "decode (commit)"),
+             "workload": "64 sequences, K=2 draft tokens per round, verify then commit of a seeded accepted "
+                         "prefix (1 or 2 tokens), same geometry and states as the decode workload; "
+                         "time between events on the launching stream"}
+    del mq, mz, ma, mb
+
     clk = clocks.summary()
     cpu = cpu_baseline(inp) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
     if rank == 0:
@@ -418,7 +475,7 @@ def run_gdn(args, rank, world, local_rank):
                                    "fp32 state from zero", "global_batch": world, "seq_len": T, "chunk": C,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": f"inputs rotate over {ROTATE} sets (> 4x L2) between steps"},
-            "roofline": roof_p, "decode": decode, "e2e": e2e, "gpu_launches": launches,
+            "roofline": roof_p, "decode": decode, "draft_verify": draft, "e2e": e2e, "gpu_launches": launches,
             "kernels": kernel_share, "clocks": clk, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

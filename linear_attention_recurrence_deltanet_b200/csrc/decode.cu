@@ -196,7 +196,7 @@ __device__ __forceinline__ float dot4(const float4& a, const float4& b, float ac
 }
 
 template <typename T, int K>
-__global__ void __launch_bounds__(kBulkThreads, K == 1 ? 8 : 4)
+__global__ void __launch_bounds__(kBulkThreads, K <= 2 ? 8 : 4)
     decode_bulk_kernel(Dims d, const float* __restrict__ conv_w, const float* __restrict__ A_log,
                        const float* __restrict__ dt_bias, const float* __restrict__ norm_w,
                        const T* __restrict__ qkv, const T* __restrict__ z, const T* __restrict__ a,

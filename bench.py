@@ -295,7 +295,8 @@ def run_gdn(args, rank, world, local_rank):
                                                                            dtype=torch.float32, device="cuda")))
     del base
     ws = torch.empty(gdn.prefill_workspace_size(cfg, T, 1, C) + 256, dtype=torch.uint8, device="cuda")
-    flags = gdn.ZERO_INIT_STATE | (gdn.PREFILL_RECURRENT if args.recurrent else 0)
+    flags = gdn.ZERO_INIT_STATE | (gdn.PREFILL_RECURRENT if args.recurrent else 0) | \
+        (gdn.PREFILL_FUSED if args.fused else 0)
 
     def prefill(i):
         s = sets[i % ROTATE]
@@ -320,17 +321,25 @@ def run_gdn(args, rank, world, local_rank):
     launches = gdn.launch_count()
     gdn.profiler_enable(False)
     ms_total = max_over_ranks(ev0.elapsed_time(ev1))
-    kid = gdn.K.PREFILL_RECURRENT if args.recurrent else None
     per_kernel = {gdn.kernel_name(k): gdn.profiler_read(k) for k in range(gdn.K.COUNT)}
-    if kid is None:  # the dominant prefill kernel is whichever mixer kernel ran
-        kid = max((gdn.K.PREFILL_CHUNKED, gdn.K.PREFILL_RECURRENT), key=lambda k: per_kernel[gdn.kernel_name(k)][1])
-    kname = gdn.kernel_name(kid)
-    n_launch, k_ms = per_kernel[kname]
-    k_avg_ms = max_over_ranks(k_ms / max(1, n_launch))
+    # The mixer kernel(s) that ran.  The three-kernel chunked path is one
+    # logical kernel: its roofline takes the prefill's algorithmic bytes over
+    # the summed average launch times of its three stages.
+    split_ids = (gdn.K.SPLIT_CONV, gdn.K.SPLIT_PREP, gdn.K.SPLIT_CHAIN)
+    if not args.recurrent and not args.fused and per_kernel[gdn.kernel_name(gdn.K.SPLIT_CHAIN)][0]:
+        kids, kname, src = split_ids, "split_conv+split_prep+split_chain", source_hash("prefill_split.cu")
+    elif args.recurrent:
+        kids, kname, src = (gdn.K.PREFILL_RECURRENT,), "prefill_recurrent", source_hash("prefill_recurrent.cu")
+    else:
+        kids, kname, src = (gdn.K.PREFILL_CHUNKED,), "prefill_chunked", source_hash("prefill_chunked.cu")
+    k_avg_ms = 0.0
+    for k in kids:
+        n_launch, k_ms = per_kernel[gdn.kernel_name(k)]
+        k_avg_ms += k_ms / max(1, n_launch)
+    k_avg_ms = max_over_ranks(k_avg_ms)
     ms_per_step = ms_total / args.steps
     value = whole_job_rate(world, T, args.steps, ms_total)
     pbytes = prefill_bytes(geo, [T], zero_state=True)
-    src = source_hash("prefill_recurrent.cu" if kid == gdn.K.PREFILL_RECURRENT else "prefill_chunked.cu")
     roof_p = {"bound": "hbm", "achieved": round(pbytes / (k_avg_ms / 1000.0) / 1e9, 1), "peak": pk["hbm"],
               "unit": "GB/s", "frac": round(pbytes / (k_avg_ms / 1000.0) / 1e9 / pk["hbm"], 4),
               "traffic": measured_traffic(kname + ":" + PREFILL_WORKLOAD, src), "kernel": kname,
@@ -493,6 +502,7 @@ def main():
     ap.add_argument("--impl", choices=["gdn", "reference"], default="gdn")
     ap.add_argument("--decode-steps", type=int, default=DECODE_STEPS)
     ap.add_argument("--recurrent", action="store_true", help="time the token-recurrent prefill kernel")
+    ap.add_argument("--fused", action="store_true", help="time the single-kernel chunked prefill")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps

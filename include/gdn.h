@@ -103,6 +103,8 @@ typedef struct {
 #define GDN_ZERO_INIT_STATE 0x1u /* ignore the incoming recurrent state: start from S = 0 */
 #define GDN_ZERO_INIT_CONV 0x2u  /* ignore the incoming conv history: treat it as zeros */
 #define GDN_PREFILL_RECURRENT 0x4u /* run the token-recurrent fp32 kernel instead of the chunked one */
+#define GDN_PREFILL_FUSED 0x8u     /* chunked path as one kernel per (sequence, value head): needs only the
+                                      schedule as workspace (see gdn_prefill) */
 
 /* --------------------------------------------------------------------------
  * Causal depthwise Conv1D + SiLU over the q/k/v channels (issue #88, Scope:
@@ -131,7 +133,12 @@ GDN_API gdn_status gdn_conv_step(const gdn_config* cfg, const void* x, const flo
  *
  * Workspace: caller-provided device scratch of at least the size that
  * gdn_prefill_workspace_size() returns for the same (cfg, total_tokens,
- * num_seqs, chunk_size); 256-byte aligned.
+ * num_seqs, chunk_size); 256-byte aligned.  For the tensor-core path (bf16,
+ * d_k = d_v = 128, chunk 64) that size holds the schedule plus the chunked
+ * form's intermediates: fp16 q^, k^ (two parts each) and v^ for every token
+ * and a 65,664-byte operand record per (chunk, value head) -- about 78 KB per
+ * token at 16 key / 48 value heads.  With GDN_PREFILL_FUSED the schedule
+ * alone suffices (a few bytes per chunk).
  */
 GDN_API gdn_status gdn_prefill_workspace_size(const gdn_config* cfg, int64_t total_tokens, int32_t num_seqs,
                                       int32_t chunk_size, size_t* bytes);
@@ -139,11 +146,16 @@ GDN_API gdn_status gdn_prefill_workspace_size(const gdn_config* cfg, int64_t tot
 /* gdn_prefill: runs the whole mixer over every token of every sequence.
  *   chunk_size: 16, 32, 64 or 128 (tokens per chunk of the chunkwise form;
  *               chunks restart at each sequence start).
- *   flags:      GDN_ZERO_INIT_STATE / GDN_ZERO_INIT_CONV / GDN_PREFILL_RECURRENT.
+ *   flags:      GDN_ZERO_INIT_STATE / GDN_ZERO_INIT_CONV / GDN_PREFILL_RECURRENT /
+ *               GDN_PREFILL_FUSED.
  *   conv_state and state are read and updated in place; o is written.
- * The chunked kernel runs when io dtype is bf16 and d_k = d_v = 128; every
- * other supported case (and GDN_PREFILL_RECURRENT) runs the token-recurrent
- * fp32 kernel.  Both compute in fp32 with an fp32 state. */
+ * When io dtype is bf16, d_k = d_v = 128 and chunk_size = 64 the chunked form
+ * runs on tensor cores: by default as three kernels (conv of every token; the
+ * state-independent operands of every chunk; the state carry across chunks),
+ * with GDN_PREFILL_FUSED as one kernel per (sequence, value head).  The two
+ * agree to fp32 rounding (not bit for bit).  Every other supported case (and
+ * GDN_PREFILL_RECURRENT) runs the token-recurrent fp32 kernel.  All compute in
+ * fp32 with an fp32 state. */
 GDN_API gdn_status gdn_prefill(const gdn_config* cfg, const gdn_params* params, const void* qkv, const void* z,
                        const void* a, const void* b, const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host,
                        int32_t num_seqs, int32_t chunk_size, uint32_t flags, void* conv_state, float* state,
@@ -264,7 +276,10 @@ typedef enum {
   GDN_K_PREFILL_CHUNKED = 5,
   GDN_K_DECODE = 6,
   GDN_K_STATE_CHECKSUM = 7,
-  GDN_K_COUNT = 8
+  GDN_K_SPLIT_CONV = 8,   /* chunked prefill, stage 1: conv + SiLU + L2 norm of every token */
+  GDN_K_SPLIT_PREP = 9,   /* stage 2: per-(chunk, value head) operands of the state carry */
+  GDN_K_SPLIT_CHAIN = 10, /* stage 3: the state carry across chunks and the output rows */
+  GDN_K_COUNT = 11
 } gdn_kernel_id;
 
 GDN_API const char* gdn_kernel_name(int32_t kernel_id);

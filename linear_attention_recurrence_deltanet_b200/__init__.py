@@ -20,7 +20,7 @@ __all__ = [
     "GdnError", "Config", "Params", "lib", "make_config", "conv_prefill", "conv_step", "prefill_workspace_size",
     "prefill", "prefill_noalloc", "decode_step", "decode_multi", "state_blob_size", "state_save", "state_restore", "device_status", "last_error",
     "abi_version", "launch_count", "launch_count_reset", "profiler_enable", "profiler_reset", "profiler_read",
-    "kernel_name", "EXPORTS", "ZERO_INIT_STATE", "ZERO_INIT_CONV", "PREFILL_RECURRENT", "K", "MAX_DRAFT_TOKENS",
+    "kernel_name", "EXPORTS", "ZERO_INIT_STATE", "ZERO_INIT_CONV", "PREFILL_RECURRENT", "PREFILL_FUSED", "K", "MAX_DRAFT_TOKENS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
@@ -28,6 +28,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
 ZERO_INIT_STATE = 0x1
 ZERO_INIT_CONV = 0x2
 PREFILL_RECURRENT = 0x4
+PREFILL_FUSED = 0x8
 MAX_DRAFT_TOKENS = 4
 
 F32, BF16 = 0, 1
@@ -39,9 +40,9 @@ STATUS = {0: "GDN_OK", -1: "GDN_E_INVAL", -2: "GDN_E_UNSUPPORTED", -3: "GDN_E_WO
 
 class K:
     """Kernel ids of the profiler (gdn_kernel_id)."""
-    CONV_PREFILL, CONV_STEP, CONV_HISTORY, SCHEDULE, PREFILL_RECURRENT, PREFILL_CHUNKED, DECODE, STATE_CHECKSUM = \
-        range(8)
-    COUNT = 8
+    (CONV_PREFILL, CONV_STEP, CONV_HISTORY, SCHEDULE, PREFILL_RECURRENT, PREFILL_CHUNKED, DECODE, STATE_CHECKSUM,
+     SPLIT_CONV, SPLIT_PREP, SPLIT_CHAIN) = range(11)
+    COUNT = 11
 
 
 # Every symbol include/gdn.h declares.

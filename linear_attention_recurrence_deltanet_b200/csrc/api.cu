@@ -198,8 +198,17 @@ int64_t chunk_bound(int64_t total_tokens, int32_t num_seqs, int32_t chunk_size) 
   return total_tokens / chunk_size + num_seqs + 1;
 }
 
-size_t prefill_ws_bytes(int64_t total_tokens, int32_t num_seqs, int32_t chunk_size) {
-  return gdn::schedule_layout(num_seqs, chunk_bound(total_tokens, num_seqs, chunk_size)).total_bytes;
+// The three-kernel chunked path runs unless GDN_PREFILL_FUSED or GDN_PREFILL_RECURRENT is given.
+bool split_path(const gdn::Dims& d, const gdn_config* cfg, int32_t chunk_size, uint32_t flags) {
+  return !(flags & (GDN_PREFILL_FUSED | GDN_PREFILL_RECURRENT)) &&
+         gdn::prefill_chunked_supported(d, cfg->io_dtype == GDN_BF16, chunk_size);
+}
+
+// schedule, then (three-kernel path only) the intermediates of the chunked form
+size_t prefill_ws_bytes(const gdn::Dims& d, bool split, int64_t total_tokens, int32_t num_seqs, int32_t chunk_size) {
+  const int64_t chunks = chunk_bound(total_tokens, num_seqs, chunk_size);
+  const size_t sched = gdn::schedule_layout(num_seqs, chunks).total_bytes;
+  return split ? sched + gdn::split_layout(d, total_tokens, chunks).total_bytes : sched;
 }
 
 // ---------------------------------------------------------------- state blob
@@ -241,6 +250,10 @@ bool is_device_ptr(const void* p) {
 namespace gdn {
 void set_error_message(const char* msg) { g_err = msg; }
 
+size_t prefill_fused_ws_bytes(int64_t total_tokens, int32_t num_seqs, int32_t chunk_size) {
+  return schedule_layout(num_seqs, chunk_bound(total_tokens, num_seqs, chunk_size)).total_bytes;
+}
+
 LaunchScope::LaunchScope(int kernel_id, cudaStream_t s) : id(kernel_id), stream(s), token(nullptr) {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (g_prof.on) {
@@ -275,8 +288,9 @@ int64_t gdn_launch_count(void) { return g_launches.load(); }
 void gdn_launch_count_reset(void) { g_launches.store(0); }
 
 const char* gdn_kernel_name(int32_t id) {
-  static const char* names[GDN_K_COUNT] = {"conv_prefill", "conv_step",  "conv_history", "schedule",
-                                           "prefill_recurrent", "prefill_chunked", "decode", "state_checksum"};
+  static const char* names[GDN_K_COUNT] = {"conv_prefill",    "conv_step",       "conv_history", "schedule",
+                                           "prefill_recurrent", "prefill_chunked", "decode",       "state_checksum",
+                                           "split_conv",        "split_prep",      "split_chain"};
   return (id >= 0 && id < GDN_K_COUNT) ? names[id] : "unknown";
 }
 
@@ -365,7 +379,7 @@ gdn_status gdn_prefill_workspace_size(const gdn_config* cfg, int64_t total_token
   if (total_tokens < 0 || num_seqs <= 0 || num_seqs > kMaxSeqs) return fail(GDN_E_INVAL, "bad sizes");
   if (chunk_size != 16 && chunk_size != 32 && chunk_size != 64 && chunk_size != 128)
     return fail(GDN_E_INVAL, "chunk_size %d (16, 32, 64 or 128)", chunk_size);
-  *bytes = prefill_ws_bytes(total_tokens, num_seqs, chunk_size);
+  *bytes = prefill_ws_bytes(d, split_path(d, cfg, chunk_size, 0), total_tokens, num_seqs, chunk_size);
   return GDN_OK;
 }
 
@@ -379,7 +393,7 @@ gdn_status gdn_prefill(const gdn_config* cfg, const gdn_params* params, const vo
   if ((s = check_params(params)) != GDN_OK) return s;
   if (chunk_size != 16 && chunk_size != 32 && chunk_size != 64 && chunk_size != 128)
     return fail(GDN_E_INVAL, "chunk_size %d (16, 32, 64 or 128)", chunk_size);
-  const uint32_t known = GDN_ZERO_INIT_STATE | GDN_ZERO_INIT_CONV | GDN_PREFILL_RECURRENT;
+  const uint32_t known = GDN_ZERO_INIT_STATE | GDN_ZERO_INIT_CONV | GDN_PREFILL_RECURRENT | GDN_PREFILL_FUSED;
   if (flags & ~known) return fail(GDN_E_INVAL, "unknown flags 0x%x", flags & ~known);
   int64_t total = 0;
   int32_t max_len = 0;
@@ -391,7 +405,8 @@ gdn_status gdn_prefill(const gdn_config* cfg, const gdn_params* params, const vo
         (s = check_ptr(o, "o")) != GDN_OK)
       return s;
   }
-  const size_t need = prefill_ws_bytes(total, num_seqs, chunk_size);
+  const bool split = split_path(d, cfg, chunk_size, flags);
+  const size_t need = prefill_ws_bytes(d, split, total, num_seqs, chunk_size);
   if (workspace_bytes < need || (need > 0 && !workspace))
     return fail(GDN_E_WORKSPACE, "workspace of %zu bytes at %p, need %zu", workspace_bytes, workspace, need);
   if (((uintptr_t)workspace & 255u) != 0) return fail(GDN_E_WORKSPACE, "workspace is not 256-byte aligned");
@@ -407,12 +422,20 @@ gdn_status gdn_prefill(const gdn_config* cfg, const gdn_params* params, const vo
   const gdn::ScheduleLayout L = gdn::schedule_layout(num_seqs, chunks);
   cudaError_t e = cudaSuccess;
   const int32_t* order = nullptr;
-  if (num_seqs > 1) {
+  if (num_seqs > 1 || split) {
     e = gdn::launch_schedule(cu_seqlens_dev, num_seqs, chunk_size, chunks, workspace, st);
-    order = (const int32_t*)((const char*)workspace + L.order_off);
+    if (num_seqs > 1) order = (const int32_t*)((const char*)workspace + L.order_off);
   }
   const bool chunked = !(flags & GDN_PREFILL_RECURRENT) && gdn::prefill_chunked_supported(d, bf16, chunk_size);
-  if (e == cudaSuccess && chunked)
+  if (e == cudaSuccess && split) {
+    // intermediates start after the schedule sized for the chunk bound (the layout the size query assumed)
+    const size_t sched = gdn::schedule_layout(num_seqs, chunk_bound(total, num_seqs, chunk_size)).total_bytes;
+    e = gdn::launch_prefill_split(d, params->conv_w, params->A_log, params->dt_bias, params->norm_w, qkv, z, a, b,
+                                  cu_seqlens_dev, order, (const int32_t*)((const char*)workspace + L.chunk_off_off),
+                                  (const int4*)((const char*)workspace + L.chunk_map_off), num_seqs, total, chunks,
+                                  zero_state, zero_conv, conv_state, state, o, (char*)workspace + sched,
+                                  g_status_ptr[dev], st);
+  } else if (e == cudaSuccess && chunked)
     e = gdn::launch_prefill_chunked(d, params->conv_w, params->A_log, params->dt_bias, params->norm_w, qkv, z, a, b,
                                     cu_seqlens_dev, order, num_seqs, total, zero_state, zero_conv, conv_state, state,
                                     o, g_status_ptr[dev], st);

@@ -2,6 +2,7 @@
 // launch error; arguments are validated by the C-ABI layer (api.cu) first.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -64,8 +65,29 @@ cudaError_t launch_prefill_chunked(const Dims& d, const float* conv_w, const flo
                                    bool zero_state, bool zero_conv, const void* conv_state, float* state, void* o,
                                    int32_t* status, cudaStream_t stream);
 
+// cuTensorMapEncodeTiled, looked up once through the runtime (NULL if the driver lacks it)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn();
+
+// prefill_split.cu (tcgen05; bf16 io, d_k = d_v = 128, chunk 64): conv, per-chunk prep and
+// state chain as three kernels over a workspace of intermediates (after the schedule)
+struct SplitLayout {
+  size_t qk_hi, qk_lo, v, records, total_bytes;
+};
+SplitLayout split_layout(const Dims& d, int64_t total_tokens, int64_t chunk_bound);
+cudaError_t launch_prefill_split(const Dims& d, const float* conv_w, const float* A_log, const float* dt_bias,
+                                 const float* norm_w, const void* qkv, const void* z, const void* a, const void* b,
+                                 const int32_t* cu, const int32_t* order, const int32_t* chunk_off,
+                                 const int4* chunk_map, int32_t N, int64_t total_tokens, int64_t total_chunks,
+                                 bool zero_state, bool zero_conv, const void* conv_state, float* state, void* o,
+                                 void* split_ws, int32_t* status, cudaStream_t stream);
+
 // api.cu: records a message for gdn_last_error() on the calling thread.
 void set_error_message(const char* msg);
+// api.cu: workspace bytes of gdn_prefill with GDN_PREFILL_FUSED (the schedule only)
+size_t prefill_fused_ws_bytes(int64_t total_tokens, int32_t num_seqs, int32_t chunk_size);
 
 // checksum.cu
 cudaError_t launch_checksum(const void* payload, size_t bytes, unsigned long long* out, cudaStream_t stream);

@@ -74,22 +74,6 @@ constexpr uint32_t COL_W = 256;    // W (M2), later K~^T Delta (M5)
 constexpr uint32_t COL_U = 384;    // U -> [Delta ; O]
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait, then report and stop
 
-__device__ __forceinline__ void st8(unsigned char* p, float a, float b, float c, float d) {
-  __half2 h0 = __floats2half2_rn(a, b), h1 = __floats2half2_rn(c, d);
-  uint2 u;
-  u.x = *reinterpret_cast<uint32_t*>(&h0);
-  u.y = *reinterpret_cast<uint32_t*>(&h1);
-  *reinterpret_cast<uint2*>(p) = u;
-}
-__device__ __forceinline__ void st16h(unsigned char* p, const float* v) {
-  uint32_t w[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    __half2 h = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
-    w[i] = *reinterpret_cast<uint32_t*>(&h);
-  }
-  *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
-}
 __device__ __forceinline__ void ld4bf(const unsigned char* p, float* f) {
   const uint2 u = *reinterpret_cast<const uint2*>(p);
   f[0] = __uint_as_float(u.x << 16);
@@ -100,13 +84,6 @@ __device__ __forceinline__ void ld4bf(const unsigned char* p, float* f) {
 // raw element offset: 64-channel box, 128-byte rows, 128-byte swizzle
 __device__ __forceinline__ int raw_off(int row, int cc) {
   return row * 128 + ((((cc >> 3) ^ (row & 7))) << 4) + (cc & 7) * 2;
-}
-__device__ __forceinline__ float silu_fast(float y) { return __fdividef(y, 1.0f + __expf(-y)); }
-
-__device__ __forceinline__ void sync_tc() {
-  fence_before();
-  __syncthreads();
-  fence_after();
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -656,11 +633,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---------------------------------------------------------------- host side
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+}  // namespace
 
-EncodeTiledFn encode_fn() {
+EncodeTiledFn encode_tiled_fn() {
   static EncodeTiledFn fn = nullptr;
   static std::once_flag once;
   std::call_once(once, []() {
@@ -675,8 +650,6 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-}  // namespace
-
 bool prefill_chunked_supported(const Dims& d, bool bf16, int chunk_size) {
   return bf16 && d.dk == kD && d.dv == kD && chunk_size == kC;
 }
@@ -687,7 +660,7 @@ cudaError_t launch_prefill_chunked(const Dims& d, const float* conv_w, const flo
                                    bool zero_state, bool zero_conv, const void* conv_state, float* state, void* o,
                                    int32_t* status, cudaStream_t stream) {
   if (N <= 0 || total_tokens <= 0) return cudaSuccess;
-  EncodeTiledFn enc = encode_fn();
+  EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return cudaErrorNotSupported;
   CUtensorMap tm, tmz;
   const cuuint64_t zdim[2] = {(cuuint64_t)d.Hv * kD, (cuuint64_t)total_tokens};

@@ -59,9 +59,9 @@ extern "C" GDN_API gdn_status gdn_prefill_noalloc(const gdn_config* cfg, const g
   gdn_status s = gdn_prefill_workspace_size(cfg, 0, num_seqs, chunk_size, &need);
   if (s != GDN_OK) return s;
   if (!cu_seqlens_host) return gdn_prefill_workspace_size(nullptr, 0, 0, 0, &need);  // reports the NULL argument
-  s = gdn_prefill_workspace_size(cfg, cu_seqlens_host[num_seqs] > 0 ? cu_seqlens_host[num_seqs] : 0, num_seqs,
-                                 chunk_size, &need);
-  if (s != GDN_OK) return s;
+  // the single-kernel chunked path needs only the schedule as scratch
+  need = gdn::prefill_fused_ws_bytes(cu_seqlens_host[num_seqs] > 0 ? cu_seqlens_host[num_seqs] : 0, num_seqs,
+                                     chunk_size);
   if (need > kScratchBytes) {
     char msg[256];
     snprintf(msg, sizeof(msg),
@@ -81,6 +81,6 @@ extern "C" GDN_API gdn_status gdn_prefill_noalloc(const gdn_config* cfg, const g
     gdn::set_error_message(msg);
     return GDN_E_DEVICE;
   }
-  return gdn_prefill(cfg, params, qkv, z, a, b, cu_seqlens_dev, cu_seqlens_host, num_seqs, chunk_size, flags,
-                     conv_state, state, o, ws, kScratchBytes, stream);
+  return gdn_prefill(cfg, params, qkv, z, a, b, cu_seqlens_dev, cu_seqlens_host, num_seqs, chunk_size,
+                     flags | GDN_PREFILL_FUSED, conv_state, state, o, ws, kScratchBytes, stream);
 }

@@ -1,0 +1,727 @@
+// Chunked GDN prefill as three kernels (bf16 io, d_k = d_v = 128, chunk 64):
+// the work that does not depend on the recurrent state runs over every chunk
+// at once, and only the state carry walks the chunks in order.
+//
+// The chunkwise (WY/UT) form of the gated delta rule ("fp32 Gated DeltaNet
+// recurrence", DS4Server issue #95, implementation comment).  Within a chunk
+// of rows r with gamma_r = sum_{i<=r} g_i:
+//   A_rj = beta_r e^{gamma_r - gamma_j} k_r.k_j (j < r),   T = (I + A)^-1
+//   W = T diag(beta e^gamma) K,   U = T diag(beta) V
+//   Delta = U - W S,   O = diag(e^gamma) Q S + (M o Q K^T) Delta
+//   S <- e^{gamma_C} S + K~^T Delta,   K~ = diag(e^{gamma_C - gamma}) K.
+//
+//   conv_qkv_kernel   grid (chunk, head slot): causal conv + SiLU of q/k/v
+//                     ("causal depthwise Conv1D", DS4Server issue #88, Scope),
+//                     L2 norm of q and k with epsilon inside the square root;
+//                     q^, k^ as fp16 hi + lo parts, v^ as fp16.
+//   prep_kernel       grid (chunk, value head): gates, [K;Q]K^T in split
+//                     precision on tcgen05, A and P, T = (I+A)^-1, W on tcgen05;
+//                     writes one record per (chunk, value head) whose parts are
+//                     byte images of the chain kernel's shared-memory operands.
+//   chain_kernel      grid (sequence, value head): per chunk, U = T' V^ and
+//                     [Delta; Qg S] on tcgen05, then [0;P] Delta and K~^T Delta,
+//                     then the state update; the output norm and gate of chunk c
+//                     run while the MMAs of chunk c+1 are in flight.
+//
+// Record of (chunk, value head), byte images of 128-byte-swizzled operands:
+//   [  0, 32768)  [-W ; Qg]  K-major 128 x 128   (Qg = diag(e^gamma) q^)
+//   [32768, 40960) T' = T diag(beta)     K-major 64 x 64  (rows 0..63 of [T';0])
+//   [40960, 49152) P                    K-major 64 x 64  (rows 64..127 of [0;P])
+//   [49152, 65536) K~                   MN-major K=64 x M=128
+//   [65536, 65552) e^{gamma_C}, gamma_C
+// Operands are fp16 (all bounded: normalised keys and queries, decay factors
+// <= 1), accumulation fp32, the state fp32.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "../../include/gdn.h"
+#include "internal.h"
+#include "tc.cuh"
+
+namespace gdn {
+namespace {
+
+using namespace tc;
+
+constexpr int kC = 64;
+constexpr int kD = 128;
+constexpr uint64_t kWaitNs = 2000000000ull;
+
+constexpr int kRec = 65664;
+constexpr int REC_A = 0, REC_T = 32768, REC_P = 40960, REC_K = 49152, REC_META = 65536;
+
+// ------------------------------------------------------------------ conv_qkv_kernel
+// Block = 4 warps = the 64 rows of one chunk for one 128-channel head slot
+// (q heads, then k heads, then v heads).  Warp w owns rows 16w .. 16w+15, lane
+// l owns channels 4l .. 4l+3.
+constexpr int kConvRows = 16;
+
+__global__ void __launch_bounds__(128)
+    conv_qkv_kernel(Dims d, const float* __restrict__ conv_w, const __nv_bfloat16* __restrict__ qkv,
+                    const __nv_bfloat16* __restrict__ hist, int zero_conv, const int4* __restrict__ chunk_map,
+                    __half* __restrict__ qk_hi, __half* __restrict__ qk_lo, __half* __restrict__ vh) {
+  const int4 cm = chunk_map[blockIdx.x];  // {seq, first token, length, chunk index}
+  const int slot = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r0 = kConvRows * warp;
+  const int L = cm.z;
+  if (r0 >= L) return;
+  const int nqk = 2 * d.Hk;
+  const int64_t C = d.C;
+  const int64_t c = (int64_t)slot * kD + 4 * lane;  // q heads, k heads and v heads are consecutive in qkv
+  float w[4][4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float4 x = __ldg(reinterpret_cast<const float4*>(conv_w + (c + e) * 4));
+    w[e][0] = x.x; w[e][1] = x.y; w[e][2] = x.z; w[e][3] = x.w;
+  }
+  // raw rows r0-3 .. r0+15 of the chunk; rows before the sequence start come
+  // from the conv history, rows past the chunk's end are never used
+  float x[kConvRows + 3][4];
+  const bool first = cm.w == 0;
+#pragma unroll
+  for (int i = 0; i < kConvRows + 3; ++i) {
+    const int rr = r0 - 3 + i;
+    uint2 u = make_uint2(0u, 0u);
+    if (rr < L) {
+      if (first && rr < 0) {
+        if (!zero_conv) u = *reinterpret_cast<const uint2*>(hist + ((int64_t)cm.x * 3 + (3 + rr)) * C + c);
+      } else {
+        u = __ldg(reinterpret_cast<const uint2*>(qkv + ((int64_t)cm.y + rr) * C + c));
+      }
+    }
+    x[i][0] = __uint_as_float(u.x << 16);
+    x[i][1] = __uint_as_float(u.x & 0xffff0000u);
+    x[i][2] = __uint_as_float(u.y << 16);
+    x[i][3] = __uint_as_float(u.y & 0xffff0000u);
+  }
+  float y[kConvRows][4];
+#pragma unroll
+  for (int i = 0; i < kConvRows; ++i)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float acc = 0.f;
+#pragma unroll
+      for (int tap = 0; tap < 4; ++tap) acc += w[e][tap] * x[i + tap][e];
+      y[i][e] = silu_fast(acc);
+    }
+  if (slot < nqk) {  // q or k: L2 norm over the head's 128 channels, then hi + lo fp16 parts
+    float ss[kConvRows];
+#pragma unroll
+    for (int i = 0; i < kConvRows; ++i) ss[i] = y[i][0] * y[i][0] + y[i][1] * y[i][1] + y[i][2] * y[i][2] + y[i][3] * y[i][3];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+      for (int i = 0; i < kConvRows; ++i) ss[i] += __shfl_xor_sync(0xffffffffu, ss[i], off);
+    const float scale = slot < d.Hk ? d.q_scale : 1.0f;
+    const int64_t W2 = (int64_t)nqk * kD;
+#pragma unroll
+    for (int i = 0; i < kConvRows; ++i) {
+      if (r0 + i < L) {
+        const float rs = scale * rsqrtf(ss[i] + d.l2_eps);
+        float hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float v = y[i][e] * rs;
+          hi[e] = __half2float(__float2half_rn(v));
+          lo[e] = v - hi[e];
+        }
+        const int64_t off = ((int64_t)cm.y + r0 + i) * W2 + c;
+        st8(reinterpret_cast<unsigned char*>(qk_hi + off), hi[0], hi[1], hi[2], hi[3]);
+        st8(reinterpret_cast<unsigned char*>(qk_lo + off), lo[0], lo[1], lo[2], lo[3]);
+      }
+    }
+  } else {
+    const int64_t WV = (int64_t)d.Hv * kD;
+    const int64_t cv = c - (int64_t)nqk * kD;
+#pragma unroll
+    for (int i = 0; i < kConvRows; ++i)
+      if (r0 + i < L)
+        st8(reinterpret_cast<unsigned char*>(vh + ((int64_t)cm.y + r0 + i) * WV + cv), y[i][0], y[i][1], y[i][2],
+            y[i][3]);
+  }
+}
+
+// ------------------------------------------------------------------ prep_kernel
+constexpr int kPrepThreads = 256;
+constexpr int LDS = 68;  // fp32 solve scratch row stride
+constexpr int P_KQ = 0;            // [k^ ; q^] hi  K-major 128 x 128
+constexpr int P_KQL = 32768;       // [k^ ; q^] lo; after M1 the solve scratch (A, T, Y: 3 x 64 x LDS floats)
+constexpr int P_TA = 86016;        // [T'' ; 0]   K-major 128 x 64
+constexpr int P_MISC = 102400;
+constexpr int kPrepSmem = P_MISC + 64 * 6 * 4 + 64 + 1024;
+constexpr uint32_t P_COL_D1 = 0, P_COL_W = 128, kPrepTmemCols = 256;
+
+__global__ void __launch_bounds__(kPrepThreads, 2)
+    prep_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constant__ CUtensorMap tm_lo, Dims d,
+                const float* __restrict__ A_log, const float* __restrict__ dt_bias,
+                const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
+                const int4* __restrict__ chunk_map, unsigned char* __restrict__ records, int32_t* status) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  __shared__ uint64_t mb_tma, mb_mma;
+  __shared__ uint32_t tslot;
+  bool bad = false;  // this thread saw a wait run out
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = blockIdx.x / d.Hv;
+  const int h = blockIdx.x - g * d.Hv;
+  const int kh = h / d.G;
+  const int4 cm = chunk_map[g];
+  const int64_t t0 = cm.y;
+  const int L = cm.z;
+  unsigned char* rec = records + ((int64_t)g * d.Hv + h) * kRec;
+
+  float* misc = reinterpret_cast<float*>(sm + P_MISC);
+  float* s_gam = misc;
+  float* s_beta = misc + 64;
+  float* s_eg = misc + 128;
+  float* s_ekd = misc + 192;
+  float* s_tb = misc + 256;    // beta_j        (columns of T')
+  float* s_tbg = misc + 320;   // beta_j e^{gamma_j} (columns of T'')
+  float* s_gC = misc + 384;
+  float* Am = reinterpret_cast<float*>(sm + P_KQL);
+  float* Tm = Am + 64 * LDS;
+  float* Ym = Tm + 64 * LDS;
+
+  if (tid == 0) {
+    mbar_init(&mb_tma, 1);
+    mbar_init(&mb_mma, 1);
+    mbar_init_fence();
+  }
+  if (warp == 0) tmem_alloc(&tslot, kPrepTmemCols);
+  for (int i = tid; i < 512; i += kPrepThreads)  // rows 64..127 of [T'';0] stay zero
+    reinterpret_cast<uint4*>(sm + P_TA + 8192)[i] = make_uint4(0, 0, 0, 0);
+  sync_tc();
+  const uint32_t tbase = tslot;
+  if (tid == 0) {
+    mbar_expect_tx(&mb_tma, 8 * 8192);
+    const int qx = kh * kD, kx = d.Hk * kD + kh * kD;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      tma_load_2d(sm + P_KQ + j * 16384, &tm_hi, kx + 64 * j, (int)t0, &mb_tma);
+      tma_load_2d(sm + P_KQ + j * 16384 + 8192, &tm_hi, qx + 64 * j, (int)t0, &mb_tma);
+      tma_load_2d(sm + P_KQL + j * 16384, &tm_lo, kx + 64 * j, (int)t0, &mb_tma);
+      tma_load_2d(sm + P_KQL + j * 16384 + 8192, &tm_lo, qx + 64 * j, (int)t0, &mb_tma);
+    }
+  }
+  if (warp == 0) {  // gates of rows 2 lane, 2 lane + 1; inclusive scan of g
+    const float negA = -expf(A_log[h]);
+    const float dtb = dt_bias[h];
+    float g2[2], be2[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int r = 2 * lane + e;
+      g2[e] = 0.f;
+      be2[e] = 0.f;
+      if (r < L) {
+        g2[e] = negA * softplus_f(__bfloat162float(a[(t0 + r) * d.Hv + h]) + dtb);
+        be2[e] = 1.0f / (1.0f + expf(-__bfloat162float(b[(t0 + r) * d.Hv + h])));
+      }
+    }
+    float incl = g2[0] + g2[1];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    const float gam1 = incl, gam0 = incl - g2[1];
+    const float gC = __shfl_sync(0xffffffffu, incl, 31);
+    const float gm[2] = {gam0, gam1};
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int r = 2 * lane + e;
+      const float eg = expf(gm[e]);
+      s_gam[r] = gm[e];
+      s_beta[r] = be2[e];
+      s_eg[r] = eg;
+      s_ekd[r] = expf(gC - gm[e]);
+      s_tb[r] = be2[e];
+      s_tbg[r] = be2[e] * eg;
+    }
+    if (lane == 0) {
+      *s_gC = gC;
+      reinterpret_cast<float2*>(rec + REC_META)[0] = make_float2(expf(gC), gC);
+    }
+  }
+  if (!mbar_wait(&mb_tma, 0, kWaitNs)) bad = true;
+  if (sync_tc_any(bad)) {
+    if (tid == 0) set_status(status, kStatusWaitTimeout);
+    if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
+    return;
+  }
+
+  // M1: [K;Q] K^T as hi.hi + hi.lo + lo.hi
+  if (tid == 0) {
+    const uint32_t kq = smem_u32(sm + P_KQ), kql = smem_u32(sm + P_KQL);
+    constexpr uint32_t id = idesc_f16(128, 64, false, false);
+#pragma unroll
+    for (int s = 0; s < 8; ++s) mma_f16(tbase + P_COL_D1, desc_kmaj(kq, 128, s), desc_kmaj(kq, 128, s), id, s > 0);
+#pragma unroll
+    for (int s = 0; s < 8; ++s) mma_f16(tbase + P_COL_D1, desc_kmaj(kq, 128, s), desc_kmaj(kql, 128, s), id, 1);
+#pragma unroll
+    for (int s = 0; s < 8; ++s) mma_f16(tbase + P_COL_D1, desc_kmaj(kql, 128, s), desc_kmaj(kq, 128, s), id, 1);
+    mma_commit(&mb_mma);
+  }
+  if (!mbar_wait(&mb_mma, 0, kWaitNs)) bad = true;
+  if (sync_tc_any(bad)) {
+    if (tid == 0) set_status(status, kStatusWaitTimeout);
+    if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
+    return;
+  }
+
+  // A (rows 0..63, fp32 into the solve scratch) and P (rows 64..127, fp16 into the record)
+  const int si = 32 * (warp & 3) + lane, hc = warp >> 2;
+  const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+  {
+    float v[32];
+    tmem_ld32(tbase + lane_base + P_COL_D1 + 32 * hc, v);
+    if (si < 64) {
+      const float br = s_beta[si], gr = s_gam[si];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        float a4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = 32 * hc + 4 * m + e;
+          a4[e] = (j < si) ? br * __expf(gr - s_gam[j]) * v[4 * m + e] : 0.f;
+        }
+        *reinterpret_cast<float4*>(Am + si * LDS + 32 * hc + 4 * m) = make_float4(a4[0], a4[1], a4[2], a4[3]);
+      }
+    } else {
+      const int r = si - 64;
+      const float gr = s_gam[r];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        float p[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int j = 32 * hc + 8 * m + e;
+          p[e] = (j <= r) ? __expf(gr - s_gam[j]) * v[8 * m + e] : 0.f;
+        }
+        *reinterpret_cast<uint4*>(rec + REC_P + kmaj_chunk(64, r, 32 * hc + 8 * m)) = pack8h(p);
+      }
+    }
+  }
+  __syncthreads();
+  // T = (I + A)^-1 in 16x16 blocks: diagonal blocks by right-looking forward
+  // substitution (one column per thread), then the blocks below the diagonal
+  // by distance from it.
+  if (tid < 64) {
+    const int bb = tid >> 4, c16 = tid & 15;
+    const float* Ab = Am + (16 * bb) * LDS + 16 * bb;
+    float acc[16], t[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      t[k] = (k < c16) ? 0.f : (k == c16 ? 1.f : -acc[k]);
+#pragma unroll
+      for (int i = k + 1; i < 16; ++i) acc[i] += Ab[i * LDS + k] * t[k];
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) Tm[(16 * bb + i) * LDS + 16 * bb + c16] = t[i];
+  }
+  __syncthreads();
+  for (int e = tid; e < 6 * 64; e += kPrepThreads) {  // At_ij = T_ii A_ij below the diagonal
+    const int pr = e >> 6, p = (e >> 2) & 15, q = 4 * (e & 3);
+    const int bi = pr == 0 ? 1 : (pr < 3 ? 2 : 3), bj = pr == 0 ? 0 : (pr < 3 ? pr - 1 : pr - 3);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      const float t = Tm[(16 * bi + p) * LDS + 16 * bi + kk];
+      const float4 a4 = *reinterpret_cast<const float4*>(Am + (16 * bi + kk) * LDS + 16 * bj + q);
+      acc.x += t * a4.x; acc.y += t * a4.y; acc.z += t * a4.z; acc.w += t * a4.w;
+    }
+    *reinterpret_cast<float4*>(Ym + (16 * bi + p) * LDS + 16 * bj + q) = acc;
+  }
+  __syncthreads();
+  for (int dl = 1; dl < 4; ++dl) {  // T_ij = -sum_{k=j}^{i-1} At_ik T_kj
+    for (int e = tid; e < (4 - dl) * 64; e += kPrepThreads) {
+      const int bj = e >> 6, bi = bj + dl, p = (e >> 2) & 15, q = 4 * (e & 3);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int bk = bj; bk < bi; ++bk) {
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+          const float y = Ym[(16 * bi + p) * LDS + 16 * bk + kk];
+          const float4 t4 = *reinterpret_cast<const float4*>(Tm + (16 * bk + kk) * LDS + 16 * bj + q);
+          acc.x += y * t4.x; acc.y += y * t4.y; acc.z += y * t4.z; acc.w += y * t4.w;
+        }
+      }
+      *reinterpret_cast<float4*>(Tm + (16 * bi + p) * LDS + 16 * bj + q) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+    }
+    __syncthreads();
+  }
+  {  // T' = T diag(beta) -> record; T'' = T diag(beta e^gamma) -> rows 0..63 of [T'';0]
+    const int r = tid >> 2, j0 = 16 * (tid & 3);
+    float tv[16], t1[16], t2[16];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const float4 t4 = *reinterpret_cast<const float4*>(Tm + r * LDS + j0 + 4 * m);
+      tv[4 * m] = t4.x; tv[4 * m + 1] = t4.y; tv[4 * m + 2] = t4.z; tv[4 * m + 3] = t4.w;
+    }
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) {
+      const float t = (j0 + jj <= r) ? tv[jj] : 0.f;
+      t1[jj] = t * s_tb[j0 + jj];
+      t2[jj] = t * s_tbg[j0 + jj];
+    }
+    *reinterpret_cast<uint4*>(rec + REC_T + kmaj_chunk(64, r, j0)) = pack8h(t1);
+    *reinterpret_cast<uint4*>(rec + REC_T + kmaj_chunk(64, r, j0 + 8)) = pack8h(t1 + 8);
+    st16h(sm + P_TA + kmaj_chunk(128, r, j0), t2);
+    st16h(sm + P_TA + kmaj_chunk(128, r, j0 + 8), t2 + 8);
+  }
+  fence_async_smem();
+  sync_tc();
+
+  // M2: W = [T'';0] K  (B = the k^ rows of the hi tile read as MN-major: K = 64 rows, N = 128 channels)
+  if (tid == 0) {
+    const uint32_t ta = smem_u32(sm + P_TA), kq = smem_u32(sm + P_KQ);
+    constexpr uint32_t id = idesc_f16(128, 128, false, true);
+#pragma unroll
+    for (int s = 0; s < 4; ++s)
+      mma_f16(tbase + P_COL_W, desc_kmaj(ta, 128, s), sdesc(kq + s * 2048, 16384, 1024), id, s > 0);
+    mma_commit(&mb_mma);
+  }
+  // while W is computed: Qg = diag(e^gamma) q^ -> rows 64..127 of the [-W;Qg] image, K~ -> its image
+  for (int e = tid; e < 64 * 16; e += kPrepThreads) {
+    const int r = e >> 4, c8 = 8 * (e & 15);
+    const uint4 uq = *reinterpret_cast<const uint4*>(sm + P_KQ + kmaj_chunk(128, 64 + r, c8));
+    const uint4 uk = *reinterpret_cast<const uint4*>(sm + P_KQ + kmaj_chunk(128, r, c8));
+    const float eg = s_eg[r], ek = s_ekd[r];
+    const __half2* hq = reinterpret_cast<const __half2*>(&uq);
+    const __half2* hk = reinterpret_cast<const __half2*>(&uk);
+    float fq[8], fk[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 a2 = __half22float2(hq[i]), b2 = __half22float2(hk[i]);
+      fq[2 * i] = a2.x * eg;
+      fq[2 * i + 1] = a2.y * eg;
+      fk[2 * i] = b2.x * ek;
+      fk[2 * i + 1] = b2.y * ek;
+    }
+    *reinterpret_cast<uint4*>(rec + REC_A + kmaj_chunk(128, 64 + r, c8)) = pack8h(fq);
+    *reinterpret_cast<uint4*>(rec + REC_K + mnmaj_chunk(64, r, c8)) = pack8h(fk);
+  }
+  if (!mbar_wait(&mb_mma, 1, kWaitNs)) bad = true;
+  fence_after();
+  if (si < 64) {  // -W -> rows 0..63 of the [-W;Qg] image
+    float v[32];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      tmem_ld32(tbase + lane_base + P_COL_W + 64 * hc + 32 * hh, v);
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) v[jj] = -v[jj];
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        *reinterpret_cast<uint4*>(rec + REC_A + kmaj_chunk(128, si, 64 * hc + 32 * hh + 8 * m)) = pack8h(v + 8 * m);
+    }
+  }
+  if (sync_tc_any(bad) && tid == 0) set_status(status, kStatusWaitTimeout);
+  if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
+}
+
+// ------------------------------------------------------------------ chain_kernel
+constexpr int kChainThreads = 256;
+constexpr int C_A = 0;          // [-W ; Qg]   K-major 128 x 128
+constexpr int C_TA = 32768;     // [T' ; 0]    K-major 128 x 64
+constexpr int C_V = 49152;      // v^          MN-major K=64 x N=128
+constexpr int C_PA = 65536;     // [0 ; P]     K-major 128 x 64
+constexpr int C_KT = 81920;     // K~          MN-major K=64 x M=128
+constexpr int C_DB = 98304;     // Delta       MN-major K=64 x N=128
+constexpr int C_SB = 114688;    // S (fp16)    MN-major K=128 x N=128
+constexpr int C_Z = 147456;     // z           two 64-column boxes, 64 rows
+constexpr int C_MISC = 163840;  // 1 + norm_w [128], row sums of squares [2][64], meta [2][4]
+constexpr int kChainSmem = C_MISC + (128 + 128 + 8) * 4 + 1024;
+constexpr uint32_t COL_S = 0, COL_U0 = 128, COL_Y = 384, kChainTmemCols = 512;
+
+__global__ void __launch_bounds__(kChainThreads, 1)
+    chain_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_z, Dims d,
+                 const float* __restrict__ norm_w, const unsigned char* __restrict__ records,
+                 const int32_t* __restrict__ chunk_off, const int32_t* __restrict__ order,
+                 const int32_t* __restrict__ cu, int zero_state, float* __restrict__ state,
+                 __nv_bfloat16* __restrict__ o, int32_t* status) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  __shared__ uint64_t mb_ld0, mb_ld1, mb_z, mb_mma;
+  __shared__ uint32_t tslot;
+  bool bad = false;  // this thread saw a wait run out
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = blockIdx.x % d.Hv;
+  const int oi = blockIdx.x / d.Hv;
+  const int n = order ? order[oi] : oi;
+  const int64_t seq0 = cu[n];
+  const int len = cu[n + 1] - cu[n];
+  if (len <= 0) return;
+  const int nchunks = (len + kC - 1) / kC;
+  const int64_t g0 = chunk_off[n];
+  const int64_t HvD = (int64_t)d.Hv * kD;
+
+  float* s_nw = reinterpret_cast<float*>(sm + C_MISC);
+  float* s_rms = s_nw + 128;      // [2][64]
+  float* s_meta = s_rms + 128;    // [2][4]: e^{gamma_C}, gamma_C of chunks with parity 0 / 1
+
+  if (tid == 0) {
+    mbar_init(&mb_ld0, 1);
+    mbar_init(&mb_ld1, 1);
+    mbar_init(&mb_z, 1);
+    mbar_init(&mb_mma, 1);
+    mbar_init_fence();
+  }
+  if (warp == 0) tmem_alloc(&tslot, kChainTmemCols);
+  for (int i = tid; i < 512; i += kChainThreads) {  // constant zero halves of [T';0] and [0;P]
+    reinterpret_cast<uint4*>(sm + C_TA + 8192)[i] = make_uint4(0, 0, 0, 0);
+    reinterpret_cast<uint4*>(sm + C_PA)[i] = make_uint4(0, 0, 0, 0);
+  }
+  if (tid < kD) s_nw[tid] = 1.0f + norm_w[tid];
+  // state S (fp32 in TMEM): thread owns row si (d_k index), columns [64 hc, 64 hc + 64)
+  const int si = 32 * (warp & 3) + lane, hc = warp >> 2;
+  const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+  float* gst = state + ((int64_t)n * d.Hv + h) * kD * kD;  // stored [j][i]
+  sync_tc();
+  const uint32_t tbase = tslot;
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    float S[32];
+#pragma unroll
+    for (int jj = 0; jj < 32; ++jj) S[jj] = zero_state ? 0.f : gst[(int64_t)(64 * hc + 32 * hh + jj) * kD + si];
+    tmem_st32(tbase + lane_base + COL_S + 64 * hc + 32 * hh, S);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) st16h(sm + C_SB + mnmaj_chunk(kD, si, 64 * hc + 32 * hh + 8 * m), S + 8 * m);
+  }
+  fence_async_smem();
+  sync_tc();
+
+  auto rec_of = [&](int cc) { return records + ((g0 + cc) * d.Hv + h) * (int64_t)kRec; };
+  // loads of chunk cc: group 0 = [-W;Qg], T', v^ (read by the first MMA group);
+  // group 1 = P, K~ and the chunk's decay (read by the second)
+  auto issue_ld0 = [&](int cc) {
+    const unsigned char* r = rec_of(cc);
+    mbar_expect_tx(&mb_ld0, 32768 + 8192 + 2 * 8192);
+    bulk_load(sm + C_A, r + REC_A, 32768, &mb_ld0);
+    bulk_load(sm + C_TA, r + REC_T, 8192, &mb_ld0);
+    const int ty = (int)(seq0 + (int64_t)cc * kC);
+    tma_load_2d(sm + C_V, &tm_v, h * kD, ty, &mb_ld0);
+    tma_load_2d(sm + C_V + 8192, &tm_v, h * kD + 64, ty, &mb_ld0);
+  };
+  auto issue_ld1 = [&](int cc) {
+    const unsigned char* r = rec_of(cc);
+    mbar_expect_tx(&mb_ld1, 8192 + 16384 + 16);
+    bulk_load(sm + C_PA + 8192, r + REC_P, 8192, &mb_ld1);
+    bulk_load(sm + C_KT, r + REC_K, 16384, &mb_ld1);
+    bulk_load(s_meta + 4 * (cc & 1), r + REC_META, 16, &mb_ld1);
+  };
+  if (tid == 0) {
+    issue_ld0(0);
+    issue_ld1(0);
+  }
+
+  // output rows of chunk cc (O in lanes 64..127 of its U buffer): zero-centred
+  // RMSNorm over d_v times sigmoid(z), bf16 out.  Warps 2, 3, 6, 7 only.
+  auto epilogue = [&](int cc) {
+    const int r = si - 64;
+    const uint32_t col = COL_U0 + 128 * (cc & 1) + 64 * hc;
+    float v[64];
+    tmem_ld32(tbase + lane_base + col, v);
+    tmem_ld32(tbase + lane_base + col + 32, v + 32);
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < 64; ++j) ss += v[j] * v[j];
+    s_rms[64 * hc + r] = ss;
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    const int Lc = min(kC, len - cc * kC);
+    if (r < Lc) {
+      const float rinv = rsqrtf((s_rms[r] + s_rms[64 + r]) * (1.0f / kD) + d.norm_eps);
+      const unsigned char* zrow = sm + C_Z + hc * 8192 + r * 128;
+      __nv_bfloat16* orow = o + (seq0 + (int64_t)cc * kC + r) * HvD + (int64_t)h * kD + 64 * hc;
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const uint4 zr = *reinterpret_cast<const uint4*>(zrow + ((m ^ (r & 7)) << 4));
+        const uint32_t zw[4] = {zr.x, zr.y, zr.z, zr.w};
+        uint32_t ow[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = 8 * m + 2 * e;
+          const float z0 = __uint_as_float(zw[e] << 16), z1 = __uint_as_float(zw[e] & 0xffff0000u);
+          const float o0 = v[j] * rinv * s_nw[64 * hc + j] * __fdividef(1.0f, 1.0f + __expf(-z0));
+          const float o1 = v[j + 1] * rinv * s_nw[64 * hc + j + 1] * __fdividef(1.0f, 1.0f + __expf(-z1));
+          __nv_bfloat162 pr = __floats2bfloat162_rn(o0, o1);
+          ow[e] = *reinterpret_cast<uint32_t*>(&pr);
+        }
+        *reinterpret_cast<uint4*>(orow + 8 * m) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+      }
+    }
+  };
+  const bool out_warp = (warp & 3) >= 2;
+
+  uint32_t ph0 = 0, ph1 = 0, phz = 0, phm = 0;
+  for (int c = 0; c < nchunks; ++c) {
+    const uint32_t colU = COL_U0 + 128 * (c & 1);
+    if (!mbar_wait(&mb_ld0, ph0, kWaitNs)) bad = true;
+    ph0 ^= 1;
+    // U = [T';0] v^ ; U += [-W;Qg] S  ->  [Delta ; Qg S]
+    if (tid == 0 && !bad) {
+      const uint32_t ta = smem_u32(sm + C_TA), vb = smem_u32(sm + C_V), aa = smem_u32(sm + C_A),
+                     sb = smem_u32(sm + C_SB);
+      constexpr uint32_t id = idesc_f16(128, 128, false, true);
+#pragma unroll
+      for (int s = 0; s < 4; ++s) mma_f16(tbase + colU, desc_kmaj(ta, 128, s), desc_mnmaj(vb, kC, s), id, s > 0);
+#pragma unroll
+      for (int s = 0; s < 8; ++s) mma_f16(tbase + colU, desc_kmaj(aa, 128, s), desc_mnmaj(sb, kD, s), id, 1);
+      mma_commit(&mb_mma);
+    }
+    if (c > 0 && out_warp) {
+      if (!mbar_wait(&mb_z, phz, kWaitNs)) bad = true;
+      epilogue(c - 1);
+    }
+    if (c > 0) phz ^= 1;
+    if (!mbar_wait(&mb_mma, phm, kWaitNs)) bad = true;
+    phm ^= 1;
+    fence_after();
+    if (tid == 0 && c + 1 < nchunks) issue_ld0(c + 1);
+    if (si < 64) {  // Delta -> shared (MN-major B operand)
+      float v[32];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        tmem_ld32(tbase + lane_base + colU + 64 * hc + 32 * hh, v);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) st16h(sm + C_DB + mnmaj_chunk(kC, si, 64 * hc + 32 * hh + 8 * m), v + 8 * m);
+      }
+    }
+    fence_async_smem();
+    if (sync_tc_any(bad)) break;
+    if (tid == 0) {  // z rows of this chunk; the previous chunk's output is done with the z tile
+      mbar_expect_tx(&mb_z, 2 * 8192);
+      const int ty = (int)(seq0 + (int64_t)c * kC);
+      tma_load_2d(sm + C_Z, &tm_z, h * kD, ty, &mb_z);
+      tma_load_2d(sm + C_Z + 8192, &tm_z, h * kD + 64, ty, &mb_z);
+    }
+    if (!mbar_wait(&mb_ld1, ph1, kWaitNs)) bad = true;
+    ph1 ^= 1;
+    // O += [0;P] Delta ;  Y = K~^T Delta
+    if (tid == 0 && !bad) {
+      const uint32_t pa = smem_u32(sm + C_PA), db = smem_u32(sm + C_DB), kt = smem_u32(sm + C_KT);
+      constexpr uint32_t id4 = idesc_f16(128, 128, false, true);
+      constexpr uint32_t id5 = idesc_f16(128, 128, true, true);
+#pragma unroll
+      for (int s = 0; s < 4; ++s) mma_f16(tbase + colU, desc_kmaj(pa, 128, s), desc_mnmaj(db, kC, s), id4, 1);
+#pragma unroll
+      for (int s = 0; s < 4; ++s) mma_f16(tbase + COL_Y, desc_mnmaj(kt, kC, s), desc_mnmaj(db, kC, s), id5, s > 0);
+      mma_commit(&mb_mma);
+    }
+    const float egC = s_meta[4 * (c & 1)];
+    if (!mbar_wait(&mb_mma, phm, kWaitNs)) bad = true;
+    phm ^= 1;
+    fence_after();
+    if (tid == 0 && c + 1 < nchunks) issue_ld1(c + 1);
+    {  // S = e^{gamma_C} S + K~^T Delta, and its fp16 copy for the next chunk
+      float v[32], S[32];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        tmem_ld32(tbase + lane_base + COL_Y + 64 * hc + 32 * hh, v);
+        tmem_ld32(tbase + lane_base + COL_S + 64 * hc + 32 * hh, S);
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) S[jj] = egC * S[jj] + v[jj];
+        tmem_st32(tbase + lane_base + COL_S + 64 * hc + 32 * hh, S);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) st16h(sm + C_SB + mnmaj_chunk(kD, si, 64 * hc + 32 * hh + 8 * m), S + 8 * m);
+      }
+    }
+    fence_async_smem();
+    if (sync_tc_any(bad)) break;
+  }
+  // block-uniform: either every output warp reaches the epilogue's named barrier or none does
+  if (!sync_tc_any(bad) && out_warp) {
+    if (!mbar_wait(&mb_z, phz, kWaitNs)) bad = true;
+    epilogue(nchunks - 1);
+  }
+  if (sync_tc_any(bad)) {
+    if (tid == 0) set_status(status, kStatusWaitTimeout);
+  } else {
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      float S[32];
+      tmem_ld32(tbase + lane_base + COL_S + 64 * hc + 32 * hh, S);
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) gst[(int64_t)(64 * hc + 32 * hh + jj) * kD + si] = S[jj];
+    }
+  }
+  sync_tc();
+  if (warp == 0) tmem_dealloc(tbase, kChainTmemCols);
+}
+
+bool encode_2d(EncodeTiledFn enc, CUtensorMap* tm, CUtensorMapDataType dt, const void* base, uint64_t cols,
+               uint64_t rows) {
+  const cuuint64_t dim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t stride[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {64, 64};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(tm, dt, 2, const_cast<void*>(base), dim, stride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+}  // namespace
+
+SplitLayout split_layout(const Dims& d, int64_t total_tokens, int64_t chunk_bound) {
+  SplitLayout S;
+  const size_t qkw = (size_t)2 * d.Hk * kD, vw = (size_t)d.Hv * kD;
+  S.qk_hi = 0;
+  S.qk_lo = al256(S.qk_hi + (size_t)total_tokens * qkw * 2);
+  S.v = al256(S.qk_lo + (size_t)total_tokens * qkw * 2);
+  S.records = al256(S.v + (size_t)total_tokens * vw * 2);
+  S.total_bytes = al256(S.records + (size_t)chunk_bound * d.Hv * kRec);
+  return S;
+}
+
+cudaError_t launch_prefill_split(const Dims& d, const float* conv_w, const float* A_log, const float* dt_bias,
+                                 const float* norm_w, const void* qkv, const void* z, const void* a, const void* b,
+                                 const int32_t* cu, const int32_t* order, const int32_t* chunk_off,
+                                 const int4* chunk_map, int32_t N, int64_t total_tokens, int64_t total_chunks,
+                                 bool zero_state, bool zero_conv, const void* conv_state, float* state, void* o,
+                                 void* split_ws, int32_t* status, cudaStream_t stream) {
+  if (N <= 0 || total_tokens <= 0 || total_chunks <= 0) return cudaSuccess;
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const SplitLayout S = split_layout(d, total_tokens, total_chunks);
+  unsigned char* ws = (unsigned char*)split_ws;
+  __half* qk_hi = (__half*)(ws + S.qk_hi);
+  __half* qk_lo = (__half*)(ws + S.qk_lo);
+  __half* vh = (__half*)(ws + S.v);
+  unsigned char* records = ws + S.records;
+  CUtensorMap tm_hi, tm_lo, tm_v, tm_z;
+  const uint64_t qkw = (uint64_t)2 * d.Hk * kD, vw = (uint64_t)d.Hv * kD;
+  if (!encode_2d(enc, &tm_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, qk_hi, qkw, total_tokens) ||
+      !encode_2d(enc, &tm_lo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, qk_lo, qkw, total_tokens) ||
+      !encode_2d(enc, &tm_v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, vh, vw, total_tokens) ||
+      !encode_2d(enc, &tm_z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, z, vw, total_tokens))
+    return cudaErrorInvalidValue;
+  cudaError_t e;
+  {
+    LaunchScope scope(GDN_K_SPLIT_CONV, stream);
+    conv_qkv_kernel<<<dim3((unsigned)total_chunks, (unsigned)(2 * d.Hk + d.Hv)), 128, 0, stream>>>(
+        d, conv_w, (const __nv_bfloat16*)qkv, (const __nv_bfloat16*)conv_state, zero_conv ? 1 : 0, chunk_map, qk_hi,
+        qk_lo, vh);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if ((e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrepSmem)) != cudaSuccess)
+    return e;
+  {
+    LaunchScope scope(GDN_K_SPLIT_PREP, stream);
+    prep_kernel<<<(unsigned)(total_chunks * d.Hv), kPrepThreads, kPrepSmem, stream>>>(
+        tm_hi, tm_lo, d, A_log, dt_bias, (const __nv_bfloat16*)a, (const __nv_bfloat16*)b, chunk_map, records, status);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if ((e = cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kChainSmem)) != cudaSuccess)
+    return e;
+  LaunchScope scope(GDN_K_SPLIT_CHAIN, stream);
+  chain_kernel<<<(unsigned)((int64_t)N * d.Hv), kChainThreads, kChainSmem, stream>>>(
+      tm_v, tm_z, d, norm_w, records, chunk_off, order, cu, zero_state ? 1 : 0, state, (__nv_bfloat16*)o, status);
+  return cudaGetLastError();
+}
+
+}  // namespace gdn

@@ -180,5 +180,43 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
+// ---------------------------------------------------------------- operand packing
+// four / eight fp32 values -> fp16, one 8- / 16-byte store
+__device__ __forceinline__ void st8(unsigned char* p, float a, float b, float c, float d) {
+  __half2 h0 = __floats2half2_rn(a, b), h1 = __floats2half2_rn(c, d);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&h0);
+  u.y = *reinterpret_cast<uint32_t*>(&h1);
+  *reinterpret_cast<uint2*>(p) = u;
+}
+__device__ __forceinline__ uint4 pack8h(const float* v) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __half2 h = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+    w[i] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+__device__ __forceinline__ void st16h(unsigned char* p, const float* v) { *reinterpret_cast<uint4*>(p) = pack8h(v); }
+
+// SiLU(y) = y / (1 + e^-y) with the fast exponential and division
+__device__ __forceinline__ float silu_fast(float y) { return __fdividef(y, 1.0f + __expf(-y)); }
+
+// block barrier that orders tcgen05 operations before / after it
+__device__ __forceinline__ void sync_tc() {
+  fence_before();
+  __syncthreads();
+  fence_after();
+}
+// the same barrier, returning whether any thread of the block passed `pred` true
+// (a block-uniform decision, taken in the barrier itself)
+__device__ __forceinline__ bool sync_tc_any(bool pred) {
+  fence_before();
+  const int r = __syncthreads_or(pred ? 1 : 0);
+  fence_after();
+  return r != 0;
+}
+
 }  // namespace tc
 }  // namespace gdn

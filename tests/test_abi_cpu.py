@@ -64,8 +64,14 @@ def test_bad_config_rejected(kw, status):
 def test_workspace_size_and_bad_chunk():
     cfg = qwen_cfg()
     small = gdn.prefill_workspace_size(cfg, 4096, 1, 64)
-    big = gdn.prefill_workspace_size(cfg, 65536, 16, 16)
+    big = gdn.prefill_workspace_size(cfg, 65536, 16, 64)
     assert 0 < small < big
+    # chunk 64 on bf16 d=128 holds the chunked form's intermediates: per token
+    # q^, k^ (two fp16 parts) and v^, per (chunk, value head) a 65,664-byte record
+    per_token = (2 * 2 * 16 * 128 + 48 * 128) * 2
+    assert small >= 4096 * per_token + 64 * 48 * 65664
+    sched_only = gdn.prefill_workspace_size(cfg, 65536, 16, 16)  # token-recurrent path: the schedule alone
+    assert 0 < sched_only < (1 << 20)
     with pytest.raises(gdn.GdnError) as e:
         gdn.prefill_workspace_size(cfg, 4096, 1, 48)
     assert e.value.name == "GDN_E_INVAL"

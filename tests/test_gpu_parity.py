@@ -20,6 +20,7 @@ from gpu_common import (TOL_F32, TOL_O_BF16, TOL_S_BF16, U_BF16, U_F32, compare_
 pytestmark = pytest.mark.gpu
 
 RECURRENT = gdn.PREFILL_RECURRENT
+FUSED = gdn.PREFILL_FUSED
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -193,7 +194,7 @@ def test_conv_prefill_and_step(io):
 def test_prefill_t4096_matches_oracle():
     inp = gi.workload_inputs("prefill_t4096")
     o_ref, st_ref, hist_ref = oracle.prefill_inputs(inp)
-    for flags in (0, RECURRENT):
+    for flags in (0, FUSED, RECURRENT):
         _, o, st, hist = run_gpu_prefill(inp, 64, flags | gdn.ZERO_INIT_STATE)
         eo, es = compare_prefill(inp, o, st, o_ref, st_ref, TOL_O_BF16, TOL_S_BF16)
         print(f"prefill T=4096 flags={flags}: o max-rel {eo:.2e}, state max-rel {es:.2e}")
@@ -394,26 +395,47 @@ def test_launch_count_and_profiler():
 # ------------------------------------------------------------------ chunked tensor-core prefill
 
 
+@pytest.mark.parametrize("flags", [0, FUSED])
 @pytest.mark.parametrize("zero_init", [True, False])
-def test_chunked_partial_chunks_match_oracle(zero_init):
+def test_chunked_partial_chunks_match_oracle(zero_init, flags):
     # lengths around chunk boundaries (64): partial first/last chunks, exact multiples, short sequences
     geo = gi.Geometry(num_k_heads=2, num_v_heads=6, head_k_dim=128, head_v_dim=128)
     lengths = [1, 63, 64, 65, 127, 128, 129, 200, 2, 3]
     inp = gi.make_prefill_inputs(geo, lengths, seed=31, zero_init=zero_init)
     o_ref, st_ref, hist_ref = oracle.prefill_inputs(inp)
-    _, o, st, hist = run_gpu_prefill(inp, 64)
+    _, o, st, hist = run_gpu_prefill(inp, 64, flags)
     eo, es = compare_prefill(inp, o, st, o_ref, st_ref, TOL_O_BF16, TOL_S_BF16)
-    print(f"chunked partial chunks: o {eo:.2e} state {es:.2e}")
+    print(f"chunked partial chunks (flags {flags}): o {eo:.2e} state {es:.2e}")
     assert np.array_equal(hist, ref_hist_bits(inp, hist_ref))
 
 
-def test_chunked_matches_recurrent_kernel():
+@pytest.mark.parametrize("flags", [0, FUSED])
+def test_chunked_matches_recurrent_kernel(flags):
     geo = gi.Geometry(num_k_heads=4, num_v_heads=12, head_k_dim=128, head_v_dim=128)
     inp = gi.make_prefill_inputs(geo, [300, 64, 1, 517], seed=32, zero_init=False)
-    _, o1, st1, h1 = run_gpu_prefill(inp, 64)
+    _, o1, st1, h1 = run_gpu_prefill(inp, 64, flags)
     _, o2, st2, h2 = run_gpu_prefill(inp, 64, RECURRENT)
     for n in range(inp.num_seqs):
         sl = slice(inp.cu_seqlens[n], inp.cu_seqlens[n + 1])
         assert maxrel(o1[sl], o2[sl], 2 * U_BF16) <= TOL_O_BF16
         assert maxrel(st1[n], st2[n]) <= TOL_S_BF16
     assert np.array_equal(h1, h2)
+
+
+def test_split_path_workspace_and_fused_workspace():
+    """The three-kernel path needs its intermediates; GDN_PREFILL_FUSED runs
+    with the schedule alone and rejects nothing that fits it."""
+    geo = gi.Geometry(num_k_heads=2, num_v_heads=6, head_k_dim=128, head_v_dim=128)
+    inp = gi.make_prefill_inputs(geo, [130, 70], seed=33, zero_init=False)
+    dp = DeviceProblem(inp, 64)
+    full = gdn.prefill_workspace_size(dp.cfg, inp.total_tokens, inp.num_seqs, 64)
+    assert full > 4 * 65664 * geo.num_v_heads  # records of at least four chunks
+    small = torch.empty(8192, dtype=torch.uint8, device="cuda")
+    with pytest.raises(gdn.GdnError) as e:
+        gdn.prefill(dp.cfg, dp.params, dp.qkv, dp.z, dp.a, dp.b, dp.cu_dev, dp.cu_host, 64, 0, dp.conv_state,
+                    dp.state, dp.o, small)
+    assert e.value.name == "GDN_E_WORKSPACE"
+    gdn.prefill(dp.cfg, dp.params, dp.qkv, dp.z, dp.a, dp.b, dp.cu_dev, dp.cu_host, 64, FUSED, dp.conv_state,
+                dp.state, dp.o, small)
+    torch.cuda.synchronize()
+    assert gdn.device_status() == 0

@@ -74,7 +74,7 @@ EncodeTiledFn encode_tiled_fn();
 // prefill_split.cu (tcgen05; bf16 io, d_k = d_v = 128, chunk 64): conv, per-chunk prep and
 // state chain as three kernels over a workspace of intermediates (after the schedule)
 struct SplitLayout {
-  size_t qk_hi, qk_lo, v, records, total_bytes;
+  size_t qk_hi, qk_lo, records, total_bytes;
 };
 SplitLayout split_layout(const Dims& d, int64_t total_tokens, int64_t chunk_bound);
 cudaError_t launch_prefill_split(const Dims& d, const float* conv_w, const float* A_log, const float* dt_bias,

@@ -13,22 +13,28 @@
 //   conv_qkv_kernel   grid (chunk, head slot): causal conv + SiLU of q/k/v
 //                     ("causal depthwise Conv1D", DS4Server issue #88, Scope),
 //                     L2 norm of q and k with epsilon inside the square root;
-//                     q^, k^ as fp16 hi + lo parts, v^ as fp16.
+//                     q^, k^ as fp16 hi + lo parts, v^ as fp16; and the output
+//                     gate (1 + w) sigmoid(z) of every value head, fp16.
 //   prep_kernel       grid (chunk, value head): gates, [K;Q]K^T in split
 //                     precision on tcgen05, A and P, T = (I+A)^-1, W on tcgen05;
 //                     writes one record per (chunk, value head) whose parts are
 //                     byte images of the chain kernel's shared-memory operands.
 //   chain_kernel      grid (sequence, value head): per chunk, U = T' V^ and
 //                     [Delta; Qg S] on tcgen05, then [0;P] Delta and K~^T Delta,
-//                     then the state update; the output norm and gate of chunk c
-//                     run while the MMAs of chunk c+1 are in flight.
+//                     then the state update; the output rows of chunk c (RMSNorm
+//                     times the gate) are written by half of the warps while the
+//                     other half carries chunk c+1 to its second MMA group.
 //
 // Record of (chunk, value head), byte images of 128-byte-swizzled operands:
 //   [  0, 32768)  [-W ; Qg]  K-major 128 x 128   (Qg = diag(e^gamma) q^)
 //   [32768, 40960) T' = T diag(beta)     K-major 64 x 64  (rows 0..63 of [T';0])
-//   [40960, 49152) P                    K-major 64 x 64  (rows 64..127 of [0;P])
-//   [49152, 65536) K~                   MN-major K=64 x M=128
-//   [65536, 65552) e^{gamma_C}, gamma_C
+//   [40960, 57344) v^ (from the conv)   MN-major K=64 x N=128, rows past the chunk zero
+//   [57344, 65536) P                    K-major 64 x 64  (rows 64..127 of [0;P])
+//   [65536, 81920) K~                   MN-major K=64 x M=128
+//   [81920, 98304) output gate (1 + w) sigmoid(z) (from the conv), fp16, row r at 256 r,
+//                  column half at +128, 16-byte piece q at (q ^ (r % 8)) * 16
+//   [98304, 98320) e^{gamma_C}, gamma_C
+// so the chain kernel reads each chunk in four bulk copies.
 // Operands are fp16 (all bounded: normalised keys and queries, decay factors
 // <= 1), accumulation fp32, the state fp32.
 #include <cuda.h>
@@ -48,8 +54,8 @@ constexpr int kC = 64;
 constexpr int kD = 128;
 constexpr uint64_t kWaitNs = 2000000000ull;
 
-constexpr int kRec = 65664;
-constexpr int REC_A = 0, REC_T = 32768, REC_P = 40960, REC_K = 49152, REC_META = 65536;
+constexpr int kRec = 98432;
+constexpr int REC_A = 0, REC_T = 32768, REC_V = 40960, REC_P = 57344, REC_K = 65536, REC_G = 81920, REC_META = 98304;
 
 // ------------------------------------------------------------------ conv_qkv_kernel
 // Block = 4 warps = the 64 rows of one chunk for one 128-channel head slot
@@ -57,17 +63,60 @@ constexpr int REC_A = 0, REC_T = 32768, REC_P = 40960, REC_K = 49152, REC_META =
 // l owns channels 4l .. 4l+3.
 constexpr int kConvRows = 16;
 
+// Slots past the q/k/v heads compute the output gate of one value head,
+// (1 + w_j) sigmoid(z_j), which depends on no other stage of the mixer.
+__device__ __forceinline__ void gate_rows(const Dims& d, const float* __restrict__ norm_w,
+                                          const __nv_bfloat16* __restrict__ z, unsigned char* __restrict__ grec,
+                                          int64_t t0, int r0, int L, int hz, int lane) {
+  const int64_t WV = (int64_t)d.Hv * kD;
+  const int hcol = lane >> 4, q = (lane >> 1) & 7;  // channels 4 lane .. 4 lane + 3: column half, 16-byte piece
+  const int64_t col = (int64_t)hz * kD + 4 * lane;
+  const float4 w = __ldg(reinterpret_cast<const float4*>(norm_w + 4 * lane));
+  const float nw[4] = {1.0f + w.x, 1.0f + w.y, 1.0f + w.z, 1.0f + w.w};
+  uint2 u[kConvRows];
+#pragma unroll
+  for (int i = 0; i < kConvRows; ++i)
+    u[i] = (r0 + i < L) ? __ldg(reinterpret_cast<const uint2*>(z + (t0 + r0 + i) * WV + col)) : make_uint2(0u, 0u);
+#pragma unroll
+  for (int i = 0; i < kConvRows; ++i) {
+    if (r0 + i < L) {
+      const float zz[4] = {__uint_as_float(u[i].x << 16), __uint_as_float(u[i].x & 0xffff0000u),
+                           __uint_as_float(u[i].y << 16), __uint_as_float(u[i].y & 0xffff0000u)};
+      float g[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) g[e] = nw[e] * __fdividef(1.0f, 1.0f + __expf(-zz[e]));
+      const int r = r0 + i;
+      st8(grec + r * 256 + hcol * 128 + ((q ^ (r & 7)) << 4) + (lane & 1) * 8, g[0], g[1], g[2], g[3]);
+    }
+  }
+}
+
 __global__ void __launch_bounds__(128)
     conv_qkv_kernel(Dims d, const float* __restrict__ conv_w, const __nv_bfloat16* __restrict__ qkv,
                     const __nv_bfloat16* __restrict__ hist, int zero_conv, const int4* __restrict__ chunk_map,
-                    __half* __restrict__ qk_hi, __half* __restrict__ qk_lo, __half* __restrict__ vh) {
-  const int4 cm = chunk_map[blockIdx.x];  // {seq, first token, length, chunk index}
+                    const float* __restrict__ norm_w, const __nv_bfloat16* __restrict__ z,
+                    __half* __restrict__ qk_hi, __half* __restrict__ qk_lo, unsigned char* __restrict__ records) {
+  // chunks in reverse order: the first chunks' outputs are the freshest in L2 when the chain starts
+  const int g = gridDim.x - 1 - blockIdx.x;
+  const int4 cm = chunk_map[g];  // {seq, first token, length, chunk index}
   const int slot = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r0 = kConvRows * warp;
   const int L = cm.z;
-  if (r0 >= L) return;
   const int nqk = 2 * d.Hk;
+  if (slot >= nqk + d.Hv) {
+    const int hz = slot - nqk - d.Hv;
+    if (r0 < L) gate_rows(d, norm_w, z, records + ((int64_t)g * d.Hv + hz) * kRec + REC_G, cm.y, r0, L, hz, lane);
+    return;
+  }
+  // v^ goes straight into the record of (chunk, value head) as the chain kernel's operand image
+  unsigned char* vrec = slot >= nqk ? records + ((int64_t)g * d.Hv + (slot - nqk)) * kRec + REC_V : nullptr;
+  if (vrec) {
+#pragma unroll
+    for (int i = 0; i < kConvRows; ++i)
+      if (r0 + i >= L) *reinterpret_cast<uint2*>(vrec + mnmaj(kC, r0 + i, 4 * lane)) = make_uint2(0u, 0u);
+  }
+  if (r0 >= L) return;
   const int64_t C = d.C;
   const int64_t c = (int64_t)slot * kD + 4 * lane;  // q heads, k heads and v heads are consecutive in qkv
   float w[4][4];
@@ -133,13 +182,9 @@ __global__ void __launch_bounds__(128)
       }
     }
   } else {
-    const int64_t WV = (int64_t)d.Hv * kD;
-    const int64_t cv = c - (int64_t)nqk * kD;
 #pragma unroll
     for (int i = 0; i < kConvRows; ++i)
-      if (r0 + i < L)
-        st8(reinterpret_cast<unsigned char*>(vh + ((int64_t)cm.y + r0 + i) * WV + cv), y[i][0], y[i][1], y[i][2],
-            y[i][3]);
+      if (r0 + i < L) st8(vrec + mnmaj(kC, r0 + i, 4 * lane), y[i][0], y[i][1], y[i][2], y[i][3]);
   }
 }
 
@@ -165,8 +210,9 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
   bool bad = false;  // this thread saw a wait run out
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = blockIdx.x / d.Hv;
-  const int h = blockIdx.x - g * d.Hv;
+  const int gr = blockIdx.x / d.Hv;  // chunks in reverse order, as in conv_qkv_kernel
+  const int h = blockIdx.x - gr * d.Hv;
+  const int g = gridDim.x / d.Hv - 1 - gr;
   const int kh = h / d.G;
   const int4 cm = chunk_map[g];
   const int64_t t0 = cm.y;
@@ -423,7 +469,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
 }
 
 // ------------------------------------------------------------------ chain_kernel
-constexpr int kChainThreads = 256;
+constexpr int kChainThreads = 288;  // eight compute warps and one copy-issuing warp
 constexpr int C_A = 0;          // [-W ; Qg]   K-major 128 x 128
 constexpr int C_TA = 32768;     // [T' ; 0]    K-major 128 x 64
 constexpr int C_V = 49152;      // v^          MN-major K=64 x N=128
@@ -431,20 +477,27 @@ constexpr int C_PA = 65536;     // [0 ; P]     K-major 128 x 64
 constexpr int C_KT = 81920;     // K~          MN-major K=64 x M=128
 constexpr int C_DB = 98304;     // Delta       MN-major K=64 x N=128
 constexpr int C_SB = 114688;    // S (fp16)    MN-major K=128 x N=128
-constexpr int C_Z = 147456;     // z           two 64-column boxes, 64 rows
-constexpr int C_MISC = 163840;  // 1 + norm_w [128], row sums of squares [2][64], meta [2][4]
-constexpr int kChainSmem = C_MISC + (128 + 128 + 8) * 4 + 1024;
+constexpr int C_G = 147456;     // output gate rows, two buffers (the record's image)
+constexpr int C_O = 180224;     // output staging, 32 rows x 128 bytes per output warp (16-byte pieces swizzled)
+constexpr int C_MISC = 196608;  // row sums of squares [2][64]
+constexpr int kChainSmem = C_MISC + 128 * 4 + 1024;
 constexpr uint32_t COL_S = 0, COL_U0 = 128, COL_Y = 384, kChainTmemCols = 512;
 
+// Roles: warps 0, 1, 4, 5 ("delta warps", TMEM lanes 0..63) move Delta to
+// shared memory and thread 0 issues the MMAs; warps 2, 3, 6, 7 ("output
+// warps", lanes 64..127) write the previous chunk's output rows meanwhile; all
+// eight update the state; warp 8 only issues the bulk copies, as soon as the
+// MMAs that read a buffer have finished, so no compute warp waits on a copy
+// being issued.
 __global__ void __launch_bounds__(kChainThreads, 1)
-    chain_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_z, Dims d,
-                 const float* __restrict__ norm_w, const unsigned char* __restrict__ records,
-                 const int32_t* __restrict__ chunk_off, const int32_t* __restrict__ order,
-                 const int32_t* __restrict__ cu, int zero_state, float* __restrict__ state,
-                 __nv_bfloat16* __restrict__ o, int32_t* status) {
+    chain_kernel(Dims d, const unsigned char* __restrict__ records, const int32_t* __restrict__ chunk_off,
+                 const int32_t* __restrict__ order, const int32_t* __restrict__ cu, int zero_state,
+                 float* __restrict__ state, __nv_bfloat16* __restrict__ o, int32_t* status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  __shared__ uint64_t mb_ld0, mb_ld1, mb_z, mb_mma;
+  __shared__ uint64_t mb_ld0, mb_ld1;  // operands of the two MMA groups, one phase per chunk each
+  __shared__ uint64_t mb_g[2];         // gate rows, buffer cc % 2, one phase per use
+  __shared__ uint64_t mb_m3, mb_m45;   // completions of the two MMA groups, one phase per chunk each
   __shared__ uint32_t tslot;
   bool bad = false;  // this thread saw a wait run out
 
@@ -458,16 +511,21 @@ __global__ void __launch_bounds__(kChainThreads, 1)
   const int nchunks = (len + kC - 1) / kC;
   const int64_t g0 = chunk_off[n];
   const int64_t HvD = (int64_t)d.Hv * kD;
-
-  float* s_nw = reinterpret_cast<float*>(sm + C_MISC);
-  float* s_rms = s_nw + 128;      // [2][64]
-  float* s_meta = s_rms + 128;    // [2][4]: e^{gamma_C}, gamma_C of chunks with parity 0 / 1
+  float* s_rms = reinterpret_cast<float*>(sm + C_MISC);  // [2][64]
+  const bool producer = warp == 8;
+  const bool out_warp = !producer && (warp & 3) >= 2;
+  // compute warps: thread owns row si of S (d_k index) / of the accumulators, columns [64 hc, 64 hc + 64)
+  const int si = 32 * (warp & 3) + lane, hc = (warp >> 2) & 1;
+  const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+  float* gst = state + ((int64_t)n * d.Hv + h) * kD * kD;  // stored [j][i]
 
   if (tid == 0) {
     mbar_init(&mb_ld0, 1);
     mbar_init(&mb_ld1, 1);
-    mbar_init(&mb_z, 1);
-    mbar_init(&mb_mma, 1);
+    mbar_init(&mb_g[0], 1);
+    mbar_init(&mb_g[1], 1);
+    mbar_init(&mb_m3, 1);
+    mbar_init(&mb_m45, 1);
     mbar_init_fence();
   }
   if (warp == 0) tmem_alloc(&tslot, kChainTmemCols);
@@ -475,148 +533,164 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     reinterpret_cast<uint4*>(sm + C_TA + 8192)[i] = make_uint4(0, 0, 0, 0);
     reinterpret_cast<uint4*>(sm + C_PA)[i] = make_uint4(0, 0, 0, 0);
   }
-  if (tid < kD) s_nw[tid] = 1.0f + norm_w[tid];
-  // state S (fp32 in TMEM): thread owns row si (d_k index), columns [64 hc, 64 hc + 64)
-  const int si = 32 * (warp & 3) + lane, hc = warp >> 2;
-  const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-  float* gst = state + ((int64_t)n * d.Hv + h) * kD * kD;  // stored [j][i]
+
+  auto rec_of = [&](int cc) { return records + ((g0 + cc) * d.Hv + h) * (int64_t)kRec; };
+  auto issue_ld0 = [&](int cc) {  // [-W;Qg] and T' land contiguously in C_A .. C_TA + 8192; then v^
+    const unsigned char* r = rec_of(cc);
+    mbar_expect_tx(&mb_ld0, 40960 + 16384);
+    bulk_load(sm + C_A, r + REC_A, 40960, &mb_ld0);
+    bulk_load(sm + C_V, r + REC_V, 16384, &mb_ld0);
+  };
+  auto issue_ld1 = [&](int cc) {  // P and K~ land contiguously in C_PA + 8192 .. C_KT + 16384
+    mbar_expect_tx(&mb_ld1, 8192 + 16384);
+    bulk_load(sm + C_PA + 8192, rec_of(cc) + REC_P, 8192 + 16384, &mb_ld1);
+  };
+  auto issue_gate = [&](int cc) {
+    mbar_expect_tx(&mb_g[cc & 1], 16384);
+    bulk_load(sm + C_G + (cc & 1) * 16384, rec_of(cc) + REC_G, 16384, &mb_g[cc & 1]);
+  };
+  if (producer && lane == 0) {
+    issue_ld0(0);
+    issue_ld1(0);
+    issue_gate(0);
+    if (nchunks > 1) bulk_prefetch_l2(rec_of(1), REC_META + 16);
+  }
   sync_tc();
   const uint32_t tbase = tslot;
+  if (!producer) {
 #pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    float S[32];
+    for (int hh = 0; hh < 2; ++hh) {
+      float S[32];
 #pragma unroll
-    for (int jj = 0; jj < 32; ++jj) S[jj] = zero_state ? 0.f : gst[(int64_t)(64 * hc + 32 * hh + jj) * kD + si];
-    tmem_st32(tbase + lane_base + COL_S + 64 * hc + 32 * hh, S);
+      for (int jj = 0; jj < 32; ++jj) S[jj] = zero_state ? 0.f : gst[(int64_t)(64 * hc + 32 * hh + jj) * kD + si];
+      tmem_st32(tbase + lane_base + COL_S + 64 * hc + 32 * hh, S);
 #pragma unroll
-    for (int m = 0; m < 4; ++m) st16h(sm + C_SB + mnmaj_chunk(kD, si, 64 * hc + 32 * hh + 8 * m), S + 8 * m);
+      for (int m = 0; m < 4; ++m) st16h(sm + C_SB + mnmaj_chunk(kD, si, 64 * hc + 32 * hh + 8 * m), S + 8 * m);
+    }
   }
   fence_async_smem();
   sync_tc();
 
-  auto rec_of = [&](int cc) { return records + ((g0 + cc) * d.Hv + h) * (int64_t)kRec; };
-  // loads of chunk cc: group 0 = [-W;Qg], T', v^ (read by the first MMA group);
-  // group 1 = P, K~ and the chunk's decay (read by the second)
-  auto issue_ld0 = [&](int cc) {
-    const unsigned char* r = rec_of(cc);
-    mbar_expect_tx(&mb_ld0, 32768 + 8192 + 2 * 8192);
-    bulk_load(sm + C_A, r + REC_A, 32768, &mb_ld0);
-    bulk_load(sm + C_TA, r + REC_T, 8192, &mb_ld0);
-    const int ty = (int)(seq0 + (int64_t)cc * kC);
-    tma_load_2d(sm + C_V, &tm_v, h * kD, ty, &mb_ld0);
-    tma_load_2d(sm + C_V + 8192, &tm_v, h * kD + 64, ty, &mb_ld0);
-  };
-  auto issue_ld1 = [&](int cc) {
-    const unsigned char* r = rec_of(cc);
-    mbar_expect_tx(&mb_ld1, 8192 + 16384 + 16);
-    bulk_load(sm + C_PA + 8192, r + REC_P, 8192, &mb_ld1);
-    bulk_load(sm + C_KT, r + REC_K, 16384, &mb_ld1);
-    bulk_load(s_meta + 4 * (cc & 1), r + REC_META, 16, &mb_ld1);
-  };
-  if (tid == 0) {
-    issue_ld0(0);
-    issue_ld1(0);
-  }
-
-  // output rows of chunk cc (O in lanes 64..127 of its U buffer): zero-centred
-  // RMSNorm over d_v times sigmoid(z), bf16 out.  Warps 2, 3, 6, 7 only.
+  // Output rows of chunk cc (O in lanes 64..127 of its U buffer): zero-centred
+  // RMSNorm over d_v times the precomputed gate (1 + w) sigmoid(z), bf16 out.
+  // Output warps only; they meet at named barrier 1.
   auto epilogue = [&](int cc) {
     const int r = si - 64;
-    const uint32_t col = COL_U0 + 128 * (cc & 1) + 64 * hc;
-    float v[64];
-    tmem_ld32(tbase + lane_base + col, v);
-    tmem_ld32(tbase + lane_base + col + 32, v + 32);
+    const int Lc = min(kC, len - cc * kC);
+    const uint32_t col = tbase + lane_base + COL_U0 + 128 * (cc & 1) + 64 * hc;
     float ss = 0.f;
 #pragma unroll
-    for (int j = 0; j < 64; ++j) ss += v[j] * v[j];
+    for (int hh = 0; hh < 2; ++hh) {
+      float v[32];
+      tmem_ld32(col + 32 * hh, v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) ss += v[j] * v[j];
+    }
     s_rms[64 * hc + r] = ss;
     asm volatile("bar.sync 1, 128;" ::: "memory");
-    const int Lc = min(kC, len - cc * kC);
-    if (r < Lc) {
-      const float rinv = rsqrtf((s_rms[r] + s_rms[64 + r]) * (1.0f / kD) + d.norm_eps);
-      const unsigned char* zrow = sm + C_Z + hc * 8192 + r * 128;
-      __nv_bfloat16* orow = o + (seq0 + (int64_t)cc * kC + r) * HvD + (int64_t)h * kD + 64 * hc;
+    const float rinv = rsqrtf((s_rms[r] + s_rms[64 + r]) * (1.0f / kD) + d.norm_eps);
+    const unsigned char* grow = sm + C_G + (cc & 1) * 16384 + r * 256 + hc * 128;
+    unsigned char* stage = sm + C_O + (2 * hc + (warp & 1)) * 4096;  // this warp's 32 rows x 128 bytes
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const uint4 zr = *reinterpret_cast<const uint4*>(zrow + ((m ^ (r & 7)) << 4));
-        const uint32_t zw[4] = {zr.x, zr.y, zr.z, zr.w};
+    for (int hh = 0; hh < 2; ++hh) {  // the row again from TMEM: fewer live registers
+      float v[32];
+      tmem_ld32(col + 32 * hh, v);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int q = 4 * hh + m;  // 16-byte piece of the row half
+        const uint4 gq = *reinterpret_cast<const uint4*>(grow + ((q ^ (r & 7)) << 4));
+        const __half2* g2 = reinterpret_cast<const __half2*>(&gq);
         uint32_t ow[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int j = 8 * m + 2 * e;
-          const float z0 = __uint_as_float(zw[e] << 16), z1 = __uint_as_float(zw[e] & 0xffff0000u);
-          const float o0 = v[j] * rinv * s_nw[64 * hc + j] * __fdividef(1.0f, 1.0f + __expf(-z0));
-          const float o1 = v[j + 1] * rinv * s_nw[64 * hc + j + 1] * __fdividef(1.0f, 1.0f + __expf(-z1));
-          __nv_bfloat162 pr = __floats2bfloat162_rn(o0, o1);
+          const float2 gf = __half22float2(g2[e]);
+          __nv_bfloat162 pr = __floats2bfloat162_rn(v[8 * m + 2 * e] * rinv * gf.x, v[8 * m + 2 * e + 1] * rinv * gf.y);
           ow[e] = *reinterpret_cast<uint32_t*>(&pr);
         }
-        *reinterpret_cast<uint4*>(orow + 8 * m) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+        *reinterpret_cast<uint4*>(stage + lane * 128 + ((q ^ (lane & 7)) << 4)) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
       }
     }
+    __syncwarp();
+    // eight lanes per row: each store instruction writes four whole 128-byte row halves
+    const int rbase = 32 * (warp & 1);
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int rr = 4 * it + (lane >> 3), q = lane & 7;
+      if (rbase + rr < Lc) {
+        const uint4 val = *reinterpret_cast<const uint4*>(stage + rr * 128 + ((q ^ (rr & 7)) << 4));
+        *reinterpret_cast<uint4*>(o + (seq0 + (int64_t)cc * kC + rbase + rr) * HvD + (int64_t)h * kD + 64 * hc + 8 * q) =
+            val;
+      }
+    }
+    __syncwarp();
   };
-  const bool out_warp = (warp & 3) >= 2;
 
-  uint32_t ph0 = 0, ph1 = 0, phz = 0, phm = 0;
   for (int c = 0; c < nchunks; ++c) {
     const uint32_t colU = COL_U0 + 128 * (c & 1);
-    if (!mbar_wait(&mb_ld0, ph0, kWaitNs)) bad = true;
-    ph0 ^= 1;
-    // U = [T';0] v^ ; U += [-W;Qg] S  ->  [Delta ; Qg S]
-    if (tid == 0 && !bad) {
-      const uint32_t ta = smem_u32(sm + C_TA), vb = smem_u32(sm + C_V), aa = smem_u32(sm + C_A),
-                     sb = smem_u32(sm + C_SB);
-      constexpr uint32_t id = idesc_f16(128, 128, false, true);
-#pragma unroll
-      for (int s = 0; s < 4; ++s) mma_f16(tbase + colU, desc_kmaj(ta, 128, s), desc_mnmaj(vb, kC, s), id, s > 0);
-#pragma unroll
-      for (int s = 0; s < 8; ++s) mma_f16(tbase + colU, desc_kmaj(aa, 128, s), desc_mnmaj(sb, kD, s), id, 1);
-      mma_commit(&mb_mma);
-    }
-    if (c > 0 && out_warp) {
-      if (!mbar_wait(&mb_z, phz, kWaitNs)) bad = true;
-      epilogue(c - 1);
-    }
-    if (c > 0) phz ^= 1;
-    if (!mbar_wait(&mb_mma, phm, kWaitNs)) bad = true;
-    phm ^= 1;
-    fence_after();
-    if (tid == 0 && c + 1 < nchunks) issue_ld0(c + 1);
-    if (si < 64) {  // Delta -> shared (MN-major B operand)
-      float v[32];
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        tmem_ld32(tbase + lane_base + colU + 64 * hc + 32 * hh, v);
-#pragma unroll
-        for (int m = 0; m < 4; ++m) st16h(sm + C_DB + mnmaj_chunk(kC, si, 64 * hc + 32 * hh + 8 * m), v + 8 * m);
+    if (producer) {
+      if (lane == 0) {  // chunk c+1's operands once chunk c's MMA groups are done with the buffers
+        if (c + 2 < nchunks) bulk_prefetch_l2(rec_of(c + 2), REC_META + 16);
+        if (c + 1 < nchunks) {
+          if (!mbar_wait(&mb_m3, c & 1, kWaitNs)) bad = true;
+          issue_ld0(c + 1);
+          if (!mbar_wait(&mb_m45, c & 1, kWaitNs)) bad = true;
+          issue_ld1(c + 1);
+        }
       }
-    }
-    fence_async_smem();
-    if (sync_tc_any(bad)) break;
-    if (tid == 0) {  // z rows of this chunk; the previous chunk's output is done with the z tile
-      mbar_expect_tx(&mb_z, 2 * 8192);
-      const int ty = (int)(seq0 + (int64_t)c * kC);
-      tma_load_2d(sm + C_Z, &tm_z, h * kD, ty, &mb_z);
-      tma_load_2d(sm + C_Z + 8192, &tm_z, h * kD + 64, ty, &mb_z);
-    }
-    if (!mbar_wait(&mb_ld1, ph1, kWaitNs)) bad = true;
-    ph1 ^= 1;
-    // O += [0;P] Delta ;  Y = K~^T Delta
-    if (tid == 0 && !bad) {
-      const uint32_t pa = smem_u32(sm + C_PA), db = smem_u32(sm + C_DB), kt = smem_u32(sm + C_KT);
-      constexpr uint32_t id4 = idesc_f16(128, 128, false, true);
-      constexpr uint32_t id5 = idesc_f16(128, 128, true, true);
+    } else {
+      const float egC = __ldg(reinterpret_cast<const float*>(rec_of(c) + REC_META));  // used by the state update
+      // U = [T';0] v^ ;  U += [-W;Qg] S  ->  [Delta ; Qg S]
+      if (tid == 0) {
+        if (!mbar_wait(&mb_ld0, c & 1, kWaitNs)) bad = true;
+        if (!bad) {
+          const uint32_t ta = smem_u32(sm + C_TA), vb = smem_u32(sm + C_V), aa = smem_u32(sm + C_A),
+                         sb = smem_u32(sm + C_SB);
+          constexpr uint32_t id = idesc_f16(128, 128, false, true);
 #pragma unroll
-      for (int s = 0; s < 4; ++s) mma_f16(tbase + colU, desc_kmaj(pa, 128, s), desc_mnmaj(db, kC, s), id4, 1);
+          for (int s = 0; s < 4; ++s) mma_f16(tbase + colU, desc_kmaj(ta, 128, s), desc_mnmaj(vb, kC, s), id, s > 0);
 #pragma unroll
-      for (int s = 0; s < 4; ++s) mma_f16(tbase + COL_Y, desc_mnmaj(kt, kC, s), desc_mnmaj(db, kC, s), id5, s > 0);
-      mma_commit(&mb_mma);
-    }
-    const float egC = s_meta[4 * (c & 1)];
-    if (!mbar_wait(&mb_mma, phm, kWaitNs)) bad = true;
-    phm ^= 1;
-    fence_after();
-    if (tid == 0 && c + 1 < nchunks) issue_ld1(c + 1);
-    {  // S = e^{gamma_C} S + K~^T Delta, and its fp16 copy for the next chunk
+          for (int s = 0; s < 8; ++s) mma_f16(tbase + colU, desc_kmaj(aa, 128, s), desc_mnmaj(sb, kD, s), id, 1);
+          mma_commit(&mb_m3);
+        }
+      }
+      if (out_warp) {
+        if (c > 0) {
+          if (!mbar_wait(&mb_g[(c - 1) & 1], ((c - 1) >> 1) & 1, kWaitNs)) bad = true;
+          epilogue(c - 1);
+        }
+      } else {  // Delta -> shared (MN-major B operand); then the second MMA group
+        if (!mbar_wait(&mb_m3, c & 1, kWaitNs)) bad = true;
+        fence_after();
+        float v[32];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          tmem_ld32(tbase + lane_base + colU + 64 * hc + 32 * hh, v);
+#pragma unroll
+          for (int m = 0; m < 4; ++m) st16h(sm + C_DB + mnmaj_chunk(kC, si, 64 * hc + 32 * hh + 8 * m), v + 8 * m);
+        }
+        fence_async_smem();
+        fence_before();
+        asm volatile("bar.sync 2, 128;" ::: "memory");
+        fence_after();
+        if (tid == 0) {  // O += [0;P] Delta ;  Y = K~^T Delta
+          if (!mbar_wait(&mb_ld1, c & 1, kWaitNs)) bad = true;
+          if (!bad) {
+            const uint32_t pa = smem_u32(sm + C_PA), db = smem_u32(sm + C_DB), kt = smem_u32(sm + C_KT);
+            constexpr uint32_t id4 = idesc_f16(128, 128, false, true);
+            constexpr uint32_t id5 = idesc_f16(128, 128, true, true);
+#pragma unroll
+            for (int s = 0; s < 4; ++s) mma_f16(tbase + colU, desc_kmaj(pa, 128, s), desc_mnmaj(db, kC, s), id4, 1);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+              mma_f16(tbase + COL_Y, desc_mnmaj(kt, kC, s), desc_mnmaj(db, kC, s), id5, s > 0);
+            mma_commit(&mb_m45);
+          }
+        }
+      }
+      // neither MMA barrier can run a phase ahead: the next chunk's MMAs follow the block barrier below
+      if (!mbar_wait(&mb_m45, c & 1, kWaitNs)) bad = true;
+      fence_after();
+      // S = e^{gamma_C} S + K~^T Delta, and its fp16 copy for the next chunk
       float v[32], S[32];
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
@@ -631,15 +705,18 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     }
     fence_async_smem();
     if (sync_tc_any(bad)) break;
+    // the output of chunk c-1 is written: its gate buffer takes chunk c+1's rows
+    if (producer && lane == 0 && c + 1 < nchunks) issue_gate(c + 1);
   }
   // block-uniform: either every output warp reaches the epilogue's named barrier or none does
   if (!sync_tc_any(bad) && out_warp) {
-    if (!mbar_wait(&mb_z, phz, kWaitNs)) bad = true;
-    epilogue(nchunks - 1);
+    const int cl = nchunks - 1;
+    if (!mbar_wait(&mb_g[cl & 1], (cl >> 1) & 1, kWaitNs)) bad = true;
+    epilogue(cl);
   }
   if (sync_tc_any(bad)) {
     if (tid == 0) set_status(status, kStatusWaitTimeout);
-  } else {
+  } else if (!producer) {
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       float S[32];
@@ -669,11 +746,10 @@ size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 SplitLayout split_layout(const Dims& d, int64_t total_tokens, int64_t chunk_bound) {
   SplitLayout S;
-  const size_t qkw = (size_t)2 * d.Hk * kD, vw = (size_t)d.Hv * kD;
+  const size_t qkw = (size_t)2 * d.Hk * kD;
   S.qk_hi = 0;
   S.qk_lo = al256(S.qk_hi + (size_t)total_tokens * qkw * 2);
-  S.v = al256(S.qk_lo + (size_t)total_tokens * qkw * 2);
-  S.records = al256(S.v + (size_t)total_tokens * vw * 2);
+  S.records = al256(S.qk_lo + (size_t)total_tokens * qkw * 2);
   S.total_bytes = al256(S.records + (size_t)chunk_bound * d.Hv * kRec);
   return S;
 }
@@ -691,21 +767,18 @@ cudaError_t launch_prefill_split(const Dims& d, const float* conv_w, const float
   unsigned char* ws = (unsigned char*)split_ws;
   __half* qk_hi = (__half*)(ws + S.qk_hi);
   __half* qk_lo = (__half*)(ws + S.qk_lo);
-  __half* vh = (__half*)(ws + S.v);
   unsigned char* records = ws + S.records;
-  CUtensorMap tm_hi, tm_lo, tm_v, tm_z;
-  const uint64_t qkw = (uint64_t)2 * d.Hk * kD, vw = (uint64_t)d.Hv * kD;
+  CUtensorMap tm_hi, tm_lo;
+  const uint64_t qkw = (uint64_t)2 * d.Hk * kD;
   if (!encode_2d(enc, &tm_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, qk_hi, qkw, total_tokens) ||
-      !encode_2d(enc, &tm_lo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, qk_lo, qkw, total_tokens) ||
-      !encode_2d(enc, &tm_v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, vh, vw, total_tokens) ||
-      !encode_2d(enc, &tm_z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, z, vw, total_tokens))
+      !encode_2d(enc, &tm_lo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, qk_lo, qkw, total_tokens))
     return cudaErrorInvalidValue;
   cudaError_t e;
   {
     LaunchScope scope(GDN_K_SPLIT_CONV, stream);
-    conv_qkv_kernel<<<dim3((unsigned)total_chunks, (unsigned)(2 * d.Hk + d.Hv)), 128, 0, stream>>>(
-        d, conv_w, (const __nv_bfloat16*)qkv, (const __nv_bfloat16*)conv_state, zero_conv ? 1 : 0, chunk_map, qk_hi,
-        qk_lo, vh);
+    conv_qkv_kernel<<<dim3((unsigned)total_chunks, (unsigned)(2 * d.Hk + 2 * d.Hv)), 128, 0, stream>>>(
+        d, conv_w, (const __nv_bfloat16*)qkv, (const __nv_bfloat16*)conv_state, zero_conv ? 1 : 0, chunk_map, norm_w,
+        (const __nv_bfloat16*)z, qk_hi, qk_lo, records);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if ((e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrepSmem)) != cudaSuccess)
@@ -720,7 +793,7 @@ cudaError_t launch_prefill_split(const Dims& d, const float* conv_w, const float
     return e;
   LaunchScope scope(GDN_K_SPLIT_CHAIN, stream);
   chain_kernel<<<(unsigned)((int64_t)N * d.Hv), kChainThreads, kChainSmem, stream>>>(
-      tm_v, tm_z, d, norm_w, records, chunk_off, order, cu, zero_state ? 1 : 0, state, (__nv_bfloat16*)o, status);
+      d, records, chunk_off, order, cu, zero_state ? 1 : 0, state, (__nv_bfloat16*)o, status);
   return cudaGetLastError();
 }
 

@@ -473,13 +473,15 @@ constexpr int kChainThreads = 288;  // eight compute warps and one copy-issuing 
 constexpr int C_A = 0;          // [-W ; Qg]   K-major 128 x 128
 constexpr int C_TA = 32768;     // [T' ; 0]    K-major 128 x 64
 constexpr int C_V = 49152;      // v^          MN-major K=64 x N=128
-constexpr int C_PA = 65536;     // [0 ; P]     K-major 128 x 64
-constexpr int C_KT = 81920;     // K~          MN-major K=64 x M=128
+constexpr int C_PA = 65536;     // [0 ; P]     K-major 128 x 64      (buffer 0; buffer 1 at C_PA1)
+constexpr int C_KT = 81920;     // K~          MN-major K=64 x M=128 (buffer 0; buffer 1 at C_KT1)
 constexpr int C_DB = 98304;     // Delta       MN-major K=64 x N=128
 constexpr int C_SB = 114688;    // S (fp16)    MN-major K=128 x N=128
 constexpr int C_G = 147456;     // output gate rows, two buffers (the record's image)
 constexpr int C_O = 180224;     // output staging, 32 rows x 128 bytes per output warp (16-byte pieces swizzled)
-constexpr int C_MISC = 196608;  // row sums of squares [2][64]
+constexpr int C_PA1 = 196608;   // second [0 ; P] buffer
+constexpr int C_KT1 = 212992;   // second K~ buffer
+constexpr int C_MISC = 229376;  // row sums of squares [2][64]
 constexpr int kChainSmem = C_MISC + 128 * 4 + 1024;
 constexpr uint32_t COL_S = 0, COL_U0 = 128, COL_Y = 384, kChainTmemCols = 512;
 
@@ -495,7 +497,8 @@ __global__ void __launch_bounds__(kChainThreads, 1)
                  float* __restrict__ state, __nv_bfloat16* __restrict__ o, int32_t* status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  __shared__ uint64_t mb_ld0, mb_ld1;  // operands of the two MMA groups, one phase per chunk each
+  __shared__ uint64_t mb_ld0;          // operands of the first MMA group, one phase per chunk
+  __shared__ uint64_t mb_ld1[2];       // operands of the second, buffer cc % 2, one phase per use
   __shared__ uint64_t mb_g[2];         // gate rows, buffer cc % 2, one phase per use
   __shared__ uint64_t mb_m3, mb_m45;   // completions of the two MMA groups, one phase per chunk each
   __shared__ uint32_t tslot;
@@ -521,7 +524,8 @@ __global__ void __launch_bounds__(kChainThreads, 1)
 
   if (tid == 0) {
     mbar_init(&mb_ld0, 1);
-    mbar_init(&mb_ld1, 1);
+    mbar_init(&mb_ld1[0], 1);
+    mbar_init(&mb_ld1[1], 1);
     mbar_init(&mb_g[0], 1);
     mbar_init(&mb_g[1], 1);
     mbar_init(&mb_m3, 1);
@@ -529,9 +533,10 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     mbar_init_fence();
   }
   if (warp == 0) tmem_alloc(&tslot, kChainTmemCols);
-  for (int i = tid; i < 512; i += kChainThreads) {  // constant zero halves of [T';0] and [0;P]
+  for (int i = tid; i < 512; i += kChainThreads) {  // constant zero halves of [T';0] and both [0;P]
     reinterpret_cast<uint4*>(sm + C_TA + 8192)[i] = make_uint4(0, 0, 0, 0);
     reinterpret_cast<uint4*>(sm + C_PA)[i] = make_uint4(0, 0, 0, 0);
+    reinterpret_cast<uint4*>(sm + C_PA1)[i] = make_uint4(0, 0, 0, 0);
   }
 
   auto rec_of = [&](int cc) { return records + ((g0 + cc) * d.Hv + h) * (int64_t)kRec; };
@@ -541,9 +546,10 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     bulk_load(sm + C_A, r + REC_A, 40960, &mb_ld0);
     bulk_load(sm + C_V, r + REC_V, 16384, &mb_ld0);
   };
-  auto issue_ld1 = [&](int cc) {  // P and K~ land contiguously in C_PA + 8192 .. C_KT + 16384
-    mbar_expect_tx(&mb_ld1, 8192 + 16384);
-    bulk_load(sm + C_PA + 8192, rec_of(cc) + REC_P, 8192 + 16384, &mb_ld1);
+  auto issue_ld1 = [&](int cc) {  // P and K~ land contiguously in [0;P] + 8192 .. K~ + 16384 of buffer cc % 2
+    uint64_t* mb = &mb_ld1[cc & 1];
+    mbar_expect_tx(mb, 8192 + 16384);
+    bulk_load(sm + ((cc & 1) ? C_PA1 : C_PA) + 8192, rec_of(cc) + REC_P, 8192 + 16384, mb);
   };
   auto issue_gate = [&](int cc) {
     mbar_expect_tx(&mb_g[cc & 1], 16384);
@@ -553,7 +559,8 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     issue_ld0(0);
     issue_ld1(0);
     issue_gate(0);
-    if (nchunks > 1) bulk_prefetch_l2(rec_of(1), REC_META + 16);
+    if (nchunks > 1) issue_ld1(1);
+    if (nchunks > 2) bulk_prefetch_l2(rec_of(2), REC_META + 16);
   }
   sync_tc();
   const uint32_t tbase = tslot;
@@ -628,14 +635,16 @@ __global__ void __launch_bounds__(kChainThreads, 1)
   for (int c = 0; c < nchunks; ++c) {
     const uint32_t colU = COL_U0 + 128 * (c & 1);
     if (producer) {
-      if (lane == 0) {  // chunk c+1's operands once chunk c's MMA groups are done with the buffers
-        if (c + 2 < nchunks) bulk_prefetch_l2(rec_of(c + 2), REC_META + 16);
+      if (lane == 0) {  // operands as soon as chunk c's MMA groups are done with their buffers
         if (c + 1 < nchunks) {
           if (!mbar_wait(&mb_m3, c & 1, kWaitNs)) bad = true;
           issue_ld0(c + 1);
-          if (!mbar_wait(&mb_m45, c & 1, kWaitNs)) bad = true;
-          issue_ld1(c + 1);
         }
+        if (c + 2 < nchunks) {
+          if (!mbar_wait(&mb_m45, c & 1, kWaitNs)) bad = true;
+          issue_ld1(c + 2);
+        }
+        if (c + 3 < nchunks) bulk_prefetch_l2(rec_of(c + 3), REC_META + 16);  // behind the copies in the queue
       }
     } else {
       const float egC = __ldg(reinterpret_cast<const float*>(rec_of(c) + REC_META));  // used by the state update
@@ -673,9 +682,10 @@ __global__ void __launch_bounds__(kChainThreads, 1)
         asm volatile("bar.sync 2, 128;" ::: "memory");
         fence_after();
         if (tid == 0) {  // O += [0;P] Delta ;  Y = K~^T Delta
-          if (!mbar_wait(&mb_ld1, c & 1, kWaitNs)) bad = true;
+          if (!mbar_wait(&mb_ld1[c & 1], (c >> 1) & 1, kWaitNs)) bad = true;
           if (!bad) {
-            const uint32_t pa = smem_u32(sm + C_PA), db = smem_u32(sm + C_DB), kt = smem_u32(sm + C_KT);
+            const uint32_t pa = smem_u32(sm + ((c & 1) ? C_PA1 : C_PA)), db = smem_u32(sm + C_DB),
+                           kt = smem_u32(sm + ((c & 1) ? C_KT1 : C_KT));
             constexpr uint32_t id4 = idesc_f16(128, 128, false, true);
             constexpr uint32_t id5 = idesc_f16(128, 128, true, true);
 #pragma unroll

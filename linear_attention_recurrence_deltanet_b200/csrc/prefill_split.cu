@@ -33,7 +33,8 @@
 //   [65536, 81920) K~                   MN-major K=64 x M=128
 //   [81920, 98304) output gate (1 + w) sigmoid(z) (from the conv), fp16, row r at 256 r,
 //                  column half at +128, 16-byte piece q at (q ^ (r % 8)) * 16
-//   [98304, 98320) e^{gamma_C}, gamma_C
+//   [98304, 98320) e^{gamma_C}, gamma_C (from the conv)
+//   [98320, 98832) gamma_r, beta_r of the chunk's 64 rows (from the conv; 0 past the chunk's end)
 // so the chain kernel reads each chunk in four bulk copies.
 // Operands are fp16 (all bounded: normalised keys and queries, decay factors
 // <= 1), accumulation fp32, the state fp32.
@@ -54,13 +55,16 @@ constexpr int kC = 64;
 constexpr int kD = 128;
 constexpr uint64_t kWaitNs = 2000000000ull;
 
-constexpr int kRec = 98432;
-constexpr int REC_A = 0, REC_T = 32768, REC_V = 40960, REC_P = 57344, REC_K = 65536, REC_G = 81920, REC_META = 98304;
+constexpr int kRec = 98944;
+constexpr int REC_A = 0, REC_T = 32768, REC_V = 40960, REC_P = 57344, REC_K = 65536, REC_G = 81920, REC_META = 98304,
+              REC_GAM = 98320, REC_BETA = 98576;
 
 // ------------------------------------------------------------------ conv_qkv_kernel
 // Block = 4 warps = the 64 rows of one chunk for one 128-channel head slot
-// (q heads, then k heads, then v heads).  Warp w owns rows 16w .. 16w+15, lane
-// l owns channels 4l .. 4l+3.
+// (q heads, then k heads, then v heads, then the output gates of the v
+// heads).  Warp w owns rows 16w .. 16w+15, lane l owns channels 4l .. 4l+3.
+// A fifth warp computes the chunk's gates g, beta of the value head in the
+// output-gate slots and exits in the others.
 constexpr int kConvRows = 16;
 
 // Slots past the q/k/v heads compute the output gate of one value head,
@@ -91,10 +95,47 @@ __device__ __forceinline__ void gate_rows(const Dims& d, const float* __restrict
   }
 }
 
-__global__ void __launch_bounds__(128)
+// Gates of one chunk and value head ("fp32 Gated DeltaNet recurrence"):
+// g_r = -exp(A_log) softplus(a_r + dt_bias), beta_r = sigmoid(b_r), the
+// inclusive scan gamma_r of g within the chunk, into the record.  One warp:
+// lane l owns rows 2l and 2l + 1.
+__device__ __forceinline__ void chunk_gates(const Dims& d, const float* __restrict__ A_log,
+                                            const float* __restrict__ dt_bias, const __nv_bfloat16* __restrict__ a,
+                                            const __nv_bfloat16* __restrict__ b, int64_t t0, int L, int h, int lane,
+                                            unsigned char* __restrict__ rec) {
+  const float negA = -expf(A_log[h]);
+  const float dtb = dt_bias[h];
+  float g2[2], be2[2];
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int r = 2 * lane + e;
+    g2[e] = 0.f;
+    be2[e] = 0.f;
+    if (r < L) {
+      g2[e] = negA * softplus_f(__bfloat162float(a[(t0 + r) * d.Hv + h]) + dtb);
+      be2[e] = 1.0f / (1.0f + expf(-__bfloat162float(b[(t0 + r) * d.Hv + h])));
+    }
+  }
+  float incl = g2[0] + g2[1];
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  const float gC = __shfl_sync(0xffffffffu, incl, 31);
+  reinterpret_cast<float2*>(rec + REC_GAM)[lane] = make_float2(incl - g2[1], incl);
+  reinterpret_cast<float2*>(rec + REC_BETA)[lane] = make_float2(be2[0], be2[1]);
+  if (lane == 0) reinterpret_cast<float2*>(rec + REC_META)[0] = make_float2(expf(gC), gC);
+}
+
+constexpr int kConvThreads = 160;
+
+__global__ void __launch_bounds__(kConvThreads)
     conv_qkv_kernel(Dims d, const float* __restrict__ conv_w, const __nv_bfloat16* __restrict__ qkv,
                     const __nv_bfloat16* __restrict__ hist, int zero_conv, const int4* __restrict__ chunk_map,
                     const float* __restrict__ norm_w, const __nv_bfloat16* __restrict__ z,
+                    const float* __restrict__ A_log, const float* __restrict__ dt_bias,
+                    const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
                     __half* __restrict__ qk_hi, __half* __restrict__ qk_lo, unsigned char* __restrict__ records) {
   // chunks in reverse order: the first chunks' outputs are the freshest in L2 when the chain starts
   const int g = gridDim.x - 1 - blockIdx.x;
@@ -106,9 +147,12 @@ __global__ void __launch_bounds__(128)
   const int nqk = 2 * d.Hk;
   if (slot >= nqk + d.Hv) {
     const int hz = slot - nqk - d.Hv;
-    if (r0 < L) gate_rows(d, norm_w, z, records + ((int64_t)g * d.Hv + hz) * kRec + REC_G, cm.y, r0, L, hz, lane);
+    unsigned char* rec = records + ((int64_t)g * d.Hv + hz) * kRec;
+    if (warp == 4) chunk_gates(d, A_log, dt_bias, a, b, cm.y, L, hz, lane, rec);
+    else if (r0 < L) gate_rows(d, norm_w, z, rec + REC_G, cm.y, r0, L, hz, lane);
     return;
   }
+  if (warp == 4) return;
   // v^ goes straight into the record of (chunk, value head) as the chain kernel's operand image
   unsigned char* vrec = slot >= nqk ? records + ((int64_t)g * d.Hv + (slot - nqk)) * kRec + REC_V : nullptr;
   if (vrec) {
@@ -198,10 +242,45 @@ constexpr int P_MISC = 102400;
 constexpr int kPrepSmem = P_MISC + 64 * 6 * 4 + 64 + 1024;
 constexpr uint32_t P_COL_D1 = 0, P_COL_W = 128, kPrepTmemCols = 256;
 
+// One doubling level of T = (I + A)^-1 (fp32, row stride LDS): for every
+// pair of b x b diagonal blocks at offset o = 2 b p, Y = A21 T11 (into the
+// lower-left block of Ym), then T21 = -T22 Y.  Four columns per work item.
+template <int B>
+__device__ __forceinline__ void solve_level(const float* __restrict__ Am, float* __restrict__ Tm,
+                                            float* __restrict__ Ym, int tid) {
+  constexpr int kItems = (64 / (2 * B)) * B * (B / 4);
+  for (int e = tid; e < kItems; e += kPrepThreads) {
+    const int p = e / (B * B / 4), rem = e - p * (B * B / 4);
+    const int i = rem / (B / 4), j = 4 * (rem - i * (B / 4));
+    const int o = 2 * B * p;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < B; ++k) {
+      const float a = Am[(o + B + i) * LDS + o + k];
+      const float4 t = *reinterpret_cast<const float4*>(Tm + (o + k) * LDS + o + j);
+      acc.x += a * t.x; acc.y += a * t.y; acc.z += a * t.z; acc.w += a * t.w;
+    }
+    *reinterpret_cast<float4*>(Ym + (o + B + i) * LDS + o + j) = acc;
+  }
+  __syncthreads();
+  for (int e = tid; e < kItems; e += kPrepThreads) {
+    const int p = e / (B * B / 4), rem = e - p * (B * B / 4);
+    const int i = rem / (B / 4), j = 4 * (rem - i * (B / 4));
+    const int o = 2 * B * p;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < B; ++k) {
+      const float t = Tm[(o + B + i) * LDS + o + B + k];
+      const float4 y = *reinterpret_cast<const float4*>(Ym + (o + B + k) * LDS + o + j);
+      acc.x += t * y.x; acc.y += t * y.y; acc.z += t * y.z; acc.w += t * y.w;
+    }
+    *reinterpret_cast<float4*>(Tm + (o + B + i) * LDS + o + j) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+  }
+  __syncthreads();
+}
+
 __global__ void __launch_bounds__(kPrepThreads, 2)
     prep_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constant__ CUtensorMap tm_lo, Dims d,
-                const float* __restrict__ A_log, const float* __restrict__ dt_bias,
-                const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
                 const int4* __restrict__ chunk_map, unsigned char* __restrict__ records, int32_t* status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -214,9 +293,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
   const int h = blockIdx.x - gr * d.Hv;
   const int g = gridDim.x / d.Hv - 1 - gr;
   const int kh = h / d.G;
-  const int4 cm = chunk_map[g];
-  const int64_t t0 = cm.y;
-  const int L = cm.z;
+  const int64_t t0 = chunk_map[g].y;  // rows past the chunk's end carry beta = 0 (their gates are zero)
   unsigned char* rec = records + ((int64_t)g * d.Hv + h) * kRec;
 
   float* misc = reinterpret_cast<float*>(sm + P_MISC);
@@ -226,7 +303,6 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
   float* s_ekd = misc + 192;
   float* s_tb = misc + 256;    // beta_j        (columns of T')
   float* s_tbg = misc + 320;   // beta_j e^{gamma_j} (columns of T'')
-  float* s_gC = misc + 384;
   float* Am = reinterpret_cast<float*>(sm + P_KQL);
   float* Tm = Am + 64 * LDS;
   float* Ym = Tm + 64 * LDS;
@@ -252,44 +328,17 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
       tma_load_2d(sm + P_KQL + j * 16384 + 8192, &tm_lo, qx + 64 * j, (int)t0, &mb_tma);
     }
   }
-  if (warp == 0) {  // gates of rows 2 lane, 2 lane + 1; inclusive scan of g
-    const float negA = -expf(A_log[h]);
-    const float dtb = dt_bias[h];
-    float g2[2], be2[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int r = 2 * lane + e;
-      g2[e] = 0.f;
-      be2[e] = 0.f;
-      if (r < L) {
-        g2[e] = negA * softplus_f(__bfloat162float(a[(t0 + r) * d.Hv + h]) + dtb);
-        be2[e] = 1.0f / (1.0f + expf(-__bfloat162float(b[(t0 + r) * d.Hv + h])));
-      }
-    }
-    float incl = g2[0] + g2[1];
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const float y = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += y;
-    }
-    const float gam1 = incl, gam0 = incl - g2[1];
-    const float gC = __shfl_sync(0xffffffffu, incl, 31);
-    const float gm[2] = {gam0, gam1};
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int r = 2 * lane + e;
-      const float eg = expf(gm[e]);
-      s_gam[r] = gm[e];
-      s_beta[r] = be2[e];
-      s_eg[r] = eg;
-      s_ekd[r] = expf(gC - gm[e]);
-      s_tb[r] = be2[e];
-      s_tbg[r] = be2[e] * eg;
-    }
-    if (lane == 0) {
-      *s_gC = gC;
-      reinterpret_cast<float2*>(rec + REC_META)[0] = make_float2(expf(gC), gC);
-    }
+  if (tid < 64) {  // the chunk's gates (computed by the conv kernel) and their exponentials
+    const float gam = reinterpret_cast<const float*>(rec + REC_GAM)[tid];
+    const float be = reinterpret_cast<const float*>(rec + REC_BETA)[tid];
+    const float gC = reinterpret_cast<const float*>(rec + REC_META)[1];
+    const float eg = expf(gam);
+    s_gam[tid] = gam;
+    s_beta[tid] = be;
+    s_eg[tid] = eg;
+    s_ekd[tid] = expf(gC - gam);
+    s_tb[tid] = be;
+    s_tbg[tid] = be * eg;
   }
   if (!mbar_wait(&mb_tma, 0, kWaitNs)) bad = true;
   if (sync_tc_any(bad)) {
@@ -350,55 +399,32 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
       }
     }
   }
+  for (int i = tid; i < 64 * 16; i += kPrepThreads)
+    *reinterpret_cast<float4*>(Tm + (i >> 4) * LDS + 4 * (i & 15)) = make_float4(0.f, 0.f, 0.f, 0.f);
   __syncthreads();
-  // T = (I + A)^-1 in 16x16 blocks: diagonal blocks by right-looking forward
-  // substitution (one column per thread), then the blocks below the diagonal
-  // by distance from it.
+  // T = (I + A)^-1 by recursive doubling: the 8x8 diagonal blocks by forward
+  // substitution, then for block size b = 8, 16, 32 every pair of b-blocks on
+  // the diagonal is joined into a 2b-block through its lower-left block
+  // T21 = -T22 (A21 T11).  Tm starts at zero, so the upper blocks stay zero.
   if (tid < 64) {
-    const int bb = tid >> 4, c16 = tid & 15;
-    const float* Ab = Am + (16 * bb) * LDS + 16 * bb;
-    float acc[16], t[16];
+    const int bb = tid >> 3, c8 = tid & 7;
+    const float* Ab = Am + (8 * bb) * LDS + 8 * bb;
+    float acc[8], t[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      t[k] = (k < c16) ? 0.f : (k == c16 ? 1.f : -acc[k]);
+    for (int k = 0; k < 8; ++k) {
+      t[k] = (k < c8) ? 0.f : (k == c8 ? 1.f : -acc[k]);
 #pragma unroll
-      for (int i = k + 1; i < 16; ++i) acc[i] += Ab[i * LDS + k] * t[k];
+      for (int i = k + 1; i < 8; ++i) acc[i] += Ab[i * LDS + k] * t[k];
     }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) Tm[(16 * bb + i) * LDS + 16 * bb + c16] = t[i];
+    for (int i = 0; i < 8; ++i) Tm[(8 * bb + i) * LDS + 8 * bb + c8] = t[i];
   }
   __syncthreads();
-  for (int e = tid; e < 6 * 64; e += kPrepThreads) {  // At_ij = T_ii A_ij below the diagonal
-    const int pr = e >> 6, p = (e >> 2) & 15, q = 4 * (e & 3);
-    const int bi = pr == 0 ? 1 : (pr < 3 ? 2 : 3), bj = pr == 0 ? 0 : (pr < 3 ? pr - 1 : pr - 3);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int kk = 0; kk < 16; ++kk) {
-      const float t = Tm[(16 * bi + p) * LDS + 16 * bi + kk];
-      const float4 a4 = *reinterpret_cast<const float4*>(Am + (16 * bi + kk) * LDS + 16 * bj + q);
-      acc.x += t * a4.x; acc.y += t * a4.y; acc.z += t * a4.z; acc.w += t * a4.w;
-    }
-    *reinterpret_cast<float4*>(Ym + (16 * bi + p) * LDS + 16 * bj + q) = acc;
-  }
-  __syncthreads();
-  for (int dl = 1; dl < 4; ++dl) {  // T_ij = -sum_{k=j}^{i-1} At_ik T_kj
-    for (int e = tid; e < (4 - dl) * 64; e += kPrepThreads) {
-      const int bj = e >> 6, bi = bj + dl, p = (e >> 2) & 15, q = 4 * (e & 3);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int bk = bj; bk < bi; ++bk) {
-#pragma unroll
-        for (int kk = 0; kk < 16; ++kk) {
-          const float y = Ym[(16 * bi + p) * LDS + 16 * bk + kk];
-          const float4 t4 = *reinterpret_cast<const float4*>(Tm + (16 * bk + kk) * LDS + 16 * bj + q);
-          acc.x += y * t4.x; acc.y += y * t4.y; acc.z += y * t4.z; acc.w += y * t4.w;
-        }
-      }
-      *reinterpret_cast<float4*>(Tm + (16 * bi + p) * LDS + 16 * bj + q) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
-    }
-    __syncthreads();
-  }
+  solve_level<8>(Am, Tm, Ym, tid);
+  solve_level<16>(Am, Tm, Ym, tid);
+  solve_level<32>(Am, Tm, Ym, tid);
   {  // T' = T diag(beta) -> record; T'' = T diag(beta e^gamma) -> rows 0..63 of [T'';0]
     const int r = tid >> 2, j0 = 16 * (tid & 3);
     float tv[16], t1[16], t2[16];
@@ -786,9 +812,10 @@ cudaError_t launch_prefill_split(const Dims& d, const float* conv_w, const float
   cudaError_t e;
   {
     LaunchScope scope(GDN_K_SPLIT_CONV, stream);
-    conv_qkv_kernel<<<dim3((unsigned)total_chunks, (unsigned)(2 * d.Hk + 2 * d.Hv)), 128, 0, stream>>>(
+    conv_qkv_kernel<<<dim3((unsigned)total_chunks, (unsigned)(2 * d.Hk + 2 * d.Hv)), kConvThreads, 0, stream>>>(
         d, conv_w, (const __nv_bfloat16*)qkv, (const __nv_bfloat16*)conv_state, zero_conv ? 1 : 0, chunk_map, norm_w,
-        (const __nv_bfloat16*)z, qk_hi, qk_lo, records);
+        (const __nv_bfloat16*)z, A_log, dt_bias, (const __nv_bfloat16*)a, (const __nv_bfloat16*)b, qk_hi, qk_lo,
+        records);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if ((e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrepSmem)) != cudaSuccess)
@@ -796,7 +823,7 @@ cudaError_t launch_prefill_split(const Dims& d, const float* conv_w, const float
   {
     LaunchScope scope(GDN_K_SPLIT_PREP, stream);
     prep_kernel<<<(unsigned)(total_chunks * d.Hv), kPrepThreads, kPrepSmem, stream>>>(
-        tm_hi, tm_lo, d, A_log, dt_bias, (const __nv_bfloat16*)a, (const __nv_bfloat16*)b, chunk_map, records, status);
+        tm_hi, tm_lo, d, chunk_map, records, status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if ((e = cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kChainSmem)) != cudaSuccess)

@@ -233,53 +233,68 @@ __global__ void __launch_bounds__(kConvThreads)
 }
 
 // ------------------------------------------------------------------ prep_kernel
+// Three blocks per SM.  Shared memory (67 KB):
+//   P_KQ   [k^ ; q^] hi parts, K-major 128 x 128.  Once the Qg rows are out,
+//          the q^ halves of the two 64-column blocks hold the solve's Y rows
+//          0..31 and 32..63.
+//   P_KQL  [k^ ; q^] lo parts.  After M1: the solve scratch A (16 KB) and T
+//          (16 KB); after the solve, T'' (K-major 64 x 64) over A.
+// fp32 scratch rows are 64 floats with the 16-byte pieces of row r XORed by
+// r % 16, so that column accesses from 16 rows hit distinct banks.
+// TMEM: 128 columns; [K;Q]K^T in columns 0..63, then W (an M = 64 MMA) in 0..127.
 constexpr int kPrepThreads = 256;
-constexpr int LDS = 68;  // fp32 solve scratch row stride
-constexpr int P_KQ = 0;            // [k^ ; q^] hi  K-major 128 x 128
-constexpr int P_KQL = 32768;       // [k^ ; q^] lo; after M1 the solve scratch (A, T, Y: 3 x 64 x LDS floats)
-constexpr int P_TA = 86016;        // [T'' ; 0]   K-major 128 x 64
-constexpr int P_MISC = 102400;
-constexpr int kPrepSmem = P_MISC + 64 * 6 * 4 + 64 + 1024;
-constexpr uint32_t P_COL_D1 = 0, P_COL_W = 128, kPrepTmemCols = 256;
+constexpr int P_KQ = 0;
+constexpr int P_KQL = 32768;
+constexpr int P_MISC = 65536;
+constexpr int kPrepSmem = P_MISC + 64 * 6 * 4 + 1024;
+constexpr uint32_t kPrepTmemCols = 128;
 
-// One doubling level of T = (I + A)^-1 (fp32, row stride LDS): for every
-// pair of b x b diagonal blocks at offset o = 2 b p, Y = A21 T11 (into the
-// lower-left block of Ym), then T21 = -T22 Y.  Four columns per work item.
+__device__ __forceinline__ int sidx(int row, int col) { return row * 64 + ((((col >> 2) ^ (row & 15))) << 2) + (col & 3); }
+
+// Y rows 0..31 and 32..63 live in the two q^ halves of the hi tile
+__device__ __forceinline__ float* yrow(unsigned char* sm, int row) {
+  return reinterpret_cast<float*>(sm + P_KQ + (row < 32 ? 8192 : 24576)) + (row & 31) * 64;
+}
+
+// One doubling level of T = (I + A)^-1: for every pair of B x B diagonal
+// blocks at offset o = 2 B p, Y = A21 T11, then T21 = -T22 Y.  Four columns
+// per work item.
 template <int B>
-__device__ __forceinline__ void solve_level(const float* __restrict__ Am, float* __restrict__ Tm,
-                                            float* __restrict__ Ym, int tid) {
+__device__ __forceinline__ void solve_level(const float* __restrict__ Am, float* __restrict__ Tm, unsigned char* sm,
+                                            int tid) {
   constexpr int kItems = (64 / (2 * B)) * B * (B / 4);
   for (int e = tid; e < kItems; e += kPrepThreads) {
     const int p = e / (B * B / 4), rem = e - p * (B * B / 4);
     const int i = rem / (B / 4), j = 4 * (rem - i * (B / 4));
-    const int o = 2 * B * p;
+    const int o = 2 * B * p, row = o + B + i;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int k = 0; k < B; ++k) {
-      const float a = Am[(o + B + i) * LDS + o + k];
-      const float4 t = *reinterpret_cast<const float4*>(Tm + (o + k) * LDS + o + j);
+      const float a = Am[sidx(row, o + k)];
+      const float4 t = *reinterpret_cast<const float4*>(Tm + sidx(o + k, o + j));
       acc.x += a * t.x; acc.y += a * t.y; acc.z += a * t.z; acc.w += a * t.w;
     }
-    *reinterpret_cast<float4*>(Ym + (o + B + i) * LDS + o + j) = acc;
+    *reinterpret_cast<float4*>(yrow(sm, row) + (sidx(row, o + j) & 63)) = acc;
   }
   __syncthreads();
   for (int e = tid; e < kItems; e += kPrepThreads) {
     const int p = e / (B * B / 4), rem = e - p * (B * B / 4);
     const int i = rem / (B / 4), j = 4 * (rem - i * (B / 4));
-    const int o = 2 * B * p;
+    const int o = 2 * B * p, row = o + B + i;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int k = 0; k < B; ++k) {
-      const float t = Tm[(o + B + i) * LDS + o + B + k];
-      const float4 y = *reinterpret_cast<const float4*>(Ym + (o + B + k) * LDS + o + j);
+      const float t = Tm[sidx(row, o + B + k)];
+      const int yr = o + B + k;
+      const float4 y = *reinterpret_cast<const float4*>(yrow(sm, yr) + (sidx(yr, o + j) & 63));
       acc.x += t * y.x; acc.y += t * y.y; acc.z += t * y.z; acc.w += t * y.w;
     }
-    *reinterpret_cast<float4*>(Tm + (o + B + i) * LDS + o + j) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+    *reinterpret_cast<float4*>(Tm + sidx(row, o + j)) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
   }
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kPrepThreads, 2)
+__global__ void __launch_bounds__(kPrepThreads, 3)
     prep_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constant__ CUtensorMap tm_lo, Dims d,
                 const int4* __restrict__ chunk_map, unsigned char* __restrict__ records, int32_t* status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -301,11 +316,10 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
   float* s_beta = misc + 64;
   float* s_eg = misc + 128;
   float* s_ekd = misc + 192;
-  float* s_tb = misc + 256;    // beta_j        (columns of T')
+  float* s_tb = misc + 256;    // beta_j             (columns of T')
   float* s_tbg = misc + 320;   // beta_j e^{gamma_j} (columns of T'')
   float* Am = reinterpret_cast<float*>(sm + P_KQL);
-  float* Tm = Am + 64 * LDS;
-  float* Ym = Tm + 64 * LDS;
+  float* Tm = Am + 64 * 64;
 
   if (tid == 0) {
     mbar_init(&mb_tma, 1);
@@ -313,8 +327,6 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     mbar_init_fence();
   }
   if (warp == 0) tmem_alloc(&tslot, kPrepTmemCols);
-  for (int i = tid; i < 512; i += kPrepThreads)  // rows 64..127 of [T'';0] stay zero
-    reinterpret_cast<uint4*>(sm + P_TA + 8192)[i] = make_uint4(0, 0, 0, 0);
   sync_tc();
   const uint32_t tbase = tslot;
   if (tid == 0) {
@@ -352,111 +364,14 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     const uint32_t kq = smem_u32(sm + P_KQ), kql = smem_u32(sm + P_KQL);
     constexpr uint32_t id = idesc_f16(128, 64, false, false);
 #pragma unroll
-    for (int s = 0; s < 8; ++s) mma_f16(tbase + P_COL_D1, desc_kmaj(kq, 128, s), desc_kmaj(kq, 128, s), id, s > 0);
+    for (int s = 0; s < 8; ++s) mma_f16(tbase, desc_kmaj(kq, 128, s), desc_kmaj(kq, 128, s), id, s > 0);
 #pragma unroll
-    for (int s = 0; s < 8; ++s) mma_f16(tbase + P_COL_D1, desc_kmaj(kq, 128, s), desc_kmaj(kql, 128, s), id, 1);
+    for (int s = 0; s < 8; ++s) mma_f16(tbase, desc_kmaj(kq, 128, s), desc_kmaj(kql, 128, s), id, 1);
 #pragma unroll
-    for (int s = 0; s < 8; ++s) mma_f16(tbase + P_COL_D1, desc_kmaj(kql, 128, s), desc_kmaj(kq, 128, s), id, 1);
+    for (int s = 0; s < 8; ++s) mma_f16(tbase, desc_kmaj(kql, 128, s), desc_kmaj(kq, 128, s), id, 1);
     mma_commit(&mb_mma);
   }
-  if (!mbar_wait(&mb_mma, 0, kWaitNs)) bad = true;
-  if (sync_tc_any(bad)) {
-    if (tid == 0) set_status(status, kStatusWaitTimeout);
-    if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
-    return;
-  }
-
-  // A (rows 0..63, fp32 into the solve scratch) and P (rows 64..127, fp16 into the record)
-  const int si = 32 * (warp & 3) + lane, hc = warp >> 2;
-  const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-  {
-    float v[32];
-    tmem_ld32(tbase + lane_base + P_COL_D1 + 32 * hc, v);
-    if (si < 64) {
-      const float br = s_beta[si], gr = s_gam[si];
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        float a4[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int j = 32 * hc + 4 * m + e;
-          a4[e] = (j < si) ? br * __expf(gr - s_gam[j]) * v[4 * m + e] : 0.f;
-        }
-        *reinterpret_cast<float4*>(Am + si * LDS + 32 * hc + 4 * m) = make_float4(a4[0], a4[1], a4[2], a4[3]);
-      }
-    } else {
-      const int r = si - 64;
-      const float gr = s_gam[r];
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        float p[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int j = 32 * hc + 8 * m + e;
-          p[e] = (j <= r) ? __expf(gr - s_gam[j]) * v[8 * m + e] : 0.f;
-        }
-        *reinterpret_cast<uint4*>(rec + REC_P + kmaj_chunk(64, r, 32 * hc + 8 * m)) = pack8h(p);
-      }
-    }
-  }
-  for (int i = tid; i < 64 * 16; i += kPrepThreads)
-    *reinterpret_cast<float4*>(Tm + (i >> 4) * LDS + 4 * (i & 15)) = make_float4(0.f, 0.f, 0.f, 0.f);
-  __syncthreads();
-  // T = (I + A)^-1 by recursive doubling: the 8x8 diagonal blocks by forward
-  // substitution, then for block size b = 8, 16, 32 every pair of b-blocks on
-  // the diagonal is joined into a 2b-block through its lower-left block
-  // T21 = -T22 (A21 T11).  Tm starts at zero, so the upper blocks stay zero.
-  if (tid < 64) {
-    const int bb = tid >> 3, c8 = tid & 7;
-    const float* Ab = Am + (8 * bb) * LDS + 8 * bb;
-    float acc[8], t[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      t[k] = (k < c8) ? 0.f : (k == c8 ? 1.f : -acc[k]);
-#pragma unroll
-      for (int i = k + 1; i < 8; ++i) acc[i] += Ab[i * LDS + k] * t[k];
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) Tm[(8 * bb + i) * LDS + 8 * bb + c8] = t[i];
-  }
-  __syncthreads();
-  solve_level<8>(Am, Tm, Ym, tid);
-  solve_level<16>(Am, Tm, Ym, tid);
-  solve_level<32>(Am, Tm, Ym, tid);
-  {  // T' = T diag(beta) -> record; T'' = T diag(beta e^gamma) -> rows 0..63 of [T'';0]
-    const int r = tid >> 2, j0 = 16 * (tid & 3);
-    float tv[16], t1[16], t2[16];
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const float4 t4 = *reinterpret_cast<const float4*>(Tm + r * LDS + j0 + 4 * m);
-      tv[4 * m] = t4.x; tv[4 * m + 1] = t4.y; tv[4 * m + 2] = t4.z; tv[4 * m + 3] = t4.w;
-    }
-#pragma unroll
-    for (int jj = 0; jj < 16; ++jj) {
-      const float t = (j0 + jj <= r) ? tv[jj] : 0.f;
-      t1[jj] = t * s_tb[j0 + jj];
-      t2[jj] = t * s_tbg[j0 + jj];
-    }
-    *reinterpret_cast<uint4*>(rec + REC_T + kmaj_chunk(64, r, j0)) = pack8h(t1);
-    *reinterpret_cast<uint4*>(rec + REC_T + kmaj_chunk(64, r, j0 + 8)) = pack8h(t1 + 8);
-    st16h(sm + P_TA + kmaj_chunk(128, r, j0), t2);
-    st16h(sm + P_TA + kmaj_chunk(128, r, j0 + 8), t2 + 8);
-  }
-  fence_async_smem();
-  sync_tc();
-
-  // M2: W = [T'';0] K  (B = the k^ rows of the hi tile read as MN-major: K = 64 rows, N = 128 channels)
-  if (tid == 0) {
-    const uint32_t ta = smem_u32(sm + P_TA), kq = smem_u32(sm + P_KQ);
-    constexpr uint32_t id = idesc_f16(128, 128, false, true);
-#pragma unroll
-    for (int s = 0; s < 4; ++s)
-      mma_f16(tbase + P_COL_W, desc_kmaj(ta, 128, s), sdesc(kq + s * 2048, 16384, 1024), id, s > 0);
-    mma_commit(&mb_mma);
-  }
-  // while W is computed: Qg = diag(e^gamma) q^ -> rows 64..127 of the [-W;Qg] image, K~ -> its image
+  // meanwhile: Qg = diag(e^gamma) q^ (hi) -> rows 64..127 of the [-W;Qg] image, K~ = diag(e^{gC-gamma}) k^ -> its image
   for (int e = tid; e < 64 * 16; e += kPrepThreads) {
     const int r = e >> 4, c8 = 8 * (e & 15);
     const uint4 uq = *reinterpret_cast<const uint4*>(sm + P_KQ + kmaj_chunk(128, 64 + r, c8));
@@ -476,18 +391,117 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     *reinterpret_cast<uint4*>(rec + REC_A + kmaj_chunk(128, 64 + r, c8)) = pack8h(fq);
     *reinterpret_cast<uint4*>(rec + REC_K + mnmaj_chunk(64, r, c8)) = pack8h(fk);
   }
+  if (!mbar_wait(&mb_mma, 0, kWaitNs)) bad = true;
+  if (sync_tc_any(bad)) {  // also: the q^ rows are read, the lo tile is free
+    if (tid == 0) set_status(status, kStatusWaitTimeout);
+    if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
+    return;
+  }
+
+  // A (rows 0..63, fp32 into the solve scratch) and P (rows 64..127, fp16 into the record)
+  const int si = 32 * (warp & 3) + lane, hc = warp >> 2;
+  const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+  {
+    float v[32];
+    tmem_ld32(tbase + lane_base + 32 * hc, v);
+    if (si < 64) {
+      const float br = s_beta[si], gr = s_gam[si];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        float a4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = 32 * hc + 4 * m + e;
+          a4[e] = (j < si) ? br * __expf(gr - s_gam[j]) * v[4 * m + e] : 0.f;
+        }
+        *reinterpret_cast<float4*>(Am + sidx(si, 32 * hc + 4 * m)) = make_float4(a4[0], a4[1], a4[2], a4[3]);
+      }
+    } else {
+      const int r = si - 64;
+      const float gr = s_gam[r];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        float p[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int j = 32 * hc + 8 * m + e;
+          p[e] = (j <= r) ? __expf(gr - s_gam[j]) * v[8 * m + e] : 0.f;
+        }
+        *reinterpret_cast<uint4*>(rec + REC_P + kmaj_chunk(64, r, 32 * hc + 8 * m)) = pack8h(p);
+      }
+    }
+  }
+  for (int i = tid; i < 64 * 16; i += kPrepThreads)
+    *reinterpret_cast<float4*>(Tm + 4 * i) = make_float4(0.f, 0.f, 0.f, 0.f);
+  __syncthreads();
+  // T = (I + A)^-1 by recursive doubling: the 8x8 diagonal blocks by forward
+  // substitution, then for block size b = 8, 16, 32 every pair of b-blocks on
+  // the diagonal is joined into a 2b-block through its lower-left block
+  // T21 = -T22 (A21 T11).  T starts at zero, so the upper blocks stay zero.
+  if (tid < 64) {
+    const int bb = tid >> 3, c8 = tid & 7, o = 8 * bb;
+    float acc[8], t[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      t[k] = (k < c8) ? 0.f : (k == c8 ? 1.f : -acc[k]);
+#pragma unroll
+      for (int i = k + 1; i < 8; ++i) acc[i] += Am[sidx(o + i, o + k)] * t[k];
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) Tm[sidx(o + i, o + c8)] = t[i];
+  }
+  __syncthreads();
+  solve_level<8>(Am, Tm, sm, tid);
+  solve_level<16>(Am, Tm, sm, tid);
+  solve_level<32>(Am, Tm, sm, tid);
+  {  // T' = T diag(beta) -> record; T'' = T diag(beta e^gamma) -> shared memory over A (K-major 64 x 64)
+    const int r = tid >> 2, j0 = 16 * (tid & 3);
+    float tv[16], t1[16], t2[16];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const float4 t4 = *reinterpret_cast<const float4*>(Tm + sidx(r, j0 + 4 * m));
+      tv[4 * m] = t4.x; tv[4 * m + 1] = t4.y; tv[4 * m + 2] = t4.z; tv[4 * m + 3] = t4.w;
+    }
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) {
+      const float t = (j0 + jj <= r) ? tv[jj] : 0.f;
+      t1[jj] = t * s_tb[j0 + jj];
+      t2[jj] = t * s_tbg[j0 + jj];
+    }
+    *reinterpret_cast<uint4*>(rec + REC_T + kmaj_chunk(64, r, j0)) = pack8h(t1);
+    *reinterpret_cast<uint4*>(rec + REC_T + kmaj_chunk(64, r, j0 + 8)) = pack8h(t1 + 8);
+    st16h(sm + P_KQL + kmaj_chunk(64, r, j0), t2);
+    st16h(sm + P_KQL + kmaj_chunk(64, r, j0 + 8), t2 + 8);
+  }
+  fence_async_smem();
+  sync_tc();
+
+  // M2: W = T'' K  (M = 64; B = the k^ rows of the hi tile read as MN-major: K = 64 rows, N = 128 channels).
+  // An M = 64 accumulator puts row r in TMEM lane (r % 16) + 32 (r / 16).
+  if (tid == 0) {
+    const uint32_t ta = smem_u32(sm + P_KQL), kq = smem_u32(sm + P_KQ);
+    constexpr uint32_t id = idesc_f16(64, 128, false, true);
+#pragma unroll
+    for (int s = 0; s < 4; ++s) mma_f16(tbase, desc_kmaj(ta, 64, s), sdesc(kq + s * 2048, 16384, 1024), id, s > 0);
+    mma_commit(&mb_mma);
+  }
   if (!mbar_wait(&mb_mma, 1, kWaitNs)) bad = true;
   fence_after();
-  if (si < 64) {  // -W -> rows 0..63 of the [-W;Qg] image
+  {  // -W -> rows 0..63 of the [-W;Qg] image: lanes 0..15 of each lane quarter hold rows 16 q .. 16 q + 15
+    const int r = 16 * (warp & 3) + lane;
     float v[32];
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
-      tmem_ld32(tbase + lane_base + P_COL_W + 64 * hc + 32 * hh, v);
+      tmem_ld32(tbase + lane_base + 64 * hc + 32 * hh, v);
+      if (lane < 16) {
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) v[jj] = -v[jj];
+        for (int jj = 0; jj < 32; ++jj) v[jj] = -v[jj];
 #pragma unroll
-      for (int m = 0; m < 4; ++m)
-        *reinterpret_cast<uint4*>(rec + REC_A + kmaj_chunk(128, si, 64 * hc + 32 * hh + 8 * m)) = pack8h(v + 8 * m);
+        for (int m = 0; m < 4; ++m)
+          *reinterpret_cast<uint4*>(rec + REC_A + kmaj_chunk(128, r, 64 * hc + 32 * hh + 8 * m)) = pack8h(v + 8 * m);
+      }
     }
   }
   if (sync_tc_any(bad) && tid == 0) set_status(status, kStatusWaitTimeout);

@@ -526,11 +526,10 @@ constexpr int kChainSmem = C_MISC + 128 * 4 + 1024;
 constexpr uint32_t COL_S = 0, COL_U0 = 128, COL_Y = 384, kChainTmemCols = 512;
 
 // Roles: warps 0, 1, 4, 5 ("delta warps", TMEM lanes 0..63) move Delta to
-// shared memory and thread 0 issues the MMAs; warps 2, 3, 6, 7 ("output
-// warps", lanes 64..127) write the previous chunk's output rows meanwhile; all
-// eight update the state; warp 8 only issues the bulk copies, as soon as the
-// MMAs that read a buffer have finished, so no compute warp waits on a copy
-// being issued.
+// shared memory; warps 2, 3, 6, 7 ("output warps", lanes 64..127) write the
+// previous chunk's output rows meanwhile; all eight update the state;
+// warp 8 issues the MMAs and the bulk copies (each copy as soon as the MMAs
+// that read its buffer are done), so no compute warp stalls on an issue queue.
 __global__ void __launch_bounds__(kChainThreads, 1)
     chain_kernel(Dims d, const unsigned char* __restrict__ records, const int32_t* __restrict__ chunk_off,
                  const int32_t* __restrict__ order, const int32_t* __restrict__ cu, int zero_state,
@@ -540,7 +539,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
   __shared__ uint64_t mb_ld0;          // operands of the first MMA group, one phase per chunk
   __shared__ uint64_t mb_ld1[2];       // operands of the second, buffer cc % 2, one phase per use
   __shared__ uint64_t mb_g[2];         // gate rows, buffer cc % 2, one phase per use
-  __shared__ uint64_t mb_m3, mb_m45;   // completions of the two MMA groups, one phase per chunk each
+  __shared__ uint64_t mb_m3, mb_m5, mb_m4;  // completions of [Delta;QgS], K~^T Delta and [0;P] Delta, one phase per chunk
   __shared__ uint32_t tslot;
   bool bad = false;  // this thread saw a wait run out
 
@@ -569,7 +568,8 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     mbar_init(&mb_g[0], 1);
     mbar_init(&mb_g[1], 1);
     mbar_init(&mb_m3, 1);
-    mbar_init(&mb_m45, 1);
+    mbar_init(&mb_m5, 1);
+    mbar_init(&mb_m4, 1);
     mbar_init_fence();
   }
   if (warp == 0) tmem_alloc(&tslot, kChainTmemCols);
@@ -675,21 +675,8 @@ __global__ void __launch_bounds__(kChainThreads, 1)
   for (int c = 0; c < nchunks; ++c) {
     const uint32_t colU = COL_U0 + 128 * (c & 1);
     if (producer) {
-      if (lane == 0) {  // operands as soon as chunk c's MMA groups are done with their buffers
-        if (c + 1 < nchunks) {
-          if (!mbar_wait(&mb_m3, c & 1, kWaitNs)) bad = true;
-          issue_ld0(c + 1);
-        }
-        if (c + 2 < nchunks) {
-          if (!mbar_wait(&mb_m45, c & 1, kWaitNs)) bad = true;
-          issue_ld1(c + 2);
-        }
-        if (c + 3 < nchunks) bulk_prefetch_l2(rec_of(c + 3), REC_META + 16);  // behind the copies in the queue
-      }
-    } else {
-      const float egC = __ldg(reinterpret_cast<const float*>(rec_of(c) + REC_META));  // used by the state update
-      // U = [T';0] v^ ;  U += [-W;Qg] S  ->  [Delta ; Qg S]
-      if (tid == 0) {
+      if (lane == 0) {
+        // U = [T';0] v^ ;  U += [-W;Qg] S  ->  [Delta ; Qg S]
         if (!mbar_wait(&mb_ld0, c & 1, kWaitNs)) bad = true;
         if (!bad) {
           const uint32_t ta = smem_u32(sm + C_TA), vb = smem_u32(sm + C_V), aa = smem_u32(sm + C_A),
@@ -701,13 +688,43 @@ __global__ void __launch_bounds__(kChainThreads, 1)
           for (int s = 0; s < 8; ++s) mma_f16(tbase + colU, desc_kmaj(aa, 128, s), desc_mnmaj(sb, kD, s), id, 1);
           mma_commit(&mb_m3);
         }
+        if (c + 1 < nchunks) {  // the first MMA group is done with [-W;Qg], T' and v^
+          if (!mbar_wait(&mb_m3, c & 1, kWaitNs)) bad = true;
+          issue_ld0(c + 1);
+        }
       }
+      __syncwarp();
+      fence_before();
+      asm volatile("bar.sync 2, 160;" ::: "memory");  // Delta is in shared memory
+      fence_after();
+      if (lane == 0) {  // Y = K~^T Delta first (the state update waits for it), then O += [0;P] Delta
+        if (!mbar_wait(&mb_ld1[c & 1], (c >> 1) & 1, kWaitNs)) bad = true;
+        if (!bad) {
+          const uint32_t pa = smem_u32(sm + ((c & 1) ? C_PA1 : C_PA)), db = smem_u32(sm + C_DB),
+                         kt = smem_u32(sm + ((c & 1) ? C_KT1 : C_KT));
+          constexpr uint32_t id4 = idesc_f16(128, 128, false, true);
+          constexpr uint32_t id5 = idesc_f16(128, 128, true, true);
+#pragma unroll
+          for (int s = 0; s < 4; ++s) mma_f16(tbase + COL_Y, desc_mnmaj(kt, kC, s), desc_mnmaj(db, kC, s), id5, s > 0);
+          mma_commit(&mb_m5);
+#pragma unroll
+          for (int s = 0; s < 4; ++s) mma_f16(tbase + colU, desc_kmaj(pa, 128, s), desc_mnmaj(db, kC, s), id4, 1);
+          mma_commit(&mb_m4);
+        }
+        // [0;P] Delta is the last MMA to read P and K~'s buffer; O of chunk c is complete before the
+        // block barrier, so the output warps may read it during chunk c+1
+        if (!mbar_wait(&mb_m4, c & 1, kWaitNs)) bad = true;
+        if (c + 2 < nchunks) issue_ld1(c + 2);
+        if (c + 3 < nchunks) bulk_prefetch_l2(rec_of(c + 3), REC_META + 16);  // behind the copies in the queue
+      }
+    } else {
+      const float egC = __ldg(reinterpret_cast<const float*>(rec_of(c) + REC_META));  // used by the state update
       if (out_warp) {
         if (c > 0) {
           if (!mbar_wait(&mb_g[(c - 1) & 1], ((c - 1) >> 1) & 1, kWaitNs)) bad = true;
           epilogue(c - 1);
         }
-      } else {  // Delta -> shared (MN-major B operand); then the second MMA group
+      } else {  // Delta -> shared (MN-major B operand)
         if (!mbar_wait(&mb_m3, c & 1, kWaitNs)) bad = true;
         fence_after();
         float v[32];
@@ -719,26 +736,11 @@ __global__ void __launch_bounds__(kChainThreads, 1)
         }
         fence_async_smem();
         fence_before();
-        asm volatile("bar.sync 2, 128;" ::: "memory");
+        asm volatile("bar.sync 2, 160;" ::: "memory");
         fence_after();
-        if (tid == 0) {  // O += [0;P] Delta ;  Y = K~^T Delta
-          if (!mbar_wait(&mb_ld1[c & 1], (c >> 1) & 1, kWaitNs)) bad = true;
-          if (!bad) {
-            const uint32_t pa = smem_u32(sm + ((c & 1) ? C_PA1 : C_PA)), db = smem_u32(sm + C_DB),
-                           kt = smem_u32(sm + ((c & 1) ? C_KT1 : C_KT));
-            constexpr uint32_t id4 = idesc_f16(128, 128, false, true);
-            constexpr uint32_t id5 = idesc_f16(128, 128, true, true);
-#pragma unroll
-            for (int s = 0; s < 4; ++s) mma_f16(tbase + colU, desc_kmaj(pa, 128, s), desc_mnmaj(db, kC, s), id4, 1);
-#pragma unroll
-            for (int s = 0; s < 4; ++s)
-              mma_f16(tbase + COL_Y, desc_mnmaj(kt, kC, s), desc_mnmaj(db, kC, s), id5, s > 0);
-            mma_commit(&mb_m45);
-          }
-        }
       }
-      // neither MMA barrier can run a phase ahead: the next chunk's MMAs follow the block barrier below
-      if (!mbar_wait(&mb_m45, c & 1, kWaitNs)) bad = true;
+      // no MMA barrier can run a phase ahead: the next chunk's MMAs follow the block barrier below
+      if (!mbar_wait(&mb_m5, c & 1, kWaitNs)) bad = true;
       fence_after();
       // S = e^{gamma_C} S + K~^T Delta, and its fp16 copy for the next chunk
       float v[32], S[32];

@@ -27,17 +27,20 @@
 //
 // Record of (chunk, value head), byte images of 128-byte-swizzled operands:
 //   [  0, 32768)  [-W ; Qg]  K-major 128 x 128   (Qg = diag(e^gamma) q^)
-//   [32768, 40960) T' = T diag(beta)     K-major 64 x 64  (rows 0..63 of [T';0])
-//   [40960, 57344) v^ (from the conv)   MN-major K=64 x N=128, rows past the chunk zero
-//   [57344, 65536) P                    K-major 64 x 64  (rows 64..127 of [0;P])
-//   [65536, 81920) K~                   MN-major K=64 x M=128
-//   [81920, 98304) output gate (1 + w) sigmoid(z) (from the conv), fp16, row r at 256 r,
+//   [32768, 40960) T' = T diag(beta), hi part   K-major 64 x 64 (rows 0..63 of [T';0])
+//   [40960, 49152) T' lo part (T' - hi, fp16)
+//   [49152, 65536) v^ (from the conv)   MN-major K=64 x N=128, rows past the chunk zero
+//   [65536, 73728) P                    K-major 64 x 64  (rows 64..127 of [0;P])
+//   [73728, 90112) K~                   MN-major K=64 x M=128
+//   [90112, 106496) output gate (1 + w) sigmoid(z) (from the conv), fp16, row r at 256 r,
 //                  column half at +128, 16-byte piece q at (q ^ (r % 8)) * 16
-//   [98304, 98320) e^{gamma_C}, gamma_C (from the conv)
-//   [98320, 98832) gamma_r, beta_r of the chunk's 64 rows (from the conv; 0 past the chunk's end)
-// so the chain kernel reads each chunk in four bulk copies.
+//   [106496, 106512) e^{gamma_C}, gamma_C (from the conv)
+//   [106512, 107024) gamma_r, beta_r of the chunk's 64 rows (from the conv; 0 past the chunk's end)
 // Operands are fp16 (all bounded: normalised keys and queries, decay factors
-// <= 1), accumulation fp32, the state fp32.
+// <= 1), accumulation fp32, the state fp32.  U = T' v^ takes T' as hi + lo:
+// the rounding of T' and of v^ feed Delta directly, and over thousands of
+// tokens one of the two must be carried to fp32 accuracy to keep the state
+// within its tolerance.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -55,9 +58,9 @@ constexpr int kC = 64;
 constexpr int kD = 128;
 constexpr uint64_t kWaitNs = 2000000000ull;
 
-constexpr int kRec = 98944;
-constexpr int REC_A = 0, REC_T = 32768, REC_V = 40960, REC_P = 57344, REC_K = 65536, REC_G = 81920, REC_META = 98304,
-              REC_GAM = 98320, REC_BETA = 98576;
+constexpr int kRec = 107136;
+constexpr int REC_A = 0, REC_T = 32768, REC_TL = 40960, REC_V = 49152, REC_P = 65536, REC_K = 73728, REC_G = 90112,
+              REC_META = 106496, REC_GAM = 106512, REC_BETA = 106768;
 
 // ------------------------------------------------------------------ conv_qkv_kernel
 // Block = 4 warps = the 64 rows of one chunk for one 128-channel head slot
@@ -371,22 +374,29 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
     for (int s = 0; s < 8; ++s) mma_f16(tbase, desc_kmaj(kql, 128, s), desc_kmaj(kq, 128, s), id, 1);
     mma_commit(&mb_mma);
   }
-  // meanwhile: Qg = diag(e^gamma) q^ (hi) -> rows 64..127 of the [-W;Qg] image, K~ = diag(e^{gC-gamma}) k^ -> its image
+  // meanwhile: Qg = diag(e^gamma) q^ -> rows 64..127 of the [-W;Qg] image, K~ = diag(e^{gC-gamma}) k^ -> its
+  // image; q^ and k^ as hi + lo, so that each operand is rounded to fp16 once
   for (int e = tid; e < 64 * 16; e += kPrepThreads) {
     const int r = e >> 4, c8 = 8 * (e & 15);
-    const uint4 uq = *reinterpret_cast<const uint4*>(sm + P_KQ + kmaj_chunk(128, 64 + r, c8));
-    const uint4 uk = *reinterpret_cast<const uint4*>(sm + P_KQ + kmaj_chunk(128, r, c8));
+    const uint32_t oq = kmaj_chunk(128, 64 + r, c8), ok = kmaj_chunk(128, r, c8);
+    const uint4 uq = *reinterpret_cast<const uint4*>(sm + P_KQ + oq);
+    const uint4 uk = *reinterpret_cast<const uint4*>(sm + P_KQ + ok);
+    const uint4 lq = *reinterpret_cast<const uint4*>(sm + P_KQL + oq);
+    const uint4 lk = *reinterpret_cast<const uint4*>(sm + P_KQL + ok);
     const float eg = s_eg[r], ek = s_ekd[r];
     const __half2* hq = reinterpret_cast<const __half2*>(&uq);
     const __half2* hk = reinterpret_cast<const __half2*>(&uk);
+    const __half2* hql = reinterpret_cast<const __half2*>(&lq);
+    const __half2* hkl = reinterpret_cast<const __half2*>(&lk);
     float fq[8], fk[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const float2 a2 = __half22float2(hq[i]), b2 = __half22float2(hk[i]);
-      fq[2 * i] = a2.x * eg;
-      fq[2 * i + 1] = a2.y * eg;
-      fk[2 * i] = b2.x * ek;
-      fk[2 * i + 1] = b2.y * ek;
+      const float2 a3 = __half22float2(hql[i]), b3 = __half22float2(hkl[i]);
+      fq[2 * i] = (a2.x + a3.x) * eg;
+      fq[2 * i + 1] = (a2.y + a3.y) * eg;
+      fk[2 * i] = (b2.x + b3.x) * ek;
+      fk[2 * i + 1] = (b2.y + b3.y) * ek;
     }
     *reinterpret_cast<uint4*>(rec + REC_A + kmaj_chunk(128, 64 + r, c8)) = pack8h(fq);
     *reinterpret_cast<uint4*>(rec + REC_K + mnmaj_chunk(64, r, c8)) = pack8h(fk);
@@ -470,8 +480,13 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
       t1[jj] = t * s_tb[j0 + jj];
       t2[jj] = t * s_tbg[j0 + jj];
     }
+    float tl[16];
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) tl[jj] = t1[jj] - __half2float(__float2half_rn(t1[jj]));
     *reinterpret_cast<uint4*>(rec + REC_T + kmaj_chunk(64, r, j0)) = pack8h(t1);
     *reinterpret_cast<uint4*>(rec + REC_T + kmaj_chunk(64, r, j0 + 8)) = pack8h(t1 + 8);
+    *reinterpret_cast<uint4*>(rec + REC_TL + kmaj_chunk(64, r, j0)) = pack8h(tl);
+    *reinterpret_cast<uint4*>(rec + REC_TL + kmaj_chunk(64, r, j0 + 8)) = pack8h(tl + 8);
     st16h(sm + P_KQL + kmaj_chunk(64, r, j0), t2);
     st16h(sm + P_KQL + kmaj_chunk(64, r, j0 + 8), t2 + 8);
   }
@@ -510,17 +525,19 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
 
 // ------------------------------------------------------------------ chain_kernel
 constexpr int kChainThreads = 288;  // eight compute warps and one copy-issuing warp
+// Two 24 KB regions [X | zeros | P] hold [T'hi ; 0] and [0 ; P] of even chunks
+// (X = T' hi part) and [T'lo ; 0] and [0 ; P] of odd chunks, each pair of
+// K-major 128 x 64 tiles sharing its 8 KB of zero rows.
 constexpr int C_A = 0;          // [-W ; Qg]   K-major 128 x 128
-constexpr int C_TA = 32768;     // [T' ; 0]    K-major 128 x 64
-constexpr int C_V = 49152;      // v^          MN-major K=64 x N=128
-constexpr int C_PA = 65536;     // [0 ; P]     K-major 128 x 64      (buffer 0; buffer 1 at C_PA1)
-constexpr int C_KT = 81920;     // K~          MN-major K=64 x M=128 (buffer 0; buffer 1 at C_KT1)
-constexpr int C_DB = 98304;     // Delta       MN-major K=64 x N=128
-constexpr int C_SB = 114688;    // S (fp16)    MN-major K=128 x N=128
-constexpr int C_G = 147456;     // output gate rows, two buffers (the record's image)
-constexpr int C_O = 180224;     // output staging, 32 rows x 128 bytes per output warp (16-byte pieces swizzled)
-constexpr int C_PA1 = 196608;   // second [0 ; P] buffer
-constexpr int C_KT1 = 212992;   // second K~ buffer
+constexpr int C_R0 = 32768;     // T' hi | zeros | P (even chunks)
+constexpr int C_V = 57344;      // v^          MN-major K=64 x N=128
+constexpr int C_R1 = 73728;     // T' lo | zeros | P (odd chunks)
+constexpr int C_KT = 98304;     // K~          MN-major K=64 x M=128 (buffer 0; buffer 1 at C_KT1)
+constexpr int C_KT1 = 114688;
+constexpr int C_DB = 131072;    // Delta       MN-major K=64 x N=128
+constexpr int C_SB = 147456;    // S (fp16)    MN-major K=128 x N=128
+constexpr int C_G = 180224;     // output gate rows, two buffers (the record's image)
+constexpr int C_O = 212992;     // output staging, 32 rows x 128 bytes per output warp (16-byte pieces swizzled)
 constexpr int C_MISC = 229376;  // row sums of squares [2][64]
 constexpr int kChainSmem = C_MISC + 128 * 4 + 1024;
 constexpr uint32_t COL_S = 0, COL_U0 = 128, COL_Y = 384, kChainTmemCols = 512;
@@ -573,23 +590,25 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     mbar_init_fence();
   }
   if (warp == 0) tmem_alloc(&tslot, kChainTmemCols);
-  for (int i = tid; i < 512; i += kChainThreads) {  // constant zero halves of [T';0] and both [0;P]
-    reinterpret_cast<uint4*>(sm + C_TA + 8192)[i] = make_uint4(0, 0, 0, 0);
-    reinterpret_cast<uint4*>(sm + C_PA)[i] = make_uint4(0, 0, 0, 0);
-    reinterpret_cast<uint4*>(sm + C_PA1)[i] = make_uint4(0, 0, 0, 0);
+  for (int i = tid; i < 512; i += kChainThreads) {  // the shared zero rows of both regions
+    reinterpret_cast<uint4*>(sm + C_R0 + 8192)[i] = make_uint4(0, 0, 0, 0);
+    reinterpret_cast<uint4*>(sm + C_R1 + 8192)[i] = make_uint4(0, 0, 0, 0);
   }
 
   auto rec_of = [&](int cc) { return records + ((g0 + cc) * d.Hv + h) * (int64_t)kRec; };
-  auto issue_ld0 = [&](int cc) {  // [-W;Qg] and T' land contiguously in C_A .. C_TA + 8192; then v^
+  auto issue_ld0 = [&](int cc) {  // [-W;Qg] and T' hi land contiguously in C_A .. C_R0 + 8192; T' lo; v^
     const unsigned char* r = rec_of(cc);
-    mbar_expect_tx(&mb_ld0, 40960 + 16384);
+    mbar_expect_tx(&mb_ld0, 40960 + 8192 + 16384);
     bulk_load(sm + C_A, r + REC_A, 40960, &mb_ld0);
+    bulk_load(sm + C_R1, r + REC_TL, 8192, &mb_ld0);
     bulk_load(sm + C_V, r + REC_V, 16384, &mb_ld0);
   };
-  auto issue_ld1 = [&](int cc) {  // P and K~ land contiguously in [0;P] + 8192 .. K~ + 16384 of buffer cc % 2
+  auto issue_ld1 = [&](int cc) {  // P into region cc % 2, K~ into buffer cc % 2
     uint64_t* mb = &mb_ld1[cc & 1];
+    const unsigned char* r = rec_of(cc);
     mbar_expect_tx(mb, 8192 + 16384);
-    bulk_load(sm + ((cc & 1) ? C_PA1 : C_PA) + 8192, rec_of(cc) + REC_P, 8192 + 16384, mb);
+    bulk_load(sm + ((cc & 1) ? C_R1 : C_R0) + 16384, r + REC_P, 8192, mb);
+    bulk_load(sm + ((cc & 1) ? C_KT1 : C_KT), r + REC_K, 16384, mb);
   };
   auto issue_gate = [&](int cc) {
     mbar_expect_tx(&mb_g[cc & 1], 16384);
@@ -676,14 +695,16 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     const uint32_t colU = COL_U0 + 128 * (c & 1);
     if (producer) {
       if (lane == 0) {
-        // U = [T';0] v^ ;  U += [-W;Qg] S  ->  [Delta ; Qg S]
+        // U = [T'hi;0] v^ + [T'lo;0] v^ ;  U += [-W;Qg] S  ->  [Delta ; Qg S]
         if (!mbar_wait(&mb_ld0, c & 1, kWaitNs)) bad = true;
         if (!bad) {
-          const uint32_t ta = smem_u32(sm + C_TA), vb = smem_u32(sm + C_V), aa = smem_u32(sm + C_A),
-                         sb = smem_u32(sm + C_SB);
+          const uint32_t th = smem_u32(sm + C_R0), tl = smem_u32(sm + C_R1), vb = smem_u32(sm + C_V),
+                         aa = smem_u32(sm + C_A), sb = smem_u32(sm + C_SB);
           constexpr uint32_t id = idesc_f16(128, 128, false, true);
 #pragma unroll
-          for (int s = 0; s < 4; ++s) mma_f16(tbase + colU, desc_kmaj(ta, 128, s), desc_mnmaj(vb, kC, s), id, s > 0);
+          for (int s = 0; s < 4; ++s) mma_f16(tbase + colU, desc_kmaj(th, 128, s), desc_mnmaj(vb, kC, s), id, s > 0);
+#pragma unroll
+          for (int s = 0; s < 4; ++s) mma_f16(tbase + colU, desc_kmaj(tl, 128, s), desc_mnmaj(vb, kC, s), id, 1);
 #pragma unroll
           for (int s = 0; s < 8; ++s) mma_f16(tbase + colU, desc_kmaj(aa, 128, s), desc_mnmaj(sb, kD, s), id, 1);
           mma_commit(&mb_m3);
@@ -700,7 +721,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
       if (lane == 0) {  // Y = K~^T Delta first (the state update waits for it), then O += [0;P] Delta
         if (!mbar_wait(&mb_ld1[c & 1], (c >> 1) & 1, kWaitNs)) bad = true;
         if (!bad) {
-          const uint32_t pa = smem_u32(sm + ((c & 1) ? C_PA1 : C_PA)), db = smem_u32(sm + C_DB),
+          const uint32_t pa = smem_u32(sm + ((c & 1) ? C_R1 : C_R0) + 8192), db = smem_u32(sm + C_DB),
                          kt = smem_u32(sm + ((c & 1) ? C_KT1 : C_KT));
           constexpr uint32_t id4 = idesc_f16(128, 128, false, true);
           constexpr uint32_t id5 = idesc_f16(128, 128, true, true);

@@ -63,12 +63,13 @@ constexpr int REC_A = 0, REC_T = 32768, REC_TL = 40960, REC_V = 49152, REC_P = 6
               REC_META = 106496, REC_GAM = 106512, REC_BETA = 106768;
 
 // ------------------------------------------------------------------ conv_qkv_kernel
-// Block = 4 warps = the 64 rows of one chunk for one 128-channel head slot
+// Block = 8 warps = the 64 rows of one chunk for one 128-channel head slot
 // (q heads, then k heads, then v heads, then the output gates of the v
-// heads).  Warp w owns rows 16w .. 16w+15, lane l owns channels 4l .. 4l+3.
-// A fifth warp computes the chunk's gates g, beta of the value head in the
+// heads).  Warp w owns rows 8w .. 8w+7, lane l owns channels 4l .. 4l+3.
+// A ninth warp computes the chunk's gates g, beta of the value head in the
 // output-gate slots and exits in the others.
-constexpr int kConvRows = 16;
+constexpr int kConvRows = 8;
+constexpr int kConvGateWarp = 64 / kConvRows;
 
 // Slots past the q/k/v heads compute the output gate of one value head,
 // (1 + w_j) sigmoid(z_j), which depends on no other stage of the mixer.
@@ -131,7 +132,7 @@ __device__ __forceinline__ void chunk_gates(const Dims& d, const float* __restri
   if (lane == 0) reinterpret_cast<float2*>(rec + REC_META)[0] = make_float2(expf(gC), gC);
 }
 
-constexpr int kConvThreads = 160;
+constexpr int kConvThreads = 32 * (kConvGateWarp + 1);
 
 __global__ void __launch_bounds__(kConvThreads)
     conv_qkv_kernel(Dims d, const float* __restrict__ conv_w, const __nv_bfloat16* __restrict__ qkv,
@@ -151,11 +152,11 @@ __global__ void __launch_bounds__(kConvThreads)
   if (slot >= nqk + d.Hv) {
     const int hz = slot - nqk - d.Hv;
     unsigned char* rec = records + ((int64_t)g * d.Hv + hz) * kRec;
-    if (warp == 4) chunk_gates(d, A_log, dt_bias, a, b, cm.y, L, hz, lane, rec);
+    if (warp == kConvGateWarp) chunk_gates(d, A_log, dt_bias, a, b, cm.y, L, hz, lane, rec);
     else if (r0 < L) gate_rows(d, norm_w, z, rec + REC_G, cm.y, r0, L, hz, lane);
     return;
   }
-  if (warp == 4) return;
+  if (warp == kConvGateWarp) return;
   // v^ goes straight into the record of (chunk, value head) as the chain kernel's operand image
   unsigned char* vrec = slot >= nqk ? records + ((int64_t)g * d.Hv + (slot - nqk)) * kRec + REC_V : nullptr;
   if (vrec) {
@@ -174,24 +175,24 @@ __global__ void __launch_bounds__(kConvThreads)
   }
   // raw rows r0-3 .. r0+15 of the chunk; rows before the sequence start come
   // from the conv history, rows past the chunk's end are never used
-  float x[kConvRows + 3][4];
+  uint2 xr[kConvRows + 3];  // raw bf16 pairs, unpacked where used
   const bool first = cm.w == 0;
 #pragma unroll
   for (int i = 0; i < kConvRows + 3; ++i) {
     const int rr = r0 - 3 + i;
-    uint2 u = make_uint2(0u, 0u);
+    xr[i] = make_uint2(0u, 0u);
     if (rr < L) {
       if (first && rr < 0) {
-        if (!zero_conv) u = *reinterpret_cast<const uint2*>(hist + ((int64_t)cm.x * 3 + (3 + rr)) * C + c);
+        if (!zero_conv) xr[i] = *reinterpret_cast<const uint2*>(hist + ((int64_t)cm.x * 3 + (3 + rr)) * C + c);
       } else {
-        u = __ldg(reinterpret_cast<const uint2*>(qkv + ((int64_t)cm.y + rr) * C + c));
+        xr[i] = __ldg(reinterpret_cast<const uint2*>(qkv + ((int64_t)cm.y + rr) * C + c));
       }
     }
-    x[i][0] = __uint_as_float(u.x << 16);
-    x[i][1] = __uint_as_float(u.x & 0xffff0000u);
-    x[i][2] = __uint_as_float(u.y << 16);
-    x[i][3] = __uint_as_float(u.y & 0xffff0000u);
   }
+  auto xf = [&](int i, int e) {
+    const uint32_t u = (e < 2) ? xr[i].x : xr[i].y;
+    return __uint_as_float((e & 1) ? (u & 0xffff0000u) : (u << 16));
+  };
   float y[kConvRows][4];
 #pragma unroll
   for (int i = 0; i < kConvRows; ++i)
@@ -199,7 +200,7 @@ __global__ void __launch_bounds__(kConvThreads)
     for (int e = 0; e < 4; ++e) {
       float acc = 0.f;
 #pragma unroll
-      for (int tap = 0; tap < 4; ++tap) acc += w[e][tap] * x[i + tap][e];
+      for (int tap = 0; tap < 4; ++tap) acc += w[e][tap] * xf(i + tap, e);
       y[i][e] = silu_fast(acc);
     }
   if (slot < nqk) {  // q or k: L2 norm over the head's 128 channels, then hi + lo fp16 parts

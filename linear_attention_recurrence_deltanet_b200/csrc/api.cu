@@ -422,17 +422,19 @@ gdn_status gdn_prefill(const gdn_config* cfg, const gdn_params* params, const vo
   const gdn::ScheduleLayout L = gdn::schedule_layout(num_seqs, chunks);
   cudaError_t e = cudaSuccess;
   const int32_t* order = nullptr;
-  if (num_seqs > 1 || split) {
+  if (num_seqs > 1) {  // one sequence needs neither an order nor a chunk map
     e = gdn::launch_schedule(cu_seqlens_dev, num_seqs, chunk_size, chunks, workspace, st);
-    if (num_seqs > 1) order = (const int32_t*)((const char*)workspace + L.order_off);
+    order = (const int32_t*)((const char*)workspace + L.order_off);
   }
   const bool chunked = !(flags & GDN_PREFILL_RECURRENT) && gdn::prefill_chunked_supported(d, bf16, chunk_size);
   if (e == cudaSuccess && split) {
     // intermediates start after the schedule sized for the chunk bound (the layout the size query assumed)
     const size_t sched = gdn::schedule_layout(num_seqs, chunk_bound(total, num_seqs, chunk_size)).total_bytes;
     e = gdn::launch_prefill_split(d, params->conv_w, params->A_log, params->dt_bias, params->norm_w, qkv, z, a, b,
-                                  cu_seqlens_dev, order, (const int32_t*)((const char*)workspace + L.chunk_off_off),
-                                  (const int4*)((const char*)workspace + L.chunk_map_off), num_seqs, total, chunks,
+                                  cu_seqlens_dev, order,
+                                  num_seqs > 1 ? (const int32_t*)((const char*)workspace + L.chunk_off_off) : nullptr,
+                                  num_seqs > 1 ? (const int4*)((const char*)workspace + L.chunk_map_off) : nullptr,
+                                  num_seqs, total, chunks,
                                   zero_state, zero_conv, conv_state, state, o, (char*)workspace + sched,
                                   g_status_ptr[dev], st);
   } else if (e == cudaSuccess && chunked)
@@ -443,7 +445,12 @@ gdn_status gdn_prefill(const gdn_config* cfg, const gdn_params* params, const vo
     e = gdn::launch_prefill_recurrent(d, bf16, params->conv_w, params->A_log, params->dt_bias, params->norm_w, qkv,
                                       z, a, b, cu_seqlens_dev, order, num_seqs, zero_state, zero_conv, conv_state,
                                       state, o, st);
-  if (e == cudaSuccess) e = gdn::launch_conv_history(d, bf16, qkv, cu_seqlens_dev, num_seqs, zero_conv, conv_state, st);
+  // The three-kernel path writes each non-empty sequence's new history in its prep kernel; an empty
+  // sequence keeps its history unless the history is to start from zeros.
+  bool empty_zeroed = false;
+  for (int32_t n = 0; n < num_seqs && zero_conv; ++n) empty_zeroed |= cu_seqlens_host[n + 1] == cu_seqlens_host[n];
+  if (e == cudaSuccess && (!split || empty_zeroed))
+    e = gdn::launch_conv_history(d, bf16, qkv, cu_seqlens_dev, num_seqs, zero_conv, conv_state, st);
   return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_prefill launch");
 }
 

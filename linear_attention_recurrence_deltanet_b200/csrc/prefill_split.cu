@@ -140,10 +140,13 @@ __global__ void __launch_bounds__(kConvThreads)
                     const float* __restrict__ norm_w, const __nv_bfloat16* __restrict__ z,
                     const float* __restrict__ A_log, const float* __restrict__ dt_bias,
                     const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
-                    __half* __restrict__ qk_hi, __half* __restrict__ qk_lo, unsigned char* __restrict__ records) {
+                    __half* __restrict__ qk_hi, __half* __restrict__ qk_lo, unsigned char* __restrict__ records,
+                    int64_t single_len) {
   // chunks in reverse order: the first chunks' outputs are the freshest in L2 when the chain starts
   const int g = gridDim.x - 1 - blockIdx.x;
-  const int4 cm = chunk_map[g];  // {seq, first token, length, chunk index}
+  // {seq, first token, length, chunk index}; one sequence needs no map
+  const int64_t rest = single_len - (int64_t)kC * g;
+  const int4 cm = chunk_map ? chunk_map[g] : make_int4(0, kC * g, rest < kC ? (int)rest : kC, g);
   const int slot = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r0 = kConvRows * warp;
@@ -260,6 +263,34 @@ __device__ __forceinline__ float* yrow(unsigned char* sm, int row) {
   return reinterpret_cast<float*>(sm + P_KQ + (row < 32 ? 8192 : 24576)) + (row & 31) * 64;
 }
 
+// The new conv history of sequence n: the last W-1 raw rows of [history ;
+// inputs].  The prep block of the sequence's last chunk and value head h owns
+// the v channels of h and, for the first value head of a key head, the q and
+// k channels of that key head (nothing reads the old history after the conv
+// kernel).  One thread per 16 bytes of channels reads its three rows before
+// writing them.
+__device__ __forceinline__ void write_history(const Dims& d, int h, int n, int64_t seq0, int len,
+                                           const __nv_bfloat16* __restrict__ qkv, int zero_conv,
+                                           __nv_bfloat16* __restrict__ hist) {
+  const int G = d.G, kh = h / G;
+  const int nvec = (h % G == 0 ? 3 : 1) * (kD / 8);
+  for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
+    const int part = i / (kD / 8), c8 = 8 * (i % (kD / 8));
+    const int64_t ch = part == 0 ? 2LL * d.Hk * kD + (int64_t)h * kD + c8
+                                 : (part == 1 ? (int64_t)kh * kD + c8 : (int64_t)d.Hk * kD + (int64_t)kh * kD + c8);
+    uint4 v[3];
+#pragma unroll
+    for (int r = 0; r < 3; ++r) {
+      const int m = len + r - 3;
+      v[r] = m >= 0 ? *reinterpret_cast<const uint4*>(qkv + (seq0 + m) * d.C + ch)
+                    : (zero_conv ? make_uint4(0, 0, 0, 0)
+                                 : *reinterpret_cast<const uint4*>(hist + ((int64_t)n * 3 + (m + 3)) * d.C + ch));
+    }
+#pragma unroll
+    for (int r = 0; r < 3; ++r) *reinterpret_cast<uint4*>(hist + ((int64_t)n * 3 + r) * d.C + ch) = v[r];
+  }
+}
+
 // One doubling level of T = (I + A)^-1: for every pair of B x B diagonal
 // blocks at offset o = 2 B p, Y = A21 T11, then T21 = -T22 Y.  Four columns
 // per work item.
@@ -300,7 +331,9 @@ __device__ __forceinline__ void solve_level(const float* __restrict__ Am, float*
 
 __global__ void __launch_bounds__(kPrepThreads, 3)
     prep_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constant__ CUtensorMap tm_lo, Dims d,
-                const int4* __restrict__ chunk_map, unsigned char* __restrict__ records, int32_t* status) {
+                const int4* __restrict__ chunk_map, unsigned char* __restrict__ records, const int32_t* __restrict__ cu,
+                const __nv_bfloat16* __restrict__ qkv, int zero_conv, __nv_bfloat16* __restrict__ hist,
+                int64_t single_len, int32_t* status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   __shared__ uint64_t mb_tma, mb_mma;
@@ -312,7 +345,12 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
   const int h = blockIdx.x - gr * d.Hv;
   const int g = gridDim.x / d.Hv - 1 - gr;
   const int kh = h / d.G;
-  const int64_t t0 = chunk_map[g].y;  // rows past the chunk's end carry beta = 0 (their gates are zero)
+  const int4 cm = chunk_map ? chunk_map[g] : make_int4(0, kC * g, 0, g);
+  const int64_t t0 = cm.y;  // rows past the chunk's end carry beta = 0 (their gates are zero)
+  {  // the block of a sequence's last chunk writes the sequence's new conv history for its channels
+    const int64_t s0 = chunk_map ? cu[cm.x] : 0, s1 = chunk_map ? cu[cm.x + 1] : single_len;
+    if (t0 + kC >= s1) write_history(d, h, cm.x, s0, (int)(s1 - s0), qkv, zero_conv, hist);
+  }
   unsigned char* rec = records + ((int64_t)g * d.Hv + h) * kRec;
 
   float* misc = reinterpret_cast<float*>(sm + P_MISC);
@@ -569,7 +607,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
   const int len = cu[n + 1] - cu[n];
   if (len <= 0) return;
   const int nchunks = (len + kC - 1) / kC;
-  const int64_t g0 = chunk_off[n];
+  const int64_t g0 = chunk_off ? chunk_off[n] : 0;
   const int64_t HvD = (int64_t)d.Hv * kD;
   float* s_rms = reinterpret_cast<float*>(sm + C_MISC);  // [2][64]
   const bool producer = warp == 8;
@@ -853,7 +891,7 @@ cudaError_t launch_prefill_split(const Dims& d, const float* conv_w, const float
     conv_qkv_kernel<<<dim3((unsigned)total_chunks, (unsigned)(2 * d.Hk + 2 * d.Hv)), kConvThreads, 0, stream>>>(
         d, conv_w, (const __nv_bfloat16*)qkv, (const __nv_bfloat16*)conv_state, zero_conv ? 1 : 0, chunk_map, norm_w,
         (const __nv_bfloat16*)z, A_log, dt_bias, (const __nv_bfloat16*)a, (const __nv_bfloat16*)b, qk_hi, qk_lo,
-        records);
+        records, total_tokens);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if ((e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrepSmem)) != cudaSuccess)
@@ -861,7 +899,8 @@ cudaError_t launch_prefill_split(const Dims& d, const float* conv_w, const float
   {
     LaunchScope scope(GDN_K_SPLIT_PREP, stream);
     prep_kernel<<<(unsigned)(total_chunks * d.Hv), kPrepThreads, kPrepSmem, stream>>>(
-        tm_hi, tm_lo, d, chunk_map, records, status);
+        tm_hi, tm_lo, d, chunk_map, records, cu, (const __nv_bfloat16*)qkv, zero_conv ? 1 : 0,
+        (__nv_bfloat16*)const_cast<void*>(conv_state), total_tokens, status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if ((e = cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kChainSmem)) != cudaSuccess)

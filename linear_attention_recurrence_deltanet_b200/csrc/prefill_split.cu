@@ -253,7 +253,8 @@ constexpr int kPrepThreads = 256;
 constexpr int P_KQ = 0;
 constexpr int P_KQL = 32768;
 constexpr int P_MISC = 65536;
-constexpr int kPrepSmem = P_MISC + 64 * 6 * 4 + 1024;
+constexpr int P_GATES = P_MISC + 64 * 6 * 4;  // the record's e^{gamma_C}, gamma_C, gamma_r, beta_r (528 bytes)
+constexpr int kPrepSmem = P_GATES + 528 + 1024;
 constexpr uint32_t kPrepTmemCols = 128;
 
 __device__ __forceinline__ int sidx(int row, int col) { return row * 64 + ((((col >> 2) ^ (row & 15))) << 2) + (col & 3); }
@@ -363,16 +364,12 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
   float* Am = reinterpret_cast<float*>(sm + P_KQL);
   float* Tm = Am + 64 * 64;
 
-  if (tid == 0) {
+  if (tid == 0) {  // the copies go out before anything else
     mbar_init(&mb_tma, 1);
     mbar_init(&mb_mma, 1);
     mbar_init_fence();
-  }
-  if (warp == 0) tmem_alloc(&tslot, kPrepTmemCols);
-  sync_tc();
-  const uint32_t tbase = tslot;
-  if (tid == 0) {
-    mbar_expect_tx(&mb_tma, 8 * 8192);
+    mbar_expect_tx(&mb_tma, 8 * 8192 + 528);
+    bulk_load(sm + P_GATES, rec + REC_META, 528, &mb_tma);
     const int qx = kh * kD, kx = d.Hk * kD + kh * kD;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -382,10 +379,15 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
       tma_load_2d(sm + P_KQL + j * 16384 + 8192, &tm_lo, qx + 64 * j, (int)t0, &mb_tma);
     }
   }
-  if (tid < 64) {  // the chunk's gates (computed by the conv kernel) and their exponentials
-    const float gam = reinterpret_cast<const float*>(rec + REC_GAM)[tid];
-    const float be = reinterpret_cast<const float*>(rec + REC_BETA)[tid];
-    const float gC = reinterpret_cast<const float*>(rec + REC_META)[1];
+  if (warp == 0) tmem_alloc(&tslot, kPrepTmemCols);
+  sync_tc();
+  const uint32_t tbase = tslot;
+  if (!mbar_wait(&mb_tma, 0, kWaitNs)) bad = true;
+  if (tid < 64) {  // the chunk's gates (computed by the conv kernel, copied in with the tiles) and exponentials
+    const float* gr = reinterpret_cast<const float*>(sm + P_GATES);
+    const float gam = gr[(REC_GAM - REC_META) / 4 + tid];
+    const float be = gr[(REC_BETA - REC_META) / 4 + tid];
+    const float gC = gr[1];
     const float eg = expf(gam);
     s_gam[tid] = gam;
     s_beta[tid] = be;
@@ -394,7 +396,6 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
     s_tb[tid] = be;
     s_tbg[tid] = be * eg;
   }
-  if (!mbar_wait(&mb_tma, 0, kWaitNs)) bad = true;
   if (sync_tc_any(bad)) {
     if (tid == 0) set_status(status, kStatusWaitTimeout);
     if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);

@@ -16,31 +16,36 @@
 //                     q^, k^ as fp16 hi + lo parts, v^ as fp16; and the output
 //                     gate (1 + w) sigmoid(z) of every value head, fp16.
 //   prep_kernel       grid (chunk, value head): gates, [K;Q]K^T in split
-//                     precision on tcgen05, A and P, T = (I+A)^-1, W on tcgen05;
-//                     writes one record per (chunk, value head) whose parts are
-//                     byte images of the chain kernel's shared-memory operands.
-//   chain_kernel      grid (sequence, value head): per chunk, U = T' V^ and
-//                     [Delta; Qg S] on tcgen05, then [0;P] Delta and K~^T Delta,
-//                     then the state update; the output rows of chunk c (RMSNorm
-//                     times the gate) are written by half of the warps while the
-//                     other half carries chunk c+1 to its second MMA group.
+//                     precision on tcgen05, A and P, T = (I+A)^-1, then W = T''K
+//                     and U = T'v^ on tcgen05; writes one record per (chunk,
+//                     value head) whose parts are byte images of the chain
+//                     kernel's shared-memory operands.
+//   chain_kernel      grid (sequence, value head, value-channel half), clusters
+//                     of the two halves: per chunk, [-W;Qg] S on tcgen05, Delta =
+//                     U - W S, then K~^T Delta and [0;P] Delta, then the state
+//                     update, each CTA for 64 of the 128 value channels (the
+//                     columns of the state are independent); the output rows of
+//                     chunk c (RMSNorm times the gate, the row sums of squares
+//                     exchanged through distributed shared memory) are written
+//                     by half of the warps while the other half carries chunk
+//                     c+1 to its second MMA group.
 //
 // Record of (chunk, value head), byte images of 128-byte-swizzled operands:
-//   [  0, 32768)  [-W ; Qg]  K-major 128 x 128   (Qg = diag(e^gamma) q^)
-//   [32768, 40960) T' = T diag(beta), hi part   K-major 64 x 64 (rows 0..63 of [T';0])
-//   [40960, 49152) T' lo part (T' - hi, fp16)
-//   [49152, 65536) v^ (from the conv)   MN-major K=64 x N=128, rows past the chunk zero
-//   [65536, 73728) P                    K-major 64 x 64  (rows 64..127 of [0;P])
-//   [73728, 90112) K~                   MN-major K=64 x M=128
-//   [90112, 106496) output gate (1 + w) sigmoid(z) (from the conv), fp16, row r at 256 r,
-//                  column half at +128, 16-byte piece q at (q ^ (r % 8)) * 16
-//   [106496, 106512) e^{gamma_C}, gamma_C (from the conv)
-//   [106512, 107024) gamma_r, beta_r of the chunk's 64 rows (from the conv; 0 past the chunk's end)
+//   [     0,  32768) [-W ; Qg]  K-major 128 x 128   (Qg = diag(e^gamma) q^)
+//   [ 32768,  65536) U = T' v^, fp32: channel half at 16384 half, row r at +256 r,
+//                   16-byte piece j of the half row at (j ^ (r % 8)) * 16
+//   [ 65536,  81920) v^ (from the conv)   MN-major K=64 x N=128, rows past the chunk zero
+//   [ 81920,  90112) P                    K-major 64 x 64  (rows 64..127 of [0;P])
+//   [ 90112, 106496) K~                   MN-major K=64 x M=128
+//   [106496, 122880) output gate (1 + w) sigmoid(z) (from the conv), fp16: column half
+//                   at 8192 half, row r at +128 r, 16-byte piece q at (q ^ (r % 8)) * 16
+//   [122880, 122896) e^{gamma_C}, gamma_C (from the conv)
+//   [122896, 123408) gamma_r, beta_r of the chunk's 64 rows (from the conv; 0 past the chunk's end)
 // Operands are fp16 (all bounded: normalised keys and queries, decay factors
-// <= 1), accumulation fp32, the state fp32.  U = T' v^ takes T' as hi + lo:
-// the rounding of T' and of v^ feed Delta directly, and over thousands of
-// tokens one of the two must be carried to fp32 accuracy to keep the state
-// within its tolerance.
+// <= 1), accumulation fp32, the state fp32.  U = T' v^ takes T' as hi + lo and
+// is stored in fp32: the rounding of T' and of v^ feed Delta directly, and over
+// thousands of tokens one of the two must be carried to fp32 accuracy to keep
+// the state within its tolerance.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -58,9 +63,9 @@ constexpr int kC = 64;
 constexpr int kD = 128;
 constexpr uint64_t kWaitNs = 2000000000ull;
 
-constexpr int kRec = 107136;
-constexpr int REC_A = 0, REC_T = 32768, REC_TL = 40960, REC_V = 49152, REC_P = 65536, REC_K = 73728, REC_G = 90112,
-              REC_META = 106496, REC_GAM = 106512, REC_BETA = 106768;
+constexpr int kRec = 123520;  // a multiple of 128 bytes
+constexpr int REC_A = 0, REC_U = 32768, REC_V = 65536, REC_P = 81920, REC_K = 90112, REC_G = 106496,
+              REC_META = 122880, REC_GAM = 122896, REC_BETA = 123152;
 
 // ------------------------------------------------------------------ conv_qkv_kernel
 // Block = 8 warps = the 64 rows of one chunk for one 128-channel head slot
@@ -94,7 +99,7 @@ __device__ __forceinline__ void gate_rows(const Dims& d, const float* __restrict
 #pragma unroll
       for (int e = 0; e < 4; ++e) g[e] = nw[e] * __fdividef(1.0f, 1.0f + __expf(-zz[e]));
       const int r = r0 + i;
-      st8(grec + r * 256 + hcol * 128 + ((q ^ (r & 7)) << 4) + (lane & 1) * 8, g[0], g[1], g[2], g[3]);
+      st8(grec + hcol * 8192 + r * 128 + ((q ^ (r & 7)) << 4) + (lane & 1) * 8, g[0], g[1], g[2], g[3]);
     }
   }
 }
@@ -245,10 +250,12 @@ __global__ void __launch_bounds__(kConvThreads)
 //          the q^ halves of the two 64-column blocks hold the solve's Y rows
 //          0..31 and 32..63.
 //   P_KQL  [k^ ; q^] lo parts.  After M1: the solve scratch A (16 KB) and T
-//          (16 KB); after the solve, T'' (K-major 64 x 64) over A.
+//          (16 KB); after the solve, T'' and T' hi (K-major 64 x 64) over A and
+//          T' lo over T.  After the solve v^ (MN-major, its two 64-channel
+//          blocks 16 KB apart) lands in the q^ halves of the hi tile.
 // fp32 scratch rows are 64 floats with the 16-byte pieces of row r XORed by
 // r % 16, so that column accesses from 16 rows hit distinct banks.
-// TMEM: 128 columns; [K;Q]K^T in columns 0..63, then W (an M = 64 MMA) in 0..127.
+// TMEM: 128 columns; [K;Q]K^T in columns 0..63, then W and then U (M = 64 MMAs) in 0..127.
 constexpr int kPrepThreads = 256;
 constexpr int P_KQ = 0;
 constexpr int P_KQL = 32768;
@@ -337,7 +344,7 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
                 int64_t single_len, int32_t* status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  __shared__ uint64_t mb_tma, mb_mma;
+  __shared__ uint64_t mb_tma, mb_mma, mb_v;
   __shared__ uint32_t tslot;
   bool bad = false;  // this thread saw a wait run out
 
@@ -367,6 +374,7 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
   if (tid == 0) {  // the copies go out before anything else
     mbar_init(&mb_tma, 1);
     mbar_init(&mb_mma, 1);
+    mbar_init(&mb_v, 1);
     mbar_init_fence();
     mbar_expect_tx(&mb_tma, 8 * 8192 + 528);
     bulk_load(sm + P_GATES, rec + REC_META, 528, &mb_tma);
@@ -506,7 +514,15 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
   solve_level<8>(Am, Tm, sm, tid);
   solve_level<16>(Am, Tm, sm, tid);
   solve_level<32>(Am, Tm, sm, tid);
-  {  // T' = T diag(beta) -> record; T'' = T diag(beta e^gamma) -> shared memory over A (K-major 64 x 64)
+  // the Y rows are read: v^ comes into the q^ halves of the hi tile while T' and W are formed
+  if (tid == 0) {
+    fence_async_smem();
+    mbar_expect_tx(&mb_v, 16384);
+    bulk_load(sm + P_KQ + 8192, rec + REC_V, 8192, &mb_v);
+    bulk_load(sm + P_KQ + 24576, rec + REC_V + 8192, 8192, &mb_v);
+  }
+  {  // T' = T diag(beta) as fp16 hi + lo and T'' = T diag(beta e^gamma), K-major 64 x 64 A operands of
+     // U = T' v^ and W = T'' K: T'' and T' hi over A, T' lo over T once every thread has read its rows of T
     const int r = tid >> 2, j0 = 16 * (tid & 3);
     float tv[16], t1[16], t2[16];
 #pragma unroll
@@ -520,15 +536,15 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
       t1[jj] = t * s_tb[j0 + jj];
       t2[jj] = t * s_tbg[j0 + jj];
     }
-    float tl[16];
-#pragma unroll
-    for (int jj = 0; jj < 16; ++jj) tl[jj] = t1[jj] - __half2float(__float2half_rn(t1[jj]));
-    *reinterpret_cast<uint4*>(rec + REC_T + kmaj_chunk(64, r, j0)) = pack8h(t1);
-    *reinterpret_cast<uint4*>(rec + REC_T + kmaj_chunk(64, r, j0 + 8)) = pack8h(t1 + 8);
-    *reinterpret_cast<uint4*>(rec + REC_TL + kmaj_chunk(64, r, j0)) = pack8h(tl);
-    *reinterpret_cast<uint4*>(rec + REC_TL + kmaj_chunk(64, r, j0 + 8)) = pack8h(tl + 8);
     st16h(sm + P_KQL + kmaj_chunk(64, r, j0), t2);
     st16h(sm + P_KQL + kmaj_chunk(64, r, j0 + 8), t2 + 8);
+    st16h(sm + P_KQL + 8192 + kmaj_chunk(64, r, j0), t1);
+    st16h(sm + P_KQL + 8192 + kmaj_chunk(64, r, j0 + 8), t1 + 8);
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) t1[jj] -= __half2float(__float2half_rn(t1[jj]));
+    __syncthreads();
+    st16h(sm + P_KQL + 16384 + kmaj_chunk(64, r, j0), t1);
+    st16h(sm + P_KQL + 16384 + kmaj_chunk(64, r, j0 + 8), t1 + 8);
   }
   fence_async_smem();
   sync_tc();
@@ -544,8 +560,8 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
   }
   if (!mbar_wait(&mb_mma, 1, kWaitNs)) bad = true;
   fence_after();
-  {  // -W -> rows 0..63 of the [-W;Qg] image: lanes 0..15 of each lane quarter hold rows 16 q .. 16 q + 15
-    const int r = 16 * (warp & 3) + lane;
+  const int r16 = 16 * (warp & 3) + lane;  // lanes 0..15 of each lane quarter hold rows 16 q .. 16 q + 15
+  {  // -W -> rows 0..63 of the [-W;Qg] image
     float v[32];
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
@@ -555,7 +571,40 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
         for (int jj = 0; jj < 32; ++jj) v[jj] = -v[jj];
 #pragma unroll
         for (int m = 0; m < 4; ++m)
-          *reinterpret_cast<uint4*>(rec + REC_A + kmaj_chunk(128, r, 64 * hc + 32 * hh + 8 * m)) = pack8h(v + 8 * m);
+          *reinterpret_cast<uint4*>(rec + REC_A + kmaj_chunk(128, r16, 64 * hc + 32 * hh + 8 * m)) = pack8h(v + 8 * m);
+      }
+    }
+  }
+  if (tid == 0 && !mbar_wait(&mb_v, 0, kWaitNs)) bad = true;
+  if (sync_tc_any(bad)) {  // also: W is read out, its columns take U
+    if (tid == 0) set_status(status, kStatusWaitTimeout);
+    if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
+    return;
+  }
+  // MU: U = T'hi v^ + T'lo v^  (M = 64, N = 128; v^ MN-major with its 64-channel blocks 16 KB apart)
+  if (tid == 0) {
+    const uint32_t th = smem_u32(sm + P_KQL + 8192), tl = smem_u32(sm + P_KQL + 16384), vb = smem_u32(sm + P_KQ + 8192);
+    constexpr uint32_t id = idesc_f16(64, 128, false, true);
+#pragma unroll
+    for (int s = 0; s < 4; ++s) mma_f16(tbase, desc_kmaj(th, 64, s), sdesc(vb + s * 2048, 16384, 1024), id, s > 0);
+#pragma unroll
+    for (int s = 0; s < 4; ++s) mma_f16(tbase, desc_kmaj(tl, 64, s), sdesc(vb + s * 2048, 16384, 1024), id, 1);
+    mma_commit(&mb_mma);
+  }
+  if (!mbar_wait(&mb_mma, 0, kWaitNs)) bad = true;
+  fence_after();
+  {  // U -> the record, fp32: channel half c / 64 at 16384 (c / 64), row r at 256 r, 16-byte piece j of the
+     // half row at (j ^ (r % 8)) * 16
+    float v[32];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      tmem_ld32(tbase + lane_base + 64 * hc + 32 * hh, v);
+      if (lane < 16) {
+        unsigned char* urow = rec + REC_U + 16384 * hc + 256 * r16;
+#pragma unroll
+        for (int m = 0; m < 8; ++m)
+          *reinterpret_cast<float4*>(urow + (((8 * hh + m) ^ (r16 & 7)) << 4)) =
+              make_float4(v[4 * m], v[4 * m + 1], v[4 * m + 2], v[4 * m + 3]);
       }
     }
   }
@@ -564,219 +613,239 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
 }
 
 // ------------------------------------------------------------------ chain_kernel
-constexpr int kChainThreads = 288;  // eight compute warps and one copy-issuing warp
-// Two 24 KB regions [X | zeros | P] hold [T'hi ; 0] and [0 ; P] of even chunks
-// (X = T' hi part) and [T'lo ; 0] and [0 ; P] of odd chunks, each pair of
-// K-major 128 x 64 tiles sharing its 8 KB of zero rows.
-constexpr int C_A = 0;          // [-W ; Qg]   K-major 128 x 128
-constexpr int C_R0 = 32768;     // T' hi | zeros | P (even chunks)
-constexpr int C_V = 57344;      // v^          MN-major K=64 x N=128
-constexpr int C_R1 = 73728;     // T' lo | zeros | P (odd chunks)
-constexpr int C_KT = 98304;     // K~          MN-major K=64 x M=128 (buffer 0; buffer 1 at C_KT1)
-constexpr int C_KT1 = 114688;
-constexpr int C_DB = 131072;    // Delta       MN-major K=64 x N=128
-constexpr int C_SB = 147456;    // S (fp16)    MN-major K=128 x N=128
-constexpr int C_G = 180224;     // output gate rows, two buffers (the record's image)
-constexpr int C_O = 212992;     // output staging, 32 rows x 128 bytes per output warp (16-byte pieces swizzled)
-constexpr int C_MISC = 229376;  // row sums of squares [2][64]
-constexpr int kChainSmem = C_MISC + 128 * 4 + 1024;
-constexpr uint32_t COL_S = 0, COL_U0 = 128, COL_Y = 384, kChainTmemCols = 512;
+// One cluster of two CTAs per (sequence, value head); CTA `vh` of the pair
+// carries value channels [64 vh, 64 vh + 64), i.e. 64 columns of the state,
+// which evolve independently of the other 64.  Both read the chunk's shared
+// operands ([-W;Qg], P, K~; the second read hits L2) and their own half of U
+// and of the gate rows.  Every operand buffer is doubled, so that each copy
+// goes out two chunks ahead.
+constexpr int kChainThreads = 320;  // eight compute warps, the MMA-issuing warp, the copy-issuing warp
+constexpr int C_A = 0;          // [-W ; Qg]   K-major 128 x 128; buffer cc % 2 at +32768 (cc % 2)
+constexpr int C_P = 65536;      // [0 ; P]     K-major 128 x 64 (8 KB of zero rows, then P); buffer at +16384 (cc % 2)
+constexpr int C_U = 98304;      // U half      fp32 64 x 64, the record's image; buffer at +16384 (cc % 2)
+constexpr int C_KT = 131072;    // K~          MN-major K=64 x M=128; buffer at +16384 (cc % 2)
+constexpr int C_DB = 163840;    // Delta half  MN-major K=64 x N=64
+constexpr int C_SB = 172032;    // S half (fp16) MN-major K=128 x N=64
+constexpr int C_G = 188416;     // output gate rows of this half; buffer at +8192 (cc % 2)
+constexpr int C_O = 204800;     // output staging, 32 rows x 64 bytes per output warp (16-byte pieces swizzled)
+constexpr int C_MISC = 212992;  // row sums of squares: this CTA's [2][64], the peer's [2 buffers][64]
+constexpr int kChainSmem = C_MISC + 256 * 4 + 1024;
+constexpr uint32_t COL_U0 = 0, COL_Y = 128, kChainTmemCols = 256;  // accumulators of chunk cc at COL_U0 + 64 (cc % 2)
 
-// Roles: warps 0, 1, 4, 5 ("delta warps", TMEM lanes 0..63) move Delta to
-// shared memory; warps 2, 3, 6, 7 ("output warps", lanes 64..127) write the
-// previous chunk's output rows meanwhile; all eight update the state;
-// warp 8 issues the MMAs and the bulk copies (each copy as soon as the MMAs
-// that read its buffer are done), so no compute warp stalls on an issue queue.
-__global__ void __launch_bounds__(kChainThreads, 1)
+// Roles: warps 0, 1, 4, 5 ("delta warps", TMEM lanes 0..63) form Delta = U -
+// W S and store it to shared memory; warps 2, 3, 6, 7 ("output warps", lanes
+// 64..127) write the previous chunk's output rows meanwhile; all eight carry
+// the state, thread (row i, warp w) columns 32 (w / 4) .. + 31 of row i in
+// registers.  Warp 8 issues the MMAs, warp 9 the bulk copies (each as soon as
+// the MMAs that read its buffer are done), so that neither waits for the other.
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
     chain_kernel(Dims d, const unsigned char* __restrict__ records, const int32_t* __restrict__ chunk_off,
                  const int32_t* __restrict__ order, const int32_t* __restrict__ cu, int zero_state,
                  float* __restrict__ state, __nv_bfloat16* __restrict__ o, int32_t* status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  __shared__ uint64_t mb_ld0;          // operands of the first MMA group, one phase per chunk
-  __shared__ uint64_t mb_ld1[2];       // operands of the second, buffer cc % 2, one phase per use
-  __shared__ uint64_t mb_g[2];         // gate rows, buffer cc % 2, one phase per use
-  __shared__ uint64_t mb_m3, mb_m5, mb_m4;  // completions of [Delta;QgS], K~^T Delta and [0;P] Delta, one phase per chunk
+  __shared__ uint64_t mb_a[2], mb_u[2], mb_ld1[2], mb_g[2];  // copies into buffer cc % 2, one phase per use
+  __shared__ uint64_t mb_m3, mb_m5;  // completions of [-WS;QgS] and K~^T Delta, one phase per chunk
+  __shared__ uint64_t mb_m4[2];      // completion of [0;P] Delta (O of chunk cc complete), cc % 2, one phase per use
+  __shared__ uint64_t mb_x[2];       // the peer's row sums of chunk cc arrived, cc % 2, one phase per use
   __shared__ uint32_t tslot;
   bool bad = false;  // this thread saw a wait run out
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int h = blockIdx.x % d.Hv;
-  const int oi = blockIdx.x / d.Hv;
+  const int vh = (int)cluster_ctarank();  // value-channel half
+  const int pair = blockIdx.x >> 1;
+  const int h = pair % d.Hv;
+  const int oi = pair / d.Hv;
   const int n = order ? order[oi] : oi;
   const int64_t seq0 = cu[n];
   const int len = cu[n + 1] - cu[n];
-  if (len <= 0) return;
+  if (len <= 0) return;  // both CTAs of the cluster, before any cluster barrier
   const int nchunks = (len + kC - 1) / kC;
   const int64_t g0 = chunk_off ? chunk_off[n] : 0;
   const int64_t HvD = (int64_t)d.Hv * kD;
-  float* s_rms = reinterpret_cast<float*>(sm + C_MISC);  // [2][64]
-  const bool producer = warp == 8;
-  const bool out_warp = !producer && (warp & 3) >= 2;
-  // compute warps: thread owns row si of S (d_k index) / of the accumulators, columns [64 hc, 64 hc + 64)
+  float* s_rms = reinterpret_cast<float*>(sm + C_MISC);         // [2][64], this CTA's column quarters
+  float* s_peer = reinterpret_cast<float*>(sm + C_MISC) + 128;  // [2][64], written by the peer
+  const bool compute = warp < 8, mma_warp = warp == 8, copy_warp = warp == 9;
+  const bool out_warp = compute && (warp & 3) >= 2;
+  // compute warps: thread owns row si of S (d_k index) / of the accumulators, local columns [32 hc, 32 hc + 32)
   const int si = 32 * (warp & 3) + lane, hc = (warp >> 2) & 1;
   const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+  const int c0 = 64 * vh + 32 * hc;  // first value channel of this thread's columns
   float* gst = state + ((int64_t)n * d.Hv + h) * kD * kD;  // stored [j][i]
 
   if (tid == 0) {
-    mbar_init(&mb_ld0, 1);
-    mbar_init(&mb_ld1[0], 1);
-    mbar_init(&mb_ld1[1], 1);
-    mbar_init(&mb_g[0], 1);
-    mbar_init(&mb_g[1], 1);
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&mb_a[b], 1);
+      mbar_init(&mb_u[b], 1);
+      mbar_init(&mb_ld1[b], 1);
+      mbar_init(&mb_g[b], 1);
+      mbar_init(&mb_m4[b], 1);
+      mbar_init(&mb_x[b], 1);  // one local arrival with the expected bytes; the peer's stores complete them
+    }
     mbar_init(&mb_m3, 1);
     mbar_init(&mb_m5, 1);
-    mbar_init(&mb_m4, 1);
     mbar_init_fence();
   }
   if (warp == 0) tmem_alloc(&tslot, kChainTmemCols);
-  for (int i = tid; i < 512; i += kChainThreads) {  // the shared zero rows of both regions
-    reinterpret_cast<uint4*>(sm + C_R0 + 8192)[i] = make_uint4(0, 0, 0, 0);
-    reinterpret_cast<uint4*>(sm + C_R1 + 8192)[i] = make_uint4(0, 0, 0, 0);
+  for (int i = tid; i < 512; i += kChainThreads) {  // the zero rows of both [0;P] buffers
+    reinterpret_cast<uint4*>(sm + C_P)[i] = make_uint4(0, 0, 0, 0);
+    reinterpret_cast<uint4*>(sm + C_P + 16384)[i] = make_uint4(0, 0, 0, 0);
   }
 
   auto rec_of = [&](int cc) { return records + ((g0 + cc) * d.Hv + h) * (int64_t)kRec; };
-  auto issue_ld0 = [&](int cc) {  // [-W;Qg] and T' hi land contiguously in C_A .. C_R0 + 8192; T' lo; v^
-    const unsigned char* r = rec_of(cc);
-    mbar_expect_tx(&mb_ld0, 40960 + 8192 + 16384);
-    bulk_load(sm + C_A, r + REC_A, 40960, &mb_ld0);
-    bulk_load(sm + C_R1, r + REC_TL, 8192, &mb_ld0);
-    bulk_load(sm + C_V, r + REC_V, 16384, &mb_ld0);
+  auto issue_a = [&](int cc) {
+    mbar_expect_tx(&mb_a[cc & 1], 32768);
+    bulk_load(sm + C_A + 32768 * (cc & 1), rec_of(cc) + REC_A, 32768, &mb_a[cc & 1]);
   };
-  auto issue_ld1 = [&](int cc) {  // P into region cc % 2, K~ into buffer cc % 2
+  auto issue_u = [&](int cc) {
+    mbar_expect_tx(&mb_u[cc & 1], 16384);
+    bulk_load(sm + C_U + 16384 * (cc & 1), rec_of(cc) + REC_U + 16384 * vh, 16384, &mb_u[cc & 1]);
+  };
+  auto issue_ld1 = [&](int cc) {  // P and K~
     uint64_t* mb = &mb_ld1[cc & 1];
     const unsigned char* r = rec_of(cc);
     mbar_expect_tx(mb, 8192 + 16384);
-    bulk_load(sm + ((cc & 1) ? C_R1 : C_R0) + 16384, r + REC_P, 8192, mb);
-    bulk_load(sm + ((cc & 1) ? C_KT1 : C_KT), r + REC_K, 16384, mb);
+    bulk_load(sm + C_P + 16384 * (cc & 1) + 8192, r + REC_P, 8192, mb);
+    bulk_load(sm + C_KT + 16384 * (cc & 1), r + REC_K, 16384, mb);
   };
   auto issue_gate = [&](int cc) {
-    mbar_expect_tx(&mb_g[cc & 1], 16384);
-    bulk_load(sm + C_G + (cc & 1) * 16384, rec_of(cc) + REC_G, 16384, &mb_g[cc & 1]);
+    mbar_expect_tx(&mb_g[cc & 1], 8192);
+    bulk_load(sm + C_G + (cc & 1) * 8192, rec_of(cc) + REC_G + 8192 * vh, 8192, &mb_g[cc & 1]);
   };
-  if (producer && lane == 0) {
-    issue_ld0(0);
+  auto prefetch = [&](int cc) {  // the parts this kernel reads, into L2 (one CTA of the pair)
+    bulk_prefetch_l2(rec_of(cc), REC_V);
+    bulk_prefetch_l2(rec_of(cc) + REC_P, REC_META + 16 - REC_P);
+  };
+  if (copy_warp && lane == 0) {
+    issue_a(0);
+    issue_u(0);
     issue_ld1(0);
     issue_gate(0);
-    if (nchunks > 1) issue_ld1(1);
-    if (nchunks > 2) bulk_prefetch_l2(rec_of(2), REC_META + 16);
-  }
-  sync_tc();
-  const uint32_t tbase = tslot;
-  if (!producer) {
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      float S[32];
-#pragma unroll
-      for (int jj = 0; jj < 32; ++jj) S[jj] = zero_state ? 0.f : gst[(int64_t)(64 * hc + 32 * hh + jj) * kD + si];
-      tmem_st32(tbase + lane_base + COL_S + 64 * hc + 32 * hh, S);
-#pragma unroll
-      for (int m = 0; m < 4; ++m) st16h(sm + C_SB + mnmaj_chunk(kD, si, 64 * hc + 32 * hh + 8 * m), S + 8 * m);
+    if (nchunks > 1) {
+      issue_a(1);
+      issue_u(1);
+      issue_ld1(1);
     }
+    if (nchunks > 2 && vh == 0) prefetch(2);
+  }
+  float S[32];  // this thread's part of the state, fp32
+  if (compute) {
+#pragma unroll
+    for (int jj = 0; jj < 32; ++jj) S[jj] = zero_state ? 0.f : gst[(int64_t)(c0 + jj) * kD + si];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) st16h(sm + C_SB + mnmaj_chunk(kD, si, 32 * hc + 8 * m), S + 8 * m);
   }
   fence_async_smem();
   sync_tc();
+  const uint32_t tbase = tslot;
+  cluster_sync();  // the peer's mbarriers are initialised before any arrival on them
+  const uint32_t peer = (uint32_t)(vh ^ 1);
+  const uint32_t peer_x0 = mapa_shared(smem_u32(&mb_x[0]), peer), peer_x1 = mapa_shared(smem_u32(&mb_x[1]), peer);
+  const uint32_t peer_sums = mapa_shared(smem_u32(s_peer), peer);
 
-  // Output rows of chunk cc (O in lanes 64..127 of its U buffer): zero-centred
-  // RMSNorm over d_v times the precomputed gate (1 + w) sigmoid(z), bf16 out.
-  // Output warps only; they meet at named barrier 1.
+  // Output rows of chunk cc (O in lanes 64..127 of its accumulator): zero-centred
+  // RMSNorm over all d_v channels times the precomputed gate (1 + w) sigmoid(z),
+  // bf16 out.  Each CTA holds half of a row: the two 32-column sums of squares
+  // meet at named barrier 1 (the output warps), their total goes to the peer's
+  // buffer cc % 2 by asynchronous stores that complete the transaction bytes of
+  // the peer's mbarrier, and the peer's total comes back the same way.  A buffer
+  // is rewritten only two chunks later, after the peer has sent the chunk in
+  // between, which it does after reading it.
   auto epilogue = [&](int cc) {
     const int r = si - 64;
     const int Lc = min(kC, len - cc * kC);
-    const uint32_t col = tbase + lane_base + COL_U0 + 128 * (cc & 1) + 64 * hc;
+    if (!mbar_wait(&mb_m4[cc & 1], (cc >> 1) & 1, kWaitNs)) bad = true;
+    fence_after();
+    float v[32];
+    tmem_ld32(tbase + lane_base + COL_U0 + 64 * (cc & 1) + 32 * hc, v);
     float ss = 0.f;
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      float v[32];
-      tmem_ld32(col + 32 * hh, v);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) ss += v[j] * v[j];
-    }
+    for (int j = 0; j < 32; ++j) ss += v[j] * v[j];
     s_rms[64 * hc + r] = ss;
     asm volatile("bar.sync 1, 128;" ::: "memory");
-    const float rinv = rsqrtf((s_rms[r] + s_rms[64 + r]) * (1.0f / kD) + d.norm_eps);
-    const unsigned char* grow = sm + C_G + (cc & 1) * 16384 + r * 256 + hc * 128;
-    unsigned char* stage = sm + C_O + (2 * hc + (warp & 1)) * 4096;  // this warp's 32 rows x 128 bytes
+    const float part = s_rms[r] + s_rms[64 + r];
+    if (hc == 0) {
+      st_async_f32(peer_sums + 4 * (64 * (cc & 1) + r), part, (cc & 1) ? peer_x1 : peer_x0);
+      if (r == 0) mbar_expect_tx(&mb_x[cc & 1], 64 * 4);  // the local arrival of this phase
+    }
+    if (!mbar_wait_cluster(&mb_x[cc & 1], (cc >> 1) & 1, kWaitNs)) bad = true;
+    const float rinv = rsqrtf((part + s_peer[64 * (cc & 1) + r]) * (1.0f / kD) + d.norm_eps);
+    const unsigned char* grow = sm + C_G + (cc & 1) * 8192 + r * 128;
+    unsigned char* stage = sm + C_O + (2 * hc + (warp & 1)) * 2048;  // this warp's 32 rows x 64 bytes
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {  // the row again from TMEM: fewer live registers
-      float v[32];
-      tmem_ld32(col + 32 * hh, v);
+    for (int m = 0; m < 4; ++m) {
+      const int q = 4 * hc + m;  // 16-byte piece of the gate row half
+      const uint4 gq = *reinterpret_cast<const uint4*>(grow + ((q ^ (r & 7)) << 4));
+      const __half2* g2 = reinterpret_cast<const __half2*>(&gq);
+      uint32_t ow[4];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int q = 4 * hh + m;  // 16-byte piece of the row half
-        const uint4 gq = *reinterpret_cast<const uint4*>(grow + ((q ^ (r & 7)) << 4));
-        const __half2* g2 = reinterpret_cast<const __half2*>(&gq);
-        uint32_t ow[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 gf = __half22float2(g2[e]);
-          __nv_bfloat162 pr = __floats2bfloat162_rn(v[8 * m + 2 * e] * rinv * gf.x, v[8 * m + 2 * e + 1] * rinv * gf.y);
-          ow[e] = *reinterpret_cast<uint32_t*>(&pr);
-        }
-        *reinterpret_cast<uint4*>(stage + lane * 128 + ((q ^ (lane & 7)) << 4)) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+      for (int e = 0; e < 4; ++e) {
+        const float2 gf = __half22float2(g2[e]);
+        __nv_bfloat162 pr = __floats2bfloat162_rn(v[8 * m + 2 * e] * rinv * gf.x, v[8 * m + 2 * e + 1] * rinv * gf.y);
+        ow[e] = *reinterpret_cast<uint32_t*>(&pr);
       }
+      *reinterpret_cast<uint4*>(stage + lane * 64 + ((m ^ ((lane >> 1) & 3)) << 4)) =
+          make_uint4(ow[0], ow[1], ow[2], ow[3]);
     }
     __syncwarp();
-    // eight lanes per row: each store instruction writes four whole 128-byte row halves
+    // four lanes per row: each store instruction writes eight whole 64-byte row pieces
     const int rbase = 32 * (warp & 1);
 #pragma unroll
-    for (int it = 0; it < 8; ++it) {
-      const int rr = 4 * it + (lane >> 3), q = lane & 7;
+    for (int it = 0; it < 4; ++it) {
+      const int rr = 8 * it + (lane >> 2), q = lane & 3;
       if (rbase + rr < Lc) {
-        const uint4 val = *reinterpret_cast<const uint4*>(stage + rr * 128 + ((q ^ (rr & 7)) << 4));
-        *reinterpret_cast<uint4*>(o + (seq0 + (int64_t)cc * kC + rbase + rr) * HvD + (int64_t)h * kD + 64 * hc + 8 * q) =
-            val;
+        const uint4 val = *reinterpret_cast<const uint4*>(stage + rr * 64 + ((q ^ ((rr >> 1) & 3)) << 4));
+        *reinterpret_cast<uint4*>(o + (seq0 + (int64_t)cc * kC + rbase + rr) * HvD + (int64_t)h * kD + c0 + 8 * q) = val;
       }
     }
     __syncwarp();
   };
 
   for (int c = 0; c < nchunks; ++c) {
-    const uint32_t colU = COL_U0 + 128 * (c & 1);
-    if (producer) {
-      if (lane == 0) {
-        // U = [T'hi;0] v^ + [T'lo;0] v^ ;  U += [-W;Qg] S  ->  [Delta ; Qg S]
-        if (!mbar_wait(&mb_ld0, c & 1, kWaitNs)) bad = true;
+    const uint32_t colU = COL_U0 + 64 * (c & 1);
+    const uint32_t par = (c >> 1) & 1;  // phase parity of the buffers of chunk c
+    if (mma_warp) {
+      if (lane == 0) {  // [-W;Qg] S -> [-WS ; QgS]
+        if (!mbar_wait(&mb_a[c & 1], par, kWaitNs)) bad = true;
         if (!bad) {
-          const uint32_t th = smem_u32(sm + C_R0), tl = smem_u32(sm + C_R1), vb = smem_u32(sm + C_V),
-                         aa = smem_u32(sm + C_A), sb = smem_u32(sm + C_SB);
-          constexpr uint32_t id = idesc_f16(128, 128, false, true);
+          const uint32_t aa = smem_u32(sm + C_A + 32768 * (c & 1)), sb = smem_u32(sm + C_SB);
+          constexpr uint32_t id = idesc_f16(128, 64, false, true);
 #pragma unroll
-          for (int s = 0; s < 4; ++s) mma_f16(tbase + colU, desc_kmaj(th, 128, s), desc_mnmaj(vb, kC, s), id, s > 0);
-#pragma unroll
-          for (int s = 0; s < 4; ++s) mma_f16(tbase + colU, desc_kmaj(tl, 128, s), desc_mnmaj(vb, kC, s), id, 1);
-#pragma unroll
-          for (int s = 0; s < 8; ++s) mma_f16(tbase + colU, desc_kmaj(aa, 128, s), desc_mnmaj(sb, kD, s), id, 1);
+          for (int s = 0; s < 8; ++s) mma_f16(tbase + colU, desc_kmaj(aa, 128, s), desc_mnmaj(sb, kD, s), id, s > 0);
           mma_commit(&mb_m3);
         }
-        if (c + 1 < nchunks) {  // the first MMA group is done with [-W;Qg], T' and v^
-          if (!mbar_wait(&mb_m3, c & 1, kWaitNs)) bad = true;
-          issue_ld0(c + 1);
-        }
+        if (!mbar_wait(&mb_ld1[c & 1], par, kWaitNs)) bad = true;  // P and K~, long in place
       }
       __syncwarp();
       fence_before();
       asm volatile("bar.sync 2, 160;" ::: "memory");  // Delta is in shared memory
       fence_after();
       if (lane == 0) {  // Y = K~^T Delta first (the state update waits for it), then O += [0;P] Delta
-        if (!mbar_wait(&mb_ld1[c & 1], (c >> 1) & 1, kWaitNs)) bad = true;
         if (!bad) {
-          const uint32_t pa = smem_u32(sm + ((c & 1) ? C_R1 : C_R0) + 8192), db = smem_u32(sm + C_DB),
-                         kt = smem_u32(sm + ((c & 1) ? C_KT1 : C_KT));
-          constexpr uint32_t id4 = idesc_f16(128, 128, false, true);
-          constexpr uint32_t id5 = idesc_f16(128, 128, true, true);
+          const uint32_t pa = smem_u32(sm + C_P + 16384 * (c & 1)), db = smem_u32(sm + C_DB),
+                         kt = smem_u32(sm + C_KT + 16384 * (c & 1));
+          constexpr uint32_t id4 = idesc_f16(128, 64, false, true);
+          constexpr uint32_t id5 = idesc_f16(128, 64, true, true);
 #pragma unroll
           for (int s = 0; s < 4; ++s) mma_f16(tbase + COL_Y, desc_mnmaj(kt, kC, s), desc_mnmaj(db, kC, s), id5, s > 0);
           mma_commit(&mb_m5);
 #pragma unroll
           for (int s = 0; s < 4; ++s) mma_f16(tbase + colU, desc_kmaj(pa, 128, s), desc_mnmaj(db, kC, s), id4, 1);
-          mma_commit(&mb_m4);
+          mma_commit(&mb_m4[c & 1]);
         }
-        // [0;P] Delta is the last MMA to read P and K~'s buffer; O of chunk c is complete before the
-        // block barrier, so the output warps may read it during chunk c+1
-        if (!mbar_wait(&mb_m4, c & 1, kWaitNs)) bad = true;
-        if (c + 2 < nchunks) issue_ld1(c + 2);
-        if (c + 3 < nchunks) bulk_prefetch_l2(rec_of(c + 3), REC_META + 16);  // behind the copies in the queue
+      }
+    } else if (copy_warp) {
+      if (lane == 0) {  // each buffer takes the chunk two ahead once its last reader is done
+        if (c > 0) {  // [0;P] Delta of chunk c-1 was the last reader of its P and K~ buffers
+          if (!mbar_wait(&mb_m4[(c - 1) & 1], ((c - 1) >> 1) & 1, kWaitNs)) bad = true;
+          if (c + 1 < nchunks) issue_ld1(c + 1);
+          if (c + 2 < nchunks && vh == 0) prefetch(c + 2);  // behind the copies in the queue
+        }
+        if (!mbar_wait(&mb_m3, c & 1, kWaitNs)) bad = true;
+        if (c + 2 < nchunks) issue_a(c + 2);
+        if (!mbar_wait(&mb_m5, c & 1, kWaitNs)) bad = true;  // M5 follows the delta warps' reads of U
+        if (c + 2 < nchunks) issue_u(c + 2);
       }
     } else {
       const float egC = __ldg(reinterpret_cast<const float*>(rec_of(c) + REC_META));  // used by the state update
@@ -785,16 +854,23 @@ __global__ void __launch_bounds__(kChainThreads, 1)
           if (!mbar_wait(&mb_g[(c - 1) & 1], ((c - 1) >> 1) & 1, kWaitNs)) bad = true;
           epilogue(c - 1);
         }
-      } else {  // Delta -> shared (MN-major B operand)
+      } else {  // Delta = U + (-W S) -> shared (MN-major B operand)
+        if (!mbar_wait(&mb_u[c & 1], par, kWaitNs)) bad = true;
+        float u[32];
+        const unsigned char* urow = sm + C_U + 16384 * (c & 1) + 256 * si;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const float4 f = *reinterpret_cast<const float4*>(urow + (((8 * hc + m) ^ (si & 7)) << 4));
+          u[4 * m] = f.x; u[4 * m + 1] = f.y; u[4 * m + 2] = f.z; u[4 * m + 3] = f.w;
+        }
         if (!mbar_wait(&mb_m3, c & 1, kWaitNs)) bad = true;
         fence_after();
         float v[32];
+        tmem_ld32(tbase + lane_base + colU + 32 * hc, v);
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          tmem_ld32(tbase + lane_base + colU + 64 * hc + 32 * hh, v);
+        for (int j = 0; j < 32; ++j) v[j] += u[j];
 #pragma unroll
-          for (int m = 0; m < 4; ++m) st16h(sm + C_DB + mnmaj_chunk(kC, si, 64 * hc + 32 * hh + 8 * m), v + 8 * m);
-        }
+        for (int m = 0; m < 4; ++m) st16h(sm + C_DB + mnmaj_chunk(kC, si, 32 * hc + 8 * m), v + 8 * m);
         fence_async_smem();
         fence_before();
         asm volatile("bar.sync 2, 160;" ::: "memory");
@@ -804,22 +880,17 @@ __global__ void __launch_bounds__(kChainThreads, 1)
       if (!mbar_wait(&mb_m5, c & 1, kWaitNs)) bad = true;
       fence_after();
       // S = e^{gamma_C} S + K~^T Delta, and its fp16 copy for the next chunk
-      float v[32], S[32];
+      float y[32];
+      tmem_ld32(tbase + lane_base + COL_Y + 32 * hc, y);
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        tmem_ld32(tbase + lane_base + COL_Y + 64 * hc + 32 * hh, v);
-        tmem_ld32(tbase + lane_base + COL_S + 64 * hc + 32 * hh, S);
+      for (int jj = 0; jj < 32; ++jj) S[jj] = egC * S[jj] + y[jj];
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) S[jj] = egC * S[jj] + v[jj];
-        tmem_st32(tbase + lane_base + COL_S + 64 * hc + 32 * hh, S);
-#pragma unroll
-        for (int m = 0; m < 4; ++m) st16h(sm + C_SB + mnmaj_chunk(kD, si, 64 * hc + 32 * hh + 8 * m), S + 8 * m);
-      }
+      for (int m = 0; m < 4; ++m) st16h(sm + C_SB + mnmaj_chunk(kD, si, 32 * hc + 8 * m), S + 8 * m);
     }
     fence_async_smem();
     if (sync_tc_any(bad)) break;
     // the output of chunk c-1 is written: its gate buffer takes chunk c+1's rows
-    if (producer && lane == 0 && c + 1 < nchunks) issue_gate(c + 1);
+    if (copy_warp && lane == 0 && c + 1 < nchunks) issue_gate(c + 1);
   }
   // block-uniform: either every output warp reaches the epilogue's named barrier or none does
   if (!sync_tc_any(bad) && out_warp) {
@@ -829,17 +900,13 @@ __global__ void __launch_bounds__(kChainThreads, 1)
   }
   if (sync_tc_any(bad)) {
     if (tid == 0) set_status(status, kStatusWaitTimeout);
-  } else if (!producer) {
+  } else if (compute) {
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      float S[32];
-      tmem_ld32(tbase + lane_base + COL_S + 64 * hc + 32 * hh, S);
-#pragma unroll
-      for (int jj = 0; jj < 32; ++jj) gst[(int64_t)(64 * hc + 32 * hh + jj) * kD + si] = S[jj];
-    }
+    for (int jj = 0; jj < 32; ++jj) gst[(int64_t)(c0 + jj) * kD + si] = S[jj];
   }
   sync_tc();
   if (warp == 0) tmem_dealloc(tbase, kChainTmemCols);
+  cluster_sync();  // no CTA leaves while its peer may still write its row sums
 }
 
 bool encode_2d(EncodeTiledFn enc, CUtensorMap* tm, CUtensorMapDataType dt, const void* base, uint64_t cols,
@@ -907,7 +974,7 @@ cudaError_t launch_prefill_split(const Dims& d, const float* conv_w, const float
   if ((e = cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kChainSmem)) != cudaSuccess)
     return e;
   LaunchScope scope(GDN_K_SPLIT_CHAIN, stream);
-  chain_kernel<<<(unsigned)((int64_t)N * d.Hv), kChainThreads, kChainSmem, stream>>>(
+  chain_kernel<<<(unsigned)((int64_t)N * d.Hv * 2), kChainThreads, kChainSmem, stream>>>(
       d, records, chunk_off, order, cu, zero_state ? 1 : 0, state, (__nv_bfloat16*)o, status);
   return cudaGetLastError();
 }

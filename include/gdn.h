@@ -135,8 +135,8 @@ GDN_API gdn_status gdn_conv_step(const gdn_config* cfg, const void* x, const flo
  * gdn_prefill_workspace_size() returns for the same (cfg, total_tokens,
  * num_seqs, chunk_size); 256-byte aligned.  For the tensor-core path (bf16,
  * d_k = d_v = 128, chunk 64) that size holds the schedule plus the chunked
- * form's intermediates: fp16 q^, k^ (two parts each) and v^ for every token
- * and a 65,664-byte operand record per (chunk, value head) -- about 78 KB per
+ * form's intermediates: fp16 q^, k^ (two parts each) for every token and a
+ * 123,520-byte operand record per (chunk, value head) -- about 92 KB per
  * token at 16 key / 48 value heads.  With GDN_PREFILL_FUSED the schedule
  * alone suffices (a few bytes per chunk).
  */
@@ -226,6 +226,51 @@ GDN_API gdn_status gdn_decode_multi(const gdn_config* cfg, const gdn_params* par
                                     void* o, gdn_stream_t stream);
 
 /* --------------------------------------------------------------------------
+ * Slot-indexed state pools for continuous batching ("recurrent-state cache
+ * ownership", issue #88, Scope; batching listed as a gap, Core AI model card,
+ * Limitations).  conv_state and state are pools of num_slots entries,
+ * [num_slots, W-1, C_conv] (io dtype) and [num_slots, Hv, d_v, d_k] (fp32);
+ * row n of the batch reads and writes entry state_indices[n], a device array
+ * of num_seqs int32 (4-byte aligned).  Inputs and outputs stay indexed by
+ * batch row.  Non-negative indices must be distinct.
+ *   - A negative index marks a padding row: decode writes zeros to its o rows
+ *     and touches nothing else; prefill runs it from a zero state and zero
+ *     history and discards its final state and history (its o rows are
+ *     written).
+ *   - An index >= num_slots is an error found on the device: the row is
+ *     treated as padding and gdn_get_device_status reports 3.
+ * Host-side checks as for the unindexed calls, plus num_slots in
+ * [1, 65535] and state_indices non-NULL.
+ *
+ * gdn_decode_step_indexed, gdn_decode_multi_indexed: the decode kernels read
+ * and write the slots in place; results are bit-identical to the unindexed
+ * calls on a pool whose first num_seqs entries are the batch's slots.
+ *
+ * gdn_prefill_indexed: copies the batch's slots into buffers in the
+ * workspace, runs gdn_prefill on them (same flags, same path, bit-identical
+ * results) and copies them back.  A batch that mixes prefill sequences with
+ * decode steps (length-1 sequences) runs in one call.  Workspace:
+ * gdn_prefill_indexed_workspace_size() bytes (gdn_prefill's plus the two
+ * buffers, about 3.2 MB per sequence at 16 key / 48 value heads x 128). */
+GDN_API gdn_status gdn_decode_step_indexed(const gdn_config* cfg, const gdn_params* params, const void* qkv,
+                                           const void* z, const void* a, const void* b, int32_t num_seqs,
+                                           const int32_t* state_indices, int32_t num_slots, void* conv_state,
+                                           float* state, void* o, gdn_stream_t stream);
+GDN_API gdn_status gdn_decode_multi_indexed(const gdn_config* cfg, const gdn_params* params, const void* qkv,
+                                            const void* z, const void* a, const void* b, int32_t num_seqs,
+                                            int32_t num_tokens, int32_t commit, const int32_t* accept_dev,
+                                            const int32_t* state_indices, int32_t num_slots, void* conv_state,
+                                            float* state, void* o, gdn_stream_t stream);
+GDN_API gdn_status gdn_prefill_indexed_workspace_size(const gdn_config* cfg, int64_t total_tokens,
+                                                      int32_t num_seqs, int32_t chunk_size, size_t* bytes);
+GDN_API gdn_status gdn_prefill_indexed(const gdn_config* cfg, const gdn_params* params, const void* qkv,
+                                       const void* z, const void* a, const void* b, const int32_t* cu_seqlens_dev,
+                                       const int32_t* cu_seqlens_host, int32_t num_seqs,
+                                       const int32_t* state_indices, int32_t num_slots, int32_t chunk_size,
+                                       uint32_t flags, void* conv_state, float* state, void* o, void* workspace,
+                                       size_t workspace_bytes, gdn_stream_t stream);
+
+/* --------------------------------------------------------------------------
  * Versioned state checkpoint of one sequence ("Persist every GDN convolution
  * and recurrent component in session checkpoints with versioned validation",
  * issue #95, Implementation; "identical ... BF16 convolution bytes, and fp32
@@ -279,7 +324,8 @@ typedef enum {
   GDN_K_SPLIT_CONV = 8,   /* chunked prefill, stage 1: conv + SiLU + L2 norm of every token */
   GDN_K_SPLIT_PREP = 9,   /* stage 2: per-(chunk, value head) operands of the state carry */
   GDN_K_SPLIT_CHAIN = 10, /* stage 3: the state carry across chunks and the output rows */
-  GDN_K_COUNT = 11
+  GDN_K_SLOT_COPY = 11,   /* slot-indexed prefill: pool slots to and from the batch's buffers */
+  GDN_K_COUNT = 12
 } gdn_kernel_id;
 
 GDN_API const char* gdn_kernel_name(int32_t kernel_id);

@@ -18,7 +18,8 @@ import numpy as np
 
 __all__ = [
     "GdnError", "Config", "Params", "lib", "make_config", "conv_prefill", "conv_step", "prefill_workspace_size",
-    "prefill", "prefill_noalloc", "decode_step", "decode_multi", "state_blob_size", "state_save", "state_restore", "device_status", "last_error",
+    "prefill", "prefill_noalloc", "decode_step", "decode_multi", "decode_step_indexed", "decode_multi_indexed",
+    "prefill_indexed_workspace_size", "prefill_indexed", "state_blob_size", "state_save", "state_restore", "device_status", "last_error",
     "abi_version", "launch_count", "launch_count_reset", "profiler_enable", "profiler_reset", "profiler_read",
     "kernel_name", "EXPORTS", "ZERO_INIT_STATE", "ZERO_INIT_CONV", "PREFILL_RECURRENT", "PREFILL_FUSED", "K", "MAX_DRAFT_TOKENS",
 ]
@@ -41,8 +42,8 @@ STATUS = {0: "GDN_OK", -1: "GDN_E_INVAL", -2: "GDN_E_UNSUPPORTED", -3: "GDN_E_WO
 class K:
     """Kernel ids of the profiler (gdn_kernel_id)."""
     (CONV_PREFILL, CONV_STEP, CONV_HISTORY, SCHEDULE, PREFILL_RECURRENT, PREFILL_CHUNKED, DECODE, STATE_CHECKSUM,
-     SPLIT_CONV, SPLIT_PREP, SPLIT_CHAIN) = range(11)
-    COUNT = 11
+     SPLIT_CONV, SPLIT_PREP, SPLIT_CHAIN, SLOT_COPY) = range(12)
+    COUNT = 12
 
 
 # Every symbol include/gdn.h declares.
@@ -51,6 +52,8 @@ EXPORTS = [
     "gdn_state_blob_size", "gdn_state_save", "gdn_state_restore", "gdn_get_device_status", "gdn_last_error",
     "gdn_abi_version", "gdn_launch_count", "gdn_launch_count_reset", "gdn_kernel_name", "gdn_profiler_enable",
     "gdn_profiler_reset", "gdn_profiler_read", "gdn_prefill_noalloc", "gdn_decode_multi",
+    "gdn_decode_step_indexed", "gdn_decode_multi_indexed", "gdn_prefill_indexed_workspace_size",
+    "gdn_prefill_indexed",
 ]
 
 
@@ -92,6 +95,10 @@ def lib():
             "gdn_prefill_noalloc": [P, P, P, P, P, P, P, P, I32, I32, U32, P, P, P, P],
             "gdn_decode_step": [P, P, P, P, P, P, I32, P, P, P, P],
             "gdn_decode_multi": [P, P, P, P, P, P, I32, I32, I32, P, P, P, P, P],
+            "gdn_decode_step_indexed": [P, P, P, P, P, P, I32, P, I32, P, P, P, P],
+            "gdn_decode_multi_indexed": [P, P, P, P, P, P, I32, I32, I32, P, P, I32, P, P, P, P],
+            "gdn_prefill_indexed_workspace_size": [P, I64, I32, I32, P],
+            "gdn_prefill_indexed": [P, P, P, P, P, P, P, P, I32, P, I32, I32, U32, P, P, P, P, SZ, P],
             "gdn_state_blob_size": [P, P],
             "gdn_state_save": [P, P, P, I32, P, SZ, P],
             "gdn_state_restore": [P, P, SZ, I32, P, P, P],
@@ -210,6 +217,46 @@ def decode_multi(cfg, params, qkv, z, a, b, num_seqs, num_tokens, commit, accept
     _check(lib().gdn_decode_multi(ctypes.byref(cfg), ctypes.byref(prm), _p(qkv), _p(z), _p(a), _p(b), num_seqs,
                                   num_tokens, 1 if commit else 0, _p(accept),
                                   _p(conv_state), _p(state), _p(o), _stream(stream)))
+
+
+def decode_step_indexed(cfg, params, qkv, z, a, b, num_seqs, state_indices, num_slots, conv_state, state, o,
+                        stream=None):
+    """gdn_decode_step_indexed: row n of the batch uses pool slot
+    state_indices[n] (device int32; negative = padding row)."""
+    prm = _params(*params)
+    _check(lib().gdn_decode_step_indexed(ctypes.byref(cfg), ctypes.byref(prm), _p(qkv), _p(z), _p(a), _p(b),
+                                         num_seqs, _p(state_indices), num_slots, _p(conv_state), _p(state), _p(o),
+                                         _stream(stream)))
+
+
+def decode_multi_indexed(cfg, params, qkv, z, a, b, num_seqs, num_tokens, commit, accept, state_indices, num_slots,
+                         conv_state, state, o, stream=None):
+    """gdn_decode_multi_indexed: gdn_decode_multi over pool slots."""
+    prm = _params(*params)
+    _check(lib().gdn_decode_multi_indexed(ctypes.byref(cfg), ctypes.byref(prm), _p(qkv), _p(z), _p(a), _p(b),
+                                          num_seqs, num_tokens, 1 if commit else 0, _p(accept), _p(state_indices),
+                                          num_slots, _p(conv_state), _p(state), _p(o), _stream(stream)))
+
+
+def prefill_indexed_workspace_size(cfg, total_tokens: int, num_seqs: int, chunk_size: int) -> int:
+    out = ctypes.c_size_t()
+    _check(lib().gdn_prefill_indexed_workspace_size(ctypes.byref(cfg), total_tokens, num_seqs, chunk_size,
+                                                    ctypes.byref(out)))
+    return out.value
+
+
+def prefill_indexed(cfg, params, qkv, z, a, b, cu_dev, cu_host, state_indices, num_slots, chunk_size, flags,
+                    conv_state, state, o, workspace, workspace_bytes=None, stream=None):
+    """gdn_prefill_indexed: gdn_prefill over pool slots (a batch may mix
+    prefill sequences with length-1 decode steps)."""
+    cu_h = _host_cu(cu_host)
+    prm = _params(*params)
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().gdn_prefill_indexed(ctypes.byref(cfg), ctypes.byref(prm), _p(qkv), _p(z), _p(a), _p(b), _p(cu_dev),
+                                     cu_h.ctypes.data, cu_h.size - 1, _p(state_indices), num_slots, chunk_size, flags,
+                                     _p(conv_state), _p(state), _p(o), _p(workspace), workspace_bytes,
+                                     _stream(stream)))
 
 
 def state_blob_size(cfg) -> int:

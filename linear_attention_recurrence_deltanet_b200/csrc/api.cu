@@ -290,7 +290,8 @@ void gdn_launch_count_reset(void) { g_launches.store(0); }
 const char* gdn_kernel_name(int32_t id) {
   static const char* names[GDN_K_COUNT] = {"conv_prefill",    "conv_step",       "conv_history", "schedule",
                                            "prefill_recurrent", "prefill_chunked", "decode",       "state_checksum",
-                                           "split_conv",        "split_prep",      "split_chain"};
+                                           "split_conv",        "split_prep",      "split_chain",
+                                           "slot_copy"};
   return (id >= 0 && id < GDN_K_COUNT) ? names[id] : "unknown";
 }
 
@@ -454,9 +455,19 @@ gdn_status gdn_prefill(const gdn_config* cfg, const gdn_params* params, const vo
   return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_prefill launch");
 }
 
-gdn_status gdn_decode_step(const gdn_config* cfg, const gdn_params* params, const void* qkv, const void* z,
-                           const void* a, const void* b, int32_t num_seqs, void* conv_state, float* state, void* o,
-                           gdn_stream_t stream) {
+namespace {
+
+gdn_status check_slots(const int32_t* slots_dev, int32_t num_slots, int32_t num_seqs) {
+  if (!slots_dev) return fail(GDN_E_INVAL, "state_indices is NULL");
+  if ((uintptr_t)slots_dev & 3u) return fail(GDN_E_INVAL, "state_indices is not 4-byte aligned");
+  if (num_slots <= 0 || num_slots > kMaxSeqs) return fail(GDN_E_INVAL, "num_slots %d out of range", num_slots);
+  (void)num_seqs;
+  return GDN_OK;
+}
+
+gdn_status decode_step_impl(const gdn_config* cfg, const gdn_params* params, const void* qkv, const void* z,
+                            const void* a, const void* b, int32_t num_seqs, gdn::Slots slots, void* conv_state,
+                            float* state, void* o, gdn_stream_t stream, const char* what) {
   gdn::Dims d;
   gdn_status s;
   if ((s = check_cfg(cfg, &d)) != GDN_OK) return s;
@@ -471,15 +482,15 @@ gdn_status gdn_decode_step(const gdn_config* cfg, const gdn_params* params, cons
   int dev = 0;
   if ((s = check_device(&dev)) != GDN_OK) return s;
   cudaError_t e = gdn::launch_decode_step(d, cfg->io_dtype == GDN_BF16, params->conv_w, params->A_log,
-                                          params->dt_bias, params->norm_w, qkv, z, a, b, num_seqs, conv_state,
+                                          params->dt_bias, params->norm_w, qkv, z, a, b, num_seqs, slots, conv_state,
                                           state, o, g_status_ptr[dev], (cudaStream_t)stream);
-  return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_decode_step launch");
+  return e == cudaSuccess ? GDN_OK : cuda_fail(e, what);
 }
 
-gdn_status gdn_decode_multi(const gdn_config* cfg, const gdn_params* params, const void* qkv, const void* z,
-                            const void* a, const void* b, int32_t num_seqs, int32_t num_tokens, int32_t commit,
-                            const int32_t* accept_dev, void* conv_state, float* state, void* o,
-                            gdn_stream_t stream) {
+gdn_status decode_multi_impl(const gdn_config* cfg, const gdn_params* params, const void* qkv, const void* z,
+                             const void* a, const void* b, int32_t num_seqs, int32_t num_tokens, int32_t commit,
+                             const int32_t* accept_dev, gdn::Slots slots, void* conv_state, float* state, void* o,
+                             gdn_stream_t stream, const char* what) {
   gdn::Dims d;
   gdn_status s;
   if ((s = check_cfg(cfg, &d)) != GDN_OK) return s;
@@ -501,9 +512,125 @@ gdn_status gdn_decode_multi(const gdn_config* cfg, const gdn_params* params, con
   if ((s = check_device(&dev)) != GDN_OK) return s;
   cudaError_t e = gdn::launch_decode_multi(d, cfg->io_dtype == GDN_BF16, params->conv_w, params->A_log,
                                            params->dt_bias, params->norm_w, qkv, z, a, b, num_seqs, num_tokens,
-                                           accept_dev, commit ? 1 : 0, conv_state, state, o, g_status_ptr[dev],
+                                           accept_dev, commit ? 1 : 0, slots, conv_state, state, o, g_status_ptr[dev],
                                            (cudaStream_t)stream);
-  return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_decode_multi launch");
+  return e == cudaSuccess ? GDN_OK : cuda_fail(e, what);
+}
+
+}  // namespace
+
+gdn_status gdn_decode_step(const gdn_config* cfg, const gdn_params* params, const void* qkv, const void* z,
+                           const void* a, const void* b, int32_t num_seqs, void* conv_state, float* state, void* o,
+                           gdn_stream_t stream) {
+  return decode_step_impl(cfg, params, qkv, z, a, b, num_seqs, gdn::Slots{nullptr, 0}, conv_state, state, o, stream,
+                          "gdn_decode_step launch");
+}
+
+gdn_status gdn_decode_step_indexed(const gdn_config* cfg, const gdn_params* params, const void* qkv, const void* z,
+                                   const void* a, const void* b, int32_t num_seqs, const int32_t* state_indices,
+                                   int32_t num_slots, void* conv_state, float* state, void* o, gdn_stream_t stream) {
+  gdn_status s;
+  if ((s = check_slots(state_indices, num_slots, num_seqs)) != GDN_OK) return s;
+  return decode_step_impl(cfg, params, qkv, z, a, b, num_seqs, gdn::Slots{state_indices, num_slots}, conv_state,
+                          state, o, stream, "gdn_decode_step_indexed launch");
+}
+
+gdn_status gdn_decode_multi(const gdn_config* cfg, const gdn_params* params, const void* qkv, const void* z,
+                            const void* a, const void* b, int32_t num_seqs, int32_t num_tokens, int32_t commit,
+                            const int32_t* accept_dev, void* conv_state, float* state, void* o,
+                            gdn_stream_t stream) {
+  return decode_multi_impl(cfg, params, qkv, z, a, b, num_seqs, num_tokens, commit, accept_dev,
+                           gdn::Slots{nullptr, 0}, conv_state, state, o, stream, "gdn_decode_multi launch");
+}
+
+gdn_status gdn_decode_multi_indexed(const gdn_config* cfg, const gdn_params* params, const void* qkv, const void* z,
+                                    const void* a, const void* b, int32_t num_seqs, int32_t num_tokens,
+                                    int32_t commit, const int32_t* accept_dev, const int32_t* state_indices,
+                                    int32_t num_slots, void* conv_state, float* state, void* o,
+                                    gdn_stream_t stream) {
+  gdn_status s;
+  if ((s = check_slots(state_indices, num_slots, num_seqs)) != GDN_OK) return s;
+  return decode_multi_impl(cfg, params, qkv, z, a, b, num_seqs, num_tokens, commit, accept_dev,
+                           gdn::Slots{state_indices, num_slots}, conv_state, state, o, stream,
+                           "gdn_decode_multi_indexed launch");
+}
+
+namespace {
+
+// workspace of an indexed prefill: gdn_prefill's, then the batch's state and conv-history buffers
+struct IndexedLayout {
+  size_t state_off, conv_off, total;
+};
+IndexedLayout indexed_layout(const gdn::Dims& d, bool bf16, size_t base, int32_t num_seqs) {
+  auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  IndexedLayout L;
+  L.state_off = al(base);
+  L.conv_off = al(L.state_off + (size_t)num_seqs * d.Hv * d.dv * d.dk * sizeof(float));
+  L.total = al(L.conv_off + (size_t)num_seqs * (d.W - 1) * d.C * (bf16 ? 2 : 4));
+  return L;
+}
+
+}  // namespace
+
+gdn_status gdn_prefill_indexed_workspace_size(const gdn_config* cfg, int64_t total_tokens, int32_t num_seqs,
+                                              int32_t chunk_size, size_t* bytes) {
+  size_t base = 0;
+  gdn_status s = gdn_prefill_workspace_size(cfg, total_tokens, num_seqs, chunk_size, &base);
+  if (s != GDN_OK) return s;
+  gdn::Dims d;
+  if ((s = check_cfg(cfg, &d)) != GDN_OK) return s;
+  *bytes = indexed_layout(d, cfg->io_dtype == GDN_BF16, base, num_seqs).total;
+  return GDN_OK;
+}
+
+gdn_status gdn_prefill_indexed(const gdn_config* cfg, const gdn_params* params, const void* qkv, const void* z,
+                               const void* a, const void* b, const int32_t* cu_seqlens_dev,
+                               const int32_t* cu_seqlens_host, int32_t num_seqs, const int32_t* state_indices,
+                               int32_t num_slots, int32_t chunk_size, uint32_t flags, void* conv_state, float* state,
+                               void* o, void* workspace, size_t workspace_bytes, gdn_stream_t stream) {
+  // every check gdn_prefill makes comes first, so that an error launches nothing
+  gdn::Dims d;
+  gdn_status s;
+  if ((s = check_cfg(cfg, &d)) != GDN_OK) return s;
+  if ((s = check_params(params)) != GDN_OK) return s;
+  if ((s = check_slots(state_indices, num_slots, num_seqs)) != GDN_OK) return s;
+  if (chunk_size != 16 && chunk_size != 32 && chunk_size != 64 && chunk_size != 128)
+    return fail(GDN_E_INVAL, "chunk_size %d (16, 32, 64 or 128)", chunk_size);
+  const uint32_t known = GDN_ZERO_INIT_STATE | GDN_ZERO_INIT_CONV | GDN_PREFILL_RECURRENT | GDN_PREFILL_FUSED;
+  if (flags & ~known) return fail(GDN_E_INVAL, "unknown flags 0x%x", flags & ~known);
+  int64_t total = 0;
+  int32_t max_len = 0;
+  if ((s = check_cu(cu_seqlens_dev, cu_seqlens_host, num_seqs, &total, &max_len)) != GDN_OK) return s;
+  if ((s = check_ptr(conv_state, "conv_state")) != GDN_OK || (s = check_ptr(state, "state")) != GDN_OK) return s;
+  if (total > 0) {
+    if ((s = check_ptr(qkv, "qkv")) != GDN_OK || (s = check_ptr(z, "z")) != GDN_OK ||
+        (s = check_gate_ptr(a, "a", cfg)) != GDN_OK || (s = check_gate_ptr(b, "b", cfg)) != GDN_OK ||
+        (s = check_ptr(o, "o")) != GDN_OK)
+      return s;
+  }
+  const bool bf16 = cfg->io_dtype == GDN_BF16;
+  const size_t base = prefill_ws_bytes(d, split_path(d, cfg, chunk_size, flags), total, num_seqs, chunk_size);
+  const IndexedLayout L = indexed_layout(d, bf16, base, num_seqs);
+  if (workspace_bytes < L.total || !workspace)
+    return fail(GDN_E_WORKSPACE, "workspace of %zu bytes at %p, need %zu", workspace_bytes, workspace, L.total);
+  if (((uintptr_t)workspace & 255u) != 0) return fail(GDN_E_WORKSPACE, "workspace is not 256-byte aligned");
+  int dev = 0;
+  if ((s = check_device(&dev)) != GDN_OK) return s;
+  if (total == 0) return GDN_OK;  // every sequence empty: nothing changes
+
+  cudaStream_t st = (cudaStream_t)stream;
+  const gdn::Slots slots{state_indices, num_slots};
+  float* buf_state = (float*)((char*)workspace + L.state_off);
+  void* buf_conv = (char*)workspace + L.conv_off;
+  cudaError_t e = gdn::launch_slot_copy(d, bf16, slots, num_seqs, true, state, conv_state, buf_state, buf_conv,
+                                        g_status_ptr[dev], st);
+  if (e != cudaSuccess) return cuda_fail(e, "gdn_prefill_indexed gather");
+  if ((s = gdn_prefill(cfg, params, qkv, z, a, b, cu_seqlens_dev, cu_seqlens_host, num_seqs, chunk_size, flags,
+                       buf_conv, buf_state, o, workspace, L.state_off, stream)) != GDN_OK)
+    return s;
+  e = gdn::launch_slot_copy(d, bf16, slots, num_seqs, false, state, conv_state, buf_state, buf_conv,
+                            g_status_ptr[dev], st);
+  return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_prefill_indexed scatter");
 }
 
 gdn_status gdn_state_blob_size(const gdn_config* cfg, size_t* bytes) {

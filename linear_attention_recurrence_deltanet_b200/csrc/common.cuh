@@ -19,10 +19,29 @@ enum : int32_t {
   kStatusOk = 0,
   kStatusWaitTimeout = 1,   // a bounded wait gave up
   kStatusBoundsCheck = 2,   // a debug bounds check failed
+  kStatusBadSlot = 3,       // a state slot index past the end of the pool (the row was skipped)
 };
 
 __device__ __forceinline__ void set_status(int32_t* status, int32_t code) {
   if (status) atomicCAS(status, 0, code);
+}
+
+// State slots of a batch: row n of the batch reads and writes slot idx[n] of
+// the state and conv-history pools (slot n when idx is NULL).  A negative slot
+// marks a padding row; a slot at or past `count` is reported and treated as
+// padding.
+struct Slots {
+  const int32_t* idx;
+  int32_t count;
+};
+__device__ __forceinline__ int slot_of(const Slots& s, int n, int32_t* status) {
+  if (!s.idx) return n;
+  const int v = s.idx[n];
+  if (v >= s.count) {
+    set_status(status, kStatusBadSlot);
+    return -1;
+  }
+  return v;
 }
 
 // io element access: fp32 or bf16 storage, fp32 arithmetic.

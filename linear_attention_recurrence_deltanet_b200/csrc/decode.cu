@@ -30,8 +30,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kDecThreads, 2)
     decode_kernel(Dims d, const float* __restrict__ conv_w, const float* __restrict__ A_log,
                   const float* __restrict__ dt_bias, const float* __restrict__ norm_w, const T* __restrict__ qkv,
-                  const T* __restrict__ z, const T* __restrict__ a, const T* __restrict__ b, T* __restrict__ hist,
-                  float* __restrict__ state, T* __restrict__ o) {
+                  const T* __restrict__ z, const T* __restrict__ a, const T* __restrict__ b, Slots slots,
+                  T* __restrict__ hist, float* __restrict__ state, T* __restrict__ o, int32_t* status) {
   constexpr int F4 = D / 32;  // float4s of a row held by one lane (8 lanes per row)
   extern __shared__ float smem[];
   const int G = d.G;
@@ -46,13 +46,18 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t C = d.C;
   const int h0 = G * kh;  // first value head of this key head
+  const int sl = slot_of(slots, n, status);  // state and history slot of batch row n
+  if (sl < 0) {  // padding row: zero output, nothing else touched
+    for (int i = tid; i < G * D; i += kDecThreads) o[((int64_t)n * d.Hv + h0) * D + i] = from_f<T>(0.f);
+    return;
+  }
 
   // ---- conv step + SiLU for the owned channels; rotate the history
   for (int idx = tid; idx < nch; idx += kDecThreads) {
     const int64_t c = idx < D ? (int64_t)kh * D + idx
                               : (idx < 2 * D ? (int64_t)d.Hk * D + (int64_t)kh * D + (idx - D)
                                              : 2LL * d.Hk * D + (int64_t)h0 * D + (idx - 2 * D));
-    T* hp = hist + (int64_t)n * 3 * C + c;
+    T* hp = hist + (int64_t)sl * 3 * C + c;
     const T h0v = hp[0], h1v = hp[C], h2v = hp[2 * C];
     const T xv = qkv[(int64_t)n * C + c];
     const float4 w = __ldg(reinterpret_cast<const float4*>(conv_w + c * 4));
@@ -108,7 +113,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   const float qk = red[2];
   const int rows = G * D;
   const int groups = rows / 4;
-  float* st = state + ((int64_t)n * d.Hv + h0) * D * D;  // the G heads' rows are contiguous
+  float* st = state + ((int64_t)sl * d.Hv + h0) * D * D;  // the G heads' rows are contiguous
   for (int base = warp; base < groups; base += kDecWarps * kUnroll) {
     float4 r[kUnroll][F4];
 #pragma unroll
@@ -200,7 +205,7 @@ __global__ void __launch_bounds__(kBulkThreads, K <= 2 ? 8 : 4)
     decode_bulk_kernel(Dims d, const float* __restrict__ conv_w, const float* __restrict__ A_log,
                        const float* __restrict__ dt_bias, const float* __restrict__ norm_w,
                        const T* __restrict__ qkv, const T* __restrict__ z, const T* __restrict__ a,
-                       const T* __restrict__ b, const int32_t* __restrict__ accept, int write_state,
+                       const T* __restrict__ b, const int32_t* __restrict__ accept, int write_state, Slots slots,
                        T* __restrict__ hist, float* __restrict__ state, T* __restrict__ o, int32_t* status) {
   constexpr int D = 128;
   constexpr int kStageFloats = kBulkRows * D;
@@ -221,7 +226,15 @@ __global__ void __launch_bounds__(kBulkThreads, K <= 2 ? 8 : 4)
   const int64_t C = d.C;
   const int h0 = G * kh;
   const int nst = G * D / kBulkRows;
-  float* st = state + ((int64_t)n * d.Hv + h0) * D * D;   // the G heads' rows are contiguous
+  const int sl = slot_of(slots, n, status);  // state and history slot of batch row n
+  if (sl < 0) {  // padding row: zero output for every token, nothing else touched
+    for (int i = tid; i < K * G * D; i += kBulkThreads) {
+      const int t = i / (G * D);
+      o[(((int64_t)n * K + t) * d.Hv + h0) * D + (i - t * G * D)] = from_f<T>(0.f);
+    }
+    return;
+  }
+  float* st = state + ((int64_t)sl * d.Hv + h0) * D * D;  // the G heads' rows are contiguous
   // tokens applied to the state and history (and outputs written)
   int nk = K;
   if (write_state && accept) nk = min(max(accept[n], 0), K);
@@ -248,7 +261,7 @@ __global__ void __launch_bounds__(kBulkThreads, K <= 2 ? 8 : 4)
     const int64_t c = idx < D ? (int64_t)kh * D + idx
                               : (idx < 2 * D ? (int64_t)d.Hk * D + (int64_t)kh * D + (idx - D)
                                              : 2LL * d.Hk * D + (int64_t)h0 * D + (idx - 2 * D));
-    T* hp = hist + (int64_t)n * 3 * C + c;
+    T* hp = hist + (int64_t)sl * 3 * C + c;
     T xs[3 + K];  // raw inputs, oldest first
     xs[0] = hp[0];
     xs[1] = hp[C];
@@ -394,8 +407,8 @@ __global__ void __launch_bounds__(kBulkThreads, K <= 2 ? 8 : 4)
 template <typename T, int K>
 cudaError_t launch_bulk(const Dims& d, const float* conv_w, const float* A_log, const float* dt_bias,
                         const float* norm_w, const void* qkv, const void* z, const void* a, const void* b, int32_t N,
-                        const int32_t* accept, int write_state, void* hist, float* state, void* o, int32_t* status,
-                        cudaStream_t stream) {
+                        const int32_t* accept, int write_state, Slots slots, void* hist, float* state, void* o,
+                        int32_t* status, cudaStream_t stream) {
   const size_t smem =
       (size_t)(kBulkStages * kBulkRows * 128 + K * (2 + d.G) * 128 + K * d.G * 128 + K * 2 * d.G) * sizeof(float);
   if (smem > 48 * 1024) {
@@ -406,27 +419,31 @@ cudaError_t launch_bulk(const Dims& d, const float* conv_w, const float* A_log, 
   LaunchScope scope(GDN_K_DECODE, stream);
   decode_bulk_kernel<T, K><<<(unsigned)((int64_t)N * d.Hk), kBulkThreads, smem, stream>>>(
       d, conv_w, A_log, dt_bias, norm_w, (const T*)qkv, (const T*)z, (const T*)a, (const T*)b, accept, write_state,
-      (T*)hist, state, (T*)o, status);
+      slots, (T*)hist, state, (T*)o, status);
   return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t launch_multi_t(const Dims& d, const float* conv_w, const float* A_log, const float* dt_bias,
                            const float* norm_w, const void* qkv, const void* z, const void* a, const void* b, int32_t N,
-                           int32_t K, const int32_t* accept, int write_state, void* hist, float* state, void* o,
-                           int32_t* status, cudaStream_t stream) {
+                           int32_t K, const int32_t* accept, int write_state, Slots slots, void* hist, float* state,
+                           void* o, int32_t* status, cudaStream_t stream) {
+#define GDN_MULTI(KK)                                                                                                 \
+  return launch_bulk<T, KK>(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, N, accept, write_state, slots, hist, \
+                            state, o, status, stream)
   switch (K) {
-    case 1: return launch_bulk<T, 1>(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, N, accept, write_state, hist, state, o, status, stream);
-    case 2: return launch_bulk<T, 2>(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, N, accept, write_state, hist, state, o, status, stream);
-    case 3: return launch_bulk<T, 3>(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, N, accept, write_state, hist, state, o, status, stream);
-    default: return launch_bulk<T, 4>(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, N, accept, write_state, hist, state, o, status, stream);
+    case 1: GDN_MULTI(1);
+    case 2: GDN_MULTI(2);
+    case 3: GDN_MULTI(3);
+    default: GDN_MULTI(4);
   }
+#undef GDN_MULTI
 }
 
 template <typename T, int D>
 cudaError_t launch_t(const Dims& d, const float* conv_w, const float* A_log, const float* dt_bias,
                      const float* norm_w, const void* qkv, const void* z, const void* a, const void* b, int32_t N,
-                     void* hist, float* state, void* o, cudaStream_t stream) {
+                     Slots slots, void* hist, float* state, void* o, int32_t* status, cudaStream_t stream) {
   const size_t smem = (size_t)((2 + d.G) * D + d.G * D + 2 * d.G) * sizeof(float);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -435,8 +452,8 @@ cudaError_t launch_t(const Dims& d, const float* conv_w, const float* A_log, con
   }
   LaunchScope scope(GDN_K_DECODE, stream);
   decode_kernel<T, D><<<(unsigned)((int64_t)N * d.Hk), kDecThreads, smem, stream>>>(
-      d, conv_w, A_log, dt_bias, norm_w, (const T*)qkv, (const T*)z, (const T*)a, (const T*)b, (T*)hist, state,
-      (T*)o);
+      d, conv_w, A_log, dt_bias, norm_w, (const T*)qkv, (const T*)z, (const T*)a, (const T*)b, slots, (T*)hist, state,
+      (T*)o, status);
   return cudaGetLastError();
 }
 
@@ -444,17 +461,17 @@ cudaError_t launch_t(const Dims& d, const float* conv_w, const float* A_log, con
 
 cudaError_t launch_decode_step(const Dims& d, bool bf16, const float* conv_w, const float* A_log,
                                const float* dt_bias, const float* norm_w, const void* qkv, const void* z,
-                               const void* a, const void* b, int32_t N, void* conv_state, float* state, void* o,
-                               int32_t* status, cudaStream_t stream) {
+                               const void* a, const void* b, int32_t N, Slots slots, void* conv_state, float* state,
+                               void* o, int32_t* status, cudaStream_t stream) {
   if (N <= 0) return cudaSuccess;
   if (d.dk == 128) {
-    return bf16 ? launch_bulk<__nv_bfloat16, 1>(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, N, nullptr, 1,
+    return bf16 ? launch_bulk<__nv_bfloat16, 1>(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, N, nullptr, 1, slots,
                                                 conv_state, state, o, status, stream)
-                : launch_bulk<float, 1>(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, N, nullptr, 1, conv_state,
-                                        state, o, status, stream);
+                : launch_bulk<float, 1>(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, N, nullptr, 1, slots,
+                                        conv_state, state, o, status, stream);
   }
 #define GDN_DEC(T, D) \
-  return launch_t<T, D>(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, N, conv_state, state, o, stream)
+  return launch_t<T, D>(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, N, slots, conv_state, state, o, status, stream)
   if (bf16) {
     switch (d.dk) {
       case 32: GDN_DEC(__nv_bfloat16, 32);
@@ -474,13 +491,13 @@ cudaError_t launch_decode_step(const Dims& d, bool bf16, const float* conv_w, co
 cudaError_t launch_decode_multi(const Dims& d, bool bf16, const float* conv_w, const float* A_log,
                                 const float* dt_bias, const float* norm_w, const void* qkv, const void* z,
                                 const void* a, const void* b, int32_t N, int32_t K, const int32_t* accept,
-                                int write_state, void* conv_state, float* state, void* o, int32_t* status,
-                                cudaStream_t stream) {
+                                int write_state, Slots slots, void* conv_state, float* state, void* o,
+                                int32_t* status, cudaStream_t stream) {
   if (N <= 0) return cudaSuccess;
   return bf16 ? launch_multi_t<__nv_bfloat16>(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, N, K, accept,
-                                              write_state, conv_state, state, o, status, stream)
+                                              write_state, slots, conv_state, state, o, status, stream)
               : launch_multi_t<float>(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, N, K, accept, write_state,
-                                      conv_state, state, o, status, stream);
+                                      slots, conv_state, state, o, status, stream);
 }
 
 }  // namespace gdn

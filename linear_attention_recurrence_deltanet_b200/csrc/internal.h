@@ -40,15 +40,15 @@ cudaError_t launch_schedule(const int32_t* cu, int32_t num_seqs, int32_t chunk_s
 // decode.cu
 cudaError_t launch_decode_step(const Dims& d, bool bf16, const float* conv_w, const float* A_log,
                                const float* dt_bias, const float* norm_w, const void* qkv, const void* z,
-                               const void* a, const void* b, int32_t num_seqs, void* conv_state, float* state,
-                               void* o, int32_t* status, cudaStream_t stream);
+                               const void* a, const void* b, int32_t num_seqs, Slots slots, void* conv_state,
+                               float* state, void* o, int32_t* status, cudaStream_t stream);
 
 // multi-token decode (draft-and-verify), d = 128: verify (write_state 0) or commit
 cudaError_t launch_decode_multi(const Dims& d, bool bf16, const float* conv_w, const float* A_log,
                                 const float* dt_bias, const float* norm_w, const void* qkv, const void* z,
                                 const void* a, const void* b, int32_t num_seqs, int32_t num_tokens,
-                                const int32_t* accept, int write_state, void* conv_state, float* state, void* o,
-                                int32_t* status, cudaStream_t stream);
+                                const int32_t* accept, int write_state, Slots slots, void* conv_state, float* state,
+                                void* o, int32_t* status, cudaStream_t stream);
 
 // prefill_recurrent.cu
 cudaError_t launch_prefill_recurrent(const Dims& d, bool bf16, const float* conv_w, const float* A_log,
@@ -83,6 +83,11 @@ cudaError_t launch_prefill_split(const Dims& d, const float* conv_w, const float
                                  const int4* chunk_map, int32_t N, int64_t total_tokens, int64_t total_chunks,
                                  bool zero_state, bool zero_conv, const void* conv_state, float* state, void* o,
                                  void* split_ws, int32_t* status, cudaStream_t stream);
+
+// slots.cu: the batch's pool slots to contiguous buffers (to_buffer) or back
+cudaError_t launch_slot_copy(const Dims& d, bool bf16, Slots slots, int32_t num_seqs, bool to_buffer,
+                             float* pool_state, void* pool_conv, float* buf_state, void* buf_conv, int32_t* status,
+                             cudaStream_t stream);
 
 // api.cu: records a message for gdn_last_error() on the calling thread.
 void set_error_message(const char* msg);

@@ -271,6 +271,41 @@ GDN_API gdn_status gdn_prefill_indexed(const gdn_config* cfg, const gdn_params* 
                                        size_t workspace_bytes, gdn_stream_t stream);
 
 /* --------------------------------------------------------------------------
+ * Dense projections either side of the mixer (the "GDN projection" primitive
+ * of issue #95, Verification; its "BF16 projection kernels", implementation
+ * comment).  All three are one bf16 GEMM on the tensor cores with fp32
+ * accumulation and round-to-nearest bf16 output:
+ *   Y[r, c] = sum_k X[r, k] * W[c, k]
+ * X [M, K] and W [N, K] are row-major bf16 device arrays (W is a linear
+ * layer's weight: output features x input features).  K must be a multiple
+ * of 8 (16-byte row pitch) and X, W 16-byte aligned; M, N >= 0 (0 launches
+ * nothing); M, N, K < 2^31.  No workspace.  tile_n picks the output tile
+ * width: 64, 128 or 256 columns, 0 = chosen from M and N.
+ *
+ * gdn_gemm_bf16: Y [M, N] row-major bf16 (2-byte aligned; rows 16-byte
+ *   aligned give vector stores).
+ * gdn_project_in: the input projection of one GDN layer.  W_in stacks the
+ *   rows of the four outputs, [C_conv + Hv*d_v + 2*Hv, hidden]:
+ *     rows [0, C_conv)               -> qkv [T, C_conv] (q, k, v channels)
+ *     rows [C_conv, +Hv*d_v)          -> z   [T, Hv*d_v]
+ *     next Hv rows                    -> a   [T, Hv]
+ *     last Hv rows                    -> b   [T, Hv]
+ *   with C_conv = 2*Hk*d_k + Hv*d_v; every output row-major, bf16.  The
+ *   outputs are exactly what gdn_prefill / gdn_decode_step take as qkv, z, a,
+ *   b, so a layer is project_in -> prefill or decode -> project_out.
+ *   cfg->io_dtype must be GDN_BF16.
+ * gdn_project_out: y [T, hidden] = o [T, Hv*d_v] W_out^T, W_out
+ *   [hidden, Hv*d_v].
+ * A bounded internal wait that runs out sets device status 1 (see
+ * gdn_get_device_status). */
+GDN_API gdn_status gdn_gemm_bf16(const void* x, int32_t M, int32_t K, const void* w, int32_t N, void* y,
+                                 int32_t tile_n, gdn_stream_t stream);
+GDN_API gdn_status gdn_project_in(const gdn_config* cfg, const void* x, int32_t num_tokens, int32_t hidden,
+                                  const void* w_in, void* qkv, void* z, void* a, void* b, gdn_stream_t stream);
+GDN_API gdn_status gdn_project_out(const gdn_config* cfg, const void* o, int32_t num_tokens, const void* w_out,
+                                   int32_t hidden, void* y, gdn_stream_t stream);
+
+/* --------------------------------------------------------------------------
  * Versioned state checkpoint of one sequence ("Persist every GDN convolution
  * and recurrent component in session checkpoints with versioned validation",
  * issue #95, Implementation; "identical ... BF16 convolution bytes, and fp32
@@ -325,7 +360,8 @@ typedef enum {
   GDN_K_SPLIT_PREP = 9,   /* stage 2: per-(chunk, value head) operands of the state carry */
   GDN_K_SPLIT_CHAIN = 10, /* stage 3: the state carry across chunks and the output rows */
   GDN_K_SLOT_COPY = 11,   /* slot-indexed prefill: pool slots to and from the batch's buffers */
-  GDN_K_COUNT = 12
+  GDN_K_GEMM = 12,        /* bf16 projection GEMM (gdn_gemm_bf16, gdn_project_in, gdn_project_out) */
+  GDN_K_COUNT = 13
 } gdn_kernel_id;
 
 GDN_API const char* gdn_kernel_name(int32_t kernel_id);

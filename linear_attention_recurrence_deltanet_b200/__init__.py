@@ -19,7 +19,7 @@ import numpy as np
 __all__ = [
     "GdnError", "Config", "Params", "lib", "make_config", "conv_prefill", "conv_step", "prefill_workspace_size",
     "prefill", "prefill_noalloc", "decode_step", "decode_multi", "decode_step_indexed", "decode_multi_indexed",
-    "prefill_indexed_workspace_size", "prefill_indexed", "state_blob_size", "state_save", "state_restore", "device_status", "last_error",
+    "prefill_indexed_workspace_size", "prefill_indexed", "gemm_bf16", "project_in", "project_out", "state_blob_size", "state_save", "state_restore", "device_status", "last_error",
     "abi_version", "launch_count", "launch_count_reset", "profiler_enable", "profiler_reset", "profiler_read",
     "kernel_name", "EXPORTS", "ZERO_INIT_STATE", "ZERO_INIT_CONV", "PREFILL_RECURRENT", "PREFILL_FUSED", "K", "MAX_DRAFT_TOKENS",
 ]
@@ -42,8 +42,8 @@ STATUS = {0: "GDN_OK", -1: "GDN_E_INVAL", -2: "GDN_E_UNSUPPORTED", -3: "GDN_E_WO
 class K:
     """Kernel ids of the profiler (gdn_kernel_id)."""
     (CONV_PREFILL, CONV_STEP, CONV_HISTORY, SCHEDULE, PREFILL_RECURRENT, PREFILL_CHUNKED, DECODE, STATE_CHECKSUM,
-     SPLIT_CONV, SPLIT_PREP, SPLIT_CHAIN, SLOT_COPY) = range(12)
-    COUNT = 12
+     SPLIT_CONV, SPLIT_PREP, SPLIT_CHAIN, SLOT_COPY, GEMM) = range(13)
+    COUNT = 13
 
 
 # Every symbol include/gdn.h declares.
@@ -53,7 +53,7 @@ EXPORTS = [
     "gdn_abi_version", "gdn_launch_count", "gdn_launch_count_reset", "gdn_kernel_name", "gdn_profiler_enable",
     "gdn_profiler_reset", "gdn_profiler_read", "gdn_prefill_noalloc", "gdn_decode_multi",
     "gdn_decode_step_indexed", "gdn_decode_multi_indexed", "gdn_prefill_indexed_workspace_size",
-    "gdn_prefill_indexed",
+    "gdn_prefill_indexed", "gdn_gemm_bf16", "gdn_project_in", "gdn_project_out",
 ]
 
 
@@ -99,6 +99,9 @@ def lib():
             "gdn_decode_multi_indexed": [P, P, P, P, P, P, I32, I32, I32, P, P, I32, P, P, P, P],
             "gdn_prefill_indexed_workspace_size": [P, I64, I32, I32, P],
             "gdn_prefill_indexed": [P, P, P, P, P, P, P, P, I32, P, I32, I32, U32, P, P, P, P, SZ, P],
+            "gdn_gemm_bf16": [P, I32, I32, P, I32, P, I32, P],
+            "gdn_project_in": [P, P, I32, I32, P, P, P, P, P, P],
+            "gdn_project_out": [P, P, I32, P, I32, P, P],
             "gdn_state_blob_size": [P, P],
             "gdn_state_save": [P, P, P, I32, P, SZ, P],
             "gdn_state_restore": [P, P, SZ, I32, P, P, P],
@@ -257,6 +260,25 @@ def prefill_indexed(cfg, params, qkv, z, a, b, cu_dev, cu_host, state_indices, n
                                      cu_h.ctypes.data, cu_h.size - 1, _p(state_indices), num_slots, chunk_size, flags,
                                      _p(conv_state), _p(state), _p(o), _p(workspace), workspace_bytes,
                                      _stream(stream)))
+
+
+def gemm_bf16(x, w, y, tile_n: int = 0, stream=None):
+    """gdn_gemm_bf16: y [M, N] = x [M, K] @ w [N, K]^T, all bf16 (fp32 accumulation)."""
+    M, K = x.shape[0], x.shape[1]
+    N = w.shape[0]
+    _check(lib().gdn_gemm_bf16(_p(x), M, K, _p(w), N, _p(y), tile_n, _stream(stream)))
+
+
+def project_in(cfg, x, w_in, qkv, z, a, b, stream=None):
+    """gdn_project_in: x [T, hidden] through w_in [C_conv + Hv*d_v + 2*Hv, hidden] into qkv, z, a, b."""
+    _check(lib().gdn_project_in(ctypes.byref(cfg), _p(x), x.shape[0], x.shape[1], _p(w_in), _p(qkv), _p(z), _p(a),
+                                _p(b), _stream(stream)))
+
+
+def project_out(cfg, o, w_out, y, stream=None):
+    """gdn_project_out: y [T, hidden] = o [T, Hv*d_v] @ w_out [hidden, Hv*d_v]^T."""
+    _check(lib().gdn_project_out(ctypes.byref(cfg), _p(o), o.shape[0], _p(w_out), w_out.shape[0], _p(y),
+                                 _stream(stream)))
 
 
 def state_blob_size(cfg) -> int:

@@ -291,7 +291,7 @@ const char* gdn_kernel_name(int32_t id) {
   static const char* names[GDN_K_COUNT] = {"conv_prefill",    "conv_step",       "conv_history", "schedule",
                                            "prefill_recurrent", "prefill_chunked", "decode",       "state_checksum",
                                            "split_conv",        "split_prep",      "split_chain",
-                                           "slot_copy"};
+                                           "slot_copy",         "gemm"};
   return (id >= 0 && id < GDN_K_COUNT) ? names[id] : "unknown";
 }
 
@@ -631,6 +631,80 @@ gdn_status gdn_prefill_indexed(const gdn_config* cfg, const gdn_params* params, 
   e = gdn::launch_slot_copy(d, bf16, slots, num_seqs, false, state, conv_state, buf_state, buf_conv,
                             g_status_ptr[dev], st);
   return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_prefill_indexed scatter");
+}
+
+}  // extern "C"
+
+namespace {
+
+// output k of a GEMM: columns [start, start + width) to ptr (row pitch ld elements)
+void gemm_route(gdn::GemmOutputs& g, void* ptr, int64_t ld, int32_t width) {
+  const int k = g.count++;
+  g.ptr[k] = ptr;
+  g.ld[k] = ld;
+  g.start[k + 1] = g.start[k] + width;
+  g.vec[k] = aligned16(ptr) && ld % 8 == 0 && g.start[k] % 8 == 0;
+}
+
+gdn_status gemm_impl(const void* x, int32_t M, int32_t K, const void* w, int32_t N, int32_t tile_n,
+                     const gdn::GemmOutputs& out, gdn_stream_t stream, const char* what) {
+  gdn_status s;
+  if (M < 0 || N < 0) return fail(GDN_E_INVAL, "%s: M = %d, N = %d (must be >= 0)", what, M, N);
+  if (K <= 0 || K % 8 != 0) return fail(GDN_E_INVAL, "%s: K = %d must be a positive multiple of 8", what, K);
+  if (tile_n != 0 && tile_n != 64 && tile_n != 128 && tile_n != 256)
+    return fail(GDN_E_INVAL, "%s: tile_n %d (0, 64, 128 or 256)", what, tile_n);
+  if ((s = check_ptr(x, "x")) != GDN_OK || (s = check_ptr(w, "w")) != GDN_OK) return s;
+  for (int k = 0; k < out.count; ++k)
+    if (!out.ptr[k] || ((uintptr_t)out.ptr[k] & 1u)) return fail(GDN_E_INVAL, "%s: output %d is NULL or odd", what, k);
+  int dev = 0;
+  if ((s = check_device(&dev)) != GDN_OK) return s;
+  if (M == 0 || N == 0) return GDN_OK;
+  cudaError_t e = gdn::launch_gemm_bf16(x, M, K, w, N, tile_n, out, g_status_ptr[dev], (cudaStream_t)stream);
+  return e == cudaSuccess ? GDN_OK : cuda_fail(e, what);
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_gemm_bf16(const void* x, int32_t M, int32_t K, const void* w, int32_t N, void* y, int32_t tile_n,
+                         gdn_stream_t stream) {
+  gdn::GemmOutputs g{};
+  gemm_route(g, y, N, N);
+  return gemm_impl(x, M, K, w, N, tile_n, g, stream, "gdn_gemm_bf16");
+}
+
+gdn_status gdn_project_in(const gdn_config* cfg, const void* x, int32_t num_tokens, int32_t hidden,
+                          const void* w_in, void* qkv, void* z, void* a, void* b, gdn_stream_t stream) {
+  gdn::Dims d;
+  gdn_status s;
+  if ((s = check_cfg(cfg, &d)) != GDN_OK) return s;
+  if (cfg->io_dtype != GDN_BF16) return fail(GDN_E_UNSUPPORTED, "gdn_project_in runs bf16 io only");
+  const int64_t hvd = (int64_t)d.Hv * d.dv, n = d.C + hvd + 2LL * d.Hv;
+  if (n > 0x7fffffffLL) return fail(GDN_E_UNSUPPORTED, "projection width %lld too large", (long long)n);
+  if ((s = check_ptr(qkv, "qkv")) != GDN_OK || (s = check_ptr(z, "z")) != GDN_OK ||
+      (s = check_gate_ptr(a, "a", cfg)) != GDN_OK || (s = check_gate_ptr(b, "b", cfg)) != GDN_OK)
+    return s;
+  gdn::GemmOutputs g{};
+  gemm_route(g, qkv, d.C, (int32_t)d.C);
+  gemm_route(g, z, hvd, (int32_t)hvd);
+  gemm_route(g, a, d.Hv, d.Hv);
+  gemm_route(g, b, d.Hv, d.Hv);
+  return gemm_impl(x, num_tokens, hidden, w_in, (int32_t)n, 0, g, stream, "gdn_project_in");
+}
+
+gdn_status gdn_project_out(const gdn_config* cfg, const void* o, int32_t num_tokens, const void* w_out,
+                           int32_t hidden, void* y, gdn_stream_t stream) {
+  gdn::Dims d;
+  gdn_status s;
+  if ((s = check_cfg(cfg, &d)) != GDN_OK) return s;
+  if (cfg->io_dtype != GDN_BF16) return fail(GDN_E_UNSUPPORTED, "gdn_project_out runs bf16 io only");
+  const int64_t hvd = (int64_t)d.Hv * d.dv;
+  if (hvd > 0x7fffffffLL) return fail(GDN_E_UNSUPPORTED, "Hv * d_v too large");
+  if ((s = check_ptr(y, "y")) != GDN_OK) return s;
+  gdn::GemmOutputs g{};
+  gemm_route(g, y, hidden, hidden);
+  return gemm_impl(o, num_tokens, (int32_t)hvd, w_out, hidden, 0, g, stream, "gdn_project_out");
 }
 
 gdn_status gdn_state_blob_size(const gdn_config* cfg, size_t* bytes) {

@@ -89,6 +89,24 @@ cudaError_t launch_slot_copy(const Dims& d, bool bf16, Slots slots, int32_t num_
                              float* pool_state, void* pool_conv, float* buf_state, void* buf_conv, int32_t* status,
                              cudaStream_t stream);
 
+// gemm.cu: Y = X W^T in bf16 (fp32 accumulation), X [M, K] and W [N, K] row-major.
+// Output column c goes to the output k with start[k] <= c < start[k + 1]:
+// element (r, c) is ptr[k][r * ld[k] + c - start[k]].  start[0] = 0 and
+// start[count] = N.  vec[k] says that ptr[k] is 16-byte aligned and ld[k],
+// start[k] are multiples of 8, so whole 8-column groups may be stored at once.
+constexpr int kGemmMaxOut = 4;
+struct GemmOutputs {
+  void* ptr[kGemmMaxOut];
+  int64_t ld[kGemmMaxOut];
+  int32_t start[kGemmMaxOut + 1];
+  int32_t vec[kGemmMaxOut];
+  int32_t count;
+};
+// tile width (64, 128 or 256 columns) the launch uses for tile_n (0 = chosen from M and N)
+int gemm_tile_n(int32_t M, int32_t N, int32_t tile_n);
+cudaError_t launch_gemm_bf16(const void* x, int32_t M, int32_t K, const void* w, int32_t N, int32_t tile_n,
+                             const GemmOutputs& out, int32_t* status, cudaStream_t stream);
+
 // api.cu: records a message for gdn_last_error() on the calling thread.
 void set_error_message(const char* msg);
 // api.cu: workspace bytes of gdn_prefill with GDN_PREFILL_FUSED (the schedule only)

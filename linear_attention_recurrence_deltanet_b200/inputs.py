@@ -45,6 +45,9 @@ __all__ = [
     "make_prefill_inputs",
     "make_decode_step_tokens",
     "varlen_lengths",
+    "QWEN_HIDDEN",
+    "make_projection_weights",
+    "make_hidden_states",
     "WORKLOADS",
 ]
 
@@ -186,6 +189,27 @@ def make_decode_step_tokens(geo: Geometry, num_seqs: int, seed: int, step: int):
 def varlen_lengths(seed: int = 4, num_seqs: int = 16, max_len: int = 8192) -> np.ndarray:
     """Sequence lengths drawn uniformly from 1..max_len."""
     return np.random.default_rng(seed).integers(1, max_len + 1, num_seqs)
+
+
+# hidden size of the Qwen3.8-27B configuration (DS4Server issue #89, Model and reference contract)
+QWEN_HIDDEN = 5120
+
+
+def make_projection_weights(geo: Geometry, hidden: int, seed: int):
+    """bf16 bits of a layer's two projection weights, drawn from
+    ``default_rng([seed, 3])``: w_in [C_conv + Hv*d_v + 2*Hv, hidden] ~ N(0, 1/hidden)
+    (rows stacked qkv, z, a, b) then w_out [hidden, Hv*d_v] ~ N(0, 1/(Hv*d_v))."""
+    rng = np.random.default_rng([seed, 3])
+    n_in = geo.conv_dim + geo.value_dim + 2 * geo.num_v_heads
+    w_in = rng.standard_normal((n_in, hidden), dtype=np.float32) * np.float32(1.0 / np.sqrt(hidden))
+    w_out = rng.standard_normal((hidden, geo.value_dim), dtype=np.float32) * np.float32(1.0 / np.sqrt(geo.value_dim))
+    return bf16_bits_from_f32(w_in), bf16_bits_from_f32(w_out)
+
+
+def make_hidden_states(num_tokens: int, hidden: int, seed: int) -> np.ndarray:
+    """bf16 bits of a layer's input hidden states [T, hidden] ~ N(0, 1), from ``default_rng([seed, 4])``."""
+    rng = np.random.default_rng([seed, 4])
+    return bf16_bits_from_f32(rng.standard_normal((num_tokens, hidden), dtype=np.float32))
 
 
 QWEN_GEO = Geometry()

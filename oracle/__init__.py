@@ -63,6 +63,8 @@ def lib():
         L.gdn_ref_prefill.restype = ctypes.c_int32
         L.gdn_ref_decode_step.argtypes = [P] + [P] * 8 + [ctypes.c_int32, P, P, P, P, P, ctypes.c_int32]
         L.gdn_ref_decode_step.restype = ctypes.c_int32
+        L.gdn_ref_project.argtypes = [P, ctypes.c_int64, P, ctypes.c_int64, P, ctypes.c_int64, P, ctypes.c_int32]
+        L.gdn_ref_project.restype = None
         _lib = L
     return _lib
 
@@ -184,3 +186,26 @@ def prefill_inputs(inp, heads=None, threads=None):
     params = (inp.conv_w, inp.A_log, inp.dt_bias, inp.norm_w)
     return prefill(inp.geo, params, inp.f32("qkv"), inp.f32("z"), inp.f32("a"), inp.f32("b"), inp.cu_seqlens,
                    inp.f32("conv_state"), inp.state, heads=heads, threads=threads)
+
+
+def project(x, w, rows=None, threads: Optional[int] = None) -> np.ndarray:
+    """Linear layer y = x w^T in float64 for the listed rows of x (all rows by
+    default).  x [M, K] and w [N, K] are float arrays holding the exact values
+    of their stored dtype; returns float64 [len(rows), N]."""
+    x, w = _f32(x), _f32(w)
+    rows = np.arange(x.shape[0], dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    assert x.shape[1] == w.shape[1] and (rows.size == 0 or (rows.min() >= 0 and rows.max() < x.shape[0]))
+    y = np.empty((rows.size, w.shape[0]), np.float64)
+    lib().gdn_ref_project(_ptr(x), x.shape[1], _ptr(w), w.shape[0], _ptr(rows), rows.size, _ptr(y),
+                          threads or default_threads())
+    return y
+
+
+def split_projection(geo, y):
+    """Columns of the input projection's output, in the stacking order of its
+    weight rows: (qkv [., C_conv], z [., Hv*d_v], a [., Hv], b [., Hv])."""
+    C = 2 * geo.num_k_heads * geo.head_k_dim + geo.num_v_heads * geo.head_v_dim
+    V = geo.num_v_heads * geo.head_v_dim
+    H = geo.num_v_heads
+    assert y.shape[1] == C + V + 2 * H
+    return y[:, :C], y[:, C:C + V], y[:, C + V:C + V + H], y[:, C + V + H:]

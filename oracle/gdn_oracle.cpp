@@ -223,4 +223,30 @@ int32_t gdn_ref_decode_step(const gdn_ref_geometry* geo, const float* conv_w, co
                          o, hist_out, num_threads);
 }
 
+// Dense projection of a linear layer ("GDN projection" primitive, issue #95,
+// Verification; the BF16 projection kernels of its implementation comment):
+//   y[i][c] = sum_k x[rows[i]][k] * w[c][k]
+// for the R listed rows of x [M][K]; w [N][K] holds the layer's weight (output
+// features x input features).  Every product and sum is float64, k ascending.
+void gdn_ref_project(const float* x, int64_t K, const float* w, int64_t N, const int64_t* rows, int64_t R,
+                     double* y, int32_t num_threads) {
+  std::atomic<int64_t> next{0};
+  auto worker = [&]() {
+    for (int64_t i = next++; i < R; i = next++) {
+      const float* xr = x + rows[i] * K;
+      for (int64_t c = 0; c < N; ++c) {
+        const float* wc = w + c * K;
+        double s = 0.0;
+        for (int64_t k = 0; k < K; ++k) s += (double)xr[k] * (double)wc[k];
+        y[i * N + c] = s;
+      }
+    }
+  };
+  const int32_t nt = (int32_t)std::max<int64_t>(1, std::min<int64_t>(num_threads, R));
+  std::vector<std::thread> pool;
+  for (int32_t t = 1; t < nt; ++t) pool.emplace_back(worker);
+  worker();
+  for (auto& th : pool) th.join();
+}
+
 }  // extern "C"

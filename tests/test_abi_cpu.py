@@ -247,3 +247,35 @@ def test_truncated_blob_rejected():
     with pytest.raises(gdn.GdnError) as e:
         gdn.state_restore(gdn.make_config(geo), blob, 0, FakeTensor(4096), FakeTensor(65536), stream=0)
     assert e.value.name == "GDN_E_BLOB_FORMAT"
+
+
+def test_projection_validation_rejects_before_launch():
+    """Bad K (not a positive multiple of 8), a bad tile width, a NULL or odd
+    output and a non-bf16 config are refused on the host, buffers intact."""
+    L = gdn.lib()
+    x, w, y = FakeTensor(64 * 64 * 2), FakeTensor(64 * 64 * 2), FakeTensor(64 * 64 * 2)
+    snap = {k: t.view.copy() for k, t in dict(x=x, w=w, y=y).items()}
+    cases = [
+        (dict(M=4, K=12, N=8, y=y.data_ptr(), tile_n=0), "GDN_E_INVAL"),
+        (dict(M=4, K=0, N=8, y=y.data_ptr(), tile_n=0), "GDN_E_INVAL"),
+        (dict(M=-1, K=16, N=8, y=y.data_ptr(), tile_n=0), "GDN_E_INVAL"),
+        (dict(M=4, K=16, N=8, y=y.data_ptr(), tile_n=96), "GDN_E_INVAL"),
+        (dict(M=4, K=16, N=8, y=None, tile_n=0), "GDN_E_INVAL"),
+        (dict(M=4, K=16, N=8, y=y.data_ptr() + 1, tile_n=0), "GDN_E_INVAL"),
+    ]
+    for c, status in cases:
+        rc = L.gdn_gemm_bf16(x.data_ptr(), c["M"], c["K"], w.data_ptr(), c["N"], c["y"], c["tile_n"], None)
+        assert gdn.STATUS[rc] == status, (c, gdn.last_error())
+    rc = L.gdn_gemm_bf16(x.data_ptr() + 2, 4, 16, w.data_ptr(), 8, y.data_ptr(), 0, None)
+    assert gdn.STATUS[rc] == "GDN_E_INVAL" and "aligned" in gdn.last_error()
+    geo32 = gi.Geometry(num_k_heads=2, num_v_heads=4, head_k_dim=32, head_v_dim=32, io_dtype="f32")
+    with pytest.raises(gdn.GdnError) as e:
+        L2 = np.zeros((4, 64), np.uint16)
+        gdn.project_in(gdn.make_config(geo32), L2, np.zeros((8, 64), np.uint16), y, y, y, y, stream=0)
+    assert e.value.name == "GDN_E_UNSUPPORTED"
+    with pytest.raises(gdn.GdnError) as e:
+        gdn.project_out(gdn.make_config(geo32), np.zeros((4, 128), np.uint16), np.zeros((8, 128), np.uint16), y,
+                        stream=0)
+    assert e.value.name == "GDN_E_UNSUPPORTED"
+    for k, t in dict(x=x, w=w, y=y).items():
+        assert np.array_equal(t.view, snap[k]), k

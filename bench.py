@@ -8,7 +8,10 @@ every prefill stage of the mixer.  The decode entry point (64 sequences, one
 token each, fresh bf16 inputs per step, states ~N(0, 0.02)) is timed over
 1000 consecutive steps in the same run and reported under "decode"; K=2
 draft-and-verify rounds (a verify pass, then a commit of a seeded accepted
-prefix) on the same sequences are reported under "draft_verify".
+prefix) on the same sequences are reported under "draft_verify".  The
+layer's input and output projections (bf16 tensor-core GEMMs around the
+mixer, synthetic weights) are timed at T=4096 and at 64 tokens and reported
+under "projections", with cuBLAS on the same operands for context.
 
 Inputs are synthetic (seeded numpy draws) and resident in HBM before timing.
 Between timed prefill steps the inputs rotate over 3 sets (~540 MB, > 4x L2)
@@ -501,6 +504,8 @@ def run_gdn(args, rank, world, local_rank):
                          "time between events on the launching stream"}
     del mq, mz, ma, mb
 
+    proj = run_projections(gdn, torch, pk, stream, barrier, max_over_ranks, world, args.projection_reps)
+
     clk = clocks.summary()
     cpu = cpu_baseline(inp) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
     if rank == 0:
@@ -512,7 +517,8 @@ def run_gdn(args, rank, world, local_rank):
                                    "fp32 state from zero", "global_batch": world, "seq_len": T, "chunk": C,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": f"inputs rotate over {ROTATE} sets (> 4x L2) between steps"},
-            "roofline": roof_p, "decode": decode, "draft_verify": draft, "e2e": e2e, "gpu_launches": launches,
+            "roofline": roof_p, "decode": decode, "draft_verify": draft, "projections": proj, "e2e": e2e,
+            "gpu_launches": launches,
             "kernels": kernel_share, "clocks": clk, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
@@ -520,6 +526,83 @@ def run_gdn(args, rank, world, local_rank):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def run_projections(gdn, torch, pk, stream, barrier, max_over_ranks, world, reps):
+    """The layer's input and output projections (bf16 GEMMs on the tensor
+    cores) at the prefill (T=4096) and decode (64 tokens) sizes, with
+    synthetic weights.  Each launch is timed alone with events on the
+    launching stream, after a write of 256 MB (> L2) that evicts its operands;
+    torch.matmul (cuBLAS) on the same operands is timed the same way for
+    context.  The prefill sizes are bound by the tensor cores (roofline against
+    the measured bf16 peak), the decode sizes by streaming the weights from
+    HBM (roofline against the measured copy bandwidth)."""
+    geo = gi.QWEN_GEO
+    hidden = gi.QWEN_HIDDEN
+    cfg = gdn.make_config(geo)
+    w_in_h, w_out_h = gi.make_projection_weights(geo, hidden, 5)
+    bf = torch.bfloat16
+
+    def dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits)).view(bf).cuda()
+
+    w_in, w_out = dev(w_in_h), dev(w_out_h)
+    del w_in_h, w_out_h
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        total = 0.0
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            total += a.elapsed_time(b)
+        return max_over_ranks(total / reps)
+
+    out = {}
+    for T, tag in ((4096, "prefill_t4096"), (64, "decode_b64")):
+        x = dev(gi.make_hidden_states(T, hidden, 6))
+        qkv = torch.empty((T, geo.conv_dim), dtype=bf, device="cuda")
+        z = torch.empty((T, geo.value_dim), dtype=bf, device="cuda")
+        a = torch.empty((T, geo.num_v_heads), dtype=bf, device="cuda")
+        b = torch.empty((T, geo.num_v_heads), dtype=bf, device="cuda")
+        o = dev(gi.make_hidden_states(T, geo.value_dim, 7))
+        y = torch.empty((T, hidden), dtype=bf, device="cuda")
+        y_in = torch.empty((T, w_in.shape[0]), dtype=bf, device="cuda")
+        barrier()
+        for name, fn, ref, (M, K, N) in (
+                ("project_in", lambda: gdn.project_in(cfg, x, w_in, qkv, z, a, b, stream=stream),
+                 lambda: torch.matmul(x, w_in.t(), out=y_in), (T, hidden, w_in.shape[0])),
+                ("project_out", lambda: gdn.project_out(cfg, o, w_out, y, stream=stream),
+                 lambda: torch.matmul(o, w_out.t(), out=y), (T, geo.value_dim, hidden))):
+            ms = timed(fn)
+            ms_ref = timed(ref)
+            flops = 2.0 * M * N * K
+            nbytes = 2.0 * (M * K + N * K + M * N)
+            if T >= 256:
+                achieved, peak, unit, bound = flops / (ms / 1000.0) / 1e12, pk["bf16"], "TFLOP/s", "tensor"
+            else:
+                achieved, peak, unit, bound = nbytes / (ms / 1000.0) / 1e9, pk["hbm"], "GB/s", "hbm"
+            out[f"{name}:{tag}"] = {
+                "shape": {"M": M, "K": K, "N": N}, "ms": round(ms, 5),
+                "value": round(world * M / (ms / 1000.0), 1), "unit": "tokens/s",
+                "roofline": {"bound": bound, "achieved": round(achieved, 1), "peak": peak, "unit": unit,
+                             "frac": round(achieved / peak, 4), "traffic": None, "kernel": "gemm",
+                             "peak_source": pk["src"]},
+                "tflops": round(flops / (ms / 1000.0) / 1e12, 1), "cublas_ms": round(ms_ref, 5),
+                "vs_cublas": round(ms_ref / ms, 3)}
+        del x, qkv, z, a, b, o, y, y_in
+    del w_in, w_out, flush
+    torch.cuda.empty_cache()
+    out["workload"] = ("hidden 5120 -> qkv/z/a/b (16480 columns) and 6144 -> 5120, synthetic bf16 weights "
+                       "~N(0, 1/fan_in); each launch timed alone after a 256 MB L2-evicting write; "
+                       "cublas_ms: torch.matmul on the same operands, for context")
+    return out
 
 
 def main():
@@ -532,6 +615,7 @@ def main():
     ap.add_argument("--recurrent", action="store_true", help="time the token-recurrent prefill kernel")
     ap.add_argument("--fused", action="store_true", help="time the single-kernel chunked prefill")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--projection-reps", type=int, default=20, help="timed launches per projection shape")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     rank = int(os.environ.get("RANK", "0"))

@@ -280,7 +280,8 @@ GDN_API gdn_status gdn_prefill_indexed(const gdn_config* cfg, const gdn_params* 
  * layer's weight: output features x input features).  K must be a multiple
  * of 8 (16-byte row pitch) and X, W 16-byte aligned; M, N >= 0 (0 launches
  * nothing); M, N, K < 2^31.  No workspace.  tile_n picks the output tile
- * width: 64, 128 or 256 columns, 0 = chosen from M and N.
+ * width: a multiple of 32 up to 256 columns, or 0 = chosen from M and N (a
+ * power of two: the width that fills the SMs in the fewest, widest rounds).
  *
  * gdn_gemm_bf16: Y [M, N] row-major bf16 (2-byte aligned; rows 16-byte
  *   aligned give vector stores).

@@ -651,8 +651,8 @@ gdn_status gemm_impl(const void* x, int32_t M, int32_t K, const void* w, int32_t
   gdn_status s;
   if (M < 0 || N < 0) return fail(GDN_E_INVAL, "%s: M = %d, N = %d (must be >= 0)", what, M, N);
   if (K <= 0 || K % 8 != 0) return fail(GDN_E_INVAL, "%s: K = %d must be a positive multiple of 8", what, K);
-  if (tile_n != 0 && tile_n != 64 && tile_n != 128 && tile_n != 256)
-    return fail(GDN_E_INVAL, "%s: tile_n %d (0, 64, 128 or 256)", what, tile_n);
+  if (tile_n != 0 && (tile_n % 32 != 0 || tile_n < 32 || tile_n > 256))
+    return fail(GDN_E_INVAL, "%s: tile_n %d (0, or a multiple of 32 up to 256)", what, tile_n);
   if ((s = check_ptr(x, "x")) != GDN_OK || (s = check_ptr(w, "w")) != GDN_OK) return s;
   for (int k = 0; k < out.count; ++k)
     if (!out.ptr[k] || ((uintptr_t)out.ptr[k] & 1u)) return fail(GDN_E_INVAL, "%s: output %d is NULL or odd", what, k);

@@ -5,15 +5,23 @@
 // with W stored as a linear layer's weight (output features x input
 // features), both operands K-major, fp32 accumulation in TMEM, bf16 out.
 //
-// Persistent: one CTA per SM walks the 128 x BN output tiles (m fastest, so
-// the CTAs running together share the same few weight panels in L2).  K
-// advances 64 columns per stage through a ring of TMA loads (128-byte
-// swizzle).  Warp 0 issues the loads, warp 1 the MMAs (M = 128, N = BN,
-// K = 16; each stage's commit frees its slot), warps 2..5 drain the
-// accumulator.  TMEM holds two accumulators, so the epilogue of one tile
-// overlaps the main loop of the next.  The epilogue routes every 8-column
-// group to one of up to four outputs: the input projection writes the
-// mixer's qkv, z, a and b from one GEMM.
+// Two persistent kernels walk the output tiles (m fastest, so the CTAs
+// running together share the same few weight panels in L2).  K advances 64
+// columns per TMA box (128-byte swizzle); a ring stage holds one or two boxes
+// of each operand.  Warp 0
+// issues the loads, warp 1 the MMAs (each stage's commit frees its slot),
+// warps 2..5 drain the accumulator.  TMEM holds two accumulators, so the
+// epilogue of one tile overlaps the main loop of the next.
+//   gemm_kernel       one CTA per 128 x BN tile: small M
+//   gemm_pair_kernel  a CTA pair per 256 x BN tile, MMAs of
+//                     M = 256 issued by the even CTA over both CTAs' shared
+//                     memory: each CTA loads only half of the weight panel,
+//                     which cuts the operand bytes each SM moves per MMA by a
+//                     third at BN = 256.
+// BN is any multiple of 32 up to 256 (64 up for pairs); the host picks a
+// power-of-two width from the number of tiles per wave.
+// The epilogue routes every 8-column group to one of up to four outputs: the
+// input projection writes the mixer's qkv, z, a and b from one GEMM.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -27,26 +35,62 @@ namespace {
 using namespace tc;
 
 constexpr int GM = 128, GK = 64, kMaxStages = 8;
-constexpr int kStageA = GM * GK * 2;  // 16 KB
-constexpr int kRing = 196608;         // 192 KB of stages
-constexpr int kGemmSmem = kRing + 1024;
+constexpr int kStageA = GM * GK * 2;  // 16 KB: 128 rows of X
+constexpr int kRing = 229376;         // 224 KB of stages (seven of a pair CTA's 32 KB at BN = 256)
+constexpr int kGemmSmem = kRing + 1024;  // + alignment slack: 225 KB of the 227 KB a block may have
 constexpr int kGemmThreads = 192;
 constexpr uint32_t kTmemCols = 512;  // two accumulators of up to 256 columns
 constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr uint32_t kIdescBf16 = (1u << 7) | (1u << 10);  // A and B bf16 (kind::f16)
 
+// Store columns [col0, col0 + 32) of output row `row` (fp32 in v) as bf16.
+__device__ __forceinline__ void store_block(const GemmOutputs& out, int row, int col0, int N, const float* v) {
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    const int col = col0 + 8 * g;
+    if (col >= N) break;
+    int k = 0;
+#pragma unroll
+    for (int u = 1; u < kGemmMaxOut; ++u)
+      if (u < out.count && col >= out.start[u]) k = u;
+    if (out.vec[k] && col + 8 <= out.start[k + 1]) {  // the 8 columns land in one output: one 16-byte store
+      uint32_t w4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        __nv_bfloat162 p = __floats2bfloat162_rn(v[8 * g + 2 * e], v[8 * g + 2 * e + 1]);
+        w4[e] = *reinterpret_cast<uint32_t*>(&p);
+      }
+      __nv_bfloat16* dst =
+          reinterpret_cast<__nv_bfloat16*>(out.ptr[k]) + (int64_t)row * out.ld[k] + (col - out.start[k]);
+      *reinterpret_cast<uint4*>(dst) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    } else {  // the group crosses an output boundary or the end, or its output is not 16-byte alignable
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int c = col + e;
+        if (c >= N) break;
+        while (k + 1 < out.count && c >= out.start[k + 1]) ++k;
+        reinterpret_cast<__nv_bfloat16*>(out.ptr[k])[(int64_t)row * out.ld[k] + (c - out.start[k])] =
+            __float2bfloat16_rn(v[8 * g + e]);
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ one CTA per tile
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw, int32_t M, int32_t N,
-                int32_t K, int32_t BN, const __grid_constant__ GemmOutputs out, int32_t* status) {
+                int32_t K, int32_t BN, int32_t ksub, const __grid_constant__ GemmOutputs out, int32_t* status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   __shared__ uint64_t full[kMaxStages], empty[kMaxStages], acc_full[2], acc_empty[2], drain;
   __shared__ uint32_t tslot;
   bool bad = false;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int stage_bytes = kStageA + BN * GK * 2;
+  const int blk_b = BN * GK * 2;
+  const int stage_bytes = ksub * (kStageA + blk_b);  // ksub 64-wide K blocks per stage
   const int stages = min(kMaxStages, kRing / stage_bytes);
   const int mt = (M + GM - 1) / GM, nt = (N + BN - 1) / BN, tiles = mt * nt;
-  const int nk = (K + GK - 1) / GK;
+  const int nk = (K + GK * ksub - 1) / (GK * ksub);
 
   if (tid == 0) {
     for (int s = 0; s < stages; ++s) {
@@ -79,8 +123,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           unsigned char* a = sm + s * stage_bytes;
           mbar_expect_tx(&full[s], stage_bytes);
-          tma_load_2d(a, &tx, GK * kb, m0, &full[s]);
-          tma_load_2d(a + kStageA, &tw, GK * kb, n0, &full[s]);
+          for (int u = 0; u < ksub; ++u) {
+            tma_load_2d(a + u * kStageA, &tx, GK * (kb * ksub + u), m0, &full[s]);
+            tma_load_2d(a + ksub * kStageA + u * blk_b, &tw, GK * (kb * ksub + u), n0, &full[s]);
+          }
           last[s] = i;
         }
       }
@@ -90,7 +136,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t id = idesc_f16(GM, BN, false, false) | (1u << 7) | (1u << 10);  // bf16 A and B
+      const uint32_t id = idesc_f16(GM, BN, false, false) | kIdescBf16;
       int i = 0, j = 0;
       for (int t = blockIdx.x; t < tiles && !bad; t += gridDim.x, ++j) {
         const int ab = j & 1;
@@ -107,10 +153,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           fence_after();
-          const uint32_t a = smem_u32(sm + s * stage_bytes), b = a + kStageA;
+          const uint32_t a = smem_u32(sm + s * stage_bytes), b = a + ksub * kStageA;
+          for (int u = 0; u < ksub; ++u)
 #pragma unroll
-          for (int kk = 0; kk < GK / 16; ++kk)
-            mma_f16(d, desc_kmaj(a, GM, kk), desc_kmaj(b, BN, kk), id, (kb > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < GK / 16; ++kk)
+              mma_f16(d, desc_kmaj(a + u * kStageA, GM, kk), desc_kmaj(b + u * blk_b, BN, kk), id,
+                      (kb > 0 || u > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&empty[s]);
         }
         if (!bad) mma_commit(&acc_full[ab]);
@@ -137,36 +185,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int cb = 0; cb < BN / 32; ++cb) {
         float v[32];
         tmem_ld32(src + 32 * cb, v);
-        if (row >= M) continue;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int col = n0 + 32 * cb + 8 * g;
-          if (col >= N) break;
-          int k = 0;
-#pragma unroll
-          for (int u = 1; u < kGemmMaxOut; ++u)
-            if (u < out.count && col >= out.start[u]) k = u;
-          if (out.vec[k] && col + 8 <= out.start[k + 1]) {  // the 8 columns land in one output: one 16-byte store
-            uint32_t w4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              __nv_bfloat162 p = __floats2bfloat162_rn(v[8 * g + 2 * e], v[8 * g + 2 * e + 1]);
-              w4[e] = *reinterpret_cast<uint32_t*>(&p);
-            }
-            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(out.ptr[k]) + (int64_t)row * out.ld[k] +
-                                 (col - out.start[k]);
-            *reinterpret_cast<uint4*>(dst) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-          } else {  // the group crosses an output boundary or the end, or its output is not 16-byte alignable
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int c = col + e;
-              if (c >= N) break;
-              while (k + 1 < out.count && c >= out.start[k + 1]) ++k;
-              reinterpret_cast<__nv_bfloat16*>(out.ptr[k])[(int64_t)row * out.ld[k] + (c - out.start[k])] =
-                  __float2bfloat16_rn(v[8 * g + e]);
-            }
-          }
-        }
+        if (row < M) store_block(out, row, n0 + 32 * cb, N, v);
       }
       fence_before();
       __syncwarp();
@@ -175,6 +194,191 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   if (sync_tc_any(bad) && tid == 0) set_status(status, kStatusWaitTimeout);
   if (warp == 0) tmem_dealloc(tbase, kTmemCols);
+}
+
+// ------------------------------------------------------------------ a CTA pair per tile
+// cta_group::2 forms.  The pair's TMEM columns are allocated by one warp of
+// each CTA together; an MMA issued by the even CTA reads A rows 0..127 and B
+// rows 0..BN/2-1 from its own shared memory and A rows 128..255, B rows
+// BN/2..BN-1 from the same offsets in the odd CTA's, and writes accumulator
+// rows 0..127 to the even CTA's TMEM, rows 128..255 to the odd CTA's.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void mma_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+          d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+// one arrival on the mbarrier at this shared offset in both CTAs once this thread's MMAs are done
+__device__ __forceinline__ void commit_pair_both(uint64_t* m) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(m)),
+      "h"((uint16_t)3)
+      : "memory");
+}
+__device__ __forceinline__ void commit_pair(uint64_t* m) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(m))
+               : "memory");
+}
+// 2D tiled load into this CTA's shared memory whose bytes complete on an
+// mbarrier of either CTA of the pair (`mbar` is a shared::cluster address).  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, int x, int y, uint32_t mbar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.cta_group::2 [%0], [%1, {%2, "
+      "%3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"((uint64_t)map), "r"(x), "r"(y), "r"(mbar)
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t mbar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(mbar) : "memory");
+}
+
+constexpr int kPairRows = 256;  // output rows per pair tile; each CTA holds 128 of them
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw, int32_t M,
+                     int32_t N, int32_t K, int32_t BN, int32_t ksub, const __grid_constant__ GemmOutputs out,
+                     int32_t* status) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  // full[s] and acc_empty[b] are used in the even CTA only (both CTAs complete them);
+  // empty[s], acc_full[b] in both (the even CTA's MMA commits arrive on both)
+  __shared__ uint64_t full[kMaxStages], empty[kMaxStages], acc_full[2], acc_empty[2], drain;
+  __shared__ uint32_t tslot;
+  bool bad = false;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int half = BN / 2;
+  const int blk_b = half * GK * 2;
+  const int stage_bytes = ksub * (kStageA + blk_b);  // this CTA's share of one stage: ksub 64-wide K blocks
+  const int stages = min(kMaxStages, kRing / stage_bytes);
+  const int mt = (M + kPairRows - 1) / kPairRows, nt = (N + BN - 1) / BN, tiles = mt * nt;
+  const int nk = (K + GK * ksub - 1) / (GK * ksub);
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  if (tid == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&full[s], 1);   // the even CTA's expect_tx arrival; both CTAs' loads complete its bytes
+      mbar_init(&empty[s], 1);  // the MMA commit
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 8);  // one arrival per epilogue warp of both CTAs
+    }
+    mbar_init(&drain, 1);
+    mbar_init_fence();
+  }
+  if (warp == 0) tmem_alloc_pair(&tslot, kTmemCols);
+  fence_before();
+  cluster_sync();  // both CTAs' barriers initialised and the pair's TMEM allocated
+  fence_after();
+  const uint32_t tbase = tslot;
+  const uint32_t full_lead = mapa_shared(smem_u32(&full[0]), 0);
+  const uint32_t acc_empty_lead = mapa_shared(smem_u32(&acc_empty[0]), 0);
+
+  if (warp == 0) {
+    if (lane == 0) {  // loads of this CTA's halves: A rows 128 rank .., B rows half * rank ..
+      int i = 0;
+      int last[kMaxStages];
+      for (int s = 0; s < kMaxStages; ++s) last[s] = -1;
+      for (int t = pair; t < tiles && !bad; t += npairs) {
+        const int m0 = (t % mt) * kPairRows + GM * (int)rank, n0 = (t / mt) * BN + half * (int)rank;
+        for (int kb = 0; kb < nk; ++kb, ++i) {
+          const int s = i % stages;
+          if (i >= stages && !mbar_wait_cluster(&empty[s], ((i / stages) & 1) ^ 1, kWaitNs)) {
+            bad = true;
+            break;
+          }
+          unsigned char* a = sm + s * stage_bytes;
+          if (leader) mbar_expect_tx(&full[s], 2 * stage_bytes);
+          for (int u = 0; u < ksub; ++u) {
+            tma_load_2d_pair(a + u * kStageA, &tx, GK * (kb * ksub + u), m0, full_lead + 8 * s);
+            tma_load_2d_pair(a + ksub * kStageA + u * blk_b, &tw, GK * (kb * ksub + u), n0, full_lead + 8 * s);
+          }
+          last[s] = i;
+        }
+      }
+      if (bad) {  // let the copies already issued land before the block exits
+        if (leader) {
+          for (int s = 0; s < stages; ++s)
+            if (last[s] >= 0) mbar_wait(&full[s], (last[s] / stages) & 1, kWaitNs);
+        } else {  // their completions go to the other CTA: give them a fixed grace period
+          const uint64_t t0 = globaltimer_ns();
+          while (globaltimer_ns() - t0 < 200000ull) __nanosleep(1000);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      const uint32_t id = idesc_f16(kPairRows, BN, false, false) | kIdescBf16;
+      int i = 0, j = 0;
+      for (int t = pair; t < tiles && !bad; t += npairs, ++j) {
+        const int ab = j & 1;
+        if (j >= 2 && !mbar_wait_cluster(&acc_empty[ab], ((j >> 1) & 1) ^ 1, kWaitNs)) {
+          bad = true;
+          break;
+        }
+        fence_after();
+        const uint32_t d = tbase + 256 * ab;
+        for (int kb = 0; kb < nk; ++kb, ++i) {
+          const int s = i % stages;
+          if (!mbar_wait_cluster(&full[s], (i / stages) & 1, kWaitNs)) {
+            bad = true;
+            break;
+          }
+          fence_after();
+          const uint32_t a = smem_u32(sm + s * stage_bytes), b = a + ksub * kStageA;
+          for (int u = 0; u < ksub; ++u)
+#pragma unroll
+            for (int kk = 0; kk < GK / 16; ++kk)
+              mma_pair(d, desc_kmaj(a + u * kStageA, GM, kk), desc_kmaj(b + u * blk_b, half, kk), id,
+                       (kb > 0 || u > 0 || kk > 0) ? 1u : 0u);
+          commit_pair_both(&empty[s]);
+        }
+        if (!bad) commit_pair_both(&acc_full[ab]);
+      }
+      commit_pair(&drain);  // every MMA issued has finished before the pair's TMEM is released
+      mbar_wait(&drain, 0, kWaitNs);
+    }
+  } else {  // epilogue: this CTA's 128 rows of the tile, warp w on TMEM lanes 32 (w % 4) ..
+    const int q = warp & 3;
+    int j = 0;
+    for (int t = pair; t < tiles; t += npairs, ++j) {
+      const int ab = j & 1;
+      const bool ok = mbar_wait_cluster(&acc_full[ab], (j >> 1) & 1, kWaitNs);
+      if (__any_sync(0xffffffffu, !ok)) {
+        bad = true;
+        break;
+      }
+      fence_after();
+      const int m0 = (t % mt) * kPairRows + GM * (int)rank, n0 = (t / mt) * BN;
+      const int row = m0 + 32 * q + lane;
+      const uint32_t src = tbase + 256 * ab + ((uint32_t)(32 * q) << 16);
+#pragma unroll 1
+      for (int cb = 0; cb < BN / 32; ++cb) {
+        float v[32];
+        tmem_ld32(src + 32 * cb, v);
+        if (row < M) store_block(out, row, n0 + 32 * cb, N, v);
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(acc_empty_lead + 8 * ab);
+    }
+  }
+  if (sync_tc_any(bad) && tid == 0) set_status(status, kStatusWaitTimeout);
+  __syncwarp();
+  cluster_sync();  // the even CTA's MMAs no longer read this CTA's shared memory or write its TMEM
+  fence_after();
+  if (warp == 0) tmem_dealloc_pair(tbase, kTmemCols);
 }
 
 bool encode_bf16_2d(EncodeTiledFn enc, CUtensorMap* tm, const void* base, uint64_t cols, uint64_t rows,
@@ -199,20 +403,56 @@ int num_sms() {
   return n;
 }
 
+// CTA pairs of gemm_pair_kernel that fit on the device at once
+int max_pairs() {
+  static int n = 0;
+  if (n == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * num_sms());
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = kGemmSmem;
+    int c = 0;
+    if (cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) ==
+            cudaSuccess &&
+        cudaOccupancyMaxActiveClusters(&c, gemm_pair_kernel, &cfg) == cudaSuccess && c > 0)
+      n = c;
+    else
+      n = num_sms() / 2;
+  }
+  return n;
+}
+
+// rounds of `tiles` over `slots` concurrent tiles, times the tile width plus a
+// fixed 64 columns' worth of per-tile cost (narrower MMAs and the per-tile
+// handshakes make a narrow tile cost more than its width)
+int64_t tile_cost(int64_t tiles, int64_t slots, int bn) { return (tiles + slots - 1) / slots * (bn + 64); }
+
+// K blocks per ring stage: two wherever that still leaves three stages.  Every
+// stage costs a fixed handshake (full barrier, commit, refill), so fewer,
+// larger stages keep the tensor pipe busier; measured on the Qwen-shaped
+// projections, two blocks per stage raise the pair kernel from about 1.1 to
+// 1.5 PFLOP/s.
+int ksub(int kblock_bytes) { return kRing / (2 * kblock_bytes) >= 3 ? 2 : 1; }
+
 }  // namespace
 
-int gemm_tile_n(int32_t M, int32_t N, int32_t tile_n) {
-  if (tile_n == 64 || tile_n == 128 || tile_n == 256) return tile_n;
-  // fewest (rounds of tiles over the SMs) x (cost of one tile), a tile costing
-  // its width plus a fixed 64 columns' worth of prologue and epilogue
-  const int64_t mt = (M + GM - 1) / GM, sms = num_sms();
-  int best = 256;
+GemmPlan gemm_plan(int32_t M, int32_t N, int32_t tile_n) {
+  const int64_t sms = num_sms(), pairs = max_pairs();
+  GemmPlan best{false, 256};
   int64_t best_cost = -1;
-  for (int bn = 256; bn >= 64; bn >>= 1) {
-    const int64_t rounds = (mt * ((N + bn - 1) / bn) + sms - 1) / sms;
-    const int64_t cost = rounds * (bn + 64);
-    if (best_cost < 0 || cost < best_cost) best = bn, best_cost = cost;
-  }
+  for (int pair = 0; pair < 2; ++pair)
+    for (int bn = 256; bn >= 32; bn -= 32) {
+      // widths other than powers of two only on request: measured, 224 or 192
+      // columns never beat 256 even where they fill the last wave better
+      if (tile_n != 0 ? bn != tile_n : (bn & (bn - 1)) != 0) continue;
+      if (pair && (bn < 64 || M < kPairRows)) continue;  // pairs only where both CTAs have rows to compute
+      const int64_t rows = pair ? kPairRows : GM;
+      const int64_t tiles = (M + rows - 1) / rows * ((N + bn - 1) / bn);
+      // a pair tile is two SMs' work: its cost is that of a 128-row tile on each
+      const int64_t cost = tile_cost(tiles, pair ? pairs : sms, bn);
+      if (best_cost < 0 || cost < best_cost || (cost == best_cost && pair && !best.pair))
+        best = GemmPlan{pair != 0, bn}, best_cost = cost;
+    }
   return best;
 }
 
@@ -221,17 +461,27 @@ cudaError_t launch_gemm_bf16(const void* x, int32_t M, int32_t K, const void* w,
   if (M <= 0 || N <= 0) return cudaSuccess;
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return cudaErrorNotSupported;
-  const int bn = gemm_tile_n(M, N, tile_n);
+  const GemmPlan plan = gemm_plan(M, N, tile_n);
+  const int bn = plan.tile_n;
   CUtensorMap tx, tw;
   if (!encode_bf16_2d(enc, &tx, x, (uint64_t)K, (uint64_t)M, GM) ||
-      !encode_bf16_2d(enc, &tw, w, (uint64_t)K, (uint64_t)N, (uint32_t)bn))
+      !encode_bf16_2d(enc, &tw, w, (uint64_t)K, (uint64_t)N, (uint32_t)(plan.pair ? bn / 2 : bn)))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+  const void* fn = plan.pair ? (const void*)gemm_pair_kernel : (const void*)gemm_kernel;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
   if (e != cudaSuccess) return e;
-  const int64_t tiles = (int64_t)((M + GM - 1) / GM) * ((N + bn - 1) / bn);
-  const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
   LaunchScope scope(GDN_K_GEMM, stream);
-  gemm_kernel<<<grid, kGemmThreads, kGemmSmem, stream>>>(tx, tw, M, N, K, bn, out, status);
+  if (plan.pair) {
+    const int64_t tiles = (int64_t)((M + kPairRows - 1) / kPairRows) * ((N + bn - 1) / bn);
+    const int pairs = (int)(tiles < max_pairs() ? tiles : max_pairs());
+    gemm_pair_kernel<<<2 * pairs, kGemmThreads, kGemmSmem, stream>>>(tx, tw, M, N, K, bn, ksub(kStageA + bn * GK),
+                                                                      out, status);
+  } else {
+    const int64_t tiles = (int64_t)((M + GM - 1) / GM) * ((N + bn - 1) / bn);
+    const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
+    gemm_kernel<<<grid, kGemmThreads, kGemmSmem, stream>>>(tx, tw, M, N, K, bn, ksub(kStageA + bn * GK * 2), out,
+                                                          status);
+  }
   return cudaGetLastError();
 }
 

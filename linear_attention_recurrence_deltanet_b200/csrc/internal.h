@@ -102,8 +102,12 @@ struct GemmOutputs {
   int32_t vec[kGemmMaxOut];
   int32_t count;
 };
-// tile width (64, 128 or 256 columns) the launch uses for tile_n (0 = chosen from M and N)
-int gemm_tile_n(int32_t M, int32_t N, int32_t tile_n);
+// kernel and tile width (a multiple of 32 up to 256 columns) a launch uses; tile_n 0 = chosen from M and N
+struct GemmPlan {
+  bool pair;   // CTA-pair kernel (256-row tiles) rather than one CTA per 128-row tile
+  int tile_n;
+};
+GemmPlan gemm_plan(int32_t M, int32_t N, int32_t tile_n);
 cudaError_t launch_gemm_bf16(const void* x, int32_t M, int32_t K, const void* w, int32_t N, int32_t tile_n,
                              const GemmOutputs& out, int32_t* status, cudaStream_t stream);
 

@@ -259,7 +259,8 @@ def test_projection_validation_rejects_before_launch():
         (dict(M=4, K=12, N=8, y=y.data_ptr(), tile_n=0), "GDN_E_INVAL"),
         (dict(M=4, K=0, N=8, y=y.data_ptr(), tile_n=0), "GDN_E_INVAL"),
         (dict(M=-1, K=16, N=8, y=y.data_ptr(), tile_n=0), "GDN_E_INVAL"),
-        (dict(M=4, K=16, N=8, y=y.data_ptr(), tile_n=96), "GDN_E_INVAL"),
+        (dict(M=4, K=16, N=8, y=y.data_ptr(), tile_n=80), "GDN_E_INVAL"),
+        (dict(M=4, K=16, N=8, y=y.data_ptr(), tile_n=288), "GDN_E_INVAL"),
         (dict(M=4, K=16, N=8, y=None, tile_n=0), "GDN_E_INVAL"),
         (dict(M=4, K=16, N=8, y=y.data_ptr() + 1, tile_n=0), "GDN_E_INVAL"),
     ]

@@ -1,5 +1,7 @@
 """The bf16 projection GEMM (gdn_gemm_bf16, gdn_project_in, gdn_project_out)
-through the C ABI against the float64 oracle.
+through the C ABI against the float64 oracle.  The shapes reach both kernels:
+one CTA per 128-row tile (fewer than 256 rows, or 64-column tiles) and a CTA
+pair per 256-row tile (otherwise).
 
 Inputs are bf16; the kernel accumulates in fp32 and rounds once to bf16.
 After taking off that final rounding (U_BF16 * |ref| per element), the error
@@ -50,6 +52,8 @@ def check(y_gpu, x_bits, w_bits, rows=None):
     (130, 72, 200, 64),    # ragged M tile, K not a multiple of 64, ragged 64-wide N tile
     (257, 520, 1000, 128),
     (300, 1024, 1030, 256),  # row pitch not a multiple of 8: every group takes the element path
+    (200, 256, 512, 256),  # fewer than 256 rows: one CTA per tile at the widest tile
+    (256, 128, 384, 0),    # exactly one 256-row tile for a CTA pair
     (64, 5120, 16480, 0),  # decode-sized input projection
     (512, 6144, 5120, 0),
 ])
@@ -63,7 +67,7 @@ def test_gemm_matches_oracle(M, K, N, tile_n):
     check(y, x, w)
 
 
-@pytest.mark.parametrize("tile_n", [64, 128, 256])
+@pytest.mark.parametrize("tile_n", [32, 64, 96, 128, 160, 224, 256])
 def test_every_tile_width(tile_n):
     M, K, N = 384, 640, 704
     x, w = operands(M, K, N, seed=7)
@@ -130,5 +134,5 @@ def test_project_out_qwen_prefill_sampled_rows():
     gdn.project_out(gdn.make_config(geo), io_tensor(o), io_tensor(w_out), y)
     torch.cuda.synchronize()
     assert not torch.isnan(y).any()
-    rows = sorted({0, 127, 4095} | set(np.random.default_rng(24).integers(0, T, 21).tolist()))
+    rows = sorted({0, 127, 128, 255, 256, 4095} | set(np.random.default_rng(24).integers(0, T, 21).tolist()))
     check(y, o, w_out, rows=rows)

@@ -11,7 +11,9 @@ draft-and-verify rounds (a verify pass, then a commit of a seeded accepted
 prefix) on the same sequences are reported under "draft_verify".  The
 layer's input and output projections (bf16 tensor-core GEMMs around the
 mixer, synthetic weights) are timed at T=4096 and at 64 tokens and reported
-under "projections", with cuBLAS on the same operands for context.
+under "projections", with cuBLAS on the same operands for context.  One
+65536-token sequence on a GPU holding 6 of the 48 value heads is prefilled
+with and without the sequence-parallel carry ("seq_parallel").
 
 Inputs are synthetic (seeded numpy draws) and resident in HBM before timing.
 Between timed prefill steps the inputs rotate over 3 sets (~540 MB, > 4x L2)
@@ -505,6 +507,7 @@ def run_gdn(args, rank, world, local_rank):
     del mq, mz, ma, mb
 
     proj = run_projections(gdn, torch, pk, stream, barrier, max_over_ranks, world, args.projection_reps)
+    seqpar = run_seqpar(gdn, torch, pk, stream, barrier, max_over_ranks, world)
 
     clk = clocks.summary()
     cpu = cpu_baseline(inp) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
@@ -517,7 +520,8 @@ def run_gdn(args, rank, world, local_rank):
                                    "fp32 state from zero", "global_batch": world, "seq_len": T, "chunk": C,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": f"inputs rotate over {ROTATE} sets (> 4x L2) between steps"},
-            "roofline": roof_p, "decode": decode, "draft_verify": draft, "projections": proj, "e2e": e2e,
+            "roofline": roof_p, "decode": decode, "draft_verify": draft, "projections": proj,
+            "seq_parallel": seqpar, "e2e": e2e,
             "gpu_launches": launches,
             "kernels": kernel_share, "clocks": clk, "cpu_baseline": cpu,
         }
@@ -602,6 +606,58 @@ def run_projections(gdn, torch, pk, stream, barrier, max_over_ranks, world, reps
     out["workload"] = ("hidden 5120 -> qkv/z/a/b (16480 columns) and 6144 -> 5120, synthetic bf16 weights "
                        "~N(0, 1/fan_in); each launch timed alone after a 256 MB L2-evicting write; "
                        "cublas_ms: torch.matmul on the same operands, for context")
+    return out
+
+
+def run_seqpar(gdn, torch, pk, stream, barrier, max_over_ranks, world, reps=5):
+    """One long sequence on a GPU that holds few heads: B=1, T=65536, 2 key /
+    6 value heads x 128 (one eighth of the layer's heads, as on each of 8 GPUs
+    sharding them), chunk 64, bf16, zero start.  gdn_prefill (the state carry
+    along the sequence on 2 SMs per value head) against gdn_prefill_seqpar
+    (the carry as a scan over segments; segment count from the SM count).
+    Inputs (~270 MB) exceed L2; CUDA events on the launching stream."""
+    from linear_attention_recurrence_deltanet_b200.device import DeviceProblem
+    geo = gi.Geometry(num_k_heads=2, num_v_heads=6)
+    T = 65536
+    inp = gi.make_prefill_inputs(geo, [T], seed=3, zero_init=True)
+    dp = DeviceProblem(inp, 64)
+    ws = torch.empty(gdn.prefill_seqpar_workspace_size(dp.cfg, T, 0), dtype=torch.uint8, device="cuda")
+    used = [0]
+
+    def plain():
+        dp.prefill(gdn.ZERO_INIT_STATE, stream=stream)
+
+    def segmented():
+        used[0] = gdn.prefill_seqpar(dp.cfg, dp.params, dp.qkv, dp.z, dp.a, dp.b, T, 0, gdn.ZERO_INIT_STATE,
+                                     dp.conv_state, dp.state, dp.o, ws, stream=stream)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        b.synchronize()
+        return max_over_ranks(a.elapsed_time(b) / reps)
+
+    nbytes = prefill_bytes(geo, [T], zero_state=True)
+    out = {}
+    for name, fn in (("prefill", plain), ("seqpar", segmented)):
+        ms = timed(fn)
+        gbs = nbytes / (ms / 1000.0) / 1e9
+        out[name] = {"ms": round(ms, 4), "value": round(world * T / (ms / 1000.0), 1), "unit": "tokens/s",
+                     "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm"], "unit": "GB/s",
+                                  "frac": round(gbs / pk["hbm"], 4), "traffic": None, "algorithmic_bytes": nbytes,
+                                  "peak_source": pk["src"]}}
+    out["seqpar"]["segments"] = used[0]
+    out["speedup"] = round(out["prefill"]["ms"] / out["seqpar"]["ms"], 3)
+    out["workload"] = ("B=1, T=65536, 2 key / 6 value heads x 128 (an eighth of the layer's heads), chunk 64, "
+                       "bf16 inputs, fp32 state from zero; time per whole prefill (all kernels)")
+    del dp, ws
+    torch.cuda.empty_cache()
     return out
 
 

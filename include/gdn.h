@@ -271,6 +271,40 @@ GDN_API gdn_status gdn_prefill_indexed(const gdn_config* cfg, const gdn_params* 
                                        size_t workspace_bytes, gdn_stream_t stream);
 
 /* --------------------------------------------------------------------------
+ * Sequence-parallel prefill of ONE long sequence (the long contexts, up to
+ * 262K tokens, that issue #89 measures under Measurements and gates; the
+ * state carry is the only step of the mixer that runs along the sequence).  The total_tokens tokens are cut into P chunk-aligned
+ * segments.  Over one segment the state carry is affine in the state it
+ * starts from, S -> A S + B: A depends only on keys and gates, B is linear
+ * in the values.  So one chain pass computes every segment's A and B at
+ * once, a short pass over the P segments composes them into each segment's
+ * starting state, and a second chain pass writes the outputs.  Results match
+ * gdn_prefill of the same sequence within floating-point rounding (the
+ * composition reassociates the state products); same layouts, conv-history
+ * update and flags (GDN_ZERO_INIT_STATE, GDN_ZERO_INIT_CONV) as gdn_prefill
+ * with num_seqs = 1 and chunk 64.  bf16 io, d_k = d_v = 128 only.
+ *
+ * It pays when the GPU would otherwise sit idle during the carry: few value
+ * heads on the GPU (as when heads are sharded across GPUs).  The carry of
+ * gdn_prefill occupies 2 SMs per value head for the whole sequence; this
+ * path runs 4 P per value head over segments P times shorter, at about three
+ * times the carry's arithmetic (two output-free passes, then one with outputs).
+ * segments: P, or 0 = as many as fill the SMs (SMs / (4 Hv)); the count used
+ * (at most the number of 64-token chunks, every segment non-empty) is
+ * written to *segments_used when that pointer is non-NULL.  With one segment
+ * (e.g. 0 at 48 value heads on 148 SMs) it runs gdn_prefill's carry as is.
+ * Workspace: gdn_prefill_seqpar_workspace_size() bytes for the same
+ * (cfg, total_tokens, segments), 256-byte aligned: the chunked form's
+ * intermediates plus 3 P fp32 states per value head. */
+GDN_API gdn_status gdn_prefill_seqpar_workspace_size(const gdn_config* cfg, int64_t total_tokens,
+                                                     int32_t segments, size_t* bytes);
+GDN_API gdn_status gdn_prefill_seqpar(const gdn_config* cfg, const gdn_params* params, const void* qkv,
+                                      const void* z, const void* a, const void* b, int64_t total_tokens,
+                                      int32_t segments, uint32_t flags, void* conv_state, float* state, void* o,
+                                      void* workspace, size_t workspace_bytes, int32_t* segments_used,
+                                      gdn_stream_t stream);
+
+/* --------------------------------------------------------------------------
  * Dense projections either side of the mixer (the "GDN projection" primitive
  * of issue #95, Verification; its "BF16 projection kernels", implementation
  * comment).  All three are one bf16 GEMM on the tensor cores with fp32
@@ -362,7 +396,8 @@ typedef enum {
   GDN_K_SPLIT_CHAIN = 10, /* stage 3: the state carry across chunks and the output rows */
   GDN_K_SLOT_COPY = 11,   /* slot-indexed prefill: pool slots to and from the batch's buffers */
   GDN_K_GEMM = 12,        /* bf16 projection GEMM (gdn_gemm_bf16, gdn_project_in, gdn_project_out) */
-  GDN_K_COUNT = 13
+  GDN_K_SEQPAR = 13,      /* sequence-parallel prefill: segment set-up and the combine across segments */
+  GDN_K_COUNT = 14
 } gdn_kernel_id;
 
 GDN_API const char* gdn_kernel_name(int32_t kernel_id);

@@ -19,7 +19,7 @@ import numpy as np
 __all__ = [
     "GdnError", "Config", "Params", "lib", "make_config", "conv_prefill", "conv_step", "prefill_workspace_size",
     "prefill", "prefill_noalloc", "decode_step", "decode_multi", "decode_step_indexed", "decode_multi_indexed",
-    "prefill_indexed_workspace_size", "prefill_indexed", "gemm_bf16", "project_in", "project_out", "state_blob_size", "state_save", "state_restore", "device_status", "last_error",
+    "prefill_indexed_workspace_size", "prefill_indexed", "gemm_bf16", "project_in", "project_out", "prefill_seqpar_workspace_size", "prefill_seqpar", "state_blob_size", "state_save", "state_restore", "device_status", "last_error",
     "abi_version", "launch_count", "launch_count_reset", "profiler_enable", "profiler_reset", "profiler_read",
     "kernel_name", "EXPORTS", "ZERO_INIT_STATE", "ZERO_INIT_CONV", "PREFILL_RECURRENT", "PREFILL_FUSED", "K", "MAX_DRAFT_TOKENS",
 ]
@@ -42,8 +42,8 @@ STATUS = {0: "GDN_OK", -1: "GDN_E_INVAL", -2: "GDN_E_UNSUPPORTED", -3: "GDN_E_WO
 class K:
     """Kernel ids of the profiler (gdn_kernel_id)."""
     (CONV_PREFILL, CONV_STEP, CONV_HISTORY, SCHEDULE, PREFILL_RECURRENT, PREFILL_CHUNKED, DECODE, STATE_CHECKSUM,
-     SPLIT_CONV, SPLIT_PREP, SPLIT_CHAIN, SLOT_COPY, GEMM) = range(13)
-    COUNT = 13
+     SPLIT_CONV, SPLIT_PREP, SPLIT_CHAIN, SLOT_COPY, GEMM, SEQPAR) = range(14)
+    COUNT = 14
 
 
 # Every symbol include/gdn.h declares.
@@ -54,6 +54,7 @@ EXPORTS = [
     "gdn_profiler_reset", "gdn_profiler_read", "gdn_prefill_noalloc", "gdn_decode_multi",
     "gdn_decode_step_indexed", "gdn_decode_multi_indexed", "gdn_prefill_indexed_workspace_size",
     "gdn_prefill_indexed", "gdn_gemm_bf16", "gdn_project_in", "gdn_project_out",
+    "gdn_prefill_seqpar_workspace_size", "gdn_prefill_seqpar",
 ]
 
 
@@ -102,6 +103,8 @@ def lib():
             "gdn_gemm_bf16": [P, I32, I32, P, I32, P, I32, P],
             "gdn_project_in": [P, P, I32, I32, P, P, P, P, P, P],
             "gdn_project_out": [P, P, I32, P, I32, P, P],
+            "gdn_prefill_seqpar_workspace_size": [P, I64, I32, P],
+            "gdn_prefill_seqpar": [P, P, P, P, P, P, I64, I32, U32, P, P, P, P, SZ, P, P],
             "gdn_state_blob_size": [P, P],
             "gdn_state_save": [P, P, P, I32, P, SZ, P],
             "gdn_state_restore": [P, P, SZ, I32, P, P, P],
@@ -279,6 +282,26 @@ def project_out(cfg, o, w_out, y, stream=None):
     """gdn_project_out: y [T, hidden] = o [T, Hv*d_v] @ w_out [hidden, Hv*d_v]^T."""
     _check(lib().gdn_project_out(ctypes.byref(cfg), _p(o), o.shape[0], _p(w_out), w_out.shape[0], _p(y),
                                  _stream(stream)))
+
+
+def prefill_seqpar_workspace_size(cfg, total_tokens: int, segments: int = 0) -> int:
+    out = ctypes.c_size_t()
+    _check(lib().gdn_prefill_seqpar_workspace_size(ctypes.byref(cfg), total_tokens, segments, ctypes.byref(out)))
+    return out.value
+
+
+def prefill_seqpar(cfg, params, qkv, z, a, b, total_tokens, segments, flags, conv_state, state, o, workspace,
+                   workspace_bytes=None, stream=None) -> int:
+    """gdn_prefill_seqpar: one sequence of total_tokens tokens in `segments`
+    chunk-aligned segments (0 = from the SM count); returns the count used."""
+    prm = _params(*params)
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    used = ctypes.c_int32(0)
+    _check(lib().gdn_prefill_seqpar(ctypes.byref(cfg), ctypes.byref(prm), _p(qkv), _p(z), _p(a), _p(b), total_tokens,
+                                    segments, flags, _p(conv_state), _p(state), _p(o), _p(workspace),
+                                    workspace_bytes, ctypes.byref(used), _stream(stream)))
+    return used.value
 
 
 def state_blob_size(cfg) -> int:

@@ -291,7 +291,7 @@ const char* gdn_kernel_name(int32_t id) {
   static const char* names[GDN_K_COUNT] = {"conv_prefill",    "conv_step",       "conv_history", "schedule",
                                            "prefill_recurrent", "prefill_chunked", "decode",       "state_checksum",
                                            "split_conv",        "split_prep",      "split_chain",
-                                           "slot_copy",         "gemm"};
+                                           "slot_copy",         "gemm",            "seqpar"};
   return (id >= 0 && id < GDN_K_COUNT) ? names[id] : "unknown";
 }
 
@@ -631,6 +631,75 @@ gdn_status gdn_prefill_indexed(const gdn_config* cfg, const gdn_params* params, 
   e = gdn::launch_slot_copy(d, bf16, slots, num_seqs, false, state, conv_state, buf_state, buf_conv,
                             g_status_ptr[dev], st);
   return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_prefill_indexed scatter");
+}
+
+namespace {
+
+int device_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      n <= 0) {
+    cudaGetLastError();
+    n = 148;
+  }
+  return n;
+}
+
+gdn_status seqpar_check(const gdn_config* cfg, gdn::Dims* d, int64_t total_tokens, int32_t segments) {
+  gdn_status s;
+  if ((s = check_cfg(cfg, d)) != GDN_OK) return s;
+  if (cfg->io_dtype != GDN_BF16 || d->dk != 128 || d->dv != 128)
+    return fail(GDN_E_UNSUPPORTED, "the sequence-parallel prefill runs bf16 io with d_k = d_v = 128");
+  if (total_tokens < 0 || total_tokens > 0x7fffffffLL)
+    return fail(GDN_E_INVAL, "total_tokens %lld out of range", (long long)total_tokens);
+  if (segments < 0 || segments > 4096) return fail(GDN_E_INVAL, "segments %d outside 0..4096", segments);
+  return GDN_OK;
+}
+
+}  // namespace
+
+gdn_status gdn_prefill_seqpar_workspace_size(const gdn_config* cfg, int64_t total_tokens, int32_t segments,
+                                             size_t* bytes) {
+  gdn::Dims d;
+  gdn_status s;
+  if ((s = seqpar_check(cfg, &d, total_tokens, segments)) != GDN_OK) return s;
+  if (!bytes) return fail(GDN_E_INVAL, "bytes is NULL");
+  const int P = gdn::seqpar_segments(d, total_tokens, segments, device_sms());
+  *bytes = gdn::seqpar_layout(d, total_tokens, P).total_bytes;
+  return GDN_OK;
+}
+
+gdn_status gdn_prefill_seqpar(const gdn_config* cfg, const gdn_params* params, const void* qkv, const void* z,
+                              const void* a, const void* b, int64_t total_tokens, int32_t segments, uint32_t flags,
+                              void* conv_state, float* state, void* o, void* workspace, size_t workspace_bytes,
+                              int32_t* segments_used, gdn_stream_t stream) {
+  gdn::Dims d;
+  gdn_status s;
+  if ((s = seqpar_check(cfg, &d, total_tokens, segments)) != GDN_OK) return s;
+  if ((s = check_params(params)) != GDN_OK) return s;
+  const uint32_t known = GDN_ZERO_INIT_STATE | GDN_ZERO_INIT_CONV;
+  if (flags & ~known) return fail(GDN_E_INVAL, "flags 0x%x: only GDN_ZERO_INIT_STATE and GDN_ZERO_INIT_CONV", flags);
+  if ((s = check_ptr(conv_state, "conv_state")) != GDN_OK || (s = check_ptr(state, "state")) != GDN_OK) return s;
+  if (total_tokens > 0) {
+    if ((s = check_ptr(qkv, "qkv")) != GDN_OK || (s = check_ptr(z, "z")) != GDN_OK ||
+        (s = check_gate_ptr(a, "a", cfg)) != GDN_OK || (s = check_gate_ptr(b, "b", cfg)) != GDN_OK ||
+        (s = check_ptr(o, "o")) != GDN_OK)
+      return s;
+  }
+  const int P = gdn::seqpar_segments(d, total_tokens, segments, device_sms());
+  const size_t need = gdn::seqpar_layout(d, total_tokens, P).total_bytes;
+  if (workspace_bytes < need || !workspace)
+    return fail(GDN_E_WORKSPACE, "workspace of %zu bytes at %p, need %zu", workspace_bytes, workspace, need);
+  if (((uintptr_t)workspace & 255u) != 0) return fail(GDN_E_WORKSPACE, "workspace is not 256-byte aligned");
+  int dev = 0;
+  if ((s = check_device(&dev)) != GDN_OK) return s;
+  if (segments_used) *segments_used = P;
+  if (total_tokens == 0) return GDN_OK;
+  cudaError_t e = gdn::launch_prefill_seqpar(d, params->conv_w, params->A_log, params->dt_bias, params->norm_w, qkv,
+                                             z, a, b, total_tokens, P, flags & GDN_ZERO_INIT_STATE,
+                                             flags & GDN_ZERO_INIT_CONV, conv_state, state, o, workspace,
+                                             g_status_ptr[dev], (cudaStream_t)stream);
+  return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_prefill_seqpar launch");
 }
 
 }  // extern "C"

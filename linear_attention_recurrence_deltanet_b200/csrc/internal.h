@@ -84,6 +84,19 @@ cudaError_t launch_prefill_split(const Dims& d, const float* conv_w, const float
                                  bool zero_state, bool zero_conv, const void* conv_state, float* state, void* o,
                                  void* split_ws, int32_t* status, cudaStream_t stream);
 
+// prefill_split.cu, sequence-parallel chain (one sequence, P chunk-aligned segments): segment count for a
+// request (0 = from the SM count), workspace layout, launch
+struct SeqparLayout {
+  size_t cu1, cu_seg, coff, split, s1, s3, total_bytes;
+};
+int seqpar_segments(const Dims& d, int64_t total_tokens, int32_t requested, int32_t sms);
+SeqparLayout seqpar_layout(const Dims& d, int64_t total_tokens, int32_t P);
+cudaError_t launch_prefill_seqpar(const Dims& d, const float* conv_w, const float* A_log, const float* dt_bias,
+                                  const float* norm_w, const void* qkv, const void* z, const void* a, const void* b,
+                                  int64_t total_tokens, int32_t P, bool zero_state, bool zero_conv,
+                                  const void* conv_state, float* state, void* o, void* ws, int32_t* status,
+                                  cudaStream_t stream);
+
 // slots.cu: the batch's pool slots to contiguous buffers (to_buffer) or back
 cudaError_t launch_slot_copy(const Dims& d, bool bf16, Slots slots, int32_t num_seqs, bool to_buffer,
                              float* pool_state, void* pool_conv, float* buf_state, void* buf_conv, int32_t* status,

@@ -620,6 +620,10 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
 // and of the gate rows.  Every operand buffer is doubled, so that each copy
 // goes out two chunks ahead.
 constexpr int kChainThreads = 320;  // eight compute warps, the MMA-issuing warp, the copy-issuing warp
+struct ChainScan {
+  int32_t nseg;         // > 0: segmented use (see chain_kernel)
+  int32_t zero_u_from;  // first cluster-pair index whose U is taken as zero
+};
 constexpr int C_A = 0;          // [-W ; Qg]   K-major 128 x 128; buffer cc % 2 at +32768 (cc % 2)
 constexpr int C_P = 65536;      // [0 ; P]     K-major 128 x 64 (8 KB of zero rows, then P); buffer at +16384 (cc % 2)
 constexpr int C_U = 98304;      // U half      fp32 64 x 64, the record's image; buffer at +16384 (cc % 2)
@@ -638,9 +642,14 @@ constexpr uint32_t COL_U0 = 0, COL_Y = 128, kChainTmemCols = 256;  // accumulato
 // the state, thread (row i, warp w) columns 32 (w / 4) .. + 31 of row i in
 // registers.  Warp 8 issues the MMAs, warp 9 the bulk copies (each as soon as
 // the MMAs that read its buffer are done), so that neither waits for the other.
+//
+// Segmented use (the sequence-parallel prefill): with scan.nseg > 0 the grid
+// runs cluster pair oi over segment oi % nseg of the schedule (cu, chunk_off)
+// with its own state slot oi; pairs oi >= scan.zero_u_from treat U as zero
+// (the homogeneous part of the chunk maps).  o == nullptr skips the output rows.
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
     chain_kernel(Dims d, const unsigned char* __restrict__ records, const int32_t* __restrict__ chunk_off,
-                 const int32_t* __restrict__ order, const int32_t* __restrict__ cu, int zero_state,
+                 const int32_t* __restrict__ order, const int32_t* __restrict__ cu, int zero_state, ChainScan scan,
                  float* __restrict__ state, __nv_bfloat16* __restrict__ o, int32_t* status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -656,7 +665,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
   const int pair = blockIdx.x >> 1;
   const int h = pair % d.Hv;
   const int oi = pair / d.Hv;
-  const int n = order ? order[oi] : oi;
+  const int n = scan.nseg > 0 ? oi % scan.nseg : (order ? order[oi] : oi);
+  const int slot = scan.nseg > 0 ? oi : n;       // state slot read at the start and written at the end
+  const bool zero_u = oi >= scan.zero_u_from;    // cluster-uniform
+  const bool write_o = o != nullptr;
   const int64_t seq0 = cu[n];
   const int len = cu[n + 1] - cu[n];
   if (len <= 0) return;  // both CTAs of the cluster, before any cluster barrier
@@ -671,7 +683,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
   const int si = 32 * (warp & 3) + lane, hc = (warp >> 2) & 1;
   const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
   const int c0 = 64 * vh + 32 * hc;  // first value channel of this thread's columns
-  float* gst = state + ((int64_t)n * d.Hv + h) * kD * kD;  // stored [j][i]
+  float* gst = state + ((int64_t)slot * d.Hv + h) * kD * kD;  // stored [j][i]
 
   if (tid == 0) {
 #pragma unroll
@@ -719,12 +731,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
   };
   if (copy_warp && lane == 0) {
     issue_a(0);
-    issue_u(0);
+    if (!zero_u) issue_u(0);
     issue_ld1(0);
-    issue_gate(0);
+    if (write_o) issue_gate(0);
     if (nchunks > 1) {
       issue_a(1);
-      issue_u(1);
+      if (!zero_u) issue_u(1);
       issue_ld1(1);
     }
     if (nchunks > 2 && vh == 0) prefetch(2);
@@ -845,23 +857,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
         if (!mbar_wait(&mb_m3, c & 1, kWaitNs)) bad = true;
         if (c + 2 < nchunks) issue_a(c + 2);
         if (!mbar_wait(&mb_m5, c & 1, kWaitNs)) bad = true;  // M5 follows the delta warps' reads of U
-        if (c + 2 < nchunks) issue_u(c + 2);
+        if (c + 2 < nchunks && !zero_u) issue_u(c + 2);
       }
     } else {
       const float egC = __ldg(reinterpret_cast<const float*>(rec_of(c) + REC_META));  // used by the state update
       if (out_warp) {
-        if (c > 0) {
+        if (c > 0 && write_o) {
           if (!mbar_wait(&mb_g[(c - 1) & 1], ((c - 1) >> 1) & 1, kWaitNs)) bad = true;
           epilogue(c - 1);
         }
       } else {  // Delta = U + (-W S) -> shared (MN-major B operand)
-        if (!mbar_wait(&mb_u[c & 1], par, kWaitNs)) bad = true;
         float u[32];
-        const unsigned char* urow = sm + C_U + 16384 * (c & 1) + 256 * si;
+        if (zero_u) {
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          const float4 f = *reinterpret_cast<const float4*>(urow + (((8 * hc + m) ^ (si & 7)) << 4));
-          u[4 * m] = f.x; u[4 * m + 1] = f.y; u[4 * m + 2] = f.z; u[4 * m + 3] = f.w;
+          for (int j = 0; j < 32; ++j) u[j] = 0.f;
+        } else {
+          if (!mbar_wait(&mb_u[c & 1], par, kWaitNs)) bad = true;
+          const unsigned char* urow = sm + C_U + 16384 * (c & 1) + 256 * si;
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const float4 f = *reinterpret_cast<const float4*>(urow + (((8 * hc + m) ^ (si & 7)) << 4));
+            u[4 * m] = f.x; u[4 * m + 1] = f.y; u[4 * m + 2] = f.z; u[4 * m + 3] = f.w;
+          }
         }
         if (!mbar_wait(&mb_m3, c & 1, kWaitNs)) bad = true;
         fence_after();
@@ -890,10 +907,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
     fence_async_smem();
     if (sync_tc_any(bad)) break;
     // the output of chunk c-1 is written: its gate buffer takes chunk c+1's rows
-    if (copy_warp && lane == 0 && c + 1 < nchunks) issue_gate(c + 1);
+    if (copy_warp && lane == 0 && c + 1 < nchunks && write_o) issue_gate(c + 1);
   }
   // block-uniform: either every output warp reaches the epilogue's named barrier or none does
-  if (!sync_tc_any(bad) && out_warp) {
+  if (!sync_tc_any(bad) && out_warp && write_o) {
     const int cl = nchunks - 1;
     if (!mbar_wait(&mb_g[cl & 1], (cl >> 1) & 1, kWaitNs)) bad = true;
     epilogue(cl);
@@ -934,13 +951,14 @@ SplitLayout split_layout(const Dims& d, int64_t total_tokens, int64_t chunk_boun
   return S;
 }
 
-cudaError_t launch_prefill_split(const Dims& d, const float* conv_w, const float* A_log, const float* dt_bias,
-                                 const float* norm_w, const void* qkv, const void* z, const void* a, const void* b,
-                                 const int32_t* cu, const int32_t* order, const int32_t* chunk_off,
-                                 const int4* chunk_map, int32_t N, int64_t total_tokens, int64_t total_chunks,
-                                 bool zero_state, bool zero_conv, const void* conv_state, float* state, void* o,
-                                 void* split_ws, int32_t* status, cudaStream_t stream) {
-  if (N <= 0 || total_tokens <= 0 || total_chunks <= 0) return cudaSuccess;
+namespace {
+
+// conv + prep over the packed tokens: the per-token parts and the record of every (chunk, value head)
+cudaError_t launch_stages12(const Dims& d, const float* conv_w, const float* A_log, const float* dt_bias,
+                            const float* norm_w, const void* qkv, const void* z, const void* a, const void* b,
+                            const int32_t* cu, const int4* chunk_map, int64_t total_tokens, int64_t total_chunks,
+                            bool zero_conv, const void* conv_state, void* split_ws, int32_t* status,
+                            cudaStream_t stream) {
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return cudaErrorNotSupported;
   const SplitLayout S = split_layout(d, total_tokens, total_chunks);
@@ -964,19 +982,194 @@ cudaError_t launch_prefill_split(const Dims& d, const float* conv_w, const float
   }
   if ((e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrepSmem)) != cudaSuccess)
     return e;
-  {
-    LaunchScope scope(GDN_K_SPLIT_PREP, stream);
-    prep_kernel<<<(unsigned)(total_chunks * d.Hv), kPrepThreads, kPrepSmem, stream>>>(
-        tm_hi, tm_lo, d, chunk_map, records, cu, (const __nv_bfloat16*)qkv, zero_conv ? 1 : 0,
-        (__nv_bfloat16*)const_cast<void*>(conv_state), total_tokens, status);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
-  if ((e = cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kChainSmem)) != cudaSuccess)
-    return e;
-  LaunchScope scope(GDN_K_SPLIT_CHAIN, stream);
-  chain_kernel<<<(unsigned)((int64_t)N * d.Hv * 2), kChainThreads, kChainSmem, stream>>>(
-      d, records, chunk_off, order, cu, zero_state ? 1 : 0, state, (__nv_bfloat16*)o, status);
+  LaunchScope scope(GDN_K_SPLIT_PREP, stream);
+  prep_kernel<<<(unsigned)(total_chunks * d.Hv), kPrepThreads, kPrepSmem, stream>>>(
+      tm_hi, tm_lo, d, chunk_map, records, cu, (const __nv_bfloat16*)qkv, zero_conv ? 1 : 0,
+      (__nv_bfloat16*)const_cast<void*>(conv_state), total_tokens, status);
   return cudaGetLastError();
 }
 
+cudaError_t launch_chain(const Dims& d, const unsigned char* records, const int32_t* chunk_off, const int32_t* order,
+                         const int32_t* cu, int64_t pairs, bool zero_state, ChainScan scan, float* state, void* o,
+                         int32_t* status, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kChainSmem);
+  if (e != cudaSuccess) return e;
+  LaunchScope scope(GDN_K_SPLIT_CHAIN, stream);
+  chain_kernel<<<(unsigned)(pairs * 2), kChainThreads, kChainSmem, stream>>>(
+      d, records, chunk_off, order, cu, zero_state ? 1 : 0, scan, state, (__nv_bfloat16*)o, status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_split(const Dims& d, const float* conv_w, const float* A_log, const float* dt_bias,
+                                 const float* norm_w, const void* qkv, const void* z, const void* a, const void* b,
+                                 const int32_t* cu, const int32_t* order, const int32_t* chunk_off,
+                                 const int4* chunk_map, int32_t N, int64_t total_tokens, int64_t total_chunks,
+                                 bool zero_state, bool zero_conv, const void* conv_state, float* state, void* o,
+                                 void* split_ws, int32_t* status, cudaStream_t stream) {
+  if (N <= 0 || total_tokens <= 0 || total_chunks <= 0) return cudaSuccess;
+  cudaError_t e = launch_stages12(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, cu, chunk_map, total_tokens,
+                                  total_chunks, zero_conv, conv_state, split_ws, status, stream);
+  if (e != cudaSuccess) return e;
+  const unsigned char* records = (unsigned char*)split_ws + split_layout(d, total_tokens, total_chunks).records;
+  return launch_chain(d, records, chunk_off, order, cu, (int64_t)N * d.Hv, zero_state, ChainScan{0, 0x7fffffff},
+                      state, o, status, stream);
+}
+
+// ------------------------------------------------------------------ sequence-parallel chain
+// One sequence cut into P chunk-aligned segments.  Over segment j the state
+// carry is affine in the state it starts from, S -> A_j S + B_j (A_j acts on
+// the key index and depends only on the keys and gates; B_j is linear in the
+// values), so
+//   B_j = the segment's final state from S = 0,
+//   A_j = its final state from S = I with every U taken as zero (d_k = d_v),
+// both from one chain launch over all segments at once.  A sequential pass over
+// the P segments then gives every segment's true starting state, and a second
+// chain launch writes the outputs.  The per-chunk records come from one conv +
+// prep pass over the whole sequence: they do not depend on the state.
+// States are stored transposed (stored = S^T), so the update is
+//   T_{j+1} = T_j stored(A_j) + stored(B_j)   (row-major products).
+namespace {
+
+constexpr int kCombRows = 16;  // rows of T per combine block
+
+// cu1 = {0, T}; segment table; phase-1 state slots: zeros (B runs), identities (A runs)
+__global__ void __launch_bounds__(256)
+    seqpar_init_kernel(int32_t T, int32_t P, int32_t seg_chunks, int32_t Hv, int32_t* cu1, int32_t* cu_seg,
+                       int32_t* coff, float* s1) {
+  const int64_t D2 = (int64_t)kD * kD;
+  if (blockIdx.x == gridDim.x - 1) {
+    if (threadIdx.x == 0) {
+      cu1[0] = 0;
+      cu1[1] = T;
+    }
+    for (int j = threadIdx.x; j <= P; j += blockDim.x) {
+      const int64_t t = (int64_t)j * seg_chunks * kC;
+      cu_seg[j] = (int32_t)(t < T ? t : T);
+      if (j < P) coff[j] = j * seg_chunks;
+    }
+    return;
+  }
+  const int slot = blockIdx.x / Hv;  // blockIdx.x = slot * Hv + h
+  float* dst = s1 + (int64_t)blockIdx.x * D2;
+  const bool ident = slot >= P;
+  for (int i = threadIdx.x; i < D2; i += blockDim.x) dst[i] = (ident && (i / kD) == (i % kD)) ? 1.0f : 0.0f;
+}
+
+// T_0 = the sequence's starting state (or zero); s3[j] = T_j, T_{j+1} = T_j A'_j + B'_j
+// with A'_j = s1[P + j], B'_j = s1[j] (stored forms).  Block = (value head, 16 rows of T); thread = column.
+__global__ void __launch_bounds__(kD)
+    seqpar_combine_kernel(int32_t P, int32_t Hv, const float* __restrict__ s1, const float* __restrict__ s_init,
+                          float* __restrict__ s3) {
+  extern __shared__ float smc[];
+  float* As = smc;                 // [kD][kD] stored A'_j
+  float* Ts = smc + kD * kD;       // [kCombRows][kD] rows of T_j
+  const int64_t D2 = (int64_t)kD * kD;
+  const int groups = kD / kCombRows;
+  const int h = blockIdx.x / groups, r0 = (blockIdx.x % groups) * kCombRows, k = threadIdx.x;
+  float t[kCombRows];
+#pragma unroll
+  for (int r = 0; r < kCombRows; ++r) t[r] = s_init ? s_init[h * D2 + (int64_t)(r0 + r) * kD + k] : 0.0f;
+  for (int j = 0; j < P; ++j) {
+#pragma unroll
+    for (int r = 0; r < kCombRows; ++r) s3[((int64_t)j * Hv + h) * D2 + (int64_t)(r0 + r) * kD + k] = t[r];
+    if (j == P - 1) break;
+    const float* A = s1 + ((int64_t)(P + j) * Hv + h) * D2;
+    const float* B = s1 + ((int64_t)j * Hv + h) * D2;
+    __syncthreads();  // the previous step's reads of As and Ts are done
+    for (int i = k; i < D2 / 4; i += kD) reinterpret_cast<float4*>(As)[i] = reinterpret_cast<const float4*>(A)[i];
+#pragma unroll
+    for (int r = 0; r < kCombRows; ++r) Ts[r * kD + k] = t[r];
+    __syncthreads();
+    float acc[kCombRows];
+#pragma unroll
+    for (int r = 0; r < kCombRows; ++r) acc[r] = B[(int64_t)(r0 + r) * kD + k];
+#pragma unroll 4
+    for (int l = 0; l < kD; ++l) {
+      const float a = As[l * kD + k];
+#pragma unroll
+      for (int r = 0; r < kCombRows; ++r) acc[r] = fmaf(Ts[r * kD + l], a, acc[r]);
+    }
+#pragma unroll
+    for (int r = 0; r < kCombRows; ++r) t[r] = acc[r];
+  }
+}
+
+constexpr int kCombSmem = (kD * kD + kCombRows * kD) * 4;
+
+}  // namespace
+
+int seqpar_segments(const Dims& d, int64_t total_tokens, int32_t requested, int32_t sms) {
+  const int64_t nchunks = (total_tokens + kC - 1) / kC;
+  if (nchunks <= 0) return 1;
+  int64_t P = requested > 0 ? requested : (int64_t)sms / (4 * d.Hv);  // phase 1 runs 2 P Hv clusters of two CTAs
+  P = P < 1 ? 1 : (P > nchunks ? nchunks : P);
+  const int64_t seg_chunks = (nchunks + P - 1) / P;
+  return (int)((nchunks + seg_chunks - 1) / seg_chunks);  // every segment non-empty
+}
+
+SeqparLayout seqpar_layout(const Dims& d, int64_t total_tokens, int32_t P) {
+  SeqparLayout S;
+  const int64_t nchunks = (total_tokens + kC - 1) / kC;
+  const size_t st = (size_t)d.Hv * kD * kD * 4;
+  S.cu1 = 0;
+  S.cu_seg = 256;
+  S.coff = al256(S.cu_seg + 4 * (size_t)(P + 1));
+  S.split = al256(S.coff + 4 * (size_t)P);
+  S.s1 = al256(S.split + split_layout(d, total_tokens, nchunks).total_bytes);
+  S.s3 = al256(S.s1 + 2 * (size_t)P * st);
+  S.total_bytes = al256(S.s3 + (size_t)P * st);
+  return S;
+}
+
+cudaError_t launch_prefill_seqpar(const Dims& d, const float* conv_w, const float* A_log, const float* dt_bias,
+                                  const float* norm_w, const void* qkv, const void* z, const void* a, const void* b,
+                                  int64_t total_tokens, int32_t P, bool zero_state, bool zero_conv,
+                                  const void* conv_state, float* state, void* o, void* ws, int32_t* status,
+                                  cudaStream_t stream) {
+  if (total_tokens <= 0) return cudaSuccess;
+  const int64_t nchunks = (total_tokens + kC - 1) / kC;
+  const int32_t seg_chunks = (int32_t)((nchunks + P - 1) / P);
+  const SeqparLayout L = seqpar_layout(d, total_tokens, P);
+  unsigned char* w = (unsigned char*)ws;
+  int32_t* cu1 = (int32_t*)(w + L.cu1);
+  int32_t* cu_seg = (int32_t*)(w + L.cu_seg);
+  int32_t* coff = (int32_t*)(w + L.coff);
+  float* s1 = (float*)(w + L.s1);
+  float* s3 = (float*)(w + L.s3);
+  const size_t st = (size_t)d.Hv * kD * kD;
+  cudaError_t e;
+  {  // one segment needs only cu1 (the last block's tables), not the phase-1 slots
+    LaunchScope scope(GDN_K_SEQPAR, stream);
+    seqpar_init_kernel<<<(unsigned)((P > 1 ? 2 * P * d.Hv : 0) + 1), 256, 0, stream>>>(
+        (int32_t)total_tokens, P, seg_chunks, d.Hv, cu1, cu_seg, coff, s1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if ((e = launch_stages12(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, cu1, nullptr, total_tokens, nchunks,
+                           zero_conv, conv_state, w + L.split, status, stream)) != cudaSuccess)
+    return e;
+  const unsigned char* records = w + L.split + split_layout(d, total_tokens, nchunks).records;
+  if (P == 1)  // the ordinary carry over the whole sequence
+    return launch_chain(d, records, nullptr, nullptr, cu1, d.Hv, zero_state, ChainScan{0, 0x7fffffff}, state, o,
+                        status, stream);
+  // every segment's B (pairs 0 .. P-1) and A (pairs P .. 2P-1), no output
+  if ((e = launch_chain(d, records, coff, nullptr, cu_seg, 2LL * P * d.Hv, false, ChainScan{P, P}, s1, nullptr,
+                        status, stream)) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(seqpar_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kCombSmem)) !=
+      cudaSuccess)
+    return e;
+  {
+    LaunchScope scope(GDN_K_SEQPAR, stream);
+    seqpar_combine_kernel<<<(unsigned)(d.Hv * (kD / kCombRows)), kD, kCombSmem, stream>>>(
+        P, d.Hv, s1, zero_state ? nullptr : state, s3);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  // the outputs, every segment from its true starting state; slot P-1 ends with the sequence's final state
+  if ((e = launch_chain(d, records, coff, nullptr, cu_seg, (int64_t)P * d.Hv, false, ChainScan{P, 0x7fffffff}, s3,
+                        o, status, stream)) != cudaSuccess)
+    return e;
+  return cudaMemcpyAsync(state, s3 + (size_t)(P - 1) * st, st * sizeof(float), cudaMemcpyDeviceToDevice, stream);
+}
 }  // namespace gdn

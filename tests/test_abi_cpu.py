@@ -280,3 +280,38 @@ def test_projection_validation_rejects_before_launch():
     assert e.value.name == "GDN_E_UNSUPPORTED"
     for k, t in dict(x=x, w=w, y=y).items():
         assert np.array_equal(t.view, snap[k]), k
+
+
+def test_seqpar_validation_and_workspace():
+    """gdn_prefill_seqpar takes bf16 with d = 128 only; bad segment counts and
+    flags are refused on the host, buffers intact; the workspace grows with
+    the segment count (3 fp32 states per segment and value head)."""
+    geo = gi.Geometry(num_k_heads=2, num_v_heads=6)
+    cfg = gdn.make_config(geo)
+    w4 = gdn.prefill_seqpar_workspace_size(cfg, 65536, 4)
+    w8 = gdn.prefill_seqpar_workspace_size(cfg, 65536, 8)
+    assert w8 - w4 >= 3 * 4 * geo.num_v_heads * 128 * 128 * 4
+    assert w4 > gdn.prefill_workspace_size(cfg, 65536, 1, 64)  # the chunked form's intermediates plus the states
+    for g, status in [(gi.Geometry(num_k_heads=2, num_v_heads=6, head_k_dim=64, head_v_dim=64), "GDN_E_UNSUPPORTED"),
+                      (gi.Geometry(num_k_heads=2, num_v_heads=6, io_dtype="f32"), "GDN_E_UNSUPPORTED")]:
+        with pytest.raises(gdn.GdnError) as e:
+            gdn.prefill_seqpar_workspace_size(gdn.make_config(g), 1000, 0)
+        assert e.value.name == status
+    for T, seg in [(-1, 0), (1000, -2), (1000, 5000)]:
+        with pytest.raises(gdn.GdnError) as e:
+            gdn.prefill_seqpar_workspace_size(cfg, T, seg)
+        assert e.value.name == "GDN_E_INVAL"
+    t = dict(qkv=FakeTensor(100 * geo.conv_dim * 2), z=FakeTensor(100 * geo.value_dim * 2),
+             a=FakeTensor(100 * 6 * 2), b=FakeTensor(100 * 6 * 2), conv=FakeTensor(3 * geo.conv_dim * 2),
+             state=FakeTensor(6 * 128 * 128 * 4), o=FakeTensor(100 * geo.value_dim * 2), ws=FakeTensor(w4))
+    params = tuple(FakeTensor(n) for n in (geo.conv_dim * 16, 24, 24, 512))
+    snap = {k: v.view.copy() for k, v in t.items()}
+    cases = [(gdn.PREFILL_RECURRENT, t["ws"], "GDN_E_INVAL"),   # only the two ZERO_INIT flags
+             (0, None, "GDN_E_WORKSPACE")]
+    for flags, ws, status in cases:
+        with pytest.raises(gdn.GdnError) as e:
+            gdn.prefill_seqpar(cfg, params, t["qkv"], t["z"], t["a"], t["b"], 100, 2, flags, t["conv"], t["state"],
+                               t["o"], ws, workspace_bytes=0 if ws is None else None, stream=0)
+        assert e.value.name == status
+    for k, v in t.items():
+        assert np.array_equal(v.view, snap[k]), k

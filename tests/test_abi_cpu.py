@@ -315,3 +315,26 @@ def test_seqpar_validation_and_workspace():
         assert e.value.name == status
     for k, v in t.items():
         assert np.array_equal(v.view, snap[k]), k
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/gdn.h compiles as C99 and a C program links against libgdn.so
+    and calls entry points that need no GPU."""
+    import subprocess
+    src = tmp_path / "abi.c"
+    src.write_text(
+        '#include "gdn.h"\n#include <stdio.h>\n#include <string.h>\n'
+        'int main(void) {\n'
+        '  gdn_config cfg; size_t bytes = 0; memset(&cfg, 0, sizeof cfg);\n'
+        '  cfg.num_k_heads = 16; cfg.num_v_heads = 48; cfg.head_k_dim = 128; cfg.head_v_dim = 128;\n'
+        '  cfg.conv_width = 4; cfg.l2_eps = 1e-6f; cfg.norm_eps = 1e-6f; cfg.q_scale = 1.0f; cfg.io_dtype = GDN_BF16;\n'
+        '  if (gdn_prefill_workspace_size(&cfg, 4096, 1, 64, &bytes) != GDN_OK || bytes == 0) return 2;\n'
+        '  if (gdn_gemm_bf16(NULL, 4, 12, NULL, 8, NULL, 0, NULL) != GDN_E_INVAL) return 3;\n'
+        '  printf("%d %s %zu\\n", gdn_abi_version(), gdn_kernel_name(GDN_K_DECODE), bytes);\n'
+        '  return 0;\n}\n')
+    lib_dir = os.path.join(ROOT, "linear_attention_recurrence_deltanet_b200")
+    exe = tmp_path / "abi"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src), "-o",
+                    str(exe), "-L", lib_dir, "-lgdn", "-Wl,-rpath," + lib_dir], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    assert out[0] == "1" and out[1] == "decode" and int(out[2]) > 0

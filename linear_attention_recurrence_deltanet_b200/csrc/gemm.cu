@@ -25,6 +25,8 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "../../include/gdn.h"
 #include "internal.h"
 #include "tc.cuh"
@@ -194,6 +196,142 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   if (sync_tc_any(bad) && tid == 0) set_status(status, kStatusWaitTimeout);
   if (warp == 0) tmem_dealloc(tbase, kTmemCols);
+}
+
+// ------------------------------------------------------------------ split-K over a cluster (M <= 128)
+// A cluster of S CTAs per 128 x BN output tile (only one row tile: M <= 128),
+// CTA `rank` accumulating K blocks [kb0, kb1) in its own TMEM.  When M is
+// small the weight stream is the limit and few tiles leave SMs idle; slicing
+// K puts S CTAs on each tile.  After a cluster barrier (every MMA of the
+// cluster is done, the leader's ring is free) the other CTAs store their fp32
+// partial rows into the leader's ring through distributed shared memory;
+// after a second barrier the leader adds them to its own and writes the tile.
+__device__ __forceinline__ void st_cluster_v4(uint32_t caddr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(caddr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_splitk_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw, int32_t M,
+                       int32_t N, int32_t K, int32_t BN, int32_t S, int32_t Mp, uint32_t tcols,
+                       const __grid_constant__ GemmOutputs out, int32_t* status) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  __shared__ uint64_t full[kMaxStages], empty[kMaxStages], acc_full;
+  __shared__ uint32_t tslot;
+  bool bad = false;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rank = (int)cluster_ctarank(), tile = blockIdx.x / S;
+  const int n0 = tile * BN;
+  const int blk_b = BN * GK * 2, stage_bytes = kStageA + blk_b;
+  const int stages = min(kMaxStages, kRing / stage_bytes);
+  const int nkb = (K + GK - 1) / GK;
+  const int kb0 = (int)((int64_t)nkb * rank / S), kb1 = (int)((int64_t)nkb * (rank + 1) / S);
+  const int nk = kb1 - kb0;  // >= 1: the host keeps S <= nkb
+
+  if (tid == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(&acc_full, 1);
+    mbar_init_fence();
+  }
+  if (warp == 0) tmem_alloc(&tslot, tcols);
+  sync_tc();
+  const uint32_t tbase = tslot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int last[kMaxStages];
+      for (int s = 0; s < kMaxStages; ++s) last[s] = -1;
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % stages;
+        if (i >= stages && !mbar_wait(&empty[s], ((i / stages) & 1) ^ 1, kWaitNs)) {
+          bad = true;
+          break;
+        }
+        unsigned char* a = sm + s * stage_bytes;
+        mbar_expect_tx(&full[s], stage_bytes);
+        tma_load_2d(a, &tx, GK * (kb0 + i), 0, &full[s]);
+        tma_load_2d(a + kStageA, &tw, GK * (kb0 + i), n0, &full[s]);
+        last[s] = i;
+      }
+      if (bad)
+        for (int s = 0; s < stages; ++s)
+          if (last[s] >= 0) mbar_wait(&full[s], (last[s] / stages) & 1, kWaitNs);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id = idesc_f16(GM, BN, false, false) | kIdescBf16;
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % stages;
+        if (!mbar_wait(&full[s], (i / stages) & 1, kWaitNs)) {
+          bad = true;
+          break;
+        }
+        fence_after();
+        const uint32_t a = smem_u32(sm + s * stage_bytes), b = a + kStageA;
+#pragma unroll
+        for (int kk = 0; kk < GK / 16; ++kk)
+          mma_f16(tbase, desc_kmaj(a, GM, kk), desc_kmaj(b, BN, kk), id, (i > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&empty[s]);
+      }
+      mma_commit(&acc_full);  // also when a wait ran out: every MMA issued has finished once it arrives
+    }
+  } else {
+    const bool ok = mbar_wait(&acc_full, 0, kWaitNs);
+    if (__any_sync(0xffffffffu, !ok)) bad = true;
+    fence_after();
+  }
+  // every MMA of the cluster is done: the leader's ring takes the partial rows
+  fence_before();
+  __syncwarp();
+  cluster_sync();
+  fence_after();
+  const int q = warp & 3, row = 32 * q + lane;
+  const bool epi = warp >= 2;
+  if (epi && rank > 0 && !bad) {
+    const uint32_t slot = mapa_shared(smem_u32(sm), 0) + (uint32_t)((rank - 1) * Mp + row) * (uint32_t)(BN * 4);
+#pragma unroll 1
+    for (int cb = 0; cb < BN / 32; ++cb) {
+      float v[32];
+      tmem_ld32(tbase + ((uint32_t)(32 * q) << 16) + 32 * cb, v);
+      if (row < Mp)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {  // 16-byte piece c of the 32 columns, rotated by row against bank conflicts
+          const int pc = (c + row) & 7;
+          st_cluster_v4(slot + 128 * cb + 16 * pc, v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+        }
+    }
+  }
+  fence_before();
+  __syncwarp();
+  cluster_sync();  // the partial rows are in the leader's shared memory
+  fence_after();
+  if (epi && rank == 0 && !bad) {
+#pragma unroll 1
+    for (int cb = 0; cb < BN / 32; ++cb) {
+      float v[32];
+      tmem_ld32(tbase + ((uint32_t)(32 * q) << 16) + 32 * cb, v);
+      if (row < M) {
+        for (int r = 1; r < S; ++r) {
+          const float* p = reinterpret_cast<const float*>(sm + ((size_t)(r - 1) * Mp + row) * BN * 4 + 128 * cb);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const float4 f = *reinterpret_cast<const float4*>(p + 4 * ((c + row) & 7));
+            v[4 * c] += f.x;
+            v[4 * c + 1] += f.y;
+            v[4 * c + 2] += f.z;
+            v[4 * c + 3] += f.w;
+          }
+        }
+        store_block(out, row, n0 + 32 * cb, N, v);
+      }
+    }
+  }
+  if (sync_tc_any(bad) && tid == 0) set_status(status, kStatusWaitTimeout);
+  if (warp == 0) tmem_dealloc(tbase, tcols);
 }
 
 // ------------------------------------------------------------------ a CTA pair per tile
@@ -456,12 +594,69 @@ GemmPlan gemm_plan(int32_t M, int32_t N, int32_t tile_n) {
   return best;
 }
 
+SplitPlan gemm_split_plan(int32_t M, int32_t N, int32_t K, int32_t tile_n) {
+  SplitPlan best{0, 1, 0};
+  if (M > GM) return best;
+  // Up to 128 rows the weight stream bounds the time.  Measured per CTA (one
+  // per SM): about 46, 27 and 18 GB/s of weights at 256-, 128- and 64-column
+  // tiles, and about 4.2 TB/s for the whole device.  A split tile pays about
+  // 6 us more (pipeline fill, two cluster barriers, the partial rows through
+  // DSMEM), and at 256 columns its reduction outweighs the split: measured,
+  // 64 x 6144 x 5120 took 28.7 us split 3 ways at 128 columns, 38.9 us split
+  // 4 ways at 256 and 36.9 us unsplit at 64.
+  const int64_t sms = num_sms(), nkb = (K + GK - 1) / GK;
+  const int Mp = (M + 31) / 32 * 32;
+  double best_t = -1.0;
+  for (int bn = 256; bn >= 64; bn >>= 1) {
+    if (tile_n != 0 && bn != tile_n) continue;
+    const double rate = bn == 256 ? 46e9 : (bn == 128 ? 27e9 : 18e9);
+    const int64_t ntiles = (N + bn - 1) / bn;
+    for (int S = 1; S <= 8 && S <= nkb; ++S) {
+      if (S > 1 && (bn > 128 || ntiles * S > sms || (int64_t)(S - 1) * Mp * bn * 4 > kRing)) break;
+      const double per_cta = (double)bn * 128.0 * (double)((nkb + S - 1) / S);  // weight bytes of one CTA's tile
+      const double rounds = S > 1 ? 1.0 : (double)((ntiles + sms - 1) / sms);
+      const double t = std::max(rounds * per_cta / rate + (S > 1 ? 6e-6 : 0.0), (double)N * K * 2.0 / 4.2e12);
+      if (best_t < 0 || t < best_t * 0.97) best = SplitPlan{bn, S, Mp}, best_t = t;
+    }
+  }
+  return best;
+}
+
 cudaError_t launch_gemm_bf16(const void* x, int32_t M, int32_t K, const void* w, int32_t N, int32_t tile_n,
                              const GemmOutputs& out, int32_t* status, cudaStream_t stream) {
   if (M <= 0 || N <= 0) return cudaSuccess;
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return cudaErrorNotSupported;
-  const GemmPlan plan = gemm_plan(M, N, tile_n);
+  const SplitPlan sp = gemm_split_plan(M, N, K, tile_n == 0 || tile_n == 64 || tile_n == 128 || tile_n == 256
+                                                    ? tile_n : -1);
+  if (sp.split > 1) {  // a cluster of sp.split CTAs per tile, each on a slice of K
+    CUtensorMap tx, tw;
+    if (!encode_bf16_2d(enc, &tx, x, (uint64_t)K, (uint64_t)M, GM) ||
+        !encode_bf16_2d(enc, &tw, w, (uint64_t)K, (uint64_t)N, (uint32_t)sp.tile_n))
+      return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(gemm_splitk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+    if (e != cudaSuccess) return e;
+    const int ntiles = (N + sp.tile_n - 1) / sp.tile_n;
+    uint32_t tcols = 32;
+    while ((int)tcols < sp.tile_n) tcols <<= 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(ntiles * sp.split));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = kGemmSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)sp.split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    LaunchScope scope(GDN_K_GEMM, stream);
+    e = cudaLaunchKernelEx(&cfg, gemm_splitk_kernel, tx, tw, M, N, K, (int32_t)sp.tile_n, (int32_t)sp.split,
+                           (int32_t)sp.mp, tcols, out, status);
+    return e != cudaSuccess ? e : cudaGetLastError();
+  }
+  const GemmPlan plan = gemm_plan(M, N, sp.tile_n ? sp.tile_n : tile_n);
   const int bn = plan.tile_n;
   CUtensorMap tx, tw;
   if (!encode_bf16_2d(enc, &tx, x, (uint64_t)K, (uint64_t)M, GM) ||

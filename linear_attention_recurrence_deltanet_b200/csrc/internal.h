@@ -121,6 +121,13 @@ struct GemmPlan {
   int tile_n;
 };
 GemmPlan gemm_plan(int32_t M, int32_t N, int32_t tile_n);
+// up to 128 rows: tile width and K split of the cluster kernel (split 1 = not used); tile_n -1 = no split
+struct SplitPlan {
+  int tile_n;  // 0 when M > 128
+  int split;
+  int mp;      // rows of a partial tile kept for the reduction (M rounded up to 32)
+};
+SplitPlan gemm_split_plan(int32_t M, int32_t N, int32_t K, int32_t tile_n);
 cudaError_t launch_gemm_bf16(const void* x, int32_t M, int32_t K, const void* w, int32_t N, int32_t tile_n,
                              const GemmOutputs& out, int32_t* status, cudaStream_t stream);
 

@@ -1,7 +1,8 @@
 """The bf16 projection GEMM (gdn_gemm_bf16, gdn_project_in, gdn_project_out)
-through the C ABI against the float64 oracle.  The shapes reach both kernels:
-one CTA per 128-row tile (fewer than 256 rows, or 64-column tiles) and a CTA
-pair per 256-row tile (otherwise).
+through the C ABI against the float64 oracle.  The shapes reach all three
+kernels: one CTA per 128-row tile, a CTA pair per 256-row tile, and (up to
+128 rows) a cluster of CTAs per tile splitting K and reducing through
+distributed shared memory.
 
 Inputs are bf16; the kernel accumulates in fp32 and rounds once to bf16.
 After taking off that final rounding (U_BF16 * |ref| per element), the error
@@ -54,7 +55,10 @@ def check(y_gpu, x_bits, w_bits, rows=None):
     (300, 1024, 1030, 256),  # row pitch not a multiple of 8: every group takes the element path
     (200, 256, 512, 256),  # fewer than 256 rows: one CTA per tile at the widest tile
     (256, 128, 384, 0),    # exactly one 256-row tile for a CTA pair
-    (64, 5120, 16480, 0),  # decode-sized input projection
+    (64, 5120, 16480, 0),  # decode-sized input projection: K split over a cluster of 2
+    (33, 640, 1000, 0),    # ragged rows, one CTA per tile
+    (40, 6144, 5120, 128),  # K split over a cluster of 3, partial rows padded to 64
+    (128, 6144, 5120, 0),  # decode-sized output projection shape at 128 rows: K split over 3
     (512, 6144, 5120, 0),
 ])
 def test_gemm_matches_oracle(M, K, N, tile_n):
@@ -136,3 +140,16 @@ def test_project_out_qwen_prefill_sampled_rows():
     assert not torch.isnan(y).any()
     rows = sorted({0, 127, 128, 255, 256, 4095} | set(np.random.default_rng(24).integers(0, T, 21).tolist()))
     check(y, o, w_out, rows=rows)
+
+
+def test_project_out_qwen_decode_batch():
+    """64 tokens through the output projection (6144 -> 5120): the K-split
+    cluster path, every row against the oracle."""
+    geo = gi.QWEN_GEO
+    _, w_out = gi.make_projection_weights(geo, gi.QWEN_HIDDEN, 25)
+    o = gi.make_hidden_states(64, geo.value_dim, 25)
+    y = torch.full((64, gi.QWEN_HIDDEN), float("nan"), dtype=torch.bfloat16, device="cuda")
+    gdn.project_out(gdn.make_config(geo), io_tensor(o), io_tensor(w_out), y)
+    torch.cuda.synchronize()
+    assert not torch.isnan(y).any()
+    check(y, o, w_out)

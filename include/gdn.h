@@ -68,7 +68,7 @@ typedef struct CUstream_st* gdn_stream_t; /* a cudaStream_t; NULL = the legacy d
 typedef enum {
   GDN_OK = 0,
   GDN_E_INVAL = -1,          /* bad pointer, size, alignment or cu_seqlens */
-  GDN_E_UNSUPPORTED = -2,    /* geometry or dtype this build does not run */
+  GDN_E_UNSUPPORTED = -2,    /* geometry or dtype the library does not run */
   GDN_E_WORKSPACE = -3,      /* workspace missing or smaller than gdn_prefill_workspace_size() */
   GDN_E_CUDA = -4,           /* a CUDA runtime call failed; see gdn_last_error() */
   GDN_E_BLOB_FORMAT = -5,    /* state blob: bad magic, size or layout id */

@@ -597,8 +597,9 @@ def run_projections(gdn, torch, pk, stream, barrier, max_over_ranks, world, reps
                 "value": round(world * M / (ms / 1000.0), 1), "unit": "tokens/s",
                 "roofline": {"bound": bound, "achieved": round(achieved, 1), "peak": peak, "unit": unit,
                              "frac": round(achieved / peak, 4),
-                             "traffic": (measured_traffic("gemm:project_in_t4096", source_hash("gemm.cu"))
-                                         if (name, T) == ("project_in", 4096) else None),
+                             "traffic": measured_traffic({("project_in", 4096): "gemm:project_in_t4096",
+                                                          ("project_out", 64): "gemm:project_out_b64"}
+                                                         .get((name, T), ""), source_hash("gemm.cu")),
                              "kernel": "gemm", "peak_source": pk["src"]},
                 "tflops": round(flops / (ms / 1000.0) / 1e12, 1), "cublas_ms": round(ms_ref, 5),
                 "vs_cublas": round(ms_ref / ms, 3)}

@@ -5,19 +5,20 @@
 // with W stored as a linear layer's weight (output features x input
 // features), both operands K-major, fp32 accumulation in TMEM, bf16 out.
 //
-// Two persistent kernels walk the output tiles (m fastest, so the CTAs
-// running together share the same few weight panels in L2).  K advances 64
-// columns per TMA box (128-byte swizzle); a ring stage holds one or two boxes
-// of each operand.  Warp 0
-// issues the loads, warp 1 the MMAs (each stage's commit frees its slot),
-// warps 2..5 drain the accumulator.  TMEM holds two accumulators, so the
-// epilogue of one tile overlaps the main loop of the next.
-//   gemm_kernel       one CTA per 128 x BN tile: small M
-//   gemm_pair_kernel  a CTA pair per 256 x BN tile, MMAs of
-//                     M = 256 issued by the even CTA over both CTAs' shared
-//                     memory: each CTA loads only half of the weight panel,
-//                     which cuts the operand bytes each SM moves per MMA by a
-//                     third at BN = 256.
+// K advances 64 columns per TMA box (128-byte swizzle); a ring stage holds one
+// or two boxes of each operand.  Warp 0 issues the loads, warp 1 the MMAs
+// (each stage's commit frees its slot), warps 2..5 drain the accumulator.
+//   gemm_kernel         persistent, one CTA per 128 x BN tile (m fastest, so
+//                       the CTAs running together share the same few weight
+//                       panels in L2); two TMEM accumulators, so the epilogue
+//                       of one tile overlaps the main loop of the next
+//   gemm_pair_kernel    the same with a CTA pair per 256 x BN tile, MMAs of
+//                       M = 256 issued by the even CTA over both CTAs' shared
+//                       memory: each CTA loads only half of the weight panel,
+//                       which cuts the operand bytes each SM moves per MMA by
+//                       a third at BN = 256
+//   gemm_splitk_kernel  up to 128 rows: a cluster of CTAs per tile, each on a
+//                       slice of K, partial rows reduced through DSMEM
 // BN is any multiple of 32 up to 256 (64 up for pairs); the host picks a
 // power-of-two width from the number of tiles per wave.
 // The epilogue routes every 8-column group to one of up to four outputs: the

@@ -531,21 +531,24 @@ bool encode_bf16_2d(EncodeTiledFn enc, CUtensorMap* tm, const void* base, uint64
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// SMs of the current device, looked up once (thread-safe; a failed query
+// leaves no CUDA error behind for the next launch to report)
 int num_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
+  static const int n = [] {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
+      cudaGetLastError();
+      v = 148;
+    }
+    return v;
+  }();
   return n;
 }
 
-// CTA pairs of gemm_pair_kernel that fit on the device at once
+// CTA pairs of gemm_pair_kernel that fit on the device at once, looked up once
 int max_pairs() {
-  static int n = 0;
-  if (n == 0) {
+  static const int n = [] {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * num_sms());
     cfg.blockDim = dim3(kGemmThreads);
@@ -554,10 +557,10 @@ int max_pairs() {
     if (cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) ==
             cudaSuccess &&
         cudaOccupancyMaxActiveClusters(&c, gemm_pair_kernel, &cfg) == cudaSuccess && c > 0)
-      n = c;
-    else
-      n = num_sms() / 2;
-  }
+      return c;
+    cudaGetLastError();
+    return num_sms() / 2;
+  }();
   return n;
 }
 

@@ -171,10 +171,23 @@ GDN_API gdn_status gdn_prefill(const gdn_config* cfg, const gdn_params* params, 
  * Same arguments and results as gdn_prefill, minus the workspace: the scratch
  * is a fixed array of GDN_NOALLOC_SCRATCH_BYTES inside the library's device
  * memory, present on every GPU that loads the library until the process
- * exits.  The call allocates nothing.  A problem whose gdn_prefill workspace
- * would exceed that size is rejected with GDN_E_WORKSPACE before anything
- * runs.  The first call on a device looks up the array's device address (with
- * that device current); make that first call before any stream capture.
+ * exits.  The call allocates nothing.  It always runs gdn_prefill with
+ * GDN_PREFILL_FUSED added to flags: the single-kernel chunked path where it
+ * applies (bf16, d = 128, chunk 64), else the token-recurrent kernel; both
+ * need only the varlen schedule as scratch, about 16 bytes per chunk plus 8
+ * per sequence.  The limit is therefore the workspace gdn_prefill needs with
+ * GDN_PREFILL_FUSED (not gdn_prefill_workspace_size, which reports the
+ * default path's larger need): a problem whose schedule exceeds
+ * GDN_NOALLOC_SCRATCH_BYTES, i.e. more than about 250,000 chunks plus
+ * sequences, is rejected with GDN_E_WORKSPACE before anything runs.  The
+ * schedule is sized for the chunk bound total_tokens / chunk_size + num_seqs
+ * + 1 even for a single sequence, which launches no schedule, so one
+ * sequence of more than about 16M tokens at chunk 64 (4M at chunk 16) is
+ * rejected too.  The first call on a device looks up the array's device
+ * address (with that device current) and caches it for the process; make
+ * that first call before any stream capture.  The cached address does not
+ * survive cudaDeviceReset: do not call this entry point on a device after
+ * resetting it in the same process.
  * Every call on a device shares the one array, which keeps whatever the last
  * call left in it (nothing in it needs to start at zero: every kernel writes
  * the scratch it later reads), so calls whose executions overlap on the GPU --
@@ -377,6 +390,18 @@ GDN_API gdn_status gdn_state_restore(const gdn_config* cfg, const void* blob, si
  * launch count and summed device time of one kernel id (see gdn_kernel_name).
  */
 GDN_API gdn_status gdn_get_device_status(int32_t* code, gdn_stream_t stream);
+
+/* gdn_debug_wait_expiry: exercises the bounded-wait failure path on the
+ * device.  Launches one small kernel that waits, with the same bounded
+ * mbarrier wait the mixer kernels use, on an mbarrier that nothing arrives on
+ * and that no copy targets; after limit_us microseconds (1 .. 1,000,000) the
+ * wait gives up, the kernel records status 1 (wait timeout) in the device
+ * status word and returns.  No trap, no hang: the context stays usable and
+ * the next launch runs normally.  Asynchronous on `stream`; read the result
+ * with gdn_get_device_status.  GDN_E_INVAL for a limit outside the range.
+ * The pages' counterpart is the requirement to fail explicitly instead of
+ * running unsafely (DS4Server issue #95, implementation comment). */
+GDN_API gdn_status gdn_debug_wait_expiry(uint32_t limit_us, gdn_stream_t stream);
 GDN_API const char* gdn_last_error(void);
 GDN_API int32_t gdn_abi_version(void);
 GDN_API int64_t gdn_launch_count(void);
@@ -397,7 +422,8 @@ typedef enum {
   GDN_K_SLOT_COPY = 11,   /* slot-indexed prefill: pool slots to and from the batch's buffers */
   GDN_K_GEMM = 12,        /* bf16 projection GEMM (gdn_gemm_bf16, gdn_project_in, gdn_project_out) */
   GDN_K_SEQPAR = 13,      /* sequence-parallel prefill: segment set-up and the combine across segments */
-  GDN_K_COUNT = 14
+  GDN_K_DIAG = 14,        /* gdn_debug_wait_expiry */
+  GDN_K_COUNT = 15
 } gdn_kernel_id;
 
 GDN_API const char* gdn_kernel_name(int32_t kernel_id);

@@ -19,7 +19,7 @@ import numpy as np
 __all__ = [
     "GdnError", "Config", "Params", "lib", "make_config", "conv_prefill", "conv_step", "prefill_workspace_size",
     "prefill", "prefill_noalloc", "decode_step", "decode_multi", "decode_step_indexed", "decode_multi_indexed",
-    "prefill_indexed_workspace_size", "prefill_indexed", "gemm_bf16", "project_in", "project_out", "prefill_seqpar_workspace_size", "prefill_seqpar", "state_blob_size", "state_save", "state_restore", "device_status", "last_error",
+    "prefill_indexed_workspace_size", "prefill_indexed", "gemm_bf16", "project_in", "project_out", "prefill_seqpar_workspace_size", "prefill_seqpar", "state_blob_size", "state_save", "state_restore", "device_status", "debug_wait_expiry", "last_error",
     "abi_version", "launch_count", "launch_count_reset", "profiler_enable", "profiler_reset", "profiler_read",
     "kernel_name", "EXPORTS", "ZERO_INIT_STATE", "ZERO_INIT_CONV", "PREFILL_RECURRENT", "PREFILL_FUSED", "K", "MAX_DRAFT_TOKENS",
 ]
@@ -42,8 +42,8 @@ STATUS = {0: "GDN_OK", -1: "GDN_E_INVAL", -2: "GDN_E_UNSUPPORTED", -3: "GDN_E_WO
 class K:
     """Kernel ids of the profiler (gdn_kernel_id)."""
     (CONV_PREFILL, CONV_STEP, CONV_HISTORY, SCHEDULE, PREFILL_RECURRENT, PREFILL_CHUNKED, DECODE, STATE_CHECKSUM,
-     SPLIT_CONV, SPLIT_PREP, SPLIT_CHAIN, SLOT_COPY, GEMM, SEQPAR) = range(14)
-    COUNT = 14
+     SPLIT_CONV, SPLIT_PREP, SPLIT_CHAIN, SLOT_COPY, GEMM, SEQPAR, DIAG) = range(15)
+    COUNT = 15
 
 
 # Every symbol include/gdn.h declares.
@@ -54,7 +54,7 @@ EXPORTS = [
     "gdn_profiler_reset", "gdn_profiler_read", "gdn_prefill_noalloc", "gdn_decode_multi",
     "gdn_decode_step_indexed", "gdn_decode_multi_indexed", "gdn_prefill_indexed_workspace_size",
     "gdn_prefill_indexed", "gdn_gemm_bf16", "gdn_project_in", "gdn_project_out",
-    "gdn_prefill_seqpar_workspace_size", "gdn_prefill_seqpar",
+    "gdn_prefill_seqpar_workspace_size", "gdn_prefill_seqpar", "gdn_debug_wait_expiry",
 ]
 
 
@@ -109,6 +109,7 @@ def lib():
             "gdn_state_save": [P, P, P, I32, P, SZ, P],
             "gdn_state_restore": [P, P, SZ, I32, P, P, P],
             "gdn_get_device_status": [P, P],
+            "gdn_debug_wait_expiry": [ctypes.c_uint32, P],
             "gdn_profiler_enable": [I32],
             "gdn_profiler_reset": [],
             "gdn_profiler_read": [I32, P, P],
@@ -328,6 +329,12 @@ def device_status(stream=None) -> int:
     code = ctypes.c_int32()
     _check(lib().gdn_get_device_status(ctypes.byref(code), _stream(stream)))
     return code.value
+
+
+def debug_wait_expiry(limit_us: int, stream=None):
+    """gdn_debug_wait_expiry: a kernel whose bounded wait always runs out
+    after limit_us; the device status word then reads 1 (wait timeout)."""
+    _check(lib().gdn_debug_wait_expiry(limit_us, _stream(stream)))
 
 
 def abi_version() -> int:

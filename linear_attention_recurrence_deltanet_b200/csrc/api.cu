@@ -291,7 +291,8 @@ const char* gdn_kernel_name(int32_t id) {
   static const char* names[GDN_K_COUNT] = {"conv_prefill",    "conv_step",       "conv_history", "schedule",
                                            "prefill_recurrent", "prefill_chunked", "decode",       "state_checksum",
                                            "split_conv",        "split_prep",      "split_chain",
-                                           "slot_copy",         "gemm",            "seqpar"};
+                                           "slot_copy",         "gemm",            "seqpar",
+                                           "diag"};
   return (id >= 0 && id < GDN_K_COUNT) ? names[id] : "unknown";
 }
 
@@ -335,6 +336,15 @@ gdn_status gdn_get_device_status(int32_t* code, gdn_stream_t stream) {
   if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
   *code = v;
   return GDN_OK;
+}
+
+gdn_status gdn_debug_wait_expiry(uint32_t limit_us, gdn_stream_t stream) {
+  if (limit_us < 1 || limit_us > 1000000u) return fail(GDN_E_INVAL, "limit_us %u outside 1..1000000", limit_us);
+  int dev = 0;
+  gdn_status s = check_device(&dev);
+  if (s != GDN_OK) return s;
+  cudaError_t e = gdn::launch_wait_expiry((uint64_t)limit_us * 1000ull, g_status_ptr[dev], (cudaStream_t)stream);
+  return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_debug_wait_expiry launch");
 }
 
 gdn_status gdn_conv_prefill(const gdn_config* cfg, const void* x, const float* conv_w,

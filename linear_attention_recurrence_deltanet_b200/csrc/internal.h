@@ -140,4 +140,7 @@ size_t prefill_fused_ws_bytes(int64_t total_tokens, int32_t num_seqs, int32_t ch
 cudaError_t launch_checksum(const void* payload, size_t bytes, unsigned long long* out, cudaStream_t stream);
 uint64_t host_checksum(const void* payload, size_t bytes);
 
+// diag.cu: a kernel whose bounded wait always runs out (tests the status path)
+cudaError_t launch_wait_expiry(uint64_t limit_ns, int32_t* status, cudaStream_t stream);
+
 }  // namespace gdn

@@ -58,10 +58,23 @@ extern "C" GDN_API gdn_status gdn_prefill_noalloc(const gdn_config* cfg, const g
   size_t need = 0;
   gdn_status s = gdn_prefill_workspace_size(cfg, 0, num_seqs, chunk_size, &need);
   if (s != GDN_OK) return s;
-  if (!cu_seqlens_host) return gdn_prefill_workspace_size(nullptr, 0, 0, 0, &need);  // reports the NULL argument
+  if (!cu_seqlens_host) {
+    gdn::set_error_message("gdn_prefill_noalloc: cu_seqlens_host is NULL");
+    return GDN_E_INVAL;
+  }
+  // cu_seqlens_host must be valid before its last entry sizes the schedule
+  if (cu_seqlens_host[0] != 0) {
+    gdn::set_error_message("gdn_prefill_noalloc: cu_seqlens_host[0] is not 0");
+    return GDN_E_INVAL;
+  }
+  for (int32_t n = 0; n < num_seqs; ++n) {
+    if (cu_seqlens_host[n + 1] < cu_seqlens_host[n]) {
+      gdn::set_error_message("gdn_prefill_noalloc: cu_seqlens_host decreases");
+      return GDN_E_INVAL;
+    }
+  }
   // the single-kernel chunked path needs only the schedule as scratch
-  need = gdn::prefill_fused_ws_bytes(cu_seqlens_host[num_seqs] > 0 ? cu_seqlens_host[num_seqs] : 0, num_seqs,
-                                     chunk_size);
+  need = gdn::prefill_fused_ws_bytes(cu_seqlens_host[num_seqs], num_seqs, chunk_size);
   if (need > kScratchBytes) {
     char msg[256];
     snprintf(msg, sizeof(msg),

@@ -38,6 +38,13 @@ def test_every_declared_symbol_is_exported():
     assert sorted(gdn.EXPORTS) == declared
 
 
+def test_debug_wait_expiry_limit_validated_on_the_host():
+    for bad in (0, 1000001):
+        with pytest.raises(gdn.GdnError) as e:
+            gdn.debug_wait_expiry(bad)
+        assert e.value.name == "GDN_E_INVAL" and "limit_us" in str(e.value)
+
+
 def test_abi_version_and_names():
     assert gdn.abi_version() == 1
     assert gdn.kernel_name(gdn.K.DECODE) == "decode"
@@ -133,6 +140,27 @@ def test_prefill_validation_rejects_before_launch():
     assert e.value.name == "GDN_E_INVAL" and "aligned" in str(e.value)
     for k, v in t.items():
         assert np.array_equal(v.view, snapshot[k]), k
+
+
+def test_prefill_noalloc_validates_cu_seqlens_host_on_the_host():
+    """The no-scratch prefill names a NULL or malformed cu_seqlens_host itself,
+    before it sizes anything from the array's last entry."""
+    geo = gi.Geometry()
+    cfg = gdn.make_config(geo)
+    params = gdn._params(*(FakeTensor(n) for n in (geo.conv_dim * 16, 192, 192, 512)))
+    t = FakeTensor(1 << 12)
+    L = gdn.lib()
+
+    def call(cu_ptr, n):
+        return L.gdn_prefill_noalloc(ctypes.byref(cfg), ctypes.byref(params), t.data_ptr(), t.data_ptr(),
+                                     t.data_ptr(), t.data_ptr(), t.data_ptr(), cu_ptr, n, 64, 0, t.data_ptr(),
+                                     t.data_ptr(), t.data_ptr(), None)
+
+    assert call(None, 1) == -1 and "cu_seqlens_host is NULL" in gdn.last_error()
+    bad0 = np.array([4, 8], np.int32)
+    assert call(bad0.ctypes.data, 1) == -1 and "cu_seqlens_host[0]" in gdn.last_error()
+    dec = np.array([0, 8, 4], np.int32)
+    assert call(dec.ctypes.data, 2) == -1 and "decreases" in gdn.last_error()
 
 
 def test_decode_multi_validation_rejects_before_launch():

@@ -201,7 +201,9 @@ def test_prefill_t4096_matches_oracle():
         assert np.array_equal(hist, ref_hist_bits(inp, hist_ref))
 
 
-def _decode_run(steps, heads, check_every_step_all_heads=0):
+def _decode_run(steps):
+    """`steps` decode steps of the B=64 workload; every output of every value
+    head is compared with the oracle at every step, and every final state."""
     w = gi.WORKLOADS["decode_b64"]
     geo, seed, N = w["geo"], w["seed"], 64
     params = gi.make_params(geo, seed)
@@ -212,48 +214,48 @@ def _decode_run(steps, heads, check_every_step_all_heads=0):
     st = torch.from_numpy(st0).cuda()
     o = torch.empty((N, geo.value_dim), dtype=torch.bfloat16, device="cuda")
     ref_st, ref_hist = st0.astype(np.float64), gi.f32_from_bf16_bits(conv0)
-    worst = 0.0
+    worst_o = worst_s = 0.0
     for s in range(steps):
         qkv, z, a, b = gi.make_decode_step_tokens(geo, N, seed, s)
         gdn.decode_step(cfg, dparams, io_tensor(qkv), io_tensor(z), io_tensor(a), io_tensor(b), N, conv, st, o)
-        hs = None if s < check_every_step_all_heads else heads
         o_ref, ref_st, ref_hist = oracle.decode_step(geo, params, gi.f32_from_bf16_bits(qkv), gi.f32_from_bf16_bits(z),
                                                      gi.f32_from_bf16_bits(a), gi.f32_from_bf16_bits(b), ref_hist,
-                                                     ref_st, heads=hs)
-        cols = np.arange(geo.value_dim) if hs is None else np.concatenate(
-            [np.arange(h * 128, (h + 1) * 128) for h in hs])
+                                                     ref_st)
         og = io_float(o)
         for n in range(N):
-            e = maxrel(og[n, cols], o_ref[n, cols], U_BF16)
-            worst = max(worst, e)
+            e = maxrel(og[n], o_ref[n], U_BF16)
+            worst_o = max(worst_o, e)
             assert e <= TOL_O_BF16, (s, n, e)
     torch.cuda.synchronize()
     stg = st.cpu().numpy()
     for n in range(N):
-        assert maxrel(stg[n, heads], ref_st[n, heads]) <= TOL_S_BF16, n
+        e = maxrel(stg[n], ref_st[n])
+        worst_s = max(worst_s, e)
+        assert e <= TOL_S_BF16, (n, e)
     assert np.array_equal(io_numpy(conv), gi.bf16_bits_from_f32(ref_hist))
-    return worst
+    return worst_o, worst_s
 
 
 def test_decode_b64_first_steps_all_heads():
-    _decode_run(16, list(range(48)), check_every_step_all_heads=16)
+    _decode_run(16)
 
 
 @pytest.mark.slow
-def test_decode_b64_1000_steps_sampled_heads():
-    worst = _decode_run(1000, [0, 1, 2, 25, 47])
-    print(f"decode 1000 steps: worst o max-rel {worst:.2e}")
+def test_decode_b64_1000_steps_all_heads():
+    eo, es = _decode_run(1000)
+    print(f"decode B=64, 1000 steps, all 48 value heads: worst o max-rel {eo:.2e}, worst state max-rel {es:.2e}")
 
 
 @pytest.mark.slow
 def test_varlen16_chunk_sizes():
     inp = gi.workload_inputs("varlen_16")
-    heads = [0, 4, 23, 47]
-    o_ref, st_ref, _ = oracle.prefill_inputs(inp, heads=heads)
+    o_ref, st_ref, hist_ref = oracle.prefill_inputs(inp)
     outs = []
     for C in (16, 64, 128):
         _, o, st, hist = run_gpu_prefill(inp, C)
-        compare_prefill(inp, o, st, o_ref, st_ref, TOL_O_BF16, TOL_S_BF16, heads=heads)
+        eo, es = compare_prefill(inp, o, st, o_ref, st_ref, TOL_O_BF16, TOL_S_BF16)
+        print(f"varlen-16 chunk {C}, all 48 value heads: worst o max-rel {eo:.2e}, worst state max-rel {es:.2e}")
+        assert np.array_equal(hist, ref_hist_bits(inp, hist_ref))
         outs.append((o, st, hist))
     for o, st, hist in outs[1:]:  # chunk-size equivalence, all heads
         for n in range(inp.num_seqs):
@@ -267,11 +269,12 @@ def test_varlen16_chunk_sizes():
 def test_long_t65536_split_save_restore_decode():
     w = gi.WORKLOADS["prefill_t65536"]
     inp = gi.workload_inputs("prefill_t65536")
-    heads = [0, 31, 47]
-    o_ref, st_ref, hist_ref = oracle.prefill_inputs(inp, heads=heads)
+    o_ref, st_ref, hist_ref = oracle.prefill_inputs(inp)
     # run A: one pass
     _, oA, stA, hA = run_gpu_prefill(inp, 64)
-    compare_prefill(inp, oA, stA, o_ref, st_ref, TOL_O_BF16, TOL_S_BF16, heads=heads)
+    eo, es = compare_prefill(inp, oA, stA, o_ref, st_ref, TOL_O_BF16, TOL_S_BF16)
+    print(f"T=65536 one pass, all 48 value heads: o max-rel {eo:.2e}, state max-rel {es:.2e}")
+    assert np.array_equal(hA, ref_hist_bits(inp, hist_ref))
     # run B: prefill [0, 40961), save, restore into fresh buffers, prefill to 65280, decode the last 256
     split, tail = w["split"], w["decode_tail"]
     geo, cfg = inp.geo, gdn.make_config(inp.geo)
@@ -303,7 +306,8 @@ def test_long_t65536_split_save_restore_decode():
     torch.cuda.synchronize()
     oB = np.concatenate([io_float(o1), io_float(o2), io_float(od)])
     stB = st2.cpu().numpy().astype(np.float64)
-    compare_prefill(inp, oB, stB, o_ref, st_ref, TOL_O_BF16, TOL_S_BF16, heads=heads)
+    eo, es = compare_prefill(inp, oB, stB, o_ref, st_ref, TOL_O_BF16, TOL_S_BF16)
+    print(f"T=65536 split/save/restore/decode, all 48 value heads: o max-rel {eo:.2e}, state max-rel {es:.2e}")
     assert maxrel(oB, oA, 2 * U_BF16) <= TOL_O_BF16 and maxrel(stB, stA) <= TOL_S_BF16
     assert np.array_equal(io_numpy(conv2), hA)
 

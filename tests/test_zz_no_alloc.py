@@ -48,6 +48,25 @@ def test_prefill_noalloc_matches_prefill_on_two_calls():
     assert gdn.device_status() == 0
 
 
+def test_prefill_noalloc_fp32_chunk16_matches_prefill_on_two_calls():
+    """fp32 io at chunk 16 takes the token-recurrent kernel, with the varlen
+    schedule of several sequences written into the built-in scratch array."""
+    geo = gi.Geometry(num_k_heads=2, num_v_heads=4, head_k_dim=32, head_v_dim=32, io_dtype="f32")
+    problems = [gi.make_prefill_inputs(geo, [64, 3, 0, 17, 40], seed=43, zero_init=False),
+                gi.make_prefill_inputs(geo, [5, 64, 1], seed=44, zero_init=False)]
+    for inp in problems:
+        ref = DeviceProblem(inp, 16)
+        ref.prefill()
+        got = DeviceProblem(inp, 16)
+        got.workspace = None
+        _noalloc(got)
+        torch.cuda.synchronize()
+        assert _maxrel(io_float(got.o), io_float(ref.o), 2.0 ** -24) <= 1e-5
+        assert _maxrel(got.state.cpu().numpy(), ref.state.cpu().numpy()) <= 1e-5
+        assert np.array_equal(io_numpy(got.conv_state), io_numpy(ref.conv_state))
+    assert gdn.device_status() == 0
+
+
 def test_prefill_noalloc_rejects_oversized_problem():
     geo = gi.Geometry(num_k_heads=1, num_v_heads=1, head_k_dim=32, head_v_dim=32)
     cfg = gdn.make_config(geo)

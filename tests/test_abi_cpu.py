@@ -41,7 +41,7 @@ def test_every_declared_symbol_is_exported():
 def test_debug_wait_expiry_limit_validated_on_the_host():
     for bad in (0, 1000001):
         with pytest.raises(gdn.GdnError) as e:
-            gdn.debug_wait_expiry(bad)
+            gdn.debug_wait_expiry(bad, stream=0)
         assert e.value.name == "GDN_E_INVAL" and "limit_us" in str(e.value)
 
 

@@ -50,6 +50,8 @@ DECODE_WORKLOAD = "decode_b64"
 DECODE_STEPS = 1000
 ROTATE = 3
 DRAFT_ROUNDS = 200
+# arithmetic of the prefill path: bf16 inputs; fp16 hi + lo tensor-core operands; fp32 accumulation and state
+DTYPE = "bf16 in, fp16x2 MMA, fp32 acc/state"
 
 
 def peaks():
@@ -242,23 +244,26 @@ def run_reference(args, rank):
     inp = gi.workload_inputs(PREFILL_WORKLOAD)
     import oracle
     cores = oracle.default_threads()
-    # size each step so the whole run stays near a minute
-    probe = time_oracle(inp, 64) / 64
-    per_step = 60.0 / max(1, args.steps + args.warmup)
-    tokens = int(max(16, min(inp.total_tokens, per_step / max(probe, 1e-9))))
-    for _ in range(args.warmup):
+    # every step is the whole 4096-token prefill (all heads) unless the requested steps would take more than
+    # about three minutes on the host cores; then each step is the leading part of it that fits
+    per_token = time_oracle(inp, 256) / 256
+    steps, warm = args.steps, args.warmup
+    tokens = int(max(256, min(inp.total_tokens, 180.0 / max(1, steps + warm) / max(per_token, 1e-9))))
+    for _ in range(warm):
         time_oracle(inp, tokens)
     t = 0.0
-    for _ in range(args.steps):
+    for _ in range(steps):
         t += time_oracle(inp, tokens)
-    value = tokens * args.steps / t
+    value = tokens * steps / t
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1000 * t / args.steps, 4),
+            "steps": steps, "warmup": warm, "ms_per_step": round(1000 * t / steps, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": "GDN prefill, B=1, T=4096, 16 key / 48 value heads x 128, chunk 64, bf16 inputs",
                        "global_batch": 1, "seq_len": 4096, "chunk": w["chunks"][0], "parallelism": "none (CPU)"},
             "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                             "sample": f"first {tokens} tokens of the 4096-token prefill per step, all heads"},
+                             "sample": (f"the whole {tokens}-token prefill per step" if tokens == inp.total_tokens
+                                        else f"the first {tokens} of the 4096 prefill tokens per step")
+                                       + ", all 48 value heads"},
             "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -301,7 +306,7 @@ def run_gdn(args, rank, world, local_rank):
     del base
     ws = torch.empty(gdn.prefill_workspace_size(cfg, T, 1, C) + 256, dtype=torch.uint8, device="cuda")
     flags = gdn.ZERO_INIT_STATE | (gdn.PREFILL_RECURRENT if args.recurrent else 0) | \
-        (gdn.PREFILL_FUSED if args.fused else 0)
+        (gdn.PREFILL_FUSED if args.fused else 0) | (gdn.PREFILL_FACTORED if args.factored else 0)
 
     def prefill(i):
         s = sets[i % ROTATE]
@@ -331,7 +336,10 @@ def run_gdn(args, rank, world, local_rank):
     # logical kernel: its roofline takes the prefill's algorithmic bytes over
     # the summed average launch times of its three stages.
     split_ids = (gdn.K.SPLIT_CONV, gdn.K.SPLIT_PREP, gdn.K.SPLIT_CHAIN)
-    if not args.recurrent and not args.fused and per_kernel[gdn.kernel_name(gdn.K.SPLIT_CHAIN)][0]:
+    wy_ids = (gdn.K.WY_CONV, gdn.K.WY_PREP, gdn.K.WY_CHAIN)
+    if per_kernel[gdn.kernel_name(gdn.K.WY_CHAIN)][0]:
+        kids, kname, src = wy_ids, "wy_conv+wy_prep+wy_chain", source_hash("prefill_wy.cu")
+    elif per_kernel[gdn.kernel_name(gdn.K.SPLIT_CHAIN)][0]:
         kids, kname, src = split_ids, "split_conv+split_prep+split_chain", source_hash("prefill_split.cu")
     elif args.recurrent:
         kids, kname, src = (gdn.K.PREFILL_RECURRENT,), "prefill_recurrent", source_hash("prefill_recurrent.cu")
@@ -508,28 +516,122 @@ def run_gdn(args, rank, world, local_rank):
 
     proj = run_projections(gdn, torch, pk, stream, barrier, max_over_ranks, world, args.projection_reps)
     seqpar = run_seqpar(gdn, torch, pk, stream, barrier, max_over_ranks, world)
+    extra = {} if args.no_workloads else run_workloads(gdn, torch, pk, stream, barrier, max_over_ranks, world, rank,
+                                                       clocks)
 
     clk = clocks.summary()
     cpu = cpu_baseline(inp) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
     if rank == 0:
+        # the long blocks first, so that a tail of the line keeps the per-workload summaries
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "vs_baseline": None, "dtype": DTYPE, "data": "synthetic",
             "config": {"workload": "GDN prefill, B=1, T=4096, 16 key / 48 value heads x 128, chunk 64, bf16 inputs, "
                                    "fp32 state from zero", "global_batch": world, "seq_len": T, "chunk": C,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": f"inputs rotate over {ROTATE} sets (> 4x L2) between steps"},
-            "roofline": roof_p, "decode": decode, "draft_verify": draft, "projections": proj,
-            "seq_parallel": seqpar, "e2e": e2e,
-            "gpu_launches": launches,
-            "kernels": kernel_share, "clocks": clk, "cpu_baseline": cpu,
+            "projections": proj, "seq_parallel": seqpar, "kernels": kernel_share,
+            "gpu_launches": launches, "clocks": clk, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roof_p,
+            **extra,
+            "draft_verify": draft, "decode": decode,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def oracle_sample(inp, budget_s=5.0):
+    """The float64 oracle, as it stands, on a bounded sample of a workload:
+    the leading tokens of the packed stream with their true sequence
+    boundaries and starting states, all value heads, all host cores."""
+    import oracle
+    cu = np.asarray(inp.cu_seqlens, np.int64)
+    params = (inp.conv_w, inp.A_log, inp.dt_bias, inp.norm_w)
+
+    def run(tokens):
+        n_used = int(np.searchsorted(cu, tokens, side="left"))  # sequences that start before `tokens`
+        cu_s = np.minimum(cu[:n_used + 1], tokens).astype(np.int32)
+        cu_s[-1] = tokens
+        sl = slice(0, tokens)
+        t0 = time.perf_counter()
+        oracle.prefill(inp.geo, params, inp.f32("qkv")[sl], inp.f32("z")[sl], inp.f32("a")[sl], inp.f32("b")[sl],
+                       cu_s, inp.f32("conv_state")[:n_used], inp.state[:n_used])
+        return time.perf_counter() - t0, n_used
+
+    probe = 128
+    dt, _ = run(probe)
+    tokens = int(min(inp.total_tokens, max(probe, budget_s / max(dt, 1e-6) * probe)))
+    dt, n_used = run(tokens)
+    cores = oracle.default_threads()
+    return {"value": round(tokens / dt, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"float64 oracle, first {tokens} of {inp.total_tokens} packed tokens ({n_used} sequence(s) "
+                      f"started), all {inp.geo.num_v_heads} value heads, {cores} threads, {dt:.2f} s wall"}
+
+
+def run_workloads(gdn, torch, pk, stream, barrier, max_over_ranks, world, rank, clocks, reps=3):
+    """The long-context one-pass prefill (B=1, T=65536) and the packed varlen
+    batch (16 sequences, lengths uniform in 1..8192) at chunk 16, 64 and 128,
+    at the full 16 key / 48 value head geometry, each prefill timed alone with
+    events on the launching stream (inputs > L2), with the oracle timed on a
+    bounded sample of the same workload beside it (rank 0, one GPU)."""
+    from linear_attention_recurrence_deltanet_b200.device import DeviceProblem, io_tensor
+    out = {}
+    for name, tag in (("prefill_t65536", "long_context"), ("varlen_16", "varlen_16")):
+        w = gi.WORKLOADS[name]
+        inp = gi.workload_inputs(name)
+        zero = w["zero_init"]
+        flags0 = (gdn.ZERO_INIT_STATE | gdn.ZERO_INIT_CONV) if zero else 0
+        res = {}
+        for C in w["chunks"]:
+            dp = DeviceProblem(inp, C)
+            conv0, st0 = dp.conv_state.clone(), dp.state.clone()
+            ms_all, per = [], {}
+            for i in range(reps + 1):
+                if not zero:
+                    dp.conv_state.copy_(conv0)
+                    dp.state.copy_(st0)
+                barrier()
+                gdn.profiler_reset()
+                gdn.profiler_enable(True)
+                clocks.active = i > 0
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                dp.prefill(flags0, stream=stream)
+                b.record(stream)
+                b.synchronize()
+                clocks.active = False
+                gdn.profiler_enable(False)
+                if i > 0:  # the first run is a warm-up
+                    ms_all.append(a.elapsed_time(b))
+                    for k in range(gdn.K.COUNT):
+                        nl, kms = gdn.profiler_read(k)
+                        if nl:
+                            per[gdn.kernel_name(k)] = per.get(gdn.kernel_name(k), 0.0) + kms / reps
+            ms = max_over_ranks(sum(ms_all) / len(ms_all))
+            nbytes = prefill_bytes(inp.geo, list(np.diff(inp.cu_seqlens)), zero_state=zero)
+            gbs = nbytes / (ms / 1000.0) / 1e9
+            res[f"chunk_{C}"] = {
+                "ms": round(ms, 4), "value": round(world * inp.total_tokens / (ms / 1000.0), 1), "unit": "tokens/s",
+                "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm"], "unit": "GB/s",
+                             "frac": round(gbs / pk["hbm"], 4), "traffic": None, "algorithmic_bytes": nbytes,
+                             "kernel": "whole prefill (every launch)", "peak_source": pk["src"]},
+                "kernels_ms": {k: round(v, 4) for k, v in per.items()}}
+            del dp, conv0, st0
+            torch.cuda.empty_cache()
+        lengths = [int(x) for x in np.diff(inp.cu_seqlens)]
+        res["workload"] = (f"{len(lengths)} sequence(s), {inp.total_tokens} tokens"
+                           + (f" (lengths {lengths})" if len(lengths) > 1 else "")
+                           + ", 16 key / 48 value heads x 128, bf16 inputs, "
+                           + ("zero initial states" if zero else "initial states ~N(0,0.02) and histories ~N(0,1)")
+                           + "; time per whole prefill (every launch), inputs > L2")
+        res["cpu_baseline"] = oracle_sample(inp) if (rank == 0 and world == 1) else None
+        out[tag] = res
+        del inp
+    return out
 
 
 def run_projections(gdn, torch, pk, stream, barrier, max_over_ranks, world, reps):
@@ -673,6 +775,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=DECODE_STEPS)
     ap.add_argument("--recurrent", action="store_true", help="time the token-recurrent prefill kernel")
     ap.add_argument("--fused", action="store_true", help="time the single-kernel chunked prefill")
+    ap.add_argument("--factored", action="store_true", help="time the factored three-kernel chunked prefill")
+    ap.add_argument("--no-workloads", action="store_true", help="skip the long-context and varlen workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--projection-reps", type=int, default=20, help="timed launches per projection shape")
     args = ap.parse_args()

@@ -105,6 +105,8 @@ typedef struct {
 #define GDN_PREFILL_RECURRENT 0x4u /* run the token-recurrent fp32 kernel instead of the chunked one */
 #define GDN_PREFILL_FUSED 0x8u     /* chunked path as one kernel per (sequence, value head): needs only the
                                       schedule as workspace (see gdn_prefill) */
+#define GDN_PREFILL_FACTORED 0x10u /* chunk 64 only: the three-kernel chunked path in the factored form
+                                      (W S, then K~^T Delta per chunk) instead of the affine chunk maps */
 
 /* --------------------------------------------------------------------------
  * Causal depthwise Conv1D + SiLU over the q/k/v channels (issue #88, Scope:
@@ -423,7 +425,10 @@ typedef enum {
   GDN_K_GEMM = 12,        /* bf16 projection GEMM (gdn_gemm_bf16, gdn_project_in, gdn_project_out) */
   GDN_K_SEQPAR = 13,      /* sequence-parallel prefill: segment set-up and the combine across segments */
   GDN_K_DIAG = 14,        /* gdn_debug_wait_expiry */
-  GDN_K_COUNT = 15
+  GDN_K_WY_CONV = 15,     /* chunked prefill (affine chunk maps), stage 1: conv + SiLU + L2 norm of every token */
+  GDN_K_WY_PREP = 16,     /* stage 2: per-(tile, value head) operands: T by tensor-core doubling, M', Q', U, P, K~ */
+  GDN_K_WY_CHAIN = 17,    /* stage 3: the state carry (one M' S product per chunk) and the output rows */
+  GDN_K_COUNT = 18
 } gdn_kernel_id;
 
 GDN_API const char* gdn_kernel_name(int32_t kernel_id);

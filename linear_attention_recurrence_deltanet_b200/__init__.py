@@ -21,7 +21,7 @@ __all__ = [
     "prefill", "prefill_noalloc", "decode_step", "decode_multi", "decode_step_indexed", "decode_multi_indexed",
     "prefill_indexed_workspace_size", "prefill_indexed", "gemm_bf16", "project_in", "project_out", "prefill_seqpar_workspace_size", "prefill_seqpar", "state_blob_size", "state_save", "state_restore", "device_status", "debug_wait_expiry", "last_error",
     "abi_version", "launch_count", "launch_count_reset", "profiler_enable", "profiler_reset", "profiler_read",
-    "kernel_name", "EXPORTS", "ZERO_INIT_STATE", "ZERO_INIT_CONV", "PREFILL_RECURRENT", "PREFILL_FUSED", "K", "MAX_DRAFT_TOKENS",
+    "kernel_name", "EXPORTS", "ZERO_INIT_STATE", "ZERO_INIT_CONV", "PREFILL_RECURRENT", "PREFILL_FUSED", "PREFILL_FACTORED", "K", "MAX_DRAFT_TOKENS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
@@ -30,6 +30,7 @@ ZERO_INIT_STATE = 0x1
 ZERO_INIT_CONV = 0x2
 PREFILL_RECURRENT = 0x4
 PREFILL_FUSED = 0x8
+PREFILL_FACTORED = 0x10
 MAX_DRAFT_TOKENS = 4
 
 F32, BF16 = 0, 1
@@ -42,8 +43,8 @@ STATUS = {0: "GDN_OK", -1: "GDN_E_INVAL", -2: "GDN_E_UNSUPPORTED", -3: "GDN_E_WO
 class K:
     """Kernel ids of the profiler (gdn_kernel_id)."""
     (CONV_PREFILL, CONV_STEP, CONV_HISTORY, SCHEDULE, PREFILL_RECURRENT, PREFILL_CHUNKED, DECODE, STATE_CHECKSUM,
-     SPLIT_CONV, SPLIT_PREP, SPLIT_CHAIN, SLOT_COPY, GEMM, SEQPAR, DIAG) = range(15)
-    COUNT = 15
+     SPLIT_CONV, SPLIT_PREP, SPLIT_CHAIN, SLOT_COPY, GEMM, SEQPAR, DIAG, WY_CONV, WY_PREP, WY_CHAIN) = range(18)
+    COUNT = 18
 
 
 # Every symbol include/gdn.h declares.

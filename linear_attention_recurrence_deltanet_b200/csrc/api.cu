@@ -198,17 +198,41 @@ int64_t chunk_bound(int64_t total_tokens, int32_t num_seqs, int32_t chunk_size) 
   return total_tokens / chunk_size + num_seqs + 1;
 }
 
-// The three-kernel chunked path runs unless GDN_PREFILL_FUSED or GDN_PREFILL_RECURRENT is given.
-bool split_path(const gdn::Dims& d, const gdn_config* cfg, int32_t chunk_size, uint32_t flags) {
-  return !(flags & (GDN_PREFILL_FUSED | GDN_PREFILL_RECURRENT)) &&
-         gdn::prefill_chunked_supported(d, cfg->io_dtype == GDN_BF16, chunk_size);
+// Prefill paths: the affine chunk maps (three kernels; bf16, d = 128, chunk 16/32/64) by default; the
+// factored three-kernel path (chunk 64) with GDN_PREFILL_FACTORED; one kernel per (sequence, value head)
+// with GDN_PREFILL_FUSED; the token-recurrent kernel otherwise.
+enum class Path { Wy, Split, Fused, Recurrent };
+
+Path prefill_path(const gdn::Dims& d, const gdn_config* cfg, int32_t chunk_size, uint32_t flags) {
+  const bool bf16 = cfg->io_dtype == GDN_BF16;
+  if (flags & GDN_PREFILL_RECURRENT) return Path::Recurrent;
+  if (flags & GDN_PREFILL_FUSED)
+    return gdn::prefill_chunked_supported(d, bf16, chunk_size) ? Path::Fused : Path::Recurrent;
+  if (flags & GDN_PREFILL_FACTORED)
+    return gdn::prefill_chunked_supported(d, bf16, chunk_size) ? Path::Split : Path::Recurrent;
+  if (gdn::prefill_wy_supported(d, bf16, chunk_size)) return Path::Wy;
+  return Path::Recurrent;
 }
 
-// schedule, then (three-kernel path only) the intermediates of the chunked form
-size_t prefill_ws_bytes(const gdn::Dims& d, bool split, int64_t total_tokens, int32_t num_seqs, int32_t chunk_size) {
-  const int64_t chunks = chunk_bound(total_tokens, num_seqs, chunk_size);
+// rows of the schedule's chunks: the affine path schedules tiles of 64 or 128 rows
+int32_t sched_rows(Path p, int32_t chunk_size) { return p == Path::Wy ? gdn::wy_tile(chunk_size) : chunk_size; }
+
+// schedule, then (three-kernel paths only) the intermediates of the chunked form
+size_t prefill_ws_bytes(const gdn::Dims& d, Path p, int64_t total_tokens, int32_t num_seqs, int32_t chunk_size) {
+  const int64_t chunks = chunk_bound(total_tokens, num_seqs, sched_rows(p, chunk_size));
   const size_t sched = gdn::schedule_layout(num_seqs, chunks).total_bytes;
-  return split ? sched + gdn::split_layout(d, total_tokens, chunks).total_bytes : sched;
+  if (p == Path::Split) return sched + gdn::split_layout(d, total_tokens, chunks).total_bytes;
+  if (p == Path::Wy) return sched + gdn::wy_layout(d, total_tokens, chunks, chunk_size).total_bytes;
+  return sched;
+}
+
+// what gdn_prefill_workspace_size reports: enough for every path a flag can select
+size_t prefill_ws_query(const gdn::Dims& d, const gdn_config* cfg, int64_t total_tokens, int32_t num_seqs,
+                        int32_t chunk_size) {
+  size_t m = 0;
+  for (uint32_t f : {0u, (uint32_t)GDN_PREFILL_FACTORED, (uint32_t)GDN_PREFILL_FUSED})
+    m = std::max(m, prefill_ws_bytes(d, prefill_path(d, cfg, chunk_size, f), total_tokens, num_seqs, chunk_size));
+  return m;
 }
 
 // ---------------------------------------------------------------- state blob
@@ -292,7 +316,8 @@ const char* gdn_kernel_name(int32_t id) {
                                            "prefill_recurrent", "prefill_chunked", "decode",       "state_checksum",
                                            "split_conv",        "split_prep",      "split_chain",
                                            "slot_copy",         "gemm",            "seqpar",
-                                           "diag"};
+                                           "diag",              "wy_conv",         "wy_prep",
+                                           "wy_chain"};
   return (id >= 0 && id < GDN_K_COUNT) ? names[id] : "unknown";
 }
 
@@ -390,7 +415,7 @@ gdn_status gdn_prefill_workspace_size(const gdn_config* cfg, int64_t total_token
   if (total_tokens < 0 || num_seqs <= 0 || num_seqs > kMaxSeqs) return fail(GDN_E_INVAL, "bad sizes");
   if (chunk_size != 16 && chunk_size != 32 && chunk_size != 64 && chunk_size != 128)
     return fail(GDN_E_INVAL, "chunk_size %d (16, 32, 64 or 128)", chunk_size);
-  *bytes = prefill_ws_bytes(d, split_path(d, cfg, chunk_size, 0), total_tokens, num_seqs, chunk_size);
+  *bytes = prefill_ws_query(d, cfg, total_tokens, num_seqs, chunk_size);
   return GDN_OK;
 }
 
@@ -404,7 +429,8 @@ gdn_status gdn_prefill(const gdn_config* cfg, const gdn_params* params, const vo
   if ((s = check_params(params)) != GDN_OK) return s;
   if (chunk_size != 16 && chunk_size != 32 && chunk_size != 64 && chunk_size != 128)
     return fail(GDN_E_INVAL, "chunk_size %d (16, 32, 64 or 128)", chunk_size);
-  const uint32_t known = GDN_ZERO_INIT_STATE | GDN_ZERO_INIT_CONV | GDN_PREFILL_RECURRENT | GDN_PREFILL_FUSED;
+  const uint32_t known =
+      GDN_ZERO_INIT_STATE | GDN_ZERO_INIT_CONV | GDN_PREFILL_RECURRENT | GDN_PREFILL_FUSED | GDN_PREFILL_FACTORED;
   if (flags & ~known) return fail(GDN_E_INVAL, "unknown flags 0x%x", flags & ~known);
   int64_t total = 0;
   int32_t max_len = 0;
@@ -416,8 +442,9 @@ gdn_status gdn_prefill(const gdn_config* cfg, const gdn_params* params, const vo
         (s = check_ptr(o, "o")) != GDN_OK)
       return s;
   }
-  const bool split = split_path(d, cfg, chunk_size, flags);
-  const size_t need = prefill_ws_bytes(d, split, total, num_seqs, chunk_size);
+  const Path path = prefill_path(d, cfg, chunk_size, flags);
+  const bool split = path == Path::Split || path == Path::Wy;
+  const size_t need = prefill_ws_bytes(d, path, total, num_seqs, chunk_size);
   if (workspace_bytes < need || (need > 0 && !workspace))
     return fail(GDN_E_WORKSPACE, "workspace of %zu bytes at %p, need %zu", workspace_bytes, workspace, need);
   if (((uintptr_t)workspace & 255u) != 0) return fail(GDN_E_WORKSPACE, "workspace is not 256-byte aligned");
@@ -428,19 +455,27 @@ gdn_status gdn_prefill(const gdn_config* cfg, const gdn_params* params, const vo
   cudaStream_t st = (cudaStream_t)stream;
   const bool bf16 = cfg->io_dtype == GDN_BF16;
   const bool zero_state = flags & GDN_ZERO_INIT_STATE, zero_conv = flags & GDN_ZERO_INIT_CONV;
+  const int32_t rows = sched_rows(path, chunk_size);  // rows per scheduled chunk (tiles on the affine path)
   int64_t chunks = 0;
-  for (int32_t n = 0; n < num_seqs; ++n) chunks += (cu_seqlens_host[n + 1] - cu_seqlens_host[n] + chunk_size - 1) / chunk_size;
+  for (int32_t n = 0; n < num_seqs; ++n) chunks += (cu_seqlens_host[n + 1] - cu_seqlens_host[n] + rows - 1) / rows;
   const gdn::ScheduleLayout L = gdn::schedule_layout(num_seqs, chunks);
   cudaError_t e = cudaSuccess;
   const int32_t* order = nullptr;
   if (num_seqs > 1) {  // one sequence needs neither an order nor a chunk map
-    e = gdn::launch_schedule(cu_seqlens_dev, num_seqs, chunk_size, chunks, workspace, st);
+    e = gdn::launch_schedule(cu_seqlens_dev, num_seqs, rows, chunks, workspace, st);
     order = (const int32_t*)((const char*)workspace + L.order_off);
   }
-  const bool chunked = !(flags & GDN_PREFILL_RECURRENT) && gdn::prefill_chunked_supported(d, bf16, chunk_size);
-  if (e == cudaSuccess && split) {
-    // intermediates start after the schedule sized for the chunk bound (the layout the size query assumed)
-    const size_t sched = gdn::schedule_layout(num_seqs, chunk_bound(total, num_seqs, chunk_size)).total_bytes;
+  const bool chunked = path == Path::Fused;
+  // intermediates start after the schedule sized for the chunk bound (the layout the size query assumed)
+  const size_t sched = gdn::schedule_layout(num_seqs, chunk_bound(total, num_seqs, rows)).total_bytes;
+  if (e == cudaSuccess && path == Path::Wy) {
+    e = gdn::launch_prefill_wy(d, chunk_size, params->conv_w, params->A_log, params->dt_bias, params->norm_w, qkv,
+                               z, a, b, cu_seqlens_dev, order,
+                               num_seqs > 1 ? (const int32_t*)((const char*)workspace + L.chunk_off_off) : nullptr,
+                               num_seqs > 1 ? (const int4*)((const char*)workspace + L.chunk_map_off) : nullptr,
+                               num_seqs, total, chunks, zero_state, zero_conv, conv_state, state, o,
+                               (char*)workspace + sched, g_status_ptr[dev], st);
+  } else if (e == cudaSuccess && path == Path::Split) {
     e = gdn::launch_prefill_split(d, params->conv_w, params->A_log, params->dt_bias, params->norm_w, qkv, z, a, b,
                                   cu_seqlens_dev, order,
                                   num_seqs > 1 ? (const int32_t*)((const char*)workspace + L.chunk_off_off) : nullptr,
@@ -606,7 +641,8 @@ gdn_status gdn_prefill_indexed(const gdn_config* cfg, const gdn_params* params, 
   if ((s = check_slots(state_indices, num_slots, num_seqs)) != GDN_OK) return s;
   if (chunk_size != 16 && chunk_size != 32 && chunk_size != 64 && chunk_size != 128)
     return fail(GDN_E_INVAL, "chunk_size %d (16, 32, 64 or 128)", chunk_size);
-  const uint32_t known = GDN_ZERO_INIT_STATE | GDN_ZERO_INIT_CONV | GDN_PREFILL_RECURRENT | GDN_PREFILL_FUSED;
+  const uint32_t known =
+      GDN_ZERO_INIT_STATE | GDN_ZERO_INIT_CONV | GDN_PREFILL_RECURRENT | GDN_PREFILL_FUSED | GDN_PREFILL_FACTORED;
   if (flags & ~known) return fail(GDN_E_INVAL, "unknown flags 0x%x", flags & ~known);
   int64_t total = 0;
   int32_t max_len = 0;
@@ -619,7 +655,7 @@ gdn_status gdn_prefill_indexed(const gdn_config* cfg, const gdn_params* params, 
       return s;
   }
   const bool bf16 = cfg->io_dtype == GDN_BF16;
-  const size_t base = prefill_ws_bytes(d, split_path(d, cfg, chunk_size, flags), total, num_seqs, chunk_size);
+  const size_t base = prefill_ws_bytes(d, prefill_path(d, cfg, chunk_size, flags), total, num_seqs, chunk_size);
   const IndexedLayout L = indexed_layout(d, bf16, base, num_seqs);
   if (workspace_bytes < L.total || !workspace)
     return fail(GDN_E_WORKSPACE, "workspace of %zu bytes at %p, need %zu", workspace_bytes, workspace, L.total);

@@ -140,6 +140,22 @@ size_t prefill_fused_ws_bytes(int64_t total_tokens, int32_t num_seqs, int32_t ch
 cudaError_t launch_checksum(const void* payload, size_t bytes, unsigned long long* out, cudaStream_t stream);
 uint64_t host_checksum(const void* payload, size_t bytes);
 
+// prefill_wy.cu (tcgen05; bf16 io, d_k = d_v = 128, chunk 16/32/64): conv, per-tile operands of the
+// affine chunk maps, and the state carry, over a workspace of intermediates (after the schedule, which
+// is built for tiles of wy_tile(chunk) rows)
+bool prefill_wy_supported(const Dims& d, bool bf16, int chunk_size);
+int wy_tile(int chunk_size);
+struct WyLayout {
+  size_t qk_hi, qk_lo, vimg, records, total_bytes;
+};
+WyLayout wy_layout(const Dims& d, int64_t total_tokens, int64_t tile_bound, int chunk_size);
+cudaError_t launch_prefill_wy(const Dims& d, int chunk_size, const float* conv_w, const float* A_log,
+                              const float* dt_bias, const float* norm_w, const void* qkv, const void* z,
+                              const void* a, const void* b, const int32_t* cu, const int32_t* order,
+                              const int32_t* tile_off, const int4* tile_map, int32_t N, int64_t total_tokens,
+                              int64_t total_tiles, bool zero_state, bool zero_conv, const void* conv_state,
+                              float* state, void* o, void* ws, int32_t* status, cudaStream_t stream);
+
 // diag.cu: a kernel whose bounded wait always runs out (tests the status path)
 cudaError_t launch_wait_expiry(uint64_t limit_ns, int32_t* status, cudaStream_t stream);
 

@@ -77,7 +77,12 @@ def test_workspace_size_and_bad_chunk():
     # q^, k^ (two fp16 parts) and v^, per (chunk, value head) a 65,664-byte record
     per_token = (2 * 2 * 16 * 128 + 48 * 128) * 2
     assert small >= 4096 * per_token + 64 * 48 * 65664
-    sched_only = gdn.prefill_workspace_size(cfg, 65536, 16, 16)  # token-recurrent path: the schedule alone
+    # the affine chunked path runs chunks 16, 32 and 64 on bf16 d=128: per token q^, k^ (two parts) and,
+    # per (64-row tile, value head), the two v^ images and the operand record
+    for chunk in (16, 32):
+        assert gdn.prefill_workspace_size(cfg, 4096, 1, chunk) >= 4096 * 2 * 2 * 16 * 128 * 2 + 64 * 48 * 32768
+    f32 = gdn.make_config(gi.Geometry(io_dtype="f32"))
+    sched_only = gdn.prefill_workspace_size(f32, 65536, 16, 16)  # token-recurrent path: the schedule alone
     assert 0 < sched_only < (1 << 20)
     with pytest.raises(gdn.GdnError) as e:
         gdn.prefill_workspace_size(cfg, 4096, 1, 48)
@@ -319,7 +324,9 @@ def test_seqpar_validation_and_workspace():
     w4 = gdn.prefill_seqpar_workspace_size(cfg, 65536, 4)
     w8 = gdn.prefill_seqpar_workspace_size(cfg, 65536, 8)
     assert w8 - w4 >= 3 * 4 * geo.num_v_heads * 128 * 128 * 4
-    assert w4 > gdn.prefill_workspace_size(cfg, 65536, 1, 64)  # the chunked form's intermediates plus the states
+    # the factored chunked form's intermediates (q^, k^ in two parts; a 123,520-byte record per (chunk,
+    # value head)) plus the segment states
+    assert w4 > 65536 * 2 * 2 * geo.num_k_heads * 128 * 2 + 1024 * geo.num_v_heads * 123520
     for g, status in [(gi.Geometry(num_k_heads=2, num_v_heads=6, head_k_dim=64, head_v_dim=64), "GDN_E_UNSUPPORTED"),
                       (gi.Geometry(num_k_heads=2, num_v_heads=6, io_dtype="f32"), "GDN_E_UNSUPPORTED")]:
         with pytest.raises(gdn.GdnError) as e:

@@ -51,8 +51,8 @@ def _guards_intact(raw: torch.Tensor) -> bool:
     return bool((g == PATTERN).all())
 
 
-@pytest.mark.parametrize("chunk,flags", [(64, 0), (64, gdn.PREFILL_FUSED), (64, gdn.PREFILL_RECURRENT), (16, 0),
-                                         (32, 0), (128, 0)])
+@pytest.mark.parametrize("chunk,flags", [(64, 0), (64, gdn.PREFILL_FACTORED), (64, gdn.PREFILL_FUSED),
+                                         (64, gdn.PREFILL_RECURRENT), (16, 0), (32, 0), (128, 0)])
 def test_prefill_writes_nothing_outside_its_buffers(chunk, flags):
     geo = gi.Geometry(num_k_heads=2, num_v_heads=6, head_k_dim=128, head_v_dim=128)
     inp = gi.make_prefill_inputs(geo, [1, 63, 64, 65, 130, 0, 3], seed=52, zero_init=False)

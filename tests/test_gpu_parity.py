@@ -21,6 +21,7 @@ pytestmark = pytest.mark.gpu
 
 RECURRENT = gdn.PREFILL_RECURRENT
 FUSED = gdn.PREFILL_FUSED
+FACTORED = gdn.PREFILL_FACTORED
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -194,7 +195,7 @@ def test_conv_prefill_and_step(io):
 def test_prefill_t4096_matches_oracle():
     inp = gi.workload_inputs("prefill_t4096")
     o_ref, st_ref, hist_ref = oracle.prefill_inputs(inp)
-    for flags in (0, FUSED, RECURRENT):
+    for flags in (0, FACTORED, FUSED, RECURRENT):
         _, o, st, hist = run_gpu_prefill(inp, 64, flags | gdn.ZERO_INIT_STATE)
         eo, es = compare_prefill(inp, o, st, o_ref, st_ref, TOL_O_BF16, TOL_S_BF16)
         print(f"prefill T=4096 flags={flags}: o max-rel {eo:.2e}, state max-rel {es:.2e}")
@@ -399,21 +400,39 @@ def test_launch_count_and_profiler():
 # ------------------------------------------------------------------ chunked tensor-core prefill
 
 
-@pytest.mark.parametrize("flags", [0, FUSED])
+@pytest.mark.parametrize("chunk,flags", [(16, 0), (32, 0), (64, 0), (128, 0), (64, FACTORED), (64, FUSED)])
 @pytest.mark.parametrize("zero_init", [True, False])
-def test_chunked_partial_chunks_match_oracle(zero_init, flags):
-    # lengths around chunk boundaries (64): partial first/last chunks, exact multiples, short sequences
+def test_chunked_partial_chunks_match_oracle(zero_init, chunk, flags):
+    # lengths around chunk and 64-row tile boundaries: partial first/last chunks, exact multiples, short sequences
     geo = gi.Geometry(num_k_heads=2, num_v_heads=6, head_k_dim=128, head_v_dim=128)
-    lengths = [1, 63, 64, 65, 127, 128, 129, 200, 2, 3]
+    lengths = [1, 15, 16, 17, 31, 33, 63, 64, 65, 127, 128, 129, 200, 257, 2, 3]
     inp = gi.make_prefill_inputs(geo, lengths, seed=31, zero_init=zero_init)
     o_ref, st_ref, hist_ref = oracle.prefill_inputs(inp)
-    _, o, st, hist = run_gpu_prefill(inp, 64, flags)
+    _, o, st, hist = run_gpu_prefill(inp, chunk, flags)
     eo, es = compare_prefill(inp, o, st, o_ref, st_ref, TOL_O_BF16, TOL_S_BF16)
-    print(f"chunked partial chunks (flags {flags}): o {eo:.2e} state {es:.2e}")
+    print(f"chunked partial chunks (chunk {chunk}, flags {flags}): o {eo:.2e} state {es:.2e}")
     assert np.array_equal(hist, ref_hist_bits(inp, hist_ref))
 
 
-@pytest.mark.parametrize("flags", [0, FUSED])
+@pytest.mark.parametrize("chunk", [16, 32, 64, 128])
+def test_affine_path_runs_its_tensor_core_kernels(chunk):
+    """bf16 d=128 at chunk 16, 32, 64 and 128 runs the three kernels of the affine
+    chunked path (no token-recurrent kernel), so the chunk-size comparisons
+    below compare different chunkwise computations."""
+    geo = gi.Geometry(num_k_heads=2, num_v_heads=6, head_k_dim=128, head_v_dim=128)
+    inp = gi.make_prefill_inputs(geo, [100, 37], seed=34, zero_init=False)
+    dp = DeviceProblem(inp, chunk)
+    gdn.profiler_reset()
+    gdn.profiler_enable(True)
+    dp.prefill()
+    torch.cuda.synchronize()
+    gdn.profiler_enable(False)
+    ran = {k for k in range(gdn.K.COUNT) if gdn.profiler_read(k)[0] > 0}
+    assert {gdn.K.WY_CONV, gdn.K.WY_PREP, gdn.K.WY_CHAIN} <= ran
+    assert gdn.K.PREFILL_RECURRENT not in ran and gdn.K.SPLIT_CHAIN not in ran
+
+
+@pytest.mark.parametrize("flags", [0, FACTORED, FUSED])
 def test_chunked_matches_recurrent_kernel(flags):
     geo = gi.Geometry(num_k_heads=4, num_v_heads=12, head_k_dim=128, head_v_dim=128)
     inp = gi.make_prefill_inputs(geo, [300, 64, 1, 517], seed=32, zero_init=False)

@@ -306,7 +306,7 @@ def run_gdn(args, rank, world, local_rank):
     del base
     ws = torch.empty(gdn.prefill_workspace_size(cfg, T, 1, C) + 256, dtype=torch.uint8, device="cuda")
     flags = gdn.ZERO_INIT_STATE | (gdn.PREFILL_RECURRENT if args.recurrent else 0) | \
-        (gdn.PREFILL_FUSED if args.fused else 0) | (gdn.PREFILL_FACTORED if args.factored else 0)
+        (gdn.PREFILL_FUSED if args.fused else 0) | (gdn.PREFILL_AFFINE if args.affine else 0)
 
     def prefill(i):
         s = sets[i % ROTATE]
@@ -775,7 +775,7 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=DECODE_STEPS)
     ap.add_argument("--recurrent", action="store_true", help="time the token-recurrent prefill kernel")
     ap.add_argument("--fused", action="store_true", help="time the single-kernel chunked prefill")
-    ap.add_argument("--factored", action="store_true", help="time the factored three-kernel chunked prefill")
+    ap.add_argument("--affine", action="store_true", help="time the affine three-kernel chunked prefill at chunk 64")
     ap.add_argument("--no-workloads", action="store_true", help="skip the long-context and varlen workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--projection-reps", type=int, default=20, help="timed launches per projection shape")

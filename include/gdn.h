@@ -105,8 +105,10 @@ typedef struct {
 #define GDN_PREFILL_RECURRENT 0x4u /* run the token-recurrent fp32 kernel instead of the chunked one */
 #define GDN_PREFILL_FUSED 0x8u     /* chunked path as one kernel per (sequence, value head): needs only the
                                       schedule as workspace (see gdn_prefill) */
-#define GDN_PREFILL_FACTORED 0x10u /* chunk 64 only: the three-kernel chunked path in the factored form
-                                      (W S, then K~^T Delta per chunk) instead of the affine chunk maps */
+#define GDN_PREFILL_FACTORED 0x10u /* chunk 64: the three-kernel chunked path in the factored form (W S,
+                                      then K~^T Delta per chunk); the default at chunk 64 */
+#define GDN_PREFILL_AFFINE 0x20u   /* bf16, d = 128: the three-kernel chunked path in the affine form (one
+                                      M' S product per chunk on the carry); the default at 16, 32, 128 */
 
 /* --------------------------------------------------------------------------
  * Causal depthwise Conv1D + SiLU over the q/k/v channels (issue #88, Scope:
@@ -148,16 +150,19 @@ GDN_API gdn_status gdn_prefill_workspace_size(const gdn_config* cfg, int64_t tot
 /* gdn_prefill: runs the whole mixer over every token of every sequence.
  *   chunk_size: 16, 32, 64 or 128 (tokens per chunk of the chunkwise form;
  *               chunks restart at each sequence start).
- *   flags:      GDN_ZERO_INIT_STATE / GDN_ZERO_INIT_CONV / GDN_PREFILL_RECURRENT /
- *               GDN_PREFILL_FUSED.
+ *   flags:      GDN_ZERO_INIT_STATE / GDN_ZERO_INIT_CONV, and at most one of
+ *               GDN_PREFILL_RECURRENT / GDN_PREFILL_FUSED / GDN_PREFILL_FACTORED /
+ *               GDN_PREFILL_AFFINE (GDN_E_INVAL if more than one).
  *   conv_state and state are read and updated in place; o is written.
- * When io dtype is bf16, d_k = d_v = 128 and chunk_size = 64 the chunked form
- * runs on tensor cores: by default as three kernels (conv of every token; the
- * state-independent operands of every chunk; the state carry across chunks),
- * with GDN_PREFILL_FUSED as one kernel per (sequence, value head).  The two
- * agree to fp32 rounding (not bit for bit).  Every other supported case (and
- * GDN_PREFILL_RECURRENT) runs the token-recurrent fp32 kernel.  All compute in
- * fp32 with an fp32 state. */
+ * When io dtype is bf16 and d_k = d_v = 128 the chunked form runs on tensor
+ * cores as three kernels (conv of every token; the state-independent operands
+ * of every chunk; the state carry across chunks): at chunk 16, 32 and 128 in
+ * the affine form (GDN_PREFILL_AFFINE), at chunk 64 by default in the
+ * factored form (GDN_PREFILL_FACTORED), the affine form with
+ * GDN_PREFILL_AFFINE, or one kernel per (sequence, value head) with
+ * GDN_PREFILL_FUSED.  Paths and chunk sizes agree to fp32 rounding (not bit for
+ * bit).  Every other supported case (and GDN_PREFILL_RECURRENT) runs the
+ * token-recurrent fp32 kernel.  All compute in fp32 with an fp32 state. */
 GDN_API gdn_status gdn_prefill(const gdn_config* cfg, const gdn_params* params, const void* qkv, const void* z,
                        const void* a, const void* b, const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host,
                        int32_t num_seqs, int32_t chunk_size, uint32_t flags, void* conv_state, float* state,
@@ -383,8 +388,11 @@ GDN_API gdn_status gdn_state_restore(const gdn_config* cfg, const void* blob, si
  * Diagnostics and measurement.
  *
  * gdn_get_device_status: reads and clears the device status word, which a
- * kernel sets (never traps) when an internal wait reaches its iteration limit
- * or a debug bounds check fails.  0 = clean.  Synchronises the stream.
+ * kernel sets (never traps) when an internal wait reaches its time limit, or
+ * a state slot index lies past its pool.  0 = clean.  The low byte is the
+ * code (1 wait timeout, 3 slot past the pool); the bits above it, when set,
+ * are the gdn_kernel_id of the kernel that reported it.  The first report
+ * since the last read is kept.  Synchronises the stream.
  * gdn_last_error: message of the calling thread's last failed call.
  * gdn_launch_count: kernels this library has launched since load or reset.
  * gdn_profiler_*: when enabled, every launch is bracketed by CUDA events on

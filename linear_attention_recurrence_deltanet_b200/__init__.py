@@ -21,7 +21,7 @@ __all__ = [
     "prefill", "prefill_noalloc", "decode_step", "decode_multi", "decode_step_indexed", "decode_multi_indexed",
     "prefill_indexed_workspace_size", "prefill_indexed", "gemm_bf16", "project_in", "project_out", "prefill_seqpar_workspace_size", "prefill_seqpar", "state_blob_size", "state_save", "state_restore", "device_status", "debug_wait_expiry", "last_error",
     "abi_version", "launch_count", "launch_count_reset", "profiler_enable", "profiler_reset", "profiler_read",
-    "kernel_name", "EXPORTS", "ZERO_INIT_STATE", "ZERO_INIT_CONV", "PREFILL_RECURRENT", "PREFILL_FUSED", "PREFILL_FACTORED", "K", "MAX_DRAFT_TOKENS",
+    "kernel_name", "EXPORTS", "ZERO_INIT_STATE", "ZERO_INIT_CONV", "PREFILL_RECURRENT", "PREFILL_FUSED", "PREFILL_FACTORED", "PREFILL_AFFINE", "K", "MAX_DRAFT_TOKENS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
@@ -31,6 +31,7 @@ ZERO_INIT_CONV = 0x2
 PREFILL_RECURRENT = 0x4
 PREFILL_FUSED = 0x8
 PREFILL_FACTORED = 0x10
+PREFILL_AFFINE = 0x20
 MAX_DRAFT_TOKENS = 4
 
 F32, BF16 = 0, 1

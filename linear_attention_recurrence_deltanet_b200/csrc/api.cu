@@ -198,18 +198,21 @@ int64_t chunk_bound(int64_t total_tokens, int32_t num_seqs, int32_t chunk_size) 
   return total_tokens / chunk_size + num_seqs + 1;
 }
 
-// Prefill paths: the affine chunk maps (three kernels; bf16, d = 128, chunk 16/32/64) by default; the
-// factored three-kernel path (chunk 64) with GDN_PREFILL_FACTORED; one kernel per (sequence, value head)
-// with GDN_PREFILL_FUSED; the token-recurrent kernel otherwise.
+// Prefill paths (bf16, d = 128): the factored three-kernel path at chunk 64, the affine three-kernel
+// path at chunk 16, 32 and 128 (and at 64 with GDN_PREFILL_AFFINE), one kernel per (sequence, value head)
+// with GDN_PREFILL_FUSED (chunk 64); the token-recurrent kernel for everything else.
 enum class Path { Wy, Split, Fused, Recurrent };
+
+constexpr uint32_t kPathFlags = GDN_PREFILL_RECURRENT | GDN_PREFILL_FUSED | GDN_PREFILL_FACTORED | GDN_PREFILL_AFFINE;
 
 Path prefill_path(const gdn::Dims& d, const gdn_config* cfg, int32_t chunk_size, uint32_t flags) {
   const bool bf16 = cfg->io_dtype == GDN_BF16;
   if (flags & GDN_PREFILL_RECURRENT) return Path::Recurrent;
   if (flags & GDN_PREFILL_FUSED)
     return gdn::prefill_chunked_supported(d, bf16, chunk_size) ? Path::Fused : Path::Recurrent;
-  if (flags & GDN_PREFILL_FACTORED)
-    return gdn::prefill_chunked_supported(d, bf16, chunk_size) ? Path::Split : Path::Recurrent;
+  if (flags & GDN_PREFILL_AFFINE)
+    return gdn::prefill_wy_supported(d, bf16, chunk_size) ? Path::Wy : Path::Recurrent;
+  if (gdn::prefill_chunked_supported(d, bf16, chunk_size)) return Path::Split;  // chunk 64 (factored)
   if (gdn::prefill_wy_supported(d, bf16, chunk_size)) return Path::Wy;
   return Path::Recurrent;
 }
@@ -230,7 +233,7 @@ size_t prefill_ws_bytes(const gdn::Dims& d, Path p, int64_t total_tokens, int32_
 size_t prefill_ws_query(const gdn::Dims& d, const gdn_config* cfg, int64_t total_tokens, int32_t num_seqs,
                         int32_t chunk_size) {
   size_t m = 0;
-  for (uint32_t f : {0u, (uint32_t)GDN_PREFILL_FACTORED, (uint32_t)GDN_PREFILL_FUSED})
+  for (uint32_t f : {0u, (uint32_t)GDN_PREFILL_FACTORED, (uint32_t)GDN_PREFILL_AFFINE, (uint32_t)GDN_PREFILL_FUSED})
     m = std::max(m, prefill_ws_bytes(d, prefill_path(d, cfg, chunk_size, f), total_tokens, num_seqs, chunk_size));
   return m;
 }
@@ -429,9 +432,10 @@ gdn_status gdn_prefill(const gdn_config* cfg, const gdn_params* params, const vo
   if ((s = check_params(params)) != GDN_OK) return s;
   if (chunk_size != 16 && chunk_size != 32 && chunk_size != 64 && chunk_size != 128)
     return fail(GDN_E_INVAL, "chunk_size %d (16, 32, 64 or 128)", chunk_size);
-  const uint32_t known =
-      GDN_ZERO_INIT_STATE | GDN_ZERO_INIT_CONV | GDN_PREFILL_RECURRENT | GDN_PREFILL_FUSED | GDN_PREFILL_FACTORED;
+  const uint32_t known = GDN_ZERO_INIT_STATE | GDN_ZERO_INIT_CONV | kPathFlags;
   if (flags & ~known) return fail(GDN_E_INVAL, "unknown flags 0x%x", flags & ~known);
+  if (__builtin_popcount(flags & kPathFlags) > 1)
+    return fail(GDN_E_INVAL, "flags 0x%x select more than one prefill path", flags & kPathFlags);
   int64_t total = 0;
   int32_t max_len = 0;
   if ((s = check_cu(cu_seqlens_dev, cu_seqlens_host, num_seqs, &total, &max_len)) != GDN_OK) return s;
@@ -641,9 +645,10 @@ gdn_status gdn_prefill_indexed(const gdn_config* cfg, const gdn_params* params, 
   if ((s = check_slots(state_indices, num_slots, num_seqs)) != GDN_OK) return s;
   if (chunk_size != 16 && chunk_size != 32 && chunk_size != 64 && chunk_size != 128)
     return fail(GDN_E_INVAL, "chunk_size %d (16, 32, 64 or 128)", chunk_size);
-  const uint32_t known =
-      GDN_ZERO_INIT_STATE | GDN_ZERO_INIT_CONV | GDN_PREFILL_RECURRENT | GDN_PREFILL_FUSED | GDN_PREFILL_FACTORED;
+  const uint32_t known = GDN_ZERO_INIT_STATE | GDN_ZERO_INIT_CONV | kPathFlags;
   if (flags & ~known) return fail(GDN_E_INVAL, "unknown flags 0x%x", flags & ~known);
+  if (__builtin_popcount(flags & kPathFlags) > 1)
+    return fail(GDN_E_INVAL, "flags 0x%x select more than one prefill path", flags & kPathFlags);
   int64_t total = 0;
   int32_t max_len = 0;
   if ((s = check_cu(cu_seqlens_dev, cu_seqlens_host, num_seqs, &total, &max_len)) != GDN_OK) return s;

@@ -18,7 +18,6 @@ struct Dims {
 enum : int32_t {
   kStatusOk = 0,
   kStatusWaitTimeout = 1,   // a bounded wait gave up
-  kStatusBoundsCheck = 2,   // a debug bounds check failed
   kStatusBadSlot = 3,       // a state slot index past the end of the pool (the row was skipped)
 };
 

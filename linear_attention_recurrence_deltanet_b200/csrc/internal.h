@@ -146,7 +146,7 @@ uint64_t host_checksum(const void* payload, size_t bytes);
 bool prefill_wy_supported(const Dims& d, bool bf16, int chunk_size);
 int wy_tile(int chunk_size);
 struct WyLayout {
-  size_t qk_hi, qk_lo, vimg, records, total_bytes;
+  size_t qk_hi, qk_lo, vimg, gate, records, total_bytes;
 };
 WyLayout wy_layout(const Dims& d, int64_t total_tokens, int64_t tile_bound, int chunk_size);
 cudaError_t launch_prefill_wy(const Dims& d, int chunk_size, const float* conv_w, const float* A_log,

@@ -729,6 +729,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
     bulk_prefetch_l2(rec_of(cc), REC_V);
     bulk_prefetch_l2(rec_of(cc) + REC_P, REC_META + 16 - REC_P);
   };
+  float S[32];  // this thread's part of the state, fp32
+  if (compute) {
+#pragma unroll
+    for (int jj = 0; jj < 32; ++jj) S[jj] = zero_state ? 0.f : gst[(int64_t)(c0 + jj) * kD + si];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) st16h(sm + C_SB + mnmaj_chunk(kD, si, 32 * hc + 8 * m), S + 8 * m);
+  }
+  fence_async_smem();
+  sync_tc();
+  const uint32_t tbase = tslot;
+  // the first copies go out only after the block barrier that publishes the mbarriers' initialisation
   if (copy_warp && lane == 0) {
     issue_a(0);
     if (!zero_u) issue_u(0);
@@ -741,16 +752,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
     }
     if (nchunks > 2 && vh == 0) prefetch(2);
   }
-  float S[32];  // this thread's part of the state, fp32
-  if (compute) {
-#pragma unroll
-    for (int jj = 0; jj < 32; ++jj) S[jj] = zero_state ? 0.f : gst[(int64_t)(c0 + jj) * kD + si];
-#pragma unroll
-    for (int m = 0; m < 4; ++m) st16h(sm + C_SB + mnmaj_chunk(kD, si, 32 * hc + 8 * m), S + 8 * m);
-  }
-  fence_async_smem();
-  sync_tc();
-  const uint32_t tbase = tslot;
   cluster_sync();  // the peer's mbarriers are initialised before any arrival on them
   const uint32_t peer = (uint32_t)(vh ^ 1);
   const uint32_t peer_x0 = mapa_shared(smem_u32(&mb_x[0]), peer), peer_x1 = mapa_shared(smem_u32(&mb_x[1]), peer);

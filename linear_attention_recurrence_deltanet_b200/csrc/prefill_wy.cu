@@ -20,7 +20,8 @@
 //                    ("causal depthwise Conv1D", DS4Server issue #88, Scope),
 //                    L2 norms of q and k with epsilon inside the square root;
 //                    q^, k^ as fp16 hi + lo parts (row-major) and v^ as fp16
-//                    hi + lo operand images per (tile, value head).
+//                    hi + lo operand images per (tile, value head); and the
+//                    output gate (1 + w) sigmoid(z) of every value head, fp16.
 //   wy_prep_kernel   grid (tile, value head): gates and their per-chunk scan,
 //                    [K;Q]K^T in split precision, A and P, T = (I+A)^-1 by
 //                    recursive doubling whose merges are tcgen05 MMAs, W and
@@ -31,7 +32,7 @@
 //                    of the two halves: per chunk Y = K~^T U + M' S and O =
 //                    P U + Q' S on tcgen05, S = e^{gamma_C} S + Y in fp32
 //                    registers, and the output rows (RMSNorm over d_v times
-//                    (1 + w) sigmoid(z)) by separate warps.
+//                    the gate) by separate warps.
 //
 // Tiles: the prep and chain kernels work on tiles of 64 rows (chunk sizes 16,
 // 32 and 64: a tile holds 64 / C chunks, and every intra-chunk matrix is block
@@ -52,6 +53,9 @@ using namespace tc;
 
 constexpr int kD = 128;
 constexpr uint64_t kWaitNs = 2000000000ull;
+// a wait that runs out is reported as the code in the low byte and the reporting kernel's id above it
+constexpr int32_t kTimeoutPrep = kStatusWaitTimeout | (GDN_K_WY_PREP << 8);
+constexpr int32_t kTimeoutChain = kStatusWaitTimeout | (GDN_K_WY_CHAIN << 8);
 
 // ------------------------------------------------------------------ record of one (tile, value head)
 // Byte images of the chain kernel's operands (fp16, 128-byte swizzle):
@@ -89,7 +93,8 @@ __global__ void __launch_bounds__(256)
     wy_conv_kernel(Dims d, const float* __restrict__ conv_w, const __nv_bfloat16* __restrict__ qkv,
                    const __nv_bfloat16* __restrict__ hist, int zero_conv, const int4* __restrict__ tile_map,
                    int64_t single_len, __half* __restrict__ qk_hi, __half* __restrict__ qk_lo,
-                   unsigned char* __restrict__ vimg) {
+                   unsigned char* __restrict__ vimg, const float* __restrict__ norm_w,
+                   const __nv_bfloat16* __restrict__ z, __half* __restrict__ gate) {
   constexpr int SUB = TILE / 64;
   const int gt = blockIdx.x / SUB, part = blockIdx.x - gt * SUB;
   const int64_t rest = single_len - (int64_t)TILE * gt;
@@ -99,6 +104,28 @@ __global__ void __launch_bounds__(256)
   const int r0 = 64 * part + kConvRows * warp;  // first row of this warp within the tile
   const int L = cm.z;
   const int nqk = 2 * d.Hk;
+  if (slot >= nqk + d.Hv) {  // the output gate (1 + w_j) sigmoid(z_j) of one value head, fp16
+    const int64_t HvD = (int64_t)d.Hv * kD;
+    const int64_t col = (int64_t)(slot - nqk - d.Hv) * kD + 4 * lane;
+    const float4 w = __ldg(reinterpret_cast<const float4*>(norm_w + 4 * lane));
+    const float nw[4] = {1.0f + w.x, 1.0f + w.y, 1.0f + w.z, 1.0f + w.w};
+    uint2 u[kConvRows];
+#pragma unroll
+    for (int i = 0; i < kConvRows; ++i)
+      u[i] = (r0 + i < L) ? __ldg(reinterpret_cast<const uint2*>(z + (cm.y + r0 + i) * HvD + col)) : make_uint2(0u, 0u);
+#pragma unroll
+    for (int i = 0; i < kConvRows; ++i) {
+      if (r0 + i < L) {
+        const float zz[4] = {__uint_as_float(u[i].x << 16), __uint_as_float(u[i].x & 0xffff0000u),
+                             __uint_as_float(u[i].y << 16), __uint_as_float(u[i].y & 0xffff0000u)};
+        float g[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) g[e] = nw[e] * __fdividef(1.0f, 1.0f + __expf(-zz[e]));
+        st8(reinterpret_cast<unsigned char*>(gate + (cm.y + r0 + i) * HvD + col), g[0], g[1], g[2], g[3]);
+      }
+    }
+    return;
+  }
   unsigned char* vrec = slot >= nqk ? vimg + ((int64_t)gt * d.Hv + (slot - nqk)) * kVImg<TILE> : nullptr;
   if (vrec) {  // rows past the tile's end are zero in both parts
 #pragma unroll
@@ -355,7 +382,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
   const uint32_t tbase = tslot;
   if (!mbar_wait(&mb_tma, 0, kWaitNs)) bad = true;
   if (sync_tc_any(bad)) {
-    if (tid == 0) set_status(status, kStatusWaitTimeout);
+    if (tid == 0) set_status(status, kTimeoutPrep);
     if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
     return;
   }
@@ -427,7 +454,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
   if (!mbar_wait(&mb_mma, mma_phase, kWaitNs)) bad = true;
   mma_phase ^= 1;
   if (sync_tc_any(bad)) {  // also: the tiles are read; KQL and the Q halves of KQH are free
-    if (tid == 0) set_status(status, kStatusWaitTimeout);
+    if (tid == 0) set_status(status, kTimeoutPrep);
     if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
     return;
   }
@@ -459,7 +486,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
           const int x = r ^ j;
           a16[e] = (x >= 16 && x < 32) ? av : 0.f;
           a32[e] = (x >= 32) ? av : 0.f;
-          if (x < 16) reinterpret_cast<float*>(sm + WP_DIAG)[(r >> 4) * 256 + (r & 15) * 16 + (j & 15)] = av;
+          if (x < 16) reinterpret_cast<float*>(sm + WP_DIAG)[(r >> 4) * 272 + (r & 15) * 17 + (j & 15)] = av;
         }
         *reinterpret_cast<uint4*>(sm + WP_AOFF16 + kmaj_chunk(64, r, 32 * hc + 8 * m)) = pack8h(a16);
         *reinterpret_cast<uint4*>(sm + WP_AOFF32 + kmaj_chunk(64, r, 32 * hc + 8 * m)) = pack8h(a32);
@@ -490,13 +517,13 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
   // one column of one block per thread, in fp32, rounded to fp16 once
   if (tid < 64) {
     const int bb = tid >> 4, c = tid & 15, o = 16 * bb;
-    const float* Ad = reinterpret_cast<const float*>(sm + WP_DIAG) + bb * 256;
+    const float* Ad = reinterpret_cast<const float*>(sm + WP_DIAG) + bb * 272;
     float t[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       float acc = (i == c) ? 1.f : 0.f;
 #pragma unroll
-      for (int k = 0; k < i; ++k) acc -= Ad[i * 16 + k] * t[k];
+      for (int k = 0; k < i; ++k) acc -= Ad[i * 17 + k] * t[k];
       t[i] = (i < c) ? 0.f : acc;
     }
 #pragma unroll
@@ -569,7 +596,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     }
   }
   if (abort) {
-    if (tid == 0) set_status(status, kStatusWaitTimeout);
+    if (tid == 0) set_status(status, kTimeoutPrep);
     if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
     return;
   }
@@ -613,20 +640,6 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
   if (!mbar_wait(&mb_mma, mma_phase, kWaitNs)) bad = true;
   mma_phase ^= 1;
   fence_after();
-  if (!mbar_wait(&mb_mma, mma_phase, kWaitNs)) bad = true;
-  mma_phase ^= 1;
-  if (sync_tc_any(bad)) {  // also: the tiles are read; KQL and the Q halves of KQH are free
-    if (tid == 0) set_status(status, kStatusWaitTimeout);
-    if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
-    return;
-  }
-  if (tid == 0) {  // v^ lo into the Q halves of KQH (MN-major, LBO 16 KB), behind the generic reads of q^
-    fence_async_smem();
-    mbar_expect_tx(&mb_vlo, 16384);
-    const unsigned char* vl = vimg + ((int64_t)g * d.Hv + h) * kVImg<TILE> + TILE * 256;
-    bulk_load(sm + WP_VLO, vl, 8192, &mb_vlo);
-    bulk_load(sm + WP_VLO + 16384, vl + 8192, 8192, &mb_vlo);
-  }
   {  // -W -> MN-major K=64 x N=128 (LBO 8 KB)
     float v[32];
 #pragma unroll
@@ -643,7 +656,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
   }
   fence_async_smem();
   if (sync_tc_any(bad)) {
-    if (tid == 0) set_status(status, kStatusWaitTimeout);
+    if (tid == 0) set_status(status, kTimeoutPrep);
     if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
     return;
   }
@@ -704,7 +717,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     }
   }
   if (sync_tc_any(bad)) {  // also: columns 0..127 are read out
-    if (tid == 0) set_status(status, kStatusWaitTimeout);
+    if (tid == 0) set_status(status, kTimeoutPrep);
     if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
     return;
   }
@@ -742,7 +755,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
       break;
     }
   }
-  if (abort && tid == 0) set_status(status, kStatusWaitTimeout);
+  if (abort && tid == 0) set_status(status, kTimeoutPrep);
   if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
 }
 
@@ -857,7 +870,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
   const uint32_t tbase = tslot;
   if (!mbar_wait(&mb_tma, 0, kWaitNs)) bad = true;
   if (sync_tc_any(bad)) {
-    if (tid == 0) set_status(status, kStatusWaitTimeout);
+    if (tid == 0) set_status(status, kTimeoutPrep);
     if (warp == 0) tmem_dealloc(tbase, 512);
     return;
   }
@@ -930,7 +943,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
   if (!mbar_wait(&mb_mma, ph, kWaitNs)) bad = true;
   ph ^= 1;
   if (sync_tc_any(bad)) {
-    if (tid == 0) set_status(status, kStatusWaitTimeout);
+    if (tid == 0) set_status(status, kTimeoutPrep);
     if (warp == 0) tmem_dealloc(tbase, 512);
     return;
   }
@@ -1065,7 +1078,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
     }
   }
   if (abort) {
-    if (tid == 0) set_status(status, kStatusWaitTimeout);
+    if (tid == 0) set_status(status, kTimeoutPrep);
     if (warp == 0) tmem_dealloc(tbase, 512);
     return;
   }
@@ -1129,7 +1142,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
   }
   fence_async_smem();
   if (sync_tc_any(bad)) {
-    if (tid == 0) set_status(status, kStatusWaitTimeout);
+    if (tid == 0) set_status(status, kTimeoutPrep);
     if (warp == 0) tmem_dealloc(tbase, 512);
     return;
   }
@@ -1219,7 +1232,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       }
     }
   }
-  if (sync_tc_any(bad) && tid == 0) set_status(status, kStatusWaitTimeout);
+  if (sync_tc_any(bad) && tid == 0) set_status(status, kTimeoutPrep);
   if (warp == 0) tmem_dealloc(tbase, 512);
 }
 
@@ -1260,10 +1273,10 @@ constexpr uint32_t CY0 = 0, CO0 = 128, kChainTmemCols = 256;  // Y_c at CY0 + 64
 
 template <int TILE, int C>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
-    wy_chain_kernel(Dims d, const unsigned char* __restrict__ records, const int32_t* __restrict__ tile_off,
-                    const int32_t* __restrict__ order, const int32_t* __restrict__ cu, int zero_state,
-                    const float* __restrict__ norm_w, const __nv_bfloat16* __restrict__ z, float* __restrict__ state,
-                    __nv_bfloat16* __restrict__ o, int32_t* status) {
+    wy_chain_kernel(Dims d, const unsigned char* __restrict__ records,
+                    const int32_t* __restrict__ tile_off, const int32_t* __restrict__ order,
+                    const int32_t* __restrict__ cu, int zero_state, const __half* __restrict__ gate,
+                    float* __restrict__ state, __nv_bfloat16* __restrict__ o, int32_t* status) {
   using R = Rec<TILE, C>;
   using F = ChainCfg<TILE, C>;
   constexpr int NCH = F::NCH, NM = F::NM, NB = F::NB;
@@ -1292,7 +1305,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
   const int64_t HvD = (int64_t)d.Hv * kD;
   const bool state_warp = warp < 8, out_warp = warp >= 8 && warp < 12, mma_warp = warp == 12,
              copy_warp = warp == 13;
-  float* s_nw = reinterpret_cast<float*>(sm + F::MISC + F::MS_NW);
   float* s_peer = reinterpret_cast<float*>(sm + F::MISC + F::MS_PEER);
   float* gst = state + ((int64_t)n * d.Hv + h) * kD * kD;  // stored [j][i]
 
@@ -1312,7 +1324,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
     mbar_init_fence();
   }
   if (warp == 0) tmem_alloc(&tslot, kChainTmemCols);
-  if (tid < 64) s_nw[tid] = 1.0f + norm_w[64 * vh + tid];
 
   auto rec_of = [&](int t) { return records + ((g0 + t) * d.Hv + h) * (int64_t)R::BYTES; };
   auto issue_tile = [&](int t) {
@@ -1331,10 +1342,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
     mbar_expect_tx(&mb_m[b], 32768);
     bulk_load(sm + F::MB + b * 32768, rec_of(c / NCH) + R::M + (c % NCH) * 32768, 32768, &mb_m[b]);
   };
-  if (copy_warp && lane == 0) {
-    for (int t = 0; t < NB && t < ntiles; ++t) issue_tile(t);
-    for (int c = 0; c < NM && c < nsteps; ++c) issue_m(c);
-  }
   float S[32];
   const int si = 32 * (warp & 3) + lane, hc = (warp >> 2) & 1;
   const int c0 = 64 * vh + 32 * hc;  // first value channel of a state thread's columns
@@ -1347,6 +1354,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
   fence_async_smem();
   sync_tc();
   const uint32_t tbase = tslot;
+  // the first copies go out only after the block barrier that publishes the mbarriers' initialisation
+  if (copy_warp && lane == 0) {
+    for (int t = 0; t < NB && t < ntiles; ++t) issue_tile(t);
+    for (int c = 0; c < NM && c < nsteps; ++c) issue_m(c);
+  }
   cluster_sync();  // the peer's mbarriers are initialised before any arrival on them
   const uint32_t peer = (uint32_t)(vh ^ 1);
   const uint32_t peer_x0 = mapa_shared(smem_u32(&mb_x[0]), peer), peer_x1 = mapa_shared(smem_u32(&mb_x[1]), peer);
@@ -1448,17 +1460,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
     const int q = warp - 8;
     const int r = TILE == 64 ? 16 * q + (lane & 15) : 32 * q + lane;  // this thread's row of the tile
     const bool has_row = TILE == 64 ? lane < 16 : true;
+    // the gate row (128 bytes) of this thread's row of chunk c: prefetched into L2 a few chunks ahead
+    // (a plain per-row prefetch: nothing asynchronous outlives the block), loaded one chunk ahead
+    constexpr int kGAhead = 3;
+    auto gate_row = [&](int c) -> const __half* {
+      const int t = c / NCH, s = c % NCH;
+      if (c < nsteps && has_row && (r / C) == s && (t * TILE + r) < len)
+        return gate + (seq0 + (int64_t)t * TILE + r) * HvD + (int64_t)h * kD + 64 * vh;
+      return nullptr;
+    };
+    uint4 gr[8];
+    auto load_gate = [&](int c) {
+      if (const __half* p = gate_row(c)) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) gr[i] = __ldg(reinterpret_cast<const uint4*>(p) + i);
+      }
+    };
+    for (int c = 0; c < kGAhead; ++c)
+      if (const __half* p = gate_row(c)) asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+    load_gate(0);
     for (int c = 0; c < nsteps; ++c) {
       const int t = c / NCH, s = c % NCH;
       const bool mine = has_row && (r / C) == s;
       const int64_t tok = seq0 + (int64_t)t * TILE + r;
       const bool valid = mine && (t * TILE + r) < len;
-      uint4 zr[8];
-      if (valid) {
-        const uint4* zp = reinterpret_cast<const uint4*>(z + tok * HvD + (int64_t)h * kD + 64 * vh);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) zr[i] = __ldg(zp + i);
-      }
       if (!mbar_wait(&mb_o[c & 1], (c >> 1) & 1, kWaitNs)) bad = true;
       tc::fence_after();
       float v[32], ss = 0.f;
@@ -1485,27 +1510,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
         if (valid) {
 #pragma unroll
           for (int m = 0; m < 4; ++m) {
-            const uint4 zq = zr[4 * hh + m];
-            const uint32_t zw[4] = {zq.x, zq.y, zq.z, zq.w};
+            const uint4 gq = gr[4 * hh + m];
+            const __half2* g2 = reinterpret_cast<const __half2*>(&gq);
             uint32_t ow[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int j = 32 * hh + 8 * m + 2 * e;
-              const float z0 = __uint_as_float(zw[e] << 16), z1 = __uint_as_float(zw[e] & 0xffff0000u);
-              const float g0 = s_nw[j] * __fdividef(1.0f, 1.0f + __expf(-z0));
-              const float g1 = s_nw[j + 1] * __fdividef(1.0f, 1.0f + __expf(-z1));
-              __nv_bfloat162 pr = __floats2bfloat162_rn(v[8 * m + 2 * e] * rinv * g0, v[8 * m + 2 * e + 1] * rinv * g1);
+              const float2 gf = __half22float2(g2[e]);
+              __nv_bfloat162 pr = __floats2bfloat162_rn(v[8 * m + 2 * e] * rinv * gf.x, v[8 * m + 2 * e + 1] * rinv * gf.y);
               ow[e] = *reinterpret_cast<uint32_t*>(&pr);
             }
             *reinterpret_cast<uint4*>(orow + 32 * hh + 8 * m) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
           }
         }
       }
+      if (const __half* p = gate_row(c + kGAhead)) asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+      if (c + 1 < nsteps) load_gate(c + 1);
       if (bad) break;
     }
   }
   if (sync_tc_any(bad)) {
-    if (tid == 0) set_status(status, kStatusWaitTimeout);
+    if (tid == 0) set_status(status, kTimeoutChain);
   } else if (state_warp) {
 #pragma unroll
     for (int jj = 0; jj < 32; ++jj) gst[(int64_t)(c0 + jj) * kD + si] = S[jj];
@@ -1550,6 +1574,7 @@ cudaError_t launch_wy(const Dims& d, const float* conv_w, const float* A_log, co
   __half* qk_hi = (__half*)(w + Lw.qk_hi);
   __half* qk_lo = (__half*)(w + Lw.qk_lo);
   unsigned char* vimg = w + Lw.vimg;
+  __half* gate = (__half*)(w + Lw.gate);
   unsigned char* records = w + Lw.records;
   CUtensorMap tm_hi, tm_lo;
   const uint64_t qkw = (uint64_t)2 * d.Hk * kD;
@@ -1558,9 +1583,10 @@ cudaError_t launch_wy(const Dims& d, const float* conv_w, const float* A_log, co
   cudaError_t e;
   {
     LaunchScope scope(GDN_K_WY_CONV, stream);
-    wy_conv_kernel<TILE><<<dim3((unsigned)(total_tiles * (TILE / 64)), (unsigned)(2 * d.Hk + d.Hv)), 256, 0, stream>>>(
-        d, conv_w, (const __nv_bfloat16*)qkv, (const __nv_bfloat16*)conv_state, zero_conv ? 1 : 0, tile_map,
-        total_tokens, qk_hi, qk_lo, vimg);
+    wy_conv_kernel<TILE><<<dim3((unsigned)(total_tiles * (TILE / 64)), (unsigned)(2 * d.Hk + 2 * d.Hv)), 256, 0,
+                           stream>>>(d, conv_w, (const __nv_bfloat16*)qkv, (const __nv_bfloat16*)conv_state,
+                                     zero_conv ? 1 : 0, tile_map, total_tokens, qk_hi, qk_lo, vimg, norm_w,
+                                     (const __nv_bfloat16*)z, gate);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if constexpr (TILE == 64) {
@@ -1590,8 +1616,7 @@ cudaError_t launch_wy(const Dims& d, const float* conv_w, const float* A_log, co
     return e;
   LaunchScope scope(GDN_K_WY_CHAIN, stream);
   wy_chain_kernel<TILE, C><<<(unsigned)((int64_t)N * d.Hv * 2), kChainThreads, F::SMEM, stream>>>(
-      d, records, tile_off, order, cu, zero_state ? 1 : 0, norm_w, (const __nv_bfloat16*)z, state,
-      (__nv_bfloat16*)o, status);
+      d, records, tile_off, order, cu, zero_state ? 1 : 0, gate, state, (__nv_bfloat16*)o, status);
   return cudaGetLastError();
 }
 
@@ -1611,7 +1636,8 @@ WyLayout wy_layout(const Dims& d, int64_t total_tokens, int64_t tile_bound, int 
   S.qk_hi = 0;
   S.qk_lo = al256(S.qk_hi + (size_t)total_tokens * qkw * 2);
   S.vimg = al256(S.qk_lo + (size_t)total_tokens * qkw * 2);
-  S.records = al256(S.vimg + (size_t)tile_bound * d.Hv * (tile * 512));
+  S.gate = al256(S.vimg + (size_t)tile_bound * d.Hv * (tile * 512));
+  S.records = al256(S.gate + (size_t)total_tokens * d.Hv * kD * 2);
   S.total_bytes = al256(S.records + (size_t)tile_bound * d.Hv * rec_bytes(chunk_size));
   return S;
 }

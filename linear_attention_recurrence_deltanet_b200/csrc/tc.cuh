@@ -84,18 +84,25 @@ __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.a
 // the same for every state space (e.g. generic global writes read back by a bulk copy)
 __device__ __forceinline__ void fence_async_all() { asm volatile("fence.proxy.async;" ::: "memory"); }
 
+// The tcgen05 alloc / dealloc / ld / st instructions are .sync.aligned: every lane
+// of the warp must execute them together.  Each helper first reconverges the
+// warp, since callers reach them after lane-dependent work (a lane that issued
+// and then waits for bulk copies, rows that only some lanes own).
 __device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+  __syncwarp();
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(ncols)
                : "memory");
   asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  __syncwarp();
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
 // 32 consecutive fp32 columns of this thread's lane
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   uint32_t r[32];
+  __syncwarp();
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
       "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
@@ -111,6 +118,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
 
 // store 32 consecutive fp32 columns of this thread's lane
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+  __syncwarp();
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
       "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
@@ -188,11 +196,6 @@ __device__ __forceinline__ void cp_async_wait() {
 // L2 prefetch of `bytes` (a multiple of 16) at a 16-byte aligned global address
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"((uint64_t)src), "r"(bytes) : "memory");
-}
-// L2 prefetch of the box at (x, y) of a tensor map
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"((uint64_t)map), "r"(x), "r"(y)
-               : "memory");
 }
 
 // 2D tiled load of the box at (x = inner coordinate, y = row) into shared memory,

@@ -128,6 +128,7 @@ def test_prefill_validation_rejects_before_launch():
         (dict(cu_host=[0, 8, 4]), "GDN_E_INVAL"),         # decreasing
         (dict(cu_host=[0, 8], chunk=100), "GDN_E_INVAL"),
         (dict(cu_host=[0, 8], flags=0x80), "GDN_E_INVAL"),
+        (dict(cu_host=[0, 8], flags=0x30), "GDN_E_INVAL"),   # two prefill paths at once
         (dict(cu_host=[0, 8], wsb=16), "GDN_E_WORKSPACE"),
     ]
     for kw, status in cases:

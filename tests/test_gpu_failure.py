@@ -51,7 +51,7 @@ def _guards_intact(raw: torch.Tensor) -> bool:
     return bool((g == PATTERN).all())
 
 
-@pytest.mark.parametrize("chunk,flags", [(64, 0), (64, gdn.PREFILL_FACTORED), (64, gdn.PREFILL_FUSED),
+@pytest.mark.parametrize("chunk,flags", [(64, 0), (64, gdn.PREFILL_AFFINE), (64, gdn.PREFILL_FUSED),
                                          (64, gdn.PREFILL_RECURRENT), (16, 0), (32, 0), (128, 0)])
 def test_prefill_writes_nothing_outside_its_buffers(chunk, flags):
     geo = gi.Geometry(num_k_heads=2, num_v_heads=6, head_k_dim=128, head_v_dim=128)

@@ -22,6 +22,7 @@ pytestmark = pytest.mark.gpu
 RECURRENT = gdn.PREFILL_RECURRENT
 FUSED = gdn.PREFILL_FUSED
 FACTORED = gdn.PREFILL_FACTORED
+AFFINE = gdn.PREFILL_AFFINE
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -195,7 +196,7 @@ def test_conv_prefill_and_step(io):
 def test_prefill_t4096_matches_oracle():
     inp = gi.workload_inputs("prefill_t4096")
     o_ref, st_ref, hist_ref = oracle.prefill_inputs(inp)
-    for flags in (0, FACTORED, FUSED, RECURRENT):
+    for flags in (0, AFFINE, FUSED, RECURRENT):
         _, o, st, hist = run_gpu_prefill(inp, 64, flags | gdn.ZERO_INIT_STATE)
         eo, es = compare_prefill(inp, o, st, o_ref, st_ref, TOL_O_BF16, TOL_S_BF16)
         print(f"prefill T=4096 flags={flags}: o max-rel {eo:.2e}, state max-rel {es:.2e}")
@@ -400,7 +401,7 @@ def test_launch_count_and_profiler():
 # ------------------------------------------------------------------ chunked tensor-core prefill
 
 
-@pytest.mark.parametrize("chunk,flags", [(16, 0), (32, 0), (64, 0), (128, 0), (64, FACTORED), (64, FUSED)])
+@pytest.mark.parametrize("chunk,flags", [(16, 0), (32, 0), (64, 0), (128, 0), (64, AFFINE), (64, FUSED)])
 @pytest.mark.parametrize("zero_init", [True, False])
 def test_chunked_partial_chunks_match_oracle(zero_init, chunk, flags):
     # lengths around chunk and 64-row tile boundaries: partial first/last chunks, exact multiples, short sequences
@@ -414,25 +415,38 @@ def test_chunked_partial_chunks_match_oracle(zero_init, chunk, flags):
     assert np.array_equal(hist, ref_hist_bits(inp, hist_ref))
 
 
-@pytest.mark.parametrize("chunk", [16, 32, 64, 128])
-def test_affine_path_runs_its_tensor_core_kernels(chunk):
-    """bf16 d=128 at chunk 16, 32, 64 and 128 runs the three kernels of the affine
-    chunked path (no token-recurrent kernel), so the chunk-size comparisons
-    below compare different chunkwise computations."""
+@pytest.mark.parametrize("chunk,flags,kernels", [
+    (16, 0, "wy"), (32, 0, "wy"), (128, 0, "wy"), (64, AFFINE, "wy"), (64, 0, "split"), (64, FACTORED, "split")])
+def test_chunked_paths_run_their_tensor_core_kernels(chunk, flags, kernels):
+    """bf16 d=128 runs a three-kernel tensor-core path at every chunk size (the
+    affine form at 16, 32, 128, the factored form by default at 64), never the
+    token-recurrent kernel, so the chunk-size comparisons compare different
+    chunkwise computations."""
     geo = gi.Geometry(num_k_heads=2, num_v_heads=6, head_k_dim=128, head_v_dim=128)
     inp = gi.make_prefill_inputs(geo, [100, 37], seed=34, zero_init=False)
     dp = DeviceProblem(inp, chunk)
     gdn.profiler_reset()
     gdn.profiler_enable(True)
-    dp.prefill()
+    dp.prefill(flags)
     torch.cuda.synchronize()
     gdn.profiler_enable(False)
     ran = {k for k in range(gdn.K.COUNT) if gdn.profiler_read(k)[0] > 0}
-    assert {gdn.K.WY_CONV, gdn.K.WY_PREP, gdn.K.WY_CHAIN} <= ran
-    assert gdn.K.PREFILL_RECURRENT not in ran and gdn.K.SPLIT_CHAIN not in ran
+    want = {gdn.K.WY_CONV, gdn.K.WY_PREP, gdn.K.WY_CHAIN} if kernels == "wy" else \
+        {gdn.K.SPLIT_CONV, gdn.K.SPLIT_PREP, gdn.K.SPLIT_CHAIN}
+    assert want <= ran
+    assert gdn.K.PREFILL_RECURRENT not in ran and gdn.K.PREFILL_CHUNKED not in ran
 
 
-@pytest.mark.parametrize("flags", [0, FACTORED, FUSED])
+def test_more_than_one_path_flag_is_rejected():
+    geo = gi.Geometry(num_k_heads=2, num_v_heads=6, head_k_dim=128, head_v_dim=128)
+    inp = gi.make_prefill_inputs(geo, [10], seed=35, zero_init=False)
+    dp = DeviceProblem(inp, 64)
+    with pytest.raises(gdn.GdnError) as e:
+        dp.prefill(AFFINE | FUSED)
+    assert e.value.name == "GDN_E_INVAL"
+
+
+@pytest.mark.parametrize("flags", [0, AFFINE, FUSED])
 def test_chunked_matches_recurrent_kernel(flags):
     geo = gi.Geometry(num_k_heads=4, num_v_heads=12, head_k_dim=128, head_v_dim=128)
     inp = gi.make_prefill_inputs(geo, [300, 64, 1, 517], seed=32, zero_init=False)

@@ -382,7 +382,10 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
   const uint32_t tbase = tslot;
   if (!mbar_wait(&mb_tma, 0, kWaitNs)) bad = true;
   if (sync_tc_any(bad)) {
-    if (tid == 0) set_status(status, kTimeoutPrep);
+    if (tid == 0) {
+      set_status(status, kTimeoutPrep);
+      bulk_wait<0>();  // no record image is still being read from shared memory
+    }
     if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
     return;
   }
@@ -419,10 +422,9 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
       fk[2 * i] = (b2.x + b3.x) * ek;
       fk[2 * i + 1] = (b2.y + b3.y) * ek;
     }
-    const uint4 pk = pack8h(fk);
-    *reinterpret_cast<uint4*>(sm + WP_KT + mnmaj_chunk(64, r, c8)) = pk;
-    *reinterpret_cast<uint4*>(rec + R::KT + mnmaj_chunk(64, r, c8)) = pk;
+    *reinterpret_cast<uint4*>(sm + WP_KT + mnmaj_chunk(64, r, c8)) = pack8h(fk);
   }
+  fence_async_smem();  // K~ is read by the bulk store below and by the M' products
   {
     const int r16 = 16 * (warp & 3) + (lane & 15);  // M = 64 layout: row r16 in lane (r16 % 16) + 32 (r16 / 16)
     float v[32];
@@ -454,7 +456,10 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
   if (!mbar_wait(&mb_mma, mma_phase, kWaitNs)) bad = true;
   mma_phase ^= 1;
   if (sync_tc_any(bad)) {  // also: the tiles are read; KQL and the Q halves of KQH are free
-    if (tid == 0) set_status(status, kTimeoutPrep);
+    if (tid == 0) {
+      set_status(status, kTimeoutPrep);
+      bulk_wait<0>();  // no record image is still being read from shared memory
+    }
     if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
     return;
   }
@@ -464,6 +469,8 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     const unsigned char* vl = vimg + ((int64_t)g * d.Hv + h) * kVImg<TILE> + TILE * 256;
     bulk_load(sm + WP_VLO, vl, 8192, &mb_vlo);
     bulk_load(sm + WP_VLO + 16384, vl + 8192, 8192, &mb_vlo);
+    bulk_store(rec + R::KT, sm + WP_KT, 16384);  // the K~ image goes to the record as it is
+    bulk_commit();
   }
 
   // A (rows 0..63 of M1) into the diagonal fp32 blocks and the two level images;
@@ -503,16 +510,18 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
           const bool same = (j / C) == (r / C);
           p[e] = (j <= r && same) ? __expf(gr - s_gam[j]) * v[8 * m + e] : 0.f;
         }
-        const uint4 pk = pack8h(p);
-        const uint32_t off = kmaj_chunk(64, r, 32 * hc + 8 * m);
-        *reinterpret_cast<uint4*>(sm + WP_P + off) = pk;
-        *reinterpret_cast<uint4*>(rec + R::P + off) = pk;
+        *reinterpret_cast<uint4*>(sm + WP_P + kmaj_chunk(64, r, 32 * hc + 8 * m)) = pack8h(p);
       }
     }
   }
   for (int i = tid; i < 8192 / 16; i += kPrepThreads)
     reinterpret_cast<uint4*>(sm + WP_T)[i] = make_uint4(0, 0, 0, 0);
+  fence_async_smem();
   __syncthreads();
+  if (tid == 0) {  // the P image goes to the record as it is
+    bulk_store(rec + R::P, sm + WP_P, 8192);
+    bulk_commit();
+  }
   // T = (I + A)^-1, level 0: the 16x16 diagonal blocks by forward substitution,
   // one column of one block per thread, in fp32, rounded to fp16 once
   if (tid < 64) {
@@ -596,7 +605,10 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     }
   }
   if (abort) {
-    if (tid == 0) set_status(status, kTimeoutPrep);
+    if (tid == 0) {
+      set_status(status, kTimeoutPrep);
+      bulk_wait<0>();  // no record image is still being read from shared memory
+    }
     if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
     return;
   }
@@ -656,7 +668,10 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
   }
   fence_async_smem();
   if (sync_tc_any(bad)) {
-    if (tid == 0) set_status(status, kTimeoutPrep);
+    if (tid == 0) {
+      set_status(status, kTimeoutPrep);
+      bulk_wait<0>();  // no record image is still being read from shared memory
+    }
     if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
     return;
   }
@@ -682,14 +697,14 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
   if (!mbar_wait(&mb_mma, mma_phase, kWaitNs)) bad = true;
   mma_phase ^= 1;
   fence_after();
-  {  // U -> the record as hi + lo images per value-channel half; Q' -> the record (K-major 64 x 128)
+  {  // U -> its record image (hi + lo per value-channel half) staged in KQH; Q' -> its image staged in V
     float v[32];
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       const int cb = 64 * hc + 32 * hh;  // value channels cb .. cb + 31, all in half hc
       tmem_ld32(tbase + lane_base + TP_BIG + cb, v);
       if (lane < 16) {
-        unsigned char* uh = rec + R::U + hc * 2 * R::UH;
+        unsigned char* uh = sm + WP_KQH + hc * 2 * R::UH;
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
           float hi[8], lo[8];
@@ -711,15 +726,24 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
           float q8[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) q8[e] = ok ? v[8 * m + e] : 0.f;
-          *reinterpret_cast<uint4*>(rec + R::Q + kmaj_chunk(TILE, r16, cb + 8 * m)) = pack8h(q8);
+          *reinterpret_cast<uint4*>(sm + WP_V + kmaj_chunk(TILE, r16, cb + 8 * m)) = pack8h(q8);
         }
       }
     }
   }
+  fence_async_smem();
   if (sync_tc_any(bad)) {  // also: columns 0..127 are read out
-    if (tid == 0) set_status(status, kTimeoutPrep);
+    if (tid == 0) {
+      set_status(status, kTimeoutPrep);
+      bulk_wait<0>();  // no record image is still being read from shared memory
+    }
     if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
     return;
+  }
+  if (tid == 0) {
+    bulk_store(rec + R::U, sm + WP_KQH, 4 * R::UH);
+    bulk_store(rec + R::Q, sm + WP_V, TILE * 256);
+    bulk_commit();
   }
   // M'_s = K~_s^T (-W_s) for each chunk s of the tile (M = N = 128, K = the chunk's rows)
   const int si = 32 * (warp & 3) + lane;
@@ -738,24 +762,33 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     }
     if (!mbar_wait(&mb_mma, mma_phase, kWaitNs)) bad = true;
     mma_phase ^= 1;
+    if (tid == 0) bulk_wait_read<0>();  // the staging area (KQH) has been read by the previous bulk store
+    __syncthreads();
     fence_after();
-    {
+    {  // M'_s -> its record image staged in KQH
       float v[32];
-      unsigned char* mrec = rec + R::M + s * 32768;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         tmem_ld32(tbase + lane_base + TP_BIG + 64 * hc + 32 * hh, v);
 #pragma unroll
         for (int m = 0; m < 4; ++m)
-          *reinterpret_cast<uint4*>(mrec + kmaj_chunk(128, si, 64 * hc + 32 * hh + 8 * m)) = pack8h(v + 8 * m);
+          *reinterpret_cast<uint4*>(sm + WP_KQH + kmaj_chunk(128, si, 64 * hc + 32 * hh + 8 * m)) = pack8h(v + 8 * m);
       }
     }
+    fence_async_smem();
     if (sync_tc_any(bad)) {
       abort = true;
       break;
     }
+    if (tid == 0) {
+      bulk_store(rec + R::M + s * 32768, sm + WP_KQH, 32768);
+      bulk_commit();
+    }
   }
-  if (abort && tid == 0) set_status(status, kTimeoutPrep);
+  if (tid == 0) {
+    if (abort) set_status(status, kTimeoutPrep);
+    bulk_wait<0>();  // every record image has left shared memory
+  }
   if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
 }
 
@@ -1241,12 +1274,12 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
 // carries value channels [64 vh, 64 vh + 64), i.e. 64 columns of the state,
 // which evolve independently of the other 64.  Per chunk c (chunk s of its
 // tile):
-//   Y_c = K~_s^T U_s                  (no state: issued a chunk ahead)
-//   Y_c += M'_c S_c                   (the one product on the carry's path)
-//   S_{c+1} = e^{gamma_C} S_c + Y_c   (fp32 registers; its fp16 copy is the next operand)
-//   O_c = P_s U_s + Q' S_c            (rows of chunk s; nothing waits for it)
+//   Y_c = K~_s^T U_s,  O_c = P_s U_s   (nothing from the state: issued a chunk ahead)
+//   Y_c += M'_c S_c                    (the one product on the carry's path)
+//   S_{c+1} = e^{gamma_C} S_c + Y_c    (fp32 registers; its fp16 copy is the next operand)
+//   O_c += Q' S_c                      (rows of chunk s; nothing waits for it)
 // then RMSNorm over all d_v (row sums exchanged with the peer CTA) times the
-// output gate (1 + w) sigmoid(z), bf16 out.
+// output gate, bf16 out.
 // Warps 0..7 carry the state (thread: key row 32 (w % 4) + lane, columns
 // 32 (w / 4) .. + 31 of this half); warps 8..11 write the output rows; warp 12
 // issues the MMAs and warp 13 the bulk copies.  Every wait is bounded.
@@ -1262,14 +1295,14 @@ struct ChainCfg {
   static constexpr int UB = KTB + NB * TILE * 256;              // U of this half: hi, lo MN-major K=TILE x N=64
   static constexpr int PB = UB + NB * TILE * 256;               // P K-major TILE x TILE
   static constexpr int MISC = PB + NB * TILE * TILE * 2;
-  static constexpr int MS_NW = 0;                 // (1 + w) of this half's 64 channels
-  static constexpr int MS_PEER = 256;             // the peer's row sums [2][TILE]
-  static constexpr int MS_META = MS_PEER + 2 * TILE * 4;  // e^{gamma_C} of each chunk, per tile buffer (64 floats)
-  static constexpr int MISC_BYTES = MS_META + NB * 256;
+  static constexpr int MS_PEER = 0;               // the peer's row sums [2][TILE]
+  static constexpr int MISC_BYTES = 2 * TILE * 4;
   static constexpr int SMEM = MISC + MISC_BYTES + 1024;
 };
 constexpr int kChainThreads = 448;
-constexpr uint32_t CY0 = 0, CO0 = 128, kChainTmemCols = 256;  // Y_c at CY0 + 64 (c % 2), O_c at CO0 + 64 (c % 2)
+// TMEM: Y_c in columns 64 (c % 2), O_c in 128 + 64 (c % 3)
+constexpr uint32_t CY0 = 0, CO0 = 128, kChainTmemCols = 512;
+constexpr int kOBufs = 3;
 
 template <int TILE, int C>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
@@ -1283,10 +1316,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
   constexpr int OM = TILE == 64 ? 64 : 128;  // M of the output products
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  __shared__ uint64_t mb_m[NM], mb_ta[NB], mb_tq[NB];  // copies: M', tile group (K~, U, P, meta), Q'
+  __shared__ uint64_t mb_m[NM], mb_ta[NB], mb_tq[NB];  // copies: M', tile operands (K~, U, P), Q'
   __shared__ uint64_t mb_s;                            // S_c is in shared memory (8 state warps)
-  __shared__ uint64_t mb_y[2], mb_o[2];                // commits: Y_c (+ all earlier MMAs), O_c
-  __shared__ uint64_t mb_e[2];                         // output warps done reading O_c (4 warps)
+  __shared__ uint64_t mb_ea[4];                        // commit of chunk c's state-free products, slot c % 4
+  __shared__ uint64_t mb_y[2];                         // commit of Y_c (and every earlier MMA), slot c % 2
+  __shared__ uint64_t mb_o[kOBufs];                    // commit of O_c (and every earlier MMA), slot c % 3
+  __shared__ uint64_t mb_e[kOBufs];                    // output warps done reading O_c (4 warps), slot c % 3
   __shared__ uint64_t mb_x[2];                         // the peer's row sums of chunk c arrived
   __shared__ uint32_t tslot;
   bool bad = false;
@@ -1315,27 +1350,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
       mbar_init(&mb_tq[i], 1);
     }
     mbar_init(&mb_s, 8);
+    for (int i = 0; i < 4; ++i) mbar_init(&mb_ea[i], 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&mb_y[i], 1);
+      mbar_init(&mb_x[i], 1);  // one local arrival with the expected bytes; the peer's stores complete them
+    }
+    for (int i = 0; i < kOBufs; ++i) {
       mbar_init(&mb_o[i], 1);
       mbar_init(&mb_e[i], 4);
-      mbar_init(&mb_x[i], 1);  // one local arrival with the expected bytes; the peer's stores complete them
     }
     mbar_init_fence();
   }
   if (warp == 0) tmem_alloc(&tslot, kChainTmemCols);
 
   auto rec_of = [&](int t) { return records + ((g0 + t) * d.Hv + h) * (int64_t)R::BYTES; };
-  auto issue_tile = [&](int t) {
+  auto issue_ops = [&](int t) {  // K~, U of this half, P
     const int b = t % NB;
     const unsigned char* r = rec_of(t);
-    mbar_expect_tx(&mb_ta[b], TILE * 256 + TILE * 256 + TILE * TILE * 2 + 256);
+    mbar_expect_tx(&mb_ta[b], TILE * 256 + TILE * 256 + TILE * TILE * 2);
     bulk_load(sm + F::KTB + b * TILE * 256, r + R::KT, TILE * 256, &mb_ta[b]);
     bulk_load(sm + F::UB + b * TILE * 256, r + R::U + vh * 2 * R::UH, 2 * R::UH, &mb_ta[b]);
     bulk_load(sm + F::PB + b * TILE * TILE * 2, r + R::P, TILE * TILE * 2, &mb_ta[b]);
-    bulk_load(sm + F::MISC + F::MS_META + b * 256, r + R::META, 256, &mb_ta[b]);
+  };
+  auto issue_q = [&](int t) {
+    const int b = t % NB;
     mbar_expect_tx(&mb_tq[b], TILE * 256);
-    bulk_load(sm + F::QB + b * TILE * 256, r + R::Q, TILE * 256, &mb_tq[b]);
+    bulk_load(sm + F::QB + b * TILE * 256, rec_of(t) + R::Q, TILE * 256, &mb_tq[b]);
   };
   auto issue_m = [&](int c) {
     const int b = c % NM;
@@ -1356,7 +1396,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
   const uint32_t tbase = tslot;
   // the first copies go out only after the block barrier that publishes the mbarriers' initialisation
   if (copy_warp && lane == 0) {
-    for (int t = 0; t < NB && t < ntiles; ++t) issue_tile(t);
+    for (int t = 0; t < NB && t < ntiles; ++t) {
+      issue_ops(t);
+      issue_q(t);
+    }
     for (int c = 0; c < NM && c < nsteps; ++c) issue_m(c);
   }
   cluster_sync();  // the peer's mbarriers are initialised before any arrival on them
@@ -1370,14 +1413,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
       const uint32_t id_y = idesc_f16(128, 64, true, true);    // K~^T U: A MN-major
       const uint32_t id_ys = idesc_f16(128, 64, false, true);  // M' S
       const uint32_t id_o = idesc_f16(OM, 64, false, true);    // P U, Q' S
-      // Y_c = K~_s^T U_s needs nothing from the state: it is issued a chunk ahead, right behind the
-      // output products of the chunk before, so that M'_c S_c finds its accumulator ready
-      auto y_early = [&](int c) {
+      // Y_c = K~_s^T U_s and O_c = P_s U_s need nothing from the state: they go out a chunk ahead, and
+      // their commit tells the copy warp when the tile's operand buffer is free again
+      auto early = [&](int c) {
         const int t = c / NCH, s = c % NCH, b = t % NB;
         if (s == 0 && !mbar_wait(&mb_ta[b], (t / NB) & 1, kWaitNs)) bad = true;
+        // the output buffer is free once the output warps have read chunk c-3
+        if (c >= kOBufs && !mbar_wait(&mb_e[c % kOBufs], ((c - kOBufs) / kOBufs) & 1, kWaitNs)) bad = true;
         if (bad) return;
-        const uint32_t kt = smem_u32(sm + F::KTB + b * TILE * 256), ub = smem_u32(sm + F::UB + b * TILE * 256);
-        const uint32_t y = tbase + CY0 + 64 * (c & 1);
+        const uint32_t kt = smem_u32(sm + F::KTB + b * TILE * 256), ub = smem_u32(sm + F::UB + b * TILE * 256),
+                       pb = smem_u32(sm + F::PB + b * TILE * TILE * 2);
+        const uint32_t y = tbase + CY0 + 64 * (c & 1), od = tbase + CO0 + 64 * (c % kOBufs);
 #pragma unroll
         for (int k = 0; k < C / 16; ++k) {
           const int st = s * (C / 16) + k;
@@ -1385,8 +1431,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
           mma_f16(y, sdesc(kt + st * 2048, TILE * 128, 1024), sdesc(ub + TILE * 128 + st * 2048, TILE * 128, 1024),
                   id_y, 1);
         }
+#pragma unroll
+        for (int k = 0; k < C / 16; ++k) {
+          const int st = s * (C / 16) + k;
+          mma_f16(od, desc_kmaj(pb, TILE, st), sdesc(ub + st * 2048, TILE * 128, 1024), id_o, k > 0);
+          mma_f16(od, desc_kmaj(pb, TILE, st), sdesc(ub + TILE * 128 + st * 2048, TILE * 128, 1024), id_o, 1);
+        }
+        mma_commit(&mb_ea[c & 3]);
       };
-      y_early(0);
+      early(0);
       for (int c = 0; c < nsteps && !bad; ++c) {
         const int t = c / NCH, s = c % NCH, b = t % NB;
         if (!mbar_wait(&mb_m[c % NM], (c / NM) & 1, kWaitNs)) bad = true;
@@ -1396,47 +1449,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
         if (bad) break;
         const uint32_t ma = smem_u32(sm + F::MB + (c % NM) * 32768), sb = smem_u32(sm + F::SB + (c & 1) * 16384);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mma_f16(tbase + CY0 + 64 * (c & 1), desc_kmaj(ma, 128, k), desc_mnmaj(sb, kD, k), id_ys, 1);
+        for (int k = 0; k < 8; ++k)
+          mma_f16(tbase + CY0 + 64 * (c & 1), desc_kmaj(ma, 128, k), desc_mnmaj(sb, kD, k), id_ys, 1);
         mma_commit(&mb_y[c & 1]);
-        // O_c = P_s U_s + Q' S_c, into the output buffer the output warps released after chunk c-2
-        if (c >= 2 && !mbar_wait(&mb_e[c & 1], ((c - 2) >> 1) & 1, kWaitNs)) bad = true;
         if (s == 0 && !mbar_wait(&mb_tq[b], (t / NB) & 1, kWaitNs)) bad = true;
         if (bad) break;
-        const uint32_t ub = smem_u32(sm + F::UB + b * TILE * 256), pb = smem_u32(sm + F::PB + b * TILE * TILE * 2),
-                       qb = smem_u32(sm + F::QB + b * TILE * 256), od = tbase + CO0 + 64 * (c & 1);
-#pragma unroll
-        for (int k = 0; k < C / 16; ++k) {
-          const int st = s * (C / 16) + k;
-          mma_f16(od, desc_kmaj(pb, TILE, st), sdesc(ub + st * 2048, TILE * 128, 1024), id_o, k > 0);
-          mma_f16(od, desc_kmaj(pb, TILE, st), sdesc(ub + TILE * 128 + st * 2048, TILE * 128, 1024), id_o, 1);
-        }
+        const uint32_t qb = smem_u32(sm + F::QB + b * TILE * 256), od = tbase + CO0 + 64 * (c % kOBufs);
 #pragma unroll
         for (int k = 0; k < 8; ++k) mma_f16(od, desc_kmaj(qb, TILE, k), desc_mnmaj(sb, kD, k), id_o, 1);
-        mma_commit(&mb_o[c & 1]);
-        if (c + 1 < nsteps) y_early(c + 1);
+        mma_commit(&mb_o[c % kOBufs]);
+        if (c + 1 < nsteps) early(c + 1);
       }
     }
   } else if (copy_warp) {
     if (lane == 0) {
       for (int c = 0; c < nsteps && !bad; ++c) {
-        // buffers of chunk c are free once its products are done (the commit of O_c covers every earlier MMA)
+        const int t = c / NCH;
+        const bool tile_end = c % NCH == NCH - 1 || c == nsteps - 1;
+        // the tile's K~, U, P are free once the state-free products of its last chunk are done
+        if (!mbar_wait(&mb_ea[c & 3], (c >> 2) & 1, kWaitNs)) bad = true;
+        if (bad) break;
+        if (tile_end && t + NB < ntiles) issue_ops(t + NB);
+        // M'_c and the tile's Q' are free once O_c is done (its commit covers every earlier MMA)
         if (!mbar_wait(&mb_y[c & 1], (c >> 1) & 1, kWaitNs)) bad = true;
-        if (!mbar_wait(&mb_o[c & 1], (c >> 1) & 1, kWaitNs)) bad = true;
+        if (!mbar_wait(&mb_o[c % kOBufs], (c / kOBufs) & 1, kWaitNs)) bad = true;
         if (bad) break;
         if (c + NM < nsteps) issue_m(c + NM);
-        const int t = c / NCH;
-        if ((c % NCH == NCH - 1 || c == nsteps - 1) && t + NB < ntiles) issue_tile(t + NB);
+        if (tile_end && t + NB < ntiles) issue_q(t + NB);
       }
     }
   } else if (state_warp) {
-    // e^{gamma_C} of chunk c is read before S_c is published, i.e. before the
-    // products of chunk c can complete and free the tile buffer that holds it
+    // e^{gamma_C} of chunk c, read from the record two chunks ahead (it is not on the tile buffers' path)
     auto eg_of = [&](int c) {
-      const int t = c / NCH, b = t % NB;
-      if (c % NCH == 0 && !mbar_wait(&mb_ta[b], (t / NB) & 1, kWaitNs)) bad = true;
-      return reinterpret_cast<const float*>(sm + F::MISC + F::MS_META + b * 256)[c % NCH];
+      return c < nsteps ? __ldg(reinterpret_cast<const float*>(rec_of(c / NCH) + R::META) + c % NCH) : 0.f;
     };
-    float egC = eg_of(0);
+    float egA = eg_of(0), egB = eg_of(1);
     for (int c = 0; c < nsteps; ++c) {
       if (!mbar_wait(&mb_y[c & 1], (c >> 1) & 1, kWaitNs)) bad = true;
       tc::fence_after();
@@ -1444,9 +1491,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
       float y[32];
       tmem_ld32(tbase + lane_base + CY0 + 64 * (c & 1) + 32 * hc, y);
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) S[jj] = egC * S[jj] + y[jj];
+      for (int jj = 0; jj < 32; ++jj) S[jj] = egA * S[jj] + y[jj];
       if (c + 1 < nsteps) {
-        egC = eg_of(c + 1);
 #pragma unroll
         for (int m = 0; m < 4; ++m)
           st16h(sm + F::SB + ((c + 1) & 1) * 16384 + mnmaj_chunk(kD, si, 32 * hc + 8 * m), S + 8 * m);
@@ -1455,6 +1501,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&mb_s);
       }
+      egA = egB;
+      egB = eg_of(c + 2);
     }
   } else if (out_warp) {
     const int q = warp - 8;
@@ -1484,10 +1532,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
       const bool mine = has_row && (r / C) == s;
       const int64_t tok = seq0 + (int64_t)t * TILE + r;
       const bool valid = mine && (t * TILE + r) < len;
-      if (!mbar_wait(&mb_o[c & 1], (c >> 1) & 1, kWaitNs)) bad = true;
+      if (!mbar_wait(&mb_o[c % kOBufs], (c / kOBufs) & 1, kWaitNs)) bad = true;
       tc::fence_after();
       float v[32], ss = 0.f;
-      const uint32_t ob = tbase + lane_base + CO0 + 64 * (c & 1);
+      const uint32_t ob = tbase + lane_base + CO0 + 64 * (c % kOBufs);
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         tmem_ld32(ob + 32 * hh, v);  // warp-collective: every lane takes part
@@ -1502,10 +1550,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         tmem_ld32(ob + 32 * hh, v);
-        if (hh == 1) {  // the products of chunk c are read: the buffer takes chunk c+2's
+        if (hh == 1) {  // the products of chunk c are read: the buffer takes chunk c+3's
           tc::fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&mb_e[c & 1]);
+          if (lane == 0) mbar_arrive(&mb_e[c % kOBufs]);
         }
         if (valid) {
 #pragma unroll

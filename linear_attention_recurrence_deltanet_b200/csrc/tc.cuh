@@ -180,6 +180,25 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                : "memory");
 }
 
+// 1D bulk copy shared -> global (both 16-byte aligned, size a multiple of 16)
+// in the issuing thread's bulk async-group; bulk_commit closes the group,
+// bulk_wait_read<N> waits until at most N groups still read shared memory and
+// bulk_wait<N> until at most N groups are incomplete.
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"((uint64_t)dst),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+template <int N>
+__device__ __forceinline__ void bulk_wait() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // 16-byte asynchronous copy global -> shared through the load/store path (L2
 // only); src_bytes = 0 fills the 16 bytes with zeros and reads nothing
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {

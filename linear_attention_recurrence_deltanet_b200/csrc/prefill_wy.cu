@@ -1282,7 +1282,10 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
 // output gate, bf16 out.
 // Warps 0..7 carry the state (thread: key row 32 (w % 4) + lane, columns
 // 32 (w / 4) .. + 31 of this half); warps 8..11 write the output rows; warp 12
-// issues the MMAs and warp 13 the bulk copies.  Every wait is bounded.
+// issues the products with the state (Y += M'S, O += Q'S), warp 14 the
+// state-free ones (issuing a tcgen05.mma takes its thread tens of cycles, so
+// the two streams of MMAs go out in parallel), warp 13 the bulk copies.
+// Every wait is bounded.
 template <int TILE, int C>
 struct ChainCfg {
   static constexpr int NCH = TILE / C;
@@ -1299,7 +1302,8 @@ struct ChainCfg {
   static constexpr int MISC_BYTES = 2 * TILE * 4;
   static constexpr int SMEM = MISC + MISC_BYTES + 1024;
 };
-constexpr int kChainThreads = 448;
+constexpr int kChainThreads = 480;
+constexpr int kEaSlots = 8;  // commits of the state-free products, slot c % 8
 // TMEM: Y_c in columns 64 (c % 2), O_c in 128 + 64 (c % 3)
 constexpr uint32_t CY0 = 0, CO0 = 128, kChainTmemCols = 512;
 constexpr int kOBufs = 3;
@@ -1318,7 +1322,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
   unsigned char* sm = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   __shared__ uint64_t mb_m[NM], mb_ta[NB], mb_tq[NB];  // copies: M', tile operands (K~, U, P), Q'
   __shared__ uint64_t mb_s;                            // S_c is in shared memory (8 state warps)
-  __shared__ uint64_t mb_ea[4];                        // commit of chunk c's state-free products, slot c % 4
+  __shared__ uint64_t mb_ea[kEaSlots];                 // commit of chunk c's state-free products (warp 14)
+  __shared__ uint64_t mb_yf[2];                        // the state warps have read Y_c, slot c % 2 (8 warps)
   __shared__ uint64_t mb_y[2];                         // commit of Y_c (and every earlier MMA), slot c % 2
   __shared__ uint64_t mb_o[kOBufs];                    // commit of O_c (and every earlier MMA), slot c % 3
   __shared__ uint64_t mb_e[kOBufs];                    // output warps done reading O_c (4 warps), slot c % 3
@@ -1339,7 +1344,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
   const int64_t g0 = tile_off ? tile_off[n] : 0;
   const int64_t HvD = (int64_t)d.Hv * kD;
   const bool state_warp = warp < 8, out_warp = warp >= 8 && warp < 12, mma_warp = warp == 12,
-             copy_warp = warp == 13;
+             copy_warp = warp == 13, early_warp = warp == 14;
   float* s_peer = reinterpret_cast<float*>(sm + F::MISC + F::MS_PEER);
   float* gst = state + ((int64_t)n * d.Hv + h) * kD * kD;  // stored [j][i]
 
@@ -1350,7 +1355,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
       mbar_init(&mb_tq[i], 1);
     }
     mbar_init(&mb_s, 8);
-    for (int i = 0; i < 4; ++i) mbar_init(&mb_ea[i], 1);
+    for (int i = 0; i < kEaSlots; ++i) mbar_init(&mb_ea[i], 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&mb_yf[i], 8);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&mb_y[i], 1);
       mbar_init(&mb_x[i], 1);  // one local arrival with the expected bytes; the peer's stores complete them
@@ -1408,19 +1414,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
   const uint32_t peer_sums = mapa_shared(smem_u32(s_peer), peer);
   const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
 
-  if (mma_warp) {
+  if (early_warp) {
     if (lane == 0) {
-      const uint32_t id_y = idesc_f16(128, 64, true, true);    // K~^T U: A MN-major
-      const uint32_t id_ys = idesc_f16(128, 64, false, true);  // M' S
-      const uint32_t id_o = idesc_f16(OM, 64, false, true);    // P U, Q' S
-      // Y_c = K~_s^T U_s and O_c = P_s U_s need nothing from the state: they go out a chunk ahead, and
-      // their commit tells the copy warp when the tile's operand buffer is free again
-      auto early = [&](int c) {
+      const uint32_t id_y = idesc_f16(128, 64, true, true);  // K~^T U: A MN-major
+      const uint32_t id_o = idesc_f16(OM, 64, false, true);  // P U
+      // Y_c = K~_s^T U_s and O_c = P_s U_s need nothing from the state: they go out ahead of the carry, and
+      // their commit tells warp 12 that Y_c and O_c may take the state's products, and the copy warp when
+      // the tile's operand buffer is free again
+      for (int c = 0; c < nsteps && !bad; ++c) {
         const int t = c / NCH, s = c % NCH, b = t % NB;
         if (s == 0 && !mbar_wait(&mb_ta[b], (t / NB) & 1, kWaitNs)) bad = true;
-        // the output buffer is free once the output warps have read chunk c-3
+        // Y buffer c % 2 is free once the state warps have read Y_{c-2}; O buffer c % 3 once the output
+        // warps have read O_{c-3}
+        if (c >= 2 && !mbar_wait(&mb_yf[c & 1], ((c - 2) >> 1) & 1, kWaitNs)) bad = true;
         if (c >= kOBufs && !mbar_wait(&mb_e[c % kOBufs], ((c - kOBufs) / kOBufs) & 1, kWaitNs)) bad = true;
-        if (bad) return;
+        tc::fence_after();
+        if (bad) break;
         const uint32_t kt = smem_u32(sm + F::KTB + b * TILE * 256), ub = smem_u32(sm + F::UB + b * TILE * 256),
                        pb = smem_u32(sm + F::PB + b * TILE * TILE * 2);
         const uint32_t y = tbase + CY0 + 64 * (c & 1), od = tbase + CO0 + 64 * (c % kOBufs);
@@ -1437,14 +1446,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
           mma_f16(od, desc_kmaj(pb, TILE, st), sdesc(ub + st * 2048, TILE * 128, 1024), id_o, k > 0);
           mma_f16(od, desc_kmaj(pb, TILE, st), sdesc(ub + TILE * 128 + st * 2048, TILE * 128, 1024), id_o, 1);
         }
-        mma_commit(&mb_ea[c & 3]);
-      };
-      early(0);
+        mma_commit(&mb_ea[c % kEaSlots]);
+      }
+    }
+  } else if (mma_warp) {
+    if (lane == 0) {
+      const uint32_t id_ys = idesc_f16(128, 64, false, true);  // M' S
+      const uint32_t id_o = idesc_f16(OM, 64, false, true);    // Q' S
       for (int c = 0; c < nsteps && !bad; ++c) {
         const int t = c / NCH, s = c % NCH, b = t % NB;
         if (!mbar_wait(&mb_m[c % NM], (c / NM) & 1, kWaitNs)) bad = true;
         // S_c in shared memory (S_0 was written before the block barrier; S_c, c >= 1, completes phase c - 1)
         if (c > 0 && !mbar_wait(&mb_s, (c - 1) & 1, kWaitNs)) bad = true;
+        // the state-free parts of Y_c and O_c are in place (issued by warp 14)
+        if (!mbar_wait(&mb_ea[c % kEaSlots], (c / kEaSlots) & 1, kWaitNs)) bad = true;
         tc::fence_after();
         if (bad) break;
         const uint32_t ma = smem_u32(sm + F::MB + (c % NM) * 32768), sb = smem_u32(sm + F::SB + (c & 1) * 16384);
@@ -1458,7 +1473,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
 #pragma unroll
         for (int k = 0; k < 8; ++k) mma_f16(od, desc_kmaj(qb, TILE, k), desc_mnmaj(sb, kD, k), id_o, 1);
         mma_commit(&mb_o[c % kOBufs]);
-        if (c + 1 < nsteps) early(c + 1);
       }
     }
   } else if (copy_warp) {
@@ -1467,7 +1481,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
         const int t = c / NCH;
         const bool tile_end = c % NCH == NCH - 1 || c == nsteps - 1;
         // the tile's K~, U, P are free once the state-free products of its last chunk are done
-        if (!mbar_wait(&mb_ea[c & 3], (c >> 2) & 1, kWaitNs)) bad = true;
+        if (!mbar_wait(&mb_ea[c % kEaSlots], (c / kEaSlots) & 1, kWaitNs)) bad = true;
         if (bad) break;
         if (tile_end && t + NB < ntiles) issue_ops(t + NB);
         // M'_c and the tile's Q' are free once O_c is done (its commit covers every earlier MMA)
@@ -1490,6 +1504,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
       if (bad) break;
       float y[32];
       tmem_ld32(tbase + lane_base + CY0 + 64 * (c & 1) + 32 * hc, y);
+      tc::fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&mb_yf[c & 1]);  // Y buffer c % 2 may take Y_{c+2}'s state-free part
 #pragma unroll
       for (int jj = 0; jj < 32; ++jj) S[jj] = egA * S[jj] + y[jj];
       if (c + 1 < nsteps) {

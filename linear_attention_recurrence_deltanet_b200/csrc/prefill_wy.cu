@@ -246,7 +246,7 @@ __device__ __forceinline__ void write_history(const Dims& d, int h, int n, int64
 }
 
 // ------------------------------------------------------------------ wy_prep_kernel (64-row tiles)
-// One block per (tile, value head), two blocks per SM (99 KB shared memory,
+// One block per (tile, value head), two blocks per SM (111 KB shared memory,
 // 256 TMEM columns).  Shared memory:
 //   KQH  [K;Q] hi, K-major 128 x 128 (K rows 0..63, Q rows 64..127).  Its K
 //        halves, read as MN-major K=64 x N=128 (LBO 16 KB), are the B operand
@@ -260,6 +260,7 @@ __device__ __forceinline__ void write_history(const Dims& d, int h, int n, int64
 //   V    v^ hi, MN-major K=64 x N=128 (LBO 8 KB).
 //   KT   K~, MN-major K=64 x M=128 (LBO 8 KB).
 //   PS   P, K-major 64 x 64.
+//   TF   the 16x16 diagonal blocks of T in fp32 (T' and T'' take them from here).
 // TMEM (256 columns): [K;Q]K^T in 0..63, the solve's products in 64..127,
 // diag(e^gamma) Q and then Q' in 128..255 (M = 64 layout), W, U and M' in turn
 // in 0..127.
@@ -283,7 +284,8 @@ constexpr int WP_TPH = WP_KQL;
 constexpr int WP_TPL = WP_KQL + 8192;
 constexpr int WP_TPP = WP_KQL + 24576;
 constexpr int WP_NW = WP_KQL + 16384;
-constexpr int kPrepSmem = WP_MISC + 7 * 64 * 4 + 1024;
+constexpr int WP_TF = WP_MISC + 7 * 64 * 4;  // the 16x16 diagonal blocks of T in fp32 (4 KB)
+constexpr int kPrepSmem = WP_TF + 4096 + 1024;
 constexpr uint32_t kPrepTmemCols = 256;
 constexpr uint32_t TP_M1 = 0, TP_SOLVE = 64, TP_Q = 128, TP_BIG = 0;
 
@@ -523,10 +525,12 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     bulk_commit();
   }
   // T = (I + A)^-1, level 0: the 16x16 diagonal blocks by forward substitution,
-  // one column of one block per thread, in fp32, rounded to fp16 once
+  // one column of one block per thread, in fp32: kept in fp32 for T' and T''
+  // (the doubling levels never change these blocks) and as fp16 in the T image
   if (tid < 64) {
     const int bb = tid >> 4, c = tid & 15, o = 16 * bb;
     const float* Ad = reinterpret_cast<const float*>(sm + WP_DIAG) + bb * 272;
+    float* Tf = reinterpret_cast<float*>(sm + WP_TF) + bb * 256;
     float t[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -536,8 +540,10 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
       t[i] = (i < c) ? 0.f : acc;
     }
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
+    for (int i = 0; i < 16; ++i) {
       *reinterpret_cast<__half*>(sm + WP_T + kmaj(64, o + i, o + c)) = __float2half_rn(t[i]);
+      Tf[i * 16 + c] = t[i];
+    }
   }
   fence_async_smem();
   sync_tc();
@@ -612,22 +618,34 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
     return;
   }
-  {  // T' = T diag(beta) as fp16 hi + lo, T'' = T diag(beta e^gamma), K-major 64 x 64
+  {  // T' = T diag(beta) as fp16 hi + lo, T'' = T diag(beta e^gamma), K-major 64 x 64; a thread's 16
+     // columns are one 16-column block: the diagonal one comes from the fp32 blocks
     const int r = tid >> 2, j0 = 16 * (tid & 3);
-    float t1[16], t2[16], tl[16];
+    float t1[16], t2[16], tl[16], tv[16];
+    if ((tid & 3) == (r >> 4)) {
+      const float4* tf = reinterpret_cast<const float4*>(sm + WP_TF) + (r >> 4) * 64 + (r & 15) * 4;
 #pragma unroll
-    for (int m = 0; m < 2; ++m) {
-      const uint4 tq = *reinterpret_cast<const uint4*>(sm + WP_T + kmaj_chunk(64, r, j0 + 8 * m));
-      const __half2* h2 = reinterpret_cast<const __half2*>(&tq);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f = __half22float2(h2[i]);
-        const int j = j0 + 8 * m + 2 * i;
-        t1[8 * m + 2 * i] = f.x * s_beta[j];
-        t1[8 * m + 2 * i + 1] = f.y * s_beta[j + 1];
-        t2[8 * m + 2 * i] = f.x * s_tbg[j];
-        t2[8 * m + 2 * i + 1] = f.y * s_tbg[j + 1];
+      for (int m = 0; m < 4; ++m) {
+        const float4 f = tf[m];
+        tv[4 * m] = f.x; tv[4 * m + 1] = f.y; tv[4 * m + 2] = f.z; tv[4 * m + 3] = f.w;
       }
+    } else {
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const uint4 tq = *reinterpret_cast<const uint4*>(sm + WP_T + kmaj_chunk(64, r, j0 + 8 * m));
+        const __half2* h2 = reinterpret_cast<const __half2*>(&tq);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __half22float2(h2[i]);
+          tv[8 * m + 2 * i] = f.x;
+          tv[8 * m + 2 * i + 1] = f.y;
+        }
+      }
+    }
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) {
+      t1[jj] = tv[jj] * s_beta[j0 + jj];
+      t2[jj] = tv[jj] * s_tbg[j0 + jj];
     }
 #pragma unroll
     for (int i = 0; i < 16; ++i) tl[i] = t1[i] - __half2float(__float2half_rn(t1[i]));
@@ -793,7 +811,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
 }
 
 // ------------------------------------------------------------------ wy_prep128_kernel (chunk 128)
-// One block per (128-row tile, value head); one block per SM (197 KB shared
+// One block per (128-row tile, value head); one block per SM (205 KB shared
 // memory, all 512 TMEM columns).  The same steps as the 64-row kernel on
 // 128 x 128 matrices, with one more doubling level (b = 64).  Shared memory:
 //   KH   k^ hi, K-major 128 x 128 (rows = tokens); read as MN-major (LBO 16 KB)
@@ -809,7 +827,8 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
 // products then M' in 256..383, diag(e^gamma) Q then Q' in 384..511.
 constexpr int W8_KH = 0, W8_KL = 32768, W8_QH = 65536, W8_QL = 98304, W8_X = 131072, W8_KT = 163840,
               W8_MISC = 196608;
-constexpr int kPrep128Smem = W8_MISC + 7 * 128 * 4 + 1024;
+constexpr int W8_TF = W8_MISC + 7 * 128 * 4;  // the 16x16 diagonal blocks of T in fp32 (8 KB)
+constexpr int kPrep128Smem = W8_TF + 8192 + 1024;
 constexpr uint32_t T8_KK = 0, T8_QK = 128, T8_SOLVE = 256, T8_Q = 384;
 
 __global__ void __launch_bounds__(kPrepThreads, 1)
@@ -1026,9 +1045,12 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       for (int k = 0; k < i; ++k) acc -= Ad[i * 16 + k] * t[k];
       t[i] = (i < c) ? 0.f : acc;
     }
+    float* Tf = reinterpret_cast<float*>(sm + W8_TF) + bb * 256;  // kept in fp32 for T' and T''
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
+    for (int i = 0; i < 16; ++i) {
       *reinterpret_cast<__half*>(sm + W8_KL + kmaj(128, o + i, o + c)) = __float2half_rn(t[i]);
+      Tf[i * 16 + c] = t[i];
+    }
   }
   fence_async_smem();
   sync_tc();
@@ -1120,17 +1142,26 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
 #pragma unroll 1
     for (int q = 0; q < 8; ++q) {
       const int jb = j0 + 8 * q;
-      const uint4 tq = *reinterpret_cast<const uint4*>(sm + W8_KL + kmaj_chunk(128, r, jb));
-      const __half2* h2 = reinterpret_cast<const __half2*>(&tq);
-      float t1[8], t2[8], tl[8];
+      float tv[8], t1[8], t2[8], tl[8];
+      if ((jb >> 4) == (r >> 4)) {  // the diagonal 16x16 block: its fp32 values (the levels never change it)
+        const float4* tf = reinterpret_cast<const float4*>(sm + W8_TF) + (r >> 4) * 64 + (r & 15) * 4 + ((jb & 15) >> 2);
+        const float4 f0 = tf[0], f1 = tf[1];
+        tv[0] = f0.x; tv[1] = f0.y; tv[2] = f0.z; tv[3] = f0.w;
+        tv[4] = f1.x; tv[5] = f1.y; tv[6] = f1.z; tv[7] = f1.w;
+      } else {
+        const uint4 tq = *reinterpret_cast<const uint4*>(sm + W8_KL + kmaj_chunk(128, r, jb));
+        const __half2* h2 = reinterpret_cast<const __half2*>(&tq);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f = __half22float2(h2[i]);
-        const int j = jb + 2 * i;
-        t1[2 * i] = f.x * s_beta[j];
-        t1[2 * i + 1] = f.y * s_beta[j + 1];
-        t2[2 * i] = f.x * s_tbg[j];
-        t2[2 * i + 1] = f.y * s_tbg[j + 1];
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __half22float2(h2[i]);
+          tv[2 * i] = f.x;
+          tv[2 * i + 1] = f.y;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        t1[i] = tv[i] * s_beta[jb + i];
+        t2[i] = tv[i] * s_tbg[jb + i];
       }
 #pragma unroll
       for (int i = 0; i < 8; ++i) tl[i] = t1[i] - __half2float(__float2half_rn(t1[i]));
@@ -1279,7 +1310,10 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
 //   S_{c+1} = e^{gamma_C} S_c + Y_c    (fp32 registers; its fp16 copy is the next operand)
 //   O_c += Q' S_c                      (rows of chunk s; nothing waits for it)
 // then RMSNorm over all d_v (row sums exchanged with the peer CTA) times the
-// output gate, bf16 out.
+// output gate, bf16 out.  The output products carry the state as fp16 hi + lo
+// parts (Q'S loses up to half of o's digits to cancellation when q is nearly
+// orthogonal to the state's columns): B = [S hi | S lo] and [U hi | U lo] as
+// N = 128 operands, the two column blocks of O summed by the output warps.
 // Warps 0..7 carry the state (thread: key row 32 (w % 4) + lane, columns
 // 32 (w / 4) .. + 31 of this half); warps 8..11 write the output rows; warp 12
 // issues the products with the state (Y += M'S, O += Q'S), warp 14 the
@@ -1290,11 +1324,11 @@ template <int TILE, int C>
 struct ChainCfg {
   static constexpr int NCH = TILE / C;
   static constexpr int NM = TILE == 64 ? 2 : 1;    // M' buffers
-  static constexpr int NB = TILE == 64 ? 2 : 1;    // tile operand buffers
+  static constexpr int NB = TILE == 64 ? 2 : 1;    // K~, U, P buffers (Q' has one)
   static constexpr int MB = 0;                                  // M' K-major 128 x 128, 32 KB each
-  static constexpr int SB = MB + NM * 32768;                    // S fp16 copies (2), MN-major K=128 x N=64
-  static constexpr int QB = SB + 2 * 16384;                     // Q' K-major TILE x 128
-  static constexpr int KTB = QB + NB * TILE * 256;              // K~ MN-major K=TILE x M=128
+  static constexpr int SB = MB + NM * 32768;                    // S copies (2): hi, lo MN-major K=128 x N=64
+  static constexpr int QB = SB + 2 * 32768;                     // Q' K-major TILE x 128
+  static constexpr int KTB = QB + TILE * 256;                   // K~ MN-major K=TILE x M=128
   static constexpr int UB = KTB + NB * TILE * 256;              // U of this half: hi, lo MN-major K=TILE x N=64
   static constexpr int PB = UB + NB * TILE * 256;               // P K-major TILE x TILE
   static constexpr int MISC = PB + NB * TILE * TILE * 2;
@@ -1304,7 +1338,7 @@ struct ChainCfg {
 };
 constexpr int kChainThreads = 480;
 constexpr int kEaSlots = 8;  // commits of the state-free products, slot c % 8
-// TMEM: Y_c in columns 64 (c % 2), O_c in 128 + 64 (c % 3)
+// TMEM: Y_c in columns 64 (c % 2), O_c in 128 + 128 (c % 3) (the hi and lo column blocks)
 constexpr uint32_t CY0 = 0, CO0 = 128, kChainTmemCols = 512;
 constexpr int kOBufs = 3;
 
@@ -1320,7 +1354,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
   constexpr int OM = TILE == 64 ? 64 : 128;  // M of the output products
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  __shared__ uint64_t mb_m[NM], mb_ta[NB], mb_tq[NB];  // copies: M', tile operands (K~, U, P), Q'
+  __shared__ uint64_t mb_m[NM], mb_ta[NB], mb_tq;      // copies: M', tile operands (K~, U, P), Q'
   __shared__ uint64_t mb_s;                            // S_c is in shared memory (8 state warps)
   __shared__ uint64_t mb_ea[kEaSlots];                 // commit of chunk c's state-free products (warp 14)
   __shared__ uint64_t mb_yf[2];                        // the state warps have read Y_c, slot c % 2 (8 warps)
@@ -1352,8 +1386,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
     for (int i = 0; i < NM; ++i) mbar_init(&mb_m[i], 1);
     for (int i = 0; i < NB; ++i) {
       mbar_init(&mb_ta[i], 1);
-      mbar_init(&mb_tq[i], 1);
+
     }
+    mbar_init(&mb_tq, 1);
     mbar_init(&mb_s, 8);
     for (int i = 0; i < kEaSlots; ++i) mbar_init(&mb_ea[i], 1);
     for (int i = 0; i < 2; ++i) mbar_init(&mb_yf[i], 8);
@@ -1379,9 +1414,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
     bulk_load(sm + F::PB + b * TILE * TILE * 2, r + R::P, TILE * TILE * 2, &mb_ta[b]);
   };
   auto issue_q = [&](int t) {
-    const int b = t % NB;
-    mbar_expect_tx(&mb_tq[b], TILE * 256);
-    bulk_load(sm + F::QB + b * TILE * 256, rec_of(t) + R::Q, TILE * 256, &mb_tq[b]);
+    mbar_expect_tx(&mb_tq, TILE * 256);
+    bulk_load(sm + F::QB, rec_of(t) + R::Q, TILE * 256, &mb_tq);
   };
   auto issue_m = [&](int c) {
     const int b = c % NM;
@@ -1395,17 +1429,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
 #pragma unroll
     for (int jj = 0; jj < 32; ++jj) S[jj] = zero_state ? 0.f : gst[(int64_t)(c0 + jj) * kD + si];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) st16h(sm + F::SB + mnmaj_chunk(kD, si, 32 * hc + 8 * m), S + 8 * m);
+    for (int m = 0; m < 4; ++m) {
+      float lo[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) lo[e] = S[8 * m + e] - __half2float(__float2half_rn(S[8 * m + e]));
+      st16h(sm + F::SB + mnmaj_chunk(kD, si, 32 * hc + 8 * m), S + 8 * m);
+      st16h(sm + F::SB + 16384 + mnmaj_chunk(kD, si, 32 * hc + 8 * m), lo);
+    }
   }
   fence_async_smem();
   sync_tc();
   const uint32_t tbase = tslot;
   // the first copies go out only after the block barrier that publishes the mbarriers' initialisation
   if (copy_warp && lane == 0) {
-    for (int t = 0; t < NB && t < ntiles; ++t) {
-      issue_ops(t);
-      issue_q(t);
-    }
+    for (int t = 0; t < NB && t < ntiles; ++t) issue_ops(t);
+    issue_q(0);
     for (int c = 0; c < NM && c < nsteps; ++c) issue_m(c);
   }
   cluster_sync();  // the peer's mbarriers are initialised before any arrival on them
@@ -1417,7 +1455,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
   if (early_warp) {
     if (lane == 0) {
       const uint32_t id_y = idesc_f16(128, 64, true, true);  // K~^T U: A MN-major
-      const uint32_t id_o = idesc_f16(OM, 64, false, true);  // P U
+      const uint32_t id_o = idesc_f16(OM, 128, false, true);  // P [U hi | U lo]
       // Y_c = K~_s^T U_s and O_c = P_s U_s need nothing from the state: they go out ahead of the carry, and
       // their commit tells warp 12 that Y_c and O_c may take the state's products, and the copy warp when
       // the tile's operand buffer is free again
@@ -1432,7 +1470,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
         if (bad) break;
         const uint32_t kt = smem_u32(sm + F::KTB + b * TILE * 256), ub = smem_u32(sm + F::UB + b * TILE * 256),
                        pb = smem_u32(sm + F::PB + b * TILE * TILE * 2);
-        const uint32_t y = tbase + CY0 + 64 * (c & 1), od = tbase + CO0 + 64 * (c % kOBufs);
+        const uint32_t y = tbase + CY0 + 64 * (c & 1), od = tbase + CO0 + 128 * (c % kOBufs);
 #pragma unroll
         for (int k = 0; k < C / 16; ++k) {
           const int st = s * (C / 16) + k;
@@ -1444,7 +1482,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
         for (int k = 0; k < C / 16; ++k) {
           const int st = s * (C / 16) + k;
           mma_f16(od, desc_kmaj(pb, TILE, st), sdesc(ub + st * 2048, TILE * 128, 1024), id_o, k > 0);
-          mma_f16(od, desc_kmaj(pb, TILE, st), sdesc(ub + TILE * 128 + st * 2048, TILE * 128, 1024), id_o, 1);
         }
         mma_commit(&mb_ea[c % kEaSlots]);
       }
@@ -1452,9 +1489,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
   } else if (mma_warp) {
     if (lane == 0) {
       const uint32_t id_ys = idesc_f16(128, 64, false, true);  // M' S
-      const uint32_t id_o = idesc_f16(OM, 64, false, true);    // Q' S
+      const uint32_t id_o = idesc_f16(OM, 128, false, true);   // Q' [S hi | S lo]
       for (int c = 0; c < nsteps && !bad; ++c) {
-        const int t = c / NCH, s = c % NCH, b = t % NB;
+        const int t = c / NCH, s = c % NCH;
         if (!mbar_wait(&mb_m[c % NM], (c / NM) & 1, kWaitNs)) bad = true;
         // S_c in shared memory (S_0 was written before the block barrier; S_c, c >= 1, completes phase c - 1)
         if (c > 0 && !mbar_wait(&mb_s, (c - 1) & 1, kWaitNs)) bad = true;
@@ -1462,14 +1499,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
         if (!mbar_wait(&mb_ea[c % kEaSlots], (c / kEaSlots) & 1, kWaitNs)) bad = true;
         tc::fence_after();
         if (bad) break;
-        const uint32_t ma = smem_u32(sm + F::MB + (c % NM) * 32768), sb = smem_u32(sm + F::SB + (c & 1) * 16384);
+        const uint32_t ma = smem_u32(sm + F::MB + (c % NM) * 32768), sb = smem_u32(sm + F::SB + (c & 1) * 32768);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           mma_f16(tbase + CY0 + 64 * (c & 1), desc_kmaj(ma, 128, k), desc_mnmaj(sb, kD, k), id_ys, 1);
         mma_commit(&mb_y[c & 1]);
-        if (s == 0 && !mbar_wait(&mb_tq[b], (t / NB) & 1, kWaitNs)) bad = true;
+        if (s == 0 && !mbar_wait(&mb_tq, t & 1, kWaitNs)) bad = true;
         if (bad) break;
-        const uint32_t qb = smem_u32(sm + F::QB + b * TILE * 256), od = tbase + CO0 + 64 * (c % kOBufs);
+        const uint32_t qb = smem_u32(sm + F::QB), od = tbase + CO0 + 128 * (c % kOBufs);
 #pragma unroll
         for (int k = 0; k < 8; ++k) mma_f16(od, desc_kmaj(qb, TILE, k), desc_mnmaj(sb, kD, k), id_o, 1);
         mma_commit(&mb_o[c % kOBufs]);
@@ -1489,7 +1526,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
         if (!mbar_wait(&mb_o[c % kOBufs], (c / kOBufs) & 1, kWaitNs)) bad = true;
         if (bad) break;
         if (c + NM < nsteps) issue_m(c + NM);
-        if (tile_end && t + NB < ntiles) issue_q(t + NB);
+        if (tile_end && t + 1 < ntiles) issue_q(t + 1);
       }
     }
   } else if (state_warp) {
@@ -1510,9 +1547,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
 #pragma unroll
       for (int jj = 0; jj < 32; ++jj) S[jj] = egA * S[jj] + y[jj];
       if (c + 1 < nsteps) {
+        unsigned char* sbn = sm + F::SB + ((c + 1) & 1) * 32768;
 #pragma unroll
-        for (int m = 0; m < 4; ++m)
-          st16h(sm + F::SB + ((c + 1) & 1) * 16384 + mnmaj_chunk(kD, si, 32 * hc + 8 * m), S + 8 * m);
+        for (int m = 0; m < 4; ++m) {
+          float lo[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) lo[e] = S[8 * m + e] - __half2float(__float2half_rn(S[8 * m + e]));
+          st16h(sbn + mnmaj_chunk(kD, si, 32 * hc + 8 * m), S + 8 * m);
+          st16h(sbn + 16384 + mnmaj_chunk(kD, si, 32 * hc + 8 * m), lo);
+        }
         fence_async_smem();
         tc::fence_before();
         __syncwarp();
@@ -1551,11 +1594,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
       const bool valid = mine && (t * TILE + r) < len;
       if (!mbar_wait(&mb_o[c % kOBufs], (c / kOBufs) & 1, kWaitNs)) bad = true;
       tc::fence_after();
-      float v[32], ss = 0.f;
-      const uint32_t ob = tbase + lane_base + CO0 + 64 * (c % kOBufs);
+      float v[32], vl[16], ss = 0.f;
+      const uint32_t ob = tbase + lane_base + CO0 + 128 * (c % kOBufs);
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         tmem_ld32(ob + 32 * hh, v);  // warp-collective: every lane takes part
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          tmem_ld16(ob + 64 + 32 * hh + 16 * q, vl);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[16 * q + j] += vl[j];
+        }
 #pragma unroll
         for (int j = 0; j < 32; ++j) ss += v[j] * v[j];
       }
@@ -1567,6 +1616,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         tmem_ld32(ob + 32 * hh, v);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          tmem_ld16(ob + 64 + 32 * hh + 16 * q, vl);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[16 * q + j] += vl[j];
+        }
         if (hh == 1) {  // the products of chunk c are read: the buffer takes chunk c+3's
           tc::fence_before();
           __syncwarp();

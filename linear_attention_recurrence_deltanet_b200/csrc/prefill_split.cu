@@ -41,11 +41,12 @@
 //                   at 8192 half, row r at +128 r, 16-byte piece q at (q ^ (r % 8)) * 16
 //   [122880, 122896) e^{gamma_C}, gamma_C (from the conv)
 //   [122896, 123408) gamma_r, beta_r of the chunk's 64 rows (from the conv; 0 past the chunk's end)
+//   [123520, 139904) v^ lo = v^ - fp16(v^) (from the conv), laid out as v^
 // Operands are fp16 (all bounded: normalised keys and queries, decay factors
-// <= 1), accumulation fp32, the state fp32.  U = T' v^ takes T' as hi + lo and
-// is stored in fp32: the rounding of T' and of v^ feed Delta directly, and over
-// thousands of tokens one of the two must be carried to fp32 accuracy to keep
-// the state within its tolerance.
+// <= 1), accumulation fp32, the state fp32.  U = T' v^ takes T' and v^ as hi +
+// lo (T'hi v^hi + T'lo v^hi + T'hi v^lo) and is stored in fp32: the roundings
+// of T' and of v^ feed Delta directly, and over thousands of tokens they would
+// take the state past its tolerance.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -63,9 +64,9 @@ constexpr int kC = 64;
 constexpr int kD = 128;
 constexpr uint64_t kWaitNs = 2000000000ull;
 
-constexpr int kRec = 123520;  // a multiple of 128 bytes
+constexpr int kRec = 139904;  // a multiple of 128 bytes
 constexpr int REC_A = 0, REC_U = 32768, REC_V = 65536, REC_P = 81920, REC_K = 90112, REC_G = 106496,
-              REC_META = 122880, REC_GAM = 122896, REC_BETA = 123152;
+              REC_META = 122880, REC_GAM = 122896, REC_BETA = 123152, REC_VL = 123520;
 
 // ------------------------------------------------------------------ conv_qkv_kernel
 // Block = 8 warps = the 64 rows of one chunk for one 128-channel head slot
@@ -170,7 +171,10 @@ __global__ void __launch_bounds__(kConvThreads)
   if (vrec) {
 #pragma unroll
     for (int i = 0; i < kConvRows; ++i)
-      if (r0 + i >= L) *reinterpret_cast<uint2*>(vrec + mnmaj(kC, r0 + i, 4 * lane)) = make_uint2(0u, 0u);
+      if (r0 + i >= L) {
+        *reinterpret_cast<uint2*>(vrec + mnmaj(kC, r0 + i, 4 * lane)) = make_uint2(0u, 0u);
+        *reinterpret_cast<uint2*>(vrec + (REC_VL - REC_V) + mnmaj(kC, r0 + i, 4 * lane)) = make_uint2(0u, 0u);
+      }
   }
   if (r0 >= L) return;
   const int64_t C = d.C;
@@ -240,7 +244,13 @@ __global__ void __launch_bounds__(kConvThreads)
   } else {
 #pragma unroll
     for (int i = 0; i < kConvRows; ++i)
-      if (r0 + i < L) st8(vrec + mnmaj(kC, r0 + i, 4 * lane), y[i][0], y[i][1], y[i][2], y[i][3]);
+      if (r0 + i < L) {
+        float lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) lo[e] = y[i][e] - __half2float(__float2half_rn(y[i][e]));
+        st8(vrec + mnmaj(kC, r0 + i, 4 * lane), y[i][0], y[i][1], y[i][2], y[i][3]);
+        st8(vrec + (REC_VL - REC_V) + mnmaj(kC, r0 + i, 4 * lane), lo[0], lo[1], lo[2], lo[3]);
+      }
   }
 }
 
@@ -344,7 +354,7 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
                 int64_t single_len, int32_t* status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  __shared__ uint64_t mb_tma, mb_mma, mb_v;
+  __shared__ uint64_t mb_tma, mb_mma, mb_v, mb_vl;
   __shared__ uint32_t tslot;
   bool bad = false;  // this thread saw a wait run out
 
@@ -375,6 +385,7 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
     mbar_init(&mb_tma, 1);
     mbar_init(&mb_mma, 1);
     mbar_init(&mb_v, 1);
+    mbar_init(&mb_vl, 1);
     mbar_init_fence();
     mbar_expect_tx(&mb_tma, 8 * 8192 + 528);
     bulk_load(sm + P_GATES, rec + REC_META, 528, &mb_tma);
@@ -560,6 +571,12 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
   }
   if (!mbar_wait(&mb_mma, 1, kWaitNs)) bad = true;
   fence_after();
+  if (tid == 0) {  // the k^ rows of the hi tile are read: v^ lo comes into them while -W goes out
+    fence_async_smem();
+    mbar_expect_tx(&mb_vl, 16384);
+    bulk_load(sm + P_KQ, rec + REC_VL, 8192, &mb_vl);
+    bulk_load(sm + P_KQ + 16384, rec + REC_VL + 8192, 8192, &mb_vl);
+  }
   const int r16 = 16 * (warp & 3) + lane;  // lanes 0..15 of each lane quarter hold rows 16 q .. 16 q + 15
   {  // -W -> rows 0..63 of the [-W;Qg] image
     float v[32];
@@ -581,14 +598,21 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
     if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
     return;
   }
-  // MU: U = T'hi v^ + T'lo v^  (M = 64, N = 128; v^ MN-major with its 64-channel blocks 16 KB apart)
+  // MU: U = T'hi v^hi + T'lo v^hi + T'hi v^lo  (M = 64, N = 128; v^ MN-major with its 64-channel blocks
+  // 16 KB apart: hi in the q^ halves of the hi tile, lo in its k^ halves)
   if (tid == 0) {
-    const uint32_t th = smem_u32(sm + P_KQL + 8192), tl = smem_u32(sm + P_KQL + 16384), vb = smem_u32(sm + P_KQ + 8192);
+    const uint32_t th = smem_u32(sm + P_KQL + 8192), tl = smem_u32(sm + P_KQL + 16384), vb = smem_u32(sm + P_KQ + 8192),
+                   vlb = smem_u32(sm + P_KQ);
     constexpr uint32_t id = idesc_f16(64, 128, false, true);
 #pragma unroll
     for (int s = 0; s < 4; ++s) mma_f16(tbase, desc_kmaj(th, 64, s), sdesc(vb + s * 2048, 16384, 1024), id, s > 0);
 #pragma unroll
     for (int s = 0; s < 4; ++s) mma_f16(tbase, desc_kmaj(tl, 64, s), sdesc(vb + s * 2048, 16384, 1024), id, 1);
+    if (!mbar_wait(&mb_vl, 0, kWaitNs)) bad = true;
+    if (!bad) {
+#pragma unroll
+      for (int s = 0; s < 4; ++s) mma_f16(tbase, desc_kmaj(th, 64, s), sdesc(vlb + s * 2048, 16384, 1024), id, 1);
+    }
     mma_commit(&mb_mma);
   }
   if (!mbar_wait(&mb_mma, 0, kWaitNs)) bad = true;
@@ -629,12 +653,14 @@ constexpr int C_P = 65536;      // [0 ; P]     K-major 128 x 64 (8 KB of zero ro
 constexpr int C_U = 98304;      // U half      fp32 64 x 64, the record's image; buffer at +16384 (cc % 2)
 constexpr int C_KT = 131072;    // K~          MN-major K=64 x M=128; buffer at +16384 (cc % 2)
 constexpr int C_DB = 163840;    // Delta half  MN-major K=64 x N=64
-constexpr int C_SB = 172032;    // S half (fp16) MN-major K=128 x N=64
-constexpr int C_G = 188416;     // output gate rows of this half; buffer at +8192 (cc % 2)
-constexpr int C_O = 204800;     // output staging, 32 rows x 64 bytes per output warp (16-byte pieces swizzled)
-constexpr int C_MISC = 212992;  // row sums of squares: this CTA's [2][64], the peer's [2 buffers][64]
+constexpr int C_SB = 172032;    // S half as fp16 hi (+0) and lo (+16384), MN-major K=128 x N=64 each
+constexpr int C_G = 204800;     // output gate rows of this half; buffer at +8192 (cc % 2)
+constexpr int C_O = 221184;     // output staging, 32 rows x 64 bytes per output warp (16-byte pieces swizzled)
+constexpr int C_MISC = 229376;  // row sums of squares: this CTA's [2][64], the peer's [2 buffers][64]
 constexpr int kChainSmem = C_MISC + 256 * 4 + 1024;
-constexpr uint32_t COL_U0 = 0, COL_Y = 128, kChainTmemCols = 256;  // accumulators of chunk cc at COL_U0 + 64 (cc % 2)
+// accumulators of chunk cc at COL_U0 + 128 (cc % 2): [-W;Qg] S hi in its first 64 columns, [-W;Qg] S lo in
+// the next 64 (the two are summed where they are read); K~^T Delta at COL_Y
+constexpr uint32_t COL_U0 = 0, COL_Y = 256, kChainTmemCols = 512;
 
 // Roles: warps 0, 1, 4, 5 ("delta warps", TMEM lanes 0..63) form Delta = U -
 // W S and store it to shared memory; warps 2, 3, 6, 7 ("output warps", lanes
@@ -730,11 +756,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
     bulk_prefetch_l2(rec_of(cc) + REC_P, REC_META + 16 - REC_P);
   };
   float S[32];  // this thread's part of the state, fp32
+  // its fp16 hi and lo parts, the B operand [S hi | S lo] of [-W;Qg] S (N = 128): the output Qg S + P Delta
+  // can cancel to far below |Qg||S| when q is nearly orthogonal to the state's columns, so the state's
+  // fp16 rounding alone would cost o up to about 2e-3 of its largest value
+  auto store_s = [&]() {
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      float lo[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) lo[e] = S[8 * m + e] - __half2float(__float2half_rn(S[8 * m + e]));
+      st16h(sm + C_SB + mnmaj_chunk(kD, si, 32 * hc + 8 * m), S + 8 * m);
+      st16h(sm + C_SB + 16384 + mnmaj_chunk(kD, si, 32 * hc + 8 * m), lo);
+    }
+  };
   if (compute) {
 #pragma unroll
     for (int jj = 0; jj < 32; ++jj) S[jj] = zero_state ? 0.f : gst[(int64_t)(c0 + jj) * kD + si];
-#pragma unroll
-    for (int m = 0; m < 4; ++m) st16h(sm + C_SB + mnmaj_chunk(kD, si, 32 * hc + 8 * m), S + 8 * m);
+    store_s();
   }
   fence_async_smem();
   sync_tc();
@@ -770,8 +808,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
     const int Lc = min(kC, len - cc * kC);
     if (!mbar_wait(&mb_m4[cc & 1], (cc >> 1) & 1, kWaitNs)) bad = true;
     fence_after();
-    float v[32];
-    tmem_ld32(tbase + lane_base + COL_U0 + 64 * (cc & 1) + 32 * hc, v);
+    float v[32], vl[32];
+    tmem_ld32(tbase + lane_base + COL_U0 + 128 * (cc & 1) + 32 * hc, v);
+    tmem_ld32(tbase + lane_base + COL_U0 + 128 * (cc & 1) + 64 + 32 * hc, vl);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] += vl[j];
     float ss = 0.f;
 #pragma unroll
     for (int j = 0; j < 32; ++j) ss += v[j] * v[j];
@@ -816,14 +857,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
   };
 
   for (int c = 0; c < nchunks; ++c) {
-    const uint32_t colU = COL_U0 + 64 * (c & 1);
+    const uint32_t colU = COL_U0 + 128 * (c & 1);
     const uint32_t par = (c >> 1) & 1;  // phase parity of the buffers of chunk c
     if (mma_warp) {
       if (lane == 0) {  // [-W;Qg] S -> [-WS ; QgS]
         if (!mbar_wait(&mb_a[c & 1], par, kWaitNs)) bad = true;
         if (!bad) {
           const uint32_t aa = smem_u32(sm + C_A + 32768 * (c & 1)), sb = smem_u32(sm + C_SB);
-          constexpr uint32_t id = idesc_f16(128, 64, false, true);
+          constexpr uint32_t id = idesc_f16(128, 128, false, true);  // B = [S hi | S lo]
 #pragma unroll
           for (int s = 0; s < 8; ++s) mma_f16(tbase + colU, desc_kmaj(aa, 128, s), desc_mnmaj(sb, kD, s), id, s > 0);
           mma_commit(&mb_m3);
@@ -887,6 +928,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
         tmem_ld32(tbase + lane_base + colU + 32 * hc, v);
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] += u[j];
+        tmem_ld32(tbase + lane_base + colU + 64 + 32 * hc, u);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] += u[j];
 #pragma unroll
         for (int m = 0; m < 4; ++m) st16h(sm + C_DB + mnmaj_chunk(kC, si, 32 * hc + 8 * m), v + 8 * m);
         fence_async_smem();
@@ -902,8 +946,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
       tmem_ld32(tbase + lane_base + COL_Y + 32 * hc, y);
 #pragma unroll
       for (int jj = 0; jj < 32; ++jj) S[jj] = egC * S[jj] + y[jj];
-#pragma unroll
-      for (int m = 0; m < 4; ++m) st16h(sm + C_SB + mnmaj_chunk(kD, si, 32 * hc + 8 * m), S + 8 * m);
+      store_s();
     }
     fence_async_smem();
     if (sync_tc_any(bad)) break;

@@ -60,7 +60,8 @@ constexpr int32_t kTimeoutChain = kStatusWaitTimeout | (GDN_K_WY_CHAIN << 8);
 // ------------------------------------------------------------------ record of one (tile, value head)
 // Byte images of the chain kernel's operands (fp16, 128-byte swizzle):
 //   [0, NCH * 32768)   M'_s of each chunk s of the tile, K-major 128 x 128 (row = output key index)
-//   REC_Q              Q', K-major TILE x 128
+//   REC_Q              Q', K-major TILE x 128; at chunk 16 followed by its fp16 low part (the
+//                      output's error from Q' alone otherwise reaches 2e-3 of o on long sequences)
 //   REC_KT             K~, MN-major K=TILE x M=128
 //   REC_U              U = T diag(beta) V per value-channel half: [half][hi, lo], MN-major K=TILE x N=64
 //   REC_P              P, K-major TILE x TILE
@@ -69,8 +70,10 @@ template <int TILE, int C>
 struct Rec {
   static constexpr int NCH = TILE / C;
   static constexpr int M = 0;
+  static constexpr bool QLO = C == 16;
   static constexpr int Q = NCH * 32768;
-  static constexpr int KT = Q + TILE * 256;
+  static constexpr int QBYTES = (QLO ? 2 : 1) * TILE * 256;
+  static constexpr int KT = Q + QBYTES;
   static constexpr int U = KT + TILE * 256;
   static constexpr int UH = TILE * 128;  // one hi or lo image of one half
   static constexpr int P = U + 4 * UH;
@@ -745,6 +748,11 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
 #pragma unroll
           for (int e = 0; e < 8; ++e) q8[e] = ok ? v[8 * m + e] : 0.f;
           *reinterpret_cast<uint4*>(sm + WP_V + kmaj_chunk(TILE, r16, cb + 8 * m)) = pack8h(q8);
+          if (R::QLO) {  // the low part goes over T' (read by the products just completed)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) q8[e] -= __half2float(__float2half_rn(q8[e]));
+            *reinterpret_cast<uint4*>(sm + WP_KQL + kmaj_chunk(TILE, r16, cb + 8 * m)) = pack8h(q8);
+          }
         }
       }
     }
@@ -761,6 +769,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
   if (tid == 0) {
     bulk_store(rec + R::U, sm + WP_KQH, 4 * R::UH);
     bulk_store(rec + R::Q, sm + WP_V, TILE * 256);
+    if (R::QLO) bulk_store(rec + R::Q + TILE * 256, sm + WP_KQL, TILE * 256);
     bulk_commit();
   }
   // M'_s = K~_s^T (-W_s) for each chunk s of the tile (M = N = 128, K = the chunk's rows)
@@ -1324,11 +1333,11 @@ template <int TILE, int C>
 struct ChainCfg {
   static constexpr int NCH = TILE / C;
   static constexpr int NM = TILE == 64 ? 2 : 1;    // M' buffers
-  static constexpr int NB = TILE == 64 ? 2 : 1;    // K~, U, P buffers (Q' has one)
+  static constexpr int NB = TILE == 64 && C != 16 ? 2 : 1;  // K~, U, P buffers (Q' has one)
   static constexpr int MB = 0;                                  // M' K-major 128 x 128, 32 KB each
   static constexpr int SB = MB + NM * 32768;                    // S copies (2): hi, lo MN-major K=128 x N=64
-  static constexpr int QB = SB + 2 * 32768;                     // Q' K-major TILE x 128
-  static constexpr int KTB = QB + TILE * 256;                   // K~ MN-major K=TILE x M=128
+  static constexpr int QB = SB + 2 * 32768;                     // Q' (hi, and lo at chunk 16) K-major TILE x 128
+  static constexpr int KTB = QB + Rec<TILE, C>::QBYTES;         // K~ MN-major K=TILE x M=128
   static constexpr int UB = KTB + NB * TILE * 256;              // U of this half: hi, lo MN-major K=TILE x N=64
   static constexpr int PB = UB + NB * TILE * 256;               // P K-major TILE x TILE
   static constexpr int MISC = PB + NB * TILE * TILE * 2;
@@ -1414,8 +1423,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
     bulk_load(sm + F::PB + b * TILE * TILE * 2, r + R::P, TILE * TILE * 2, &mb_ta[b]);
   };
   auto issue_q = [&](int t) {
-    mbar_expect_tx(&mb_tq, TILE * 256);
-    bulk_load(sm + F::QB, rec_of(t) + R::Q, TILE * 256, &mb_tq);
+    mbar_expect_tx(&mb_tq, R::QBYTES);
+    bulk_load(sm + F::QB, rec_of(t) + R::Q, R::QBYTES, &mb_tq);
   };
   auto issue_m = [&](int c) {
     const int b = c % NM;
@@ -1509,6 +1518,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
         const uint32_t qb = smem_u32(sm + F::QB), od = tbase + CO0 + 128 * (c % kOBufs);
 #pragma unroll
         for (int k = 0; k < 8; ++k) mma_f16(od, desc_kmaj(qb, TILE, k), desc_mnmaj(sb, kD, k), id_o, 1);
+        if (R::QLO) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mma_f16(od, desc_kmaj(qb + TILE * 256, TILE, k), desc_mnmaj(sb, kD, k), id_o, 1);
+        }
         mma_commit(&mb_o[c % kOBufs]);
       }
     }

@@ -289,7 +289,7 @@ def run_gdn(args, rank, world, local_rank):
     # ---------------- prefill workload (B=1, T=4096)
     w = gi.WORKLOADS[PREFILL_WORKLOAD]
     inp = gi.workload_inputs(PREFILL_WORKLOAD)
-    geo, C = inp.geo, w["chunks"][0]
+    geo, C = inp.geo, (args.chunk or w["chunks"][0])
     cfg = gdn.make_config(geo)
     T = inp.total_tokens
     params = tuple(torch.from_numpy(np.ascontiguousarray(p)).cuda() for p in (inp.conv_w, inp.A_log, inp.dt_bias,
@@ -527,7 +527,7 @@ def run_gdn(args, rank, world, local_rank):
             "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": DTYPE, "data": "synthetic",
-            "config": {"workload": "GDN prefill, B=1, T=4096, 16 key / 48 value heads x 128, chunk 64, bf16 inputs, "
+            "config": {"workload": f"GDN prefill, B=1, T=4096, 16 key / 48 value heads x 128, chunk {C}, bf16 inputs, "
                                    "fp32 state from zero", "global_batch": world, "seq_len": T, "chunk": C,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": f"inputs rotate over {ROTATE} sets (> 4x L2) between steps"},
@@ -776,6 +776,8 @@ def main():
     ap.add_argument("--recurrent", action="store_true", help="time the token-recurrent prefill kernel")
     ap.add_argument("--fused", action="store_true", help="time the single-kernel chunked prefill")
     ap.add_argument("--affine", action="store_true", help="time the affine three-kernel chunked prefill at chunk 64")
+    ap.add_argument("--chunk", type=int, choices=[16, 32, 64, 128], default=0,
+                    help="chunk size of the timed prefill (default: the workload's, 64; 16/32/128 run the affine path)")
     ap.add_argument("--no-workloads", action="store_true", help="skip the long-context and varlen workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--projection-reps", type=int, default=20, help="timed launches per projection shape")

@@ -659,7 +659,7 @@ constexpr int C_O = 221184;     // output staging, 32 rows x 64 bytes per output
 constexpr int C_MISC = 229376;  // row sums of squares: this CTA's [2][64], the peer's [2 buffers][64]
 constexpr int kChainSmem = C_MISC + 256 * 4 + 1024;
 // accumulators of chunk cc at COL_U0 + 128 (cc % 2): [-W;Qg] S hi in its first 64 columns, [-W;Qg] S lo in
-// the next 64 (the two are summed where they are read); K~^T Delta at COL_Y
+// the next 64 (the output warps sum the two; Delta takes the hi block alone); K~^T Delta at COL_Y
 constexpr uint32_t COL_U0 = 0, COL_Y = 256, kChainTmemCols = 512;
 
 // Roles: warps 0, 1, 4, 5 ("delta warps", TMEM lanes 0..63) form Delta = U -
@@ -756,9 +756,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
     bulk_prefetch_l2(rec_of(cc) + REC_P, REC_META + 16 - REC_P);
   };
   float S[32];  // this thread's part of the state, fp32
-  // its fp16 hi and lo parts, the B operand [S hi | S lo] of [-W;Qg] S (N = 128): the output Qg S + P Delta
-  // can cancel to far below |Qg||S| when q is nearly orthogonal to the state's columns, so the state's
-  // fp16 rounding alone would cost o up to about 2e-3 of its largest value
+  // its fp16 hi and lo parts: the output Qg S + P Delta can cancel to far below |Qg||S| when q is nearly
+  // orthogonal to the state's columns, so the state's fp16 rounding alone would cost o up to about 2e-3 of
+  // its largest value; [-W;Qg] S lo goes out behind the critical [-W;Qg] S hi, and only the output reads it
   auto store_s = [&]() {
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
@@ -864,10 +864,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
         if (!mbar_wait(&mb_a[c & 1], par, kWaitNs)) bad = true;
         if (!bad) {
           const uint32_t aa = smem_u32(sm + C_A + 32768 * (c & 1)), sb = smem_u32(sm + C_SB);
-          constexpr uint32_t id = idesc_f16(128, 128, false, true);  // B = [S hi | S lo]
+          constexpr uint32_t id = idesc_f16(128, 64, false, true);
 #pragma unroll
           for (int s = 0; s < 8; ++s) mma_f16(tbase + colU, desc_kmaj(aa, 128, s), desc_mnmaj(sb, kD, s), id, s > 0);
           mma_commit(&mb_m3);
+#pragma unroll
+          for (int s = 0; s < 8; ++s)
+            mma_f16(tbase + colU + 64, desc_kmaj(aa, 128, s), desc_mnmaj(sb + 16384, kD, s), id, s > 0);
         }
         if (!mbar_wait(&mb_ld1[c & 1], par, kWaitNs)) bad = true;  // P and K~, long in place
       }
@@ -926,9 +929,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
         fence_after();
         float v[32];
         tmem_ld32(tbase + lane_base + colU + 32 * hc, v);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] += u[j];
-        tmem_ld32(tbase + lane_base + colU + 64 + 32 * hc, u);
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] += u[j];
 #pragma unroll

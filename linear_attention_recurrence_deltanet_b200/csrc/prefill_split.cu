@@ -16,7 +16,8 @@
 //                     q^, k^ as fp16 hi + lo parts, v^ as fp16; and the output
 //                     gate (1 + w) sigmoid(z) of every value head, fp16.
 //   prep_kernel       grid (chunk, value head): gates, [K;Q]K^T in split
-//                     precision on tcgen05, A and P, T = (I+A)^-1, then W = T''K
+//                     precision on tcgen05, A and P, T = (I+A)^-1 by recursive
+//                     doubling whose merges are tcgen05 MMAs, then W = T''K
 //                     and U = T'v^ on tcgen05; writes one record per (chunk,
 //                     value head) whose parts are byte images of the chain
 //                     kernel's shared-memory operands.
@@ -255,31 +256,28 @@ __global__ void __launch_bounds__(kConvThreads)
 }
 
 // ------------------------------------------------------------------ prep_kernel
-// Three blocks per SM.  Shared memory (67 KB):
-//   P_KQ   [k^ ; q^] hi parts, K-major 128 x 128.  Once the Qg rows are out,
-//          the q^ halves of the two 64-column blocks hold the solve's Y rows
-//          0..31 and 32..63.
-//   P_KQL  [k^ ; q^] lo parts.  After M1: the solve scratch A (16 KB) and T
-//          (16 KB); after the solve, T'' and T' hi (K-major 64 x 64) over A and
-//          T' lo over T.  After the solve v^ (MN-major, its two 64-channel
-//          blocks 16 KB apart) lands in the q^ halves of the hi tile.
-// fp32 scratch rows are 64 floats with the 16-byte pieces of row r XORed by
-// r % 16, so that column accesses from 16 rows hit distinct banks.
-// TMEM: 128 columns; [K;Q]K^T in columns 0..63, then W and then U (M = 64 MMAs) in 0..127.
+// Three blocks per SM.  Shared memory (71 KB):
+//   P_KQ   [k^ ; q^] hi parts, K-major 128 x 128.  Once [K;Q]K^T is done, v^
+//          hi (MN-major, its two 64-channel blocks 16 KB apart) comes into the
+//          q^ halves; once W = T''K is done, v^ lo into the k^ halves.
+//   P_KQL  [k^ ; q^] lo parts.  After [K;Q]K^T: the solve's images A_off16,
+//          A_off32, T and X (K-major 64 x 64 fp16 each; the fp32 16x16
+//          diagonal blocks of A in X's place until X is first written); after
+//          the solve T'' over A_off16, T' hi over A_off32 and T' lo over T.
+//   P_TF   the 16x16 diagonal blocks of T in fp32.
+// TMEM: 128 columns; [K;Q]K^T in columns 0..63, the solve's products in 0..63,
+// then W and then U (M = 64 MMAs) in 0..127.
 constexpr int kPrepThreads = 256;
 constexpr int P_KQ = 0;
 constexpr int P_KQL = 32768;
 constexpr int P_MISC = 65536;
 constexpr int P_GATES = P_MISC + 64 * 6 * 4;  // the record's e^{gamma_C}, gamma_C, gamma_r, beta_r (528 bytes)
-constexpr int kPrepSmem = P_GATES + 528 + 1024;
+constexpr int P_TF = P_GATES + 528;            // the 16x16 diagonal blocks of T in fp32 (4 KB)
+constexpr int kPrepSmem = P_TF + 4096 + 1024;
+// the solve's images in the lo tile once [K;Q]K^T is done (K-major 64 x 64 fp16 each)
+constexpr int P_AOFF16 = P_KQL, P_AOFF32 = P_KQL + 8192, P_T = P_KQL + 16384, P_X = P_KQL + 24576;
+constexpr int P_DIAG = P_X;  // the fp32 16x16 diagonal blocks of A (stride 17) until X is first written
 constexpr uint32_t kPrepTmemCols = 128;
-
-__device__ __forceinline__ int sidx(int row, int col) { return row * 64 + ((((col >> 2) ^ (row & 15))) << 2) + (col & 3); }
-
-// Y rows 0..31 and 32..63 live in the two q^ halves of the hi tile
-__device__ __forceinline__ float* yrow(unsigned char* sm, int row) {
-  return reinterpret_cast<float*>(sm + P_KQ + (row < 32 ? 8192 : 24576)) + (row & 31) * 64;
-}
 
 // The new conv history of sequence n: the last W-1 raw rows of [history ;
 // inputs].  The prep block of the sequence's last chunk and value head h owns
@@ -307,44 +305,6 @@ __device__ __forceinline__ void write_history(const Dims& d, int h, int n, int64
 #pragma unroll
     for (int r = 0; r < 3; ++r) *reinterpret_cast<uint4*>(hist + ((int64_t)n * 3 + r) * d.C + ch) = v[r];
   }
-}
-
-// One doubling level of T = (I + A)^-1: for every pair of B x B diagonal
-// blocks at offset o = 2 B p, Y = A21 T11, then T21 = -T22 Y.  Four columns
-// per work item.
-template <int B>
-__device__ __forceinline__ void solve_level(const float* __restrict__ Am, float* __restrict__ Tm, unsigned char* sm,
-                                            int tid) {
-  constexpr int kItems = (64 / (2 * B)) * B * (B / 4);
-  for (int e = tid; e < kItems; e += kPrepThreads) {
-    const int p = e / (B * B / 4), rem = e - p * (B * B / 4);
-    const int i = rem / (B / 4), j = 4 * (rem - i * (B / 4));
-    const int o = 2 * B * p, row = o + B + i;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int k = 0; k < B; ++k) {
-      const float a = Am[sidx(row, o + k)];
-      const float4 t = *reinterpret_cast<const float4*>(Tm + sidx(o + k, o + j));
-      acc.x += a * t.x; acc.y += a * t.y; acc.z += a * t.z; acc.w += a * t.w;
-    }
-    *reinterpret_cast<float4*>(yrow(sm, row) + (sidx(row, o + j) & 63)) = acc;
-  }
-  __syncthreads();
-  for (int e = tid; e < kItems; e += kPrepThreads) {
-    const int p = e / (B * B / 4), rem = e - p * (B * B / 4);
-    const int i = rem / (B / 4), j = 4 * (rem - i * (B / 4));
-    const int o = 2 * B * p, row = o + B + i;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int k = 0; k < B; ++k) {
-      const float t = Tm[sidx(row, o + B + k)];
-      const int yr = o + B + k;
-      const float4 y = *reinterpret_cast<const float4*>(yrow(sm, yr) + (sidx(yr, o + j) & 63));
-      acc.x += t * y.x; acc.y += t * y.y; acc.z += t * y.z; acc.w += t * y.w;
-    }
-    *reinterpret_cast<float4*>(Tm + sidx(row, o + j)) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
-  }
-  __syncthreads();
 }
 
 __global__ void __launch_bounds__(kPrepThreads, 3)
@@ -378,8 +338,6 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
   float* s_ekd = misc + 192;
   float* s_tb = misc + 256;    // beta_j             (columns of T')
   float* s_tbg = misc + 320;   // beta_j e^{gamma_j} (columns of T'')
-  float* Am = reinterpret_cast<float*>(sm + P_KQL);
-  float* Tm = Am + 64 * 64;
 
   if (tid == 0) {  // the copies go out before anything else
     mbar_init(&mb_tma, 1);
@@ -467,7 +425,15 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
     return;
   }
 
-  // A (rows 0..63, fp32 into the solve scratch) and P (rows 64..127, fp16 into the record)
+  if (tid == 0) {  // the q^ rows of the hi tile are read: v^ comes into them while the solve runs
+    fence_async_smem();
+    mbar_expect_tx(&mb_v, 16384);
+    bulk_load(sm + P_KQ + 8192, rec + REC_V, 8192, &mb_v);
+    bulk_load(sm + P_KQ + 24576, rec + REC_V + 8192, 8192, &mb_v);
+  }
+  // A (rows 0..63) into the fp32 16x16 diagonal blocks and the two level images; P (rows 64..127, fp16)
+  // into the record.  Element (r, j), j < r, of A belongs to the level b = 16, 32 whose blocks first put r
+  // and j in different halves, or to a 16x16 diagonal block when r ^ j < 16.
   const int si = 32 * (warp & 3) + lane, hc = warp >> 2;
   const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
   {
@@ -476,14 +442,19 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
     if (si < 64) {
       const float br = s_beta[si], gr = s_gam[si];
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        float a4[4];
+      for (int m = 0; m < 4; ++m) {
+        float a16[8], a32[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int j = 32 * hc + 4 * m + e;
-          a4[e] = (j < si) ? br * __expf(gr - s_gam[j]) * v[4 * m + e] : 0.f;
+        for (int e = 0; e < 8; ++e) {
+          const int j = 32 * hc + 8 * m + e;
+          const float av = (j < si) ? br * __expf(gr - s_gam[j]) * v[8 * m + e] : 0.f;
+          const int x = si ^ j;
+          a16[e] = (x >= 16 && x < 32) ? av : 0.f;
+          a32[e] = (x >= 32) ? av : 0.f;
+          if (x < 16) reinterpret_cast<float*>(sm + P_DIAG)[(si >> 4) * 272 + (si & 15) * 17 + (j & 15)] = av;
         }
-        *reinterpret_cast<float4*>(Am + sidx(si, 32 * hc + 4 * m)) = make_float4(a4[0], a4[1], a4[2], a4[3]);
+        *reinterpret_cast<uint4*>(sm + P_AOFF16 + kmaj_chunk(64, si, 32 * hc + 8 * m)) = pack8h(a16);
+        *reinterpret_cast<uint4*>(sm + P_AOFF32 + kmaj_chunk(64, si, 32 * hc + 8 * m)) = pack8h(a32);
       }
     } else {
       const int r = si - 64;
@@ -500,46 +471,123 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
       }
     }
   }
-  for (int i = tid; i < 64 * 16; i += kPrepThreads)
-    *reinterpret_cast<float4*>(Tm + 4 * i) = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i = tid; i < 8192 / 16; i += kPrepThreads) reinterpret_cast<uint4*>(sm + P_T)[i] = make_uint4(0, 0, 0, 0);
   __syncthreads();
-  // T = (I + A)^-1 by recursive doubling: the 8x8 diagonal blocks by forward
-  // substitution, then for block size b = 8, 16, 32 every pair of b-blocks on
-  // the diagonal is joined into a 2b-block through its lower-left block
-  // T21 = -T22 (A21 T11).  T starts at zero, so the upper blocks stay zero.
+  // T = (I + A)^-1 by recursive doubling.  Level 0: the 16x16 diagonal blocks by forward substitution, one
+  // column of one block per thread, in fp32: kept in fp32 for T' and T'' (no later level changes them) and
+  // as fp16 in the T image.  Levels b = 16, 32: T <- T - T (A_off,b T), every merge of two b-blocks at once,
+  // both products on tcgen05 (M = N = K = 64, fp16 operands, fp32 accumulation).  T starts at zero, so
+  // its upper blocks stay zero.
   if (tid < 64) {
-    const int bb = tid >> 3, c8 = tid & 7, o = 8 * bb;
-    float acc[8], t[8];
+    const int bb = tid >> 4, c = tid & 15, o = 16 * bb;
+    const float* Ad = reinterpret_cast<const float*>(sm + P_DIAG) + bb * 272;
+    float* Tf = reinterpret_cast<float*>(sm + P_TF) + bb * 256;
+    float t[16];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int i = 0; i < 16; ++i) {
+      float acc = (i == c) ? 1.f : 0.f;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      t[k] = (k < c8) ? 0.f : (k == c8 ? 1.f : -acc[k]);
-#pragma unroll
-      for (int i = k + 1; i < 8; ++i) acc[i] += Am[sidx(o + i, o + k)] * t[k];
+      for (int k = 0; k < i; ++k) acc -= Ad[i * 17 + k] * t[k];
+      t[i] = (i < c) ? 0.f : acc;
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) Tm[sidx(o + i, o + c8)] = t[i];
+    for (int i = 0; i < 16; ++i) {
+      *reinterpret_cast<__half*>(sm + P_T + kmaj(64, o + i, o + c)) = __float2half_rn(t[i]);
+      Tf[i * 16 + c] = t[i];
+    }
   }
-  __syncthreads();
-  solve_level<8>(Am, Tm, sm, tid);
-  solve_level<16>(Am, Tm, sm, tid);
-  solve_level<32>(Am, Tm, sm, tid);
-  // the Y rows are read: v^ comes into the q^ halves of the hi tile while T' and W are formed
-  if (tid == 0) {
+  fence_async_smem();
+  sync_tc();
+  const int r16 = 16 * (warp & 3) + lane;  // lanes 0..15 of each lane quarter hold rows 16 q .. 16 q + 15
+  uint32_t mma_phase = 1;  // [K;Q]K^T completed phase 0
+#pragma unroll 1
+  for (int lv = 0; lv < 2; ++lv) {
+    const uint32_t aoff = smem_u32(sm + (lv == 0 ? P_AOFF16 : P_AOFF32));
+    const uint32_t ts = smem_u32(sm + P_T), xs = smem_u32(sm + P_X);
+    constexpr uint32_t id = idesc_f16(64, 64, false, true);
+    if (tid == 0) {  // X = A_off T
+#pragma unroll
+      for (int s = 0; s < 4; ++s) mma_f16(tbase, desc_kmaj(aoff, 64, s), desc_mnmaj(ts, 64, s), id, s > 0);
+      mma_commit(&mb_mma);
+    }
+    if (!mbar_wait(&mb_mma, mma_phase, kWaitNs)) bad = true;
+    mma_phase ^= 1;
+    fence_after();
+    {
+      float v[32];
+      tmem_ld32(tbase + lane_base + 32 * hc, v);
+      if (lane < 16) {
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+          *reinterpret_cast<uint4*>(sm + P_X + kmaj_chunk(64, r16, 32 * hc + 8 * m)) = pack8h(v + 8 * m);
+      }
+    }
     fence_async_smem();
-    mbar_expect_tx(&mb_v, 16384);
-    bulk_load(sm + P_KQ + 8192, rec + REC_V, 8192, &mb_v);
-    bulk_load(sm + P_KQ + 24576, rec + REC_V + 8192, 8192, &mb_v);
+    sync_tc();
+    if (tid == 0) {  // Y = T X
+#pragma unroll
+      for (int s = 0; s < 4; ++s) mma_f16(tbase, desc_kmaj(ts, 64, s), desc_mnmaj(xs, 64, s), id, s > 0);
+      mma_commit(&mb_mma);
+    }
+    if (!mbar_wait(&mb_mma, mma_phase, kWaitNs)) bad = true;
+    mma_phase ^= 1;
+    fence_after();
+    {
+      float v[32];
+      tmem_ld32(tbase + lane_base + 32 * hc, v);
+      if (lane < 16) {
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          unsigned char* pt = sm + P_T + kmaj_chunk(64, r16, 32 * hc + 8 * m);
+          const uint4 tq = *reinterpret_cast<const uint4*>(pt);
+          const __half2* t2 = reinterpret_cast<const __half2*>(&tq);
+          float nt[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __half22float2(t2[i]);
+            nt[2 * i] = f.x - v[8 * m + 2 * i];
+            nt[2 * i + 1] = f.y - v[8 * m + 2 * i + 1];
+          }
+          *reinterpret_cast<uint4*>(pt) = pack8h(nt);
+        }
+      }
+    }
+    fence_async_smem();
+    if (sync_tc_any(bad)) break;
+  }
+  if (bad) {  // block-uniform after sync_tc_any
+    if (tid == 0) {
+      set_status(status, kStatusWaitTimeout);
+      mbar_wait(&mb_v, 0, kWaitNs);  // the v^ copy is no longer in flight when the block leaves
+    }
+    if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
+    return;
   }
   {  // T' = T diag(beta) as fp16 hi + lo and T'' = T diag(beta e^gamma), K-major 64 x 64 A operands of
-     // U = T' v^ and W = T'' K: T'' and T' hi over A, T' lo over T once every thread has read its rows of T
+     // U = T' v^ and W = T'' K: T'' over A_off16, T' hi over A_off32 and T' lo over T once every thread
+     // has read its rows of T.  A thread's 16 columns are one 16-column block: the diagonal one comes from
+     // the fp32 blocks.
     const int r = tid >> 2, j0 = 16 * (tid & 3);
     float tv[16], t1[16], t2[16];
+    if ((tid & 3) == (r >> 4)) {
+      const float4* tf = reinterpret_cast<const float4*>(sm + P_TF) + (r >> 4) * 64 + (r & 15) * 4;
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const float4 t4 = *reinterpret_cast<const float4*>(Tm + sidx(r, j0 + 4 * m));
-      tv[4 * m] = t4.x; tv[4 * m + 1] = t4.y; tv[4 * m + 2] = t4.z; tv[4 * m + 3] = t4.w;
+      for (int m = 0; m < 4; ++m) {
+        const float4 f = tf[m];
+        tv[4 * m] = f.x; tv[4 * m + 1] = f.y; tv[4 * m + 2] = f.z; tv[4 * m + 3] = f.w;
+      }
+    } else {
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const uint4 tq = *reinterpret_cast<const uint4*>(sm + P_T + kmaj_chunk(64, r, j0 + 8 * m));
+        const __half2* h2 = reinterpret_cast<const __half2*>(&tq);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __half22float2(h2[i]);
+          tv[8 * m + 2 * i] = f.x;
+          tv[8 * m + 2 * i + 1] = f.y;
+        }
+      }
     }
 #pragma unroll
     for (int jj = 0; jj < 16; ++jj) {
@@ -547,13 +595,13 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
       t1[jj] = t * s_tb[j0 + jj];
       t2[jj] = t * s_tbg[j0 + jj];
     }
+    __syncthreads();  // every thread has read its rows of T
     st16h(sm + P_KQL + kmaj_chunk(64, r, j0), t2);
     st16h(sm + P_KQL + kmaj_chunk(64, r, j0 + 8), t2 + 8);
     st16h(sm + P_KQL + 8192 + kmaj_chunk(64, r, j0), t1);
     st16h(sm + P_KQL + 8192 + kmaj_chunk(64, r, j0 + 8), t1 + 8);
 #pragma unroll
     for (int jj = 0; jj < 16; ++jj) t1[jj] -= __half2float(__float2half_rn(t1[jj]));
-    __syncthreads();
     st16h(sm + P_KQL + 16384 + kmaj_chunk(64, r, j0), t1);
     st16h(sm + P_KQL + 16384 + kmaj_chunk(64, r, j0 + 8), t1 + 8);
   }
@@ -577,7 +625,6 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
     bulk_load(sm + P_KQ, rec + REC_VL, 8192, &mb_vl);
     bulk_load(sm + P_KQ + 16384, rec + REC_VL + 8192, 8192, &mb_vl);
   }
-  const int r16 = 16 * (warp & 3) + lane;  // lanes 0..15 of each lane quarter hold rows 16 q .. 16 q + 15
   {  // -W -> rows 0..63 of the [-W;Qg] image
     float v[32];
 #pragma unroll

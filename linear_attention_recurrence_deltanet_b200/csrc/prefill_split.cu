@@ -625,8 +625,10 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
     bulk_load(sm + P_KQ, rec + REC_VL, 8192, &mb_vl);
     bulk_load(sm + P_KQ + 16384, rec + REC_VL + 8192, 8192, &mb_vl);
   }
-  {  // -W -> rows 0..63 of the [-W;Qg] image
+  {  // -W -> rows 0..63 of the [-W;Qg] image: its two 8 KB row blocks (64-column block hc at +16 KB hc of
+     // the image) are staged over T'' (read by W) and X, and go out by bulk stores
     float v[32];
+    unsigned char* stage = sm + P_KQL + 24576 * hc;
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       tmem_ld32(tbase + lane_base + 64 * hc + 32 * hh, v);
@@ -635,15 +637,24 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
         for (int jj = 0; jj < 32; ++jj) v[jj] = -v[jj];
 #pragma unroll
         for (int m = 0; m < 4; ++m)
-          *reinterpret_cast<uint4*>(rec + REC_A + kmaj_chunk(128, r16, 64 * hc + 32 * hh + 8 * m)) = pack8h(v + 8 * m);
+          *reinterpret_cast<uint4*>(stage + kmaj_chunk(64, r16, 32 * hh + 8 * m)) = pack8h(v + 8 * m);
       }
     }
   }
+  fence_async_smem();
   if (tid == 0 && !mbar_wait(&mb_v, 0, kWaitNs)) bad = true;
   if (sync_tc_any(bad)) {  // also: W is read out, its columns take U
-    if (tid == 0) set_status(status, kStatusWaitTimeout);
+    if (tid == 0) {
+      set_status(status, kStatusWaitTimeout);
+      mbar_wait(&mb_vl, 0, kWaitNs);  // no copy is still in flight when the block leaves
+    }
     if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
     return;
+  }
+  if (tid == 0) {
+    bulk_store(rec + REC_A, sm + P_KQL, 8192);
+    bulk_store(rec + REC_A + 16384, sm + P_KQL + 24576, 8192);
+    bulk_commit();
   }
   // MU: U = T'hi v^hi + T'lo v^hi + T'hi v^lo  (M = 64, N = 128; v^ MN-major with its 64-channel blocks
   // 16 KB apart: hi in the q^ halves of the hi tile, lo in its k^ halves)
@@ -663,15 +674,17 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
     mma_commit(&mb_mma);
   }
   if (!mbar_wait(&mb_mma, 0, kWaitNs)) bad = true;
+  if (tid == 0) bulk_wait_read<0>();  // the -W stores have read their staging (the U image goes over it)
+  __syncthreads();
   fence_after();
-  {  // U -> the record, fp32: channel half c / 64 at 16384 (c / 64), row r at 256 r, 16-byte piece j of the
-     // half row at (j ^ (r % 8)) * 16
+  {  // U -> its record image staged over T'' .. X (all read by the U products): fp32, channel half c / 64
+     // at 16384 (c / 64), row r at 256 r, 16-byte piece j of the half row at (j ^ (r % 8)) * 16
     float v[32];
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       tmem_ld32(tbase + lane_base + 64 * hc + 32 * hh, v);
       if (lane < 16) {
-        unsigned char* urow = rec + REC_U + 16384 * hc + 256 * r16;
+        unsigned char* urow = sm + P_KQL + 16384 * hc + 256 * r16;
 #pragma unroll
         for (int m = 0; m < 8; ++m)
           *reinterpret_cast<float4*>(urow + (((8 * hh + m) ^ (r16 & 7)) << 4)) =
@@ -679,7 +692,14 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
       }
     }
   }
-  if (sync_tc_any(bad) && tid == 0) set_status(status, kStatusWaitTimeout);
+  fence_async_smem();
+  const bool fail = sync_tc_any(bad);
+  if (tid == 0) {
+    if (fail) set_status(status, kStatusWaitTimeout);
+    bulk_store(rec + REC_U, sm + P_KQL, 32768);
+    bulk_commit();
+    bulk_wait<0>();  // every record image has left shared memory
+  }
   if (warp == 0) tmem_dealloc(tbase, kPrepTmemCols);
 }
 

@@ -141,7 +141,7 @@ __device__ __forceinline__ void chunk_gates(const Dims& d, const float* __restri
 
 constexpr int kConvThreads = 32 * (kConvGateWarp + 1);
 
-__global__ void __launch_bounds__(kConvThreads)
+__global__ void __launch_bounds__(kConvThreads, 4)
     conv_qkv_kernel(Dims d, const float* __restrict__ conv_w, const __nv_bfloat16* __restrict__ qkv,
                     const __nv_bfloat16* __restrict__ hist, int zero_conv, const int4* __restrict__ chunk_map,
                     const float* __restrict__ norm_w, const __nv_bfloat16* __restrict__ z,

@@ -224,7 +224,10 @@ int32_t sched_rows(Path p, int32_t chunk_size) { return p == Path::Wy ? gdn::wy_
 size_t prefill_ws_bytes(const gdn::Dims& d, Path p, int64_t total_tokens, int32_t num_seqs, int32_t chunk_size) {
   const int64_t chunks = chunk_bound(total_tokens, num_seqs, sched_rows(p, chunk_size));
   const size_t sched = gdn::schedule_layout(num_seqs, chunks).total_bytes;
-  if (p == Path::Split) return sched + gdn::split_layout(d, total_tokens, chunks).total_bytes;
+  if (p == Path::Split) {  // one window of chunks at a time
+    const int64_t w = gdn::split_window_chunks(chunks);
+    return sched + gdn::split_layout(d, std::min<int64_t>(total_tokens, w * chunk_size), w).total_bytes;
+  }
   if (p == Path::Wy) return sched + gdn::wy_layout(d, total_tokens, chunks, chunk_size).total_bytes;
   return sched;
 }
@@ -481,7 +484,7 @@ gdn_status gdn_prefill(const gdn_config* cfg, const gdn_params* params, const vo
                                (char*)workspace + sched, g_status_ptr[dev], st);
   } else if (e == cudaSuccess && path == Path::Split) {
     e = gdn::launch_prefill_split(d, params->conv_w, params->A_log, params->dt_bias, params->norm_w, qkv, z, a, b,
-                                  cu_seqlens_dev, order,
+                                  cu_seqlens_dev, cu_seqlens_host, order,
                                   num_seqs > 1 ? (const int32_t*)((const char*)workspace + L.chunk_off_off) : nullptr,
                                   num_seqs > 1 ? (const int4*)((const char*)workspace + L.chunk_map_off) : nullptr,
                                   num_seqs, total, chunks,

@@ -77,12 +77,16 @@ struct SplitLayout {
   size_t qk_hi, qk_lo, records, total_bytes;
 };
 SplitLayout split_layout(const Dims& d, int64_t total_tokens, int64_t chunk_bound);
+// the chunks go through conv, prep and chain in windows of at most this many chunks (16384 tokens), so the
+// workspace holds the intermediates of one window: split_layout(d, min(T, window * 64), window)
+constexpr int64_t kSplitWindowChunks = 256;
+int64_t split_window_chunks(int64_t total_chunks);
 cudaError_t launch_prefill_split(const Dims& d, const float* conv_w, const float* A_log, const float* dt_bias,
                                  const float* norm_w, const void* qkv, const void* z, const void* a, const void* b,
-                                 const int32_t* cu, const int32_t* order, const int32_t* chunk_off,
-                                 const int4* chunk_map, int32_t N, int64_t total_tokens, int64_t total_chunks,
-                                 bool zero_state, bool zero_conv, const void* conv_state, float* state, void* o,
-                                 void* split_ws, int32_t* status, cudaStream_t stream);
+                                 const int32_t* cu, const int32_t* cu_host, const int32_t* order,
+                                 const int32_t* chunk_off, const int4* chunk_map, int32_t N, int64_t total_tokens,
+                                 int64_t total_chunks, bool zero_state, bool zero_conv, const void* conv_state,
+                                 float* state, void* o, void* split_ws, int32_t* status, cudaStream_t stream);
 
 // prefill_split.cu, sequence-parallel chain (one sequence, P chunk-aligned segments): segment count for a
 // request (0 = from the SM count), workspace layout, launch

@@ -141,6 +141,14 @@ __device__ __forceinline__ void chunk_gates(const Dims& d, const float* __restri
 
 constexpr int kConvThreads = 32 * (kConvGateWarp + 1);
 
+// A window of the packed chunks handled by one conv + prep + chain pass: global chunks [g_base, g_base + the
+// grid's chunk count), whose records start at record 0 of the window's buffer and whose q^/k^ rows start at
+// row 0 of the window's hi and lo buffers (token t_base).
+struct Window {
+  int64_t g_base;
+  int64_t t_base;
+};
+
 __global__ void __launch_bounds__(kConvThreads, 4)
     conv_qkv_kernel(Dims d, const float* __restrict__ conv_w, const __nv_bfloat16* __restrict__ qkv,
                     const __nv_bfloat16* __restrict__ hist, int zero_conv, const int4* __restrict__ chunk_map,
@@ -148,9 +156,10 @@ __global__ void __launch_bounds__(kConvThreads, 4)
                     const float* __restrict__ A_log, const float* __restrict__ dt_bias,
                     const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
                     __half* __restrict__ qk_hi, __half* __restrict__ qk_lo, unsigned char* __restrict__ records,
-                    int64_t single_len) {
+                    int64_t single_len, Window win) {
   // chunks in reverse order: the first chunks' outputs are the freshest in L2 when the chain starts
-  const int g = gridDim.x - 1 - blockIdx.x;
+  const int g = (int)(win.g_base + gridDim.x - 1 - blockIdx.x);
+  const int64_t gw = g - win.g_base;  // the chunk's record in the window
   // {seq, first token, length, chunk index}; one sequence needs no map
   const int64_t rest = single_len - (int64_t)kC * g;
   const int4 cm = chunk_map ? chunk_map[g] : make_int4(0, kC * g, rest < kC ? (int)rest : kC, g);
@@ -161,14 +170,14 @@ __global__ void __launch_bounds__(kConvThreads, 4)
   const int nqk = 2 * d.Hk;
   if (slot >= nqk + d.Hv) {
     const int hz = slot - nqk - d.Hv;
-    unsigned char* rec = records + ((int64_t)g * d.Hv + hz) * kRec;
+    unsigned char* rec = records + (gw * d.Hv + hz) * kRec;
     if (warp == kConvGateWarp) chunk_gates(d, A_log, dt_bias, a, b, cm.y, L, hz, lane, rec);
     else if (r0 < L) gate_rows(d, norm_w, z, rec + REC_G, cm.y, r0, L, hz, lane);
     return;
   }
   if (warp == kConvGateWarp) return;
   // v^ goes straight into the record of (chunk, value head) as the chain kernel's operand image
-  unsigned char* vrec = slot >= nqk ? records + ((int64_t)g * d.Hv + (slot - nqk)) * kRec + REC_V : nullptr;
+  unsigned char* vrec = slot >= nqk ? records + (gw * d.Hv + (slot - nqk)) * kRec + REC_V : nullptr;
   if (vrec) {
 #pragma unroll
     for (int i = 0; i < kConvRows; ++i)
@@ -237,7 +246,7 @@ __global__ void __launch_bounds__(kConvThreads, 4)
           hi[e] = __half2float(__float2half_rn(v));
           lo[e] = v - hi[e];
         }
-        const int64_t off = ((int64_t)cm.y + r0 + i) * W2 + c;
+        const int64_t off = ((int64_t)cm.y + r0 + i - win.t_base) * W2 + c;
         st8(reinterpret_cast<unsigned char*>(qk_hi + off), hi[0], hi[1], hi[2], hi[3]);
         st8(reinterpret_cast<unsigned char*>(qk_lo + off), lo[0], lo[1], lo[2], lo[3]);
       }
@@ -311,7 +320,7 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
     prep_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constant__ CUtensorMap tm_lo, Dims d,
                 const int4* __restrict__ chunk_map, unsigned char* __restrict__ records, const int32_t* __restrict__ cu,
                 const __nv_bfloat16* __restrict__ qkv, int zero_conv, __nv_bfloat16* __restrict__ hist,
-                int64_t single_len, int32_t* status) {
+                int64_t single_len, Window win, int32_t* status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   __shared__ uint64_t mb_tma, mb_mma, mb_v, mb_vl;
@@ -321,7 +330,7 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gr = blockIdx.x / d.Hv;  // chunks in reverse order, as in conv_qkv_kernel
   const int h = blockIdx.x - gr * d.Hv;
-  const int g = gridDim.x / d.Hv - 1 - gr;
+  const int g = (int)(win.g_base + gridDim.x / d.Hv - 1 - gr);
   const int kh = h / d.G;
   const int4 cm = chunk_map ? chunk_map[g] : make_int4(0, kC * g, 0, g);
   const int64_t t0 = cm.y;  // rows past the chunk's end carry beta = 0 (their gates are zero)
@@ -329,7 +338,8 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
     const int64_t s0 = chunk_map ? cu[cm.x] : 0, s1 = chunk_map ? cu[cm.x + 1] : single_len;
     if (t0 + kC >= s1) write_history(d, h, cm.x, s0, (int)(s1 - s0), qkv, zero_conv, hist);
   }
-  unsigned char* rec = records + ((int64_t)g * d.Hv + h) * kRec;
+  unsigned char* rec = records + ((g - win.g_base) * d.Hv + h) * kRec;
+  const int trow = (int)(t0 - win.t_base);  // the chunk's first row in the window's q^/k^ buffers
 
   float* misc = reinterpret_cast<float*>(sm + P_MISC);
   float* s_gam = misc;
@@ -350,10 +360,10 @@ __global__ void __launch_bounds__(kPrepThreads, 3)
     const int qx = kh * kD, kx = d.Hk * kD + kh * kD;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-      tma_load_2d(sm + P_KQ + j * 16384, &tm_hi, kx + 64 * j, (int)t0, &mb_tma);
-      tma_load_2d(sm + P_KQ + j * 16384 + 8192, &tm_hi, qx + 64 * j, (int)t0, &mb_tma);
-      tma_load_2d(sm + P_KQL + j * 16384, &tm_lo, kx + 64 * j, (int)t0, &mb_tma);
-      tma_load_2d(sm + P_KQL + j * 16384 + 8192, &tm_lo, qx + 64 * j, (int)t0, &mb_tma);
+      tma_load_2d(sm + P_KQ + j * 16384, &tm_hi, kx + 64 * j, trow, &mb_tma);
+      tma_load_2d(sm + P_KQ + j * 16384 + 8192, &tm_hi, qx + 64 * j, trow, &mb_tma);
+      tma_load_2d(sm + P_KQL + j * 16384, &tm_lo, kx + 64 * j, trow, &mb_tma);
+      tma_load_2d(sm + P_KQL + j * 16384 + 8192, &tm_lo, qx + 64 * j, trow, &mb_tma);
     }
   }
   if (warp == 0) tmem_alloc(&tslot, kPrepTmemCols);
@@ -714,6 +724,8 @@ constexpr int kChainThreads = 320;  // eight compute warps, the MMA-issuing warp
 struct ChainScan {
   int32_t nseg;         // > 0: segmented use (see chain_kernel)
   int32_t zero_u_from;  // first cluster-pair index whose U is taken as zero
+  int32_t win_lo = 0;   // the window of global chunks [win_lo, win_hi) whose records `records` holds,
+  int32_t win_hi = 0x7fffffff;  // record 0 being chunk win_lo's
 };
 constexpr int C_A = 0;          // [-W ; Qg]   K-major 128 x 128; buffer cc % 2 at +32768 (cc % 2)
 constexpr int C_P = 65536;      // [0 ; P]     K-major 128 x 64 (8 KB of zero rows, then P); buffer at +16384 (cc % 2)
@@ -765,8 +777,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
   const int64_t seq0 = cu[n];
   const int len = cu[n + 1] - cu[n];
   if (len <= 0) return;  // both CTAs of the cluster, before any cluster barrier
-  const int nchunks = (len + kC - 1) / kC;
-  const int64_t g0 = chunk_off ? chunk_off[n] : 0;
+  // the sequence's chunks inside the window: local chunks cc0 .. cc0 + nchunks - 1; the state carries in from
+  // the previous window (or from zero at the sequence's first chunk) and out to the next
+  const int64_t gfirst = chunk_off ? chunk_off[n] : 0;
+  const int64_t ga = max(gfirst, (int64_t)scan.win_lo), gb = min(gfirst + (len + kC - 1) / kC, (int64_t)scan.win_hi);
+  if (ga >= gb) return;  // both CTAs of the cluster, before any cluster barrier
+  const int cc0 = (int)(ga - gfirst);
+  const int nchunks = (int)(gb - ga);
+  const int64_t g0 = ga - scan.win_lo;  // record of the window's first chunk of this sequence
+  const bool zero_here = zero_state && cc0 == 0;
   const int64_t HvD = (int64_t)d.Hv * kD;
   float* s_rms = reinterpret_cast<float*>(sm + C_MISC);         // [2][64], this CTA's column quarters
   float* s_peer = reinterpret_cast<float*>(sm + C_MISC) + 128;  // [2][64], written by the peer
@@ -838,7 +857,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
   };
   if (compute) {
 #pragma unroll
-    for (int jj = 0; jj < 32; ++jj) S[jj] = zero_state ? 0.f : gst[(int64_t)(c0 + jj) * kD + si];
+    for (int jj = 0; jj < 32; ++jj) S[jj] = zero_here ? 0.f : gst[(int64_t)(c0 + jj) * kD + si];
     store_s();
   }
   fence_async_smem();
@@ -872,7 +891,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
   // between, which it does after reading it.
   auto epilogue = [&](int cc) {
     const int r = si - 64;
-    const int Lc = min(kC, len - cc * kC);
+    const int Lc = min(kC, len - (cc0 + cc) * kC);
     if (!mbar_wait(&mb_m4[cc & 1], (cc >> 1) & 1, kWaitNs)) bad = true;
     fence_after();
     float v[32], vl[32];
@@ -917,7 +936,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
       const int rr = 8 * it + (lane >> 2), q = lane & 3;
       if (rbase + rr < Lc) {
         const uint4 val = *reinterpret_cast<const uint4*>(stage + rr * 64 + ((q ^ ((rr >> 1) & 3)) << 4));
-        *reinterpret_cast<uint4*>(o + (seq0 + (int64_t)cc * kC + rbase + rr) * HvD + (int64_t)h * kD + c0 + 8 * q) = val;
+        *reinterpret_cast<uint4*>(o + (seq0 + (int64_t)(cc0 + cc) * kC + rbase + rr) * HvD + (int64_t)h * kD + c0 + 8 * q) =
+            val;
       }
     }
     __syncwarp();
@@ -1065,38 +1085,39 @@ SplitLayout split_layout(const Dims& d, int64_t total_tokens, int64_t chunk_boun
 namespace {
 
 // conv + prep over the packed tokens: the per-token parts and the record of every (chunk, value head)
+// conv + prep over one window of the packed chunks (see Window): the per-token parts and the record of every
+// (chunk, value head) of the window, in the buffers of layout S (sized for the largest window)
 cudaError_t launch_stages12(const Dims& d, const float* conv_w, const float* A_log, const float* dt_bias,
                             const float* norm_w, const void* qkv, const void* z, const void* a, const void* b,
-                            const int32_t* cu, const int4* chunk_map, int64_t total_tokens, int64_t total_chunks,
-                            bool zero_conv, const void* conv_state, void* split_ws, int32_t* status,
-                            cudaStream_t stream) {
+                            const int32_t* cu, const int4* chunk_map, int64_t total_tokens, Window win,
+                            int64_t win_chunks, int64_t win_tokens, const SplitLayout& S, bool zero_conv,
+                            const void* conv_state, void* split_ws, int32_t* status, cudaStream_t stream) {
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return cudaErrorNotSupported;
-  const SplitLayout S = split_layout(d, total_tokens, total_chunks);
   unsigned char* ws = (unsigned char*)split_ws;
   __half* qk_hi = (__half*)(ws + S.qk_hi);
   __half* qk_lo = (__half*)(ws + S.qk_lo);
   unsigned char* records = ws + S.records;
   CUtensorMap tm_hi, tm_lo;
   const uint64_t qkw = (uint64_t)2 * d.Hk * kD;
-  if (!encode_2d(enc, &tm_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, qk_hi, qkw, total_tokens) ||
-      !encode_2d(enc, &tm_lo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, qk_lo, qkw, total_tokens))
+  if (!encode_2d(enc, &tm_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, qk_hi, qkw, win_tokens) ||
+      !encode_2d(enc, &tm_lo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, qk_lo, qkw, win_tokens))
     return cudaErrorInvalidValue;
   cudaError_t e;
   {
     LaunchScope scope(GDN_K_SPLIT_CONV, stream);
-    conv_qkv_kernel<<<dim3((unsigned)total_chunks, (unsigned)(2 * d.Hk + 2 * d.Hv)), kConvThreads, 0, stream>>>(
+    conv_qkv_kernel<<<dim3((unsigned)win_chunks, (unsigned)(2 * d.Hk + 2 * d.Hv)), kConvThreads, 0, stream>>>(
         d, conv_w, (const __nv_bfloat16*)qkv, (const __nv_bfloat16*)conv_state, zero_conv ? 1 : 0, chunk_map, norm_w,
         (const __nv_bfloat16*)z, A_log, dt_bias, (const __nv_bfloat16*)a, (const __nv_bfloat16*)b, qk_hi, qk_lo,
-        records, total_tokens);
+        records, total_tokens, win);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if ((e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrepSmem)) != cudaSuccess)
     return e;
   LaunchScope scope(GDN_K_SPLIT_PREP, stream);
-  prep_kernel<<<(unsigned)(total_chunks * d.Hv), kPrepThreads, kPrepSmem, stream>>>(
+  prep_kernel<<<(unsigned)(win_chunks * d.Hv), kPrepThreads, kPrepSmem, stream>>>(
       tm_hi, tm_lo, d, chunk_map, records, cu, (const __nv_bfloat16*)qkv, zero_conv ? 1 : 0,
-      (__nv_bfloat16*)const_cast<void*>(conv_state), total_tokens, status);
+      (__nv_bfloat16*)const_cast<void*>(conv_state), total_tokens, win, status);
   return cudaGetLastError();
 }
 
@@ -1113,19 +1134,49 @@ cudaError_t launch_chain(const Dims& d, const unsigned char* records, const int3
 
 }  // namespace
 
+int64_t split_window_chunks(int64_t total_chunks) { return total_chunks < kSplitWindowChunks ? total_chunks
+                                                                                            : kSplitWindowChunks; }
+
 cudaError_t launch_prefill_split(const Dims& d, const float* conv_w, const float* A_log, const float* dt_bias,
                                  const float* norm_w, const void* qkv, const void* z, const void* a, const void* b,
-                                 const int32_t* cu, const int32_t* order, const int32_t* chunk_off,
-                                 const int4* chunk_map, int32_t N, int64_t total_tokens, int64_t total_chunks,
-                                 bool zero_state, bool zero_conv, const void* conv_state, float* state, void* o,
-                                 void* split_ws, int32_t* status, cudaStream_t stream) {
+                                 const int32_t* cu, const int32_t* cu_host, const int32_t* order,
+                                 const int32_t* chunk_off, const int4* chunk_map, int32_t N, int64_t total_tokens,
+                                 int64_t total_chunks, bool zero_state, bool zero_conv, const void* conv_state,
+                                 float* state, void* o, void* split_ws, int32_t* status, cudaStream_t stream) {
   if (N <= 0 || total_tokens <= 0 || total_chunks <= 0) return cudaSuccess;
-  cudaError_t e = launch_stages12(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, cu, chunk_map, total_tokens,
-                                  total_chunks, zero_conv, conv_state, split_ws, status, stream);
-  if (e != cudaSuccess) return e;
-  const unsigned char* records = (unsigned char*)split_ws + split_layout(d, total_tokens, total_chunks).records;
-  return launch_chain(d, records, chunk_off, order, cu, (int64_t)N * d.Hv, zero_state, ChainScan{0, 0x7fffffff},
-                      state, o, status, stream);
+  // The chunks go through conv, prep and the chain one window at a time, so that the intermediates take a
+  // bounded workspace whatever the length; the chain carries each sequence's state from window to window
+  // through `state` (a sequence starts from zero only in the window that holds its first chunk).
+  const int64_t W = split_window_chunks(total_chunks);
+  const SplitLayout S = split_layout(d, std::min<int64_t>(total_tokens, W * kC), W);
+  const unsigned char* records = (unsigned char*)split_ws + S.records;
+  // first token of chunk g (chunks are numbered sequence by sequence in id order)
+  int32_t n = 0;
+  int64_t n_first_chunk = 0;
+  auto chunk_token = [&](int64_t g) -> int64_t {
+    if (N == 1 || !cu_host) return kC * g;
+    while (n < N) {
+      const int64_t nch = (cu_host[n + 1] - cu_host[n] + kC - 1) / kC;
+      if (g < n_first_chunk + nch) return cu_host[n] + kC * (g - n_first_chunk);
+      n_first_chunk += nch;
+      ++n;
+    }
+    return total_tokens;
+  };
+  cudaError_t e = cudaSuccess;
+  for (int64_t g0 = 0; g0 < total_chunks && e == cudaSuccess; g0 += W) {
+    const int64_t g1 = std::min<int64_t>(g0 + W, total_chunks);
+    const int64_t t0 = chunk_token(g0), t1 = g1 < total_chunks ? chunk_token(g1) : total_tokens;
+    e = launch_stages12(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, cu, chunk_map, total_tokens,
+                        Window{g0, t0}, g1 - g0, t1 - t0, S, zero_conv, conv_state, split_ws, status, stream);
+    if (e != cudaSuccess) break;
+    ChainScan scan{0, 0x7fffffff};
+    scan.win_lo = (int32_t)g0;
+    scan.win_hi = (int32_t)g1;
+    e = launch_chain(d, records, chunk_off, order, cu, (int64_t)N * d.Hv, zero_state, scan, state, o, status,
+                     stream);
+  }
+  return e;
 }
 
 // ------------------------------------------------------------------ sequence-parallel chain
@@ -1257,8 +1308,9 @@ cudaError_t launch_prefill_seqpar(const Dims& d, const float* conv_w, const floa
         (int32_t)total_tokens, P, seg_chunks, d.Hv, cu1, cu_seg, coff, s1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  if ((e = launch_stages12(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, cu1, nullptr, total_tokens, nchunks,
-                           zero_conv, conv_state, w + L.split, status, stream)) != cudaSuccess)
+  if ((e = launch_stages12(d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, cu1, nullptr, total_tokens, Window{0, 0},
+                           nchunks, total_tokens, split_layout(d, total_tokens, nchunks), zero_conv, conv_state,
+                           w + L.split, status, stream)) != cudaSuccess)
     return e;
   const unsigned char* records = w + L.split + split_layout(d, total_tokens, nchunks).records;
   if (P == 1)  // the ordinary carry over the whole sequence

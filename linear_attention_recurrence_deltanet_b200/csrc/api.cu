@@ -228,7 +228,11 @@ size_t prefill_ws_bytes(const gdn::Dims& d, Path p, int64_t total_tokens, int32_
     const int64_t w = gdn::split_window_chunks(chunks);
     return sched + gdn::split_layout(d, std::min<int64_t>(total_tokens, w * chunk_size), w).total_bytes;
   }
-  if (p == Path::Wy) return sched + gdn::wy_layout(d, total_tokens, chunks, chunk_size).total_bytes;
+  if (p == Path::Wy) {  // one window of tiles at a time
+    const int64_t w = gdn::wy_window_tiles(chunks, chunk_size);
+    return sched + gdn::wy_layout(d, std::min<int64_t>(total_tokens, w * gdn::wy_tile(chunk_size)), w, chunk_size)
+                       .total_bytes;
+  }
   return sched;
 }
 
@@ -477,7 +481,7 @@ gdn_status gdn_prefill(const gdn_config* cfg, const gdn_params* params, const vo
   const size_t sched = gdn::schedule_layout(num_seqs, chunk_bound(total, num_seqs, rows)).total_bytes;
   if (e == cudaSuccess && path == Path::Wy) {
     e = gdn::launch_prefill_wy(d, chunk_size, params->conv_w, params->A_log, params->dt_bias, params->norm_w, qkv,
-                               z, a, b, cu_seqlens_dev, order,
+                               z, a, b, cu_seqlens_dev, cu_seqlens_host, order,
                                num_seqs > 1 ? (const int32_t*)((const char*)workspace + L.chunk_off_off) : nullptr,
                                num_seqs > 1 ? (const int4*)((const char*)workspace + L.chunk_map_off) : nullptr,
                                num_seqs, total, chunks, zero_state, zero_conv, conv_state, state, o,

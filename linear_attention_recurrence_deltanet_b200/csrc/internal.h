@@ -153,9 +153,14 @@ struct WyLayout {
   size_t qk_hi, qk_lo, vimg, gate, records, total_bytes;
 };
 WyLayout wy_layout(const Dims& d, int64_t total_tokens, int64_t tile_bound, int chunk_size);
+// the tiles go through conv, prep and chain in windows of at most kWyWindowTokens / tile rows, so the
+// workspace holds one window: wy_layout(d, min(T, window * tile), window, chunk)
+constexpr int64_t kWyWindowTokens = 16384;
+int64_t wy_window_tiles(int64_t total_tiles, int chunk_size);
 cudaError_t launch_prefill_wy(const Dims& d, int chunk_size, const float* conv_w, const float* A_log,
                               const float* dt_bias, const float* norm_w, const void* qkv, const void* z,
-                              const void* a, const void* b, const int32_t* cu, const int32_t* order,
+                              const void* a, const void* b, const int32_t* cu, const int32_t* cu_host,
+                              const int32_t* order,
                               const int32_t* tile_off, const int4* tile_map, int32_t N, int64_t total_tokens,
                               int64_t total_tiles, bool zero_state, bool zero_conv, const void* conv_state,
                               float* state, void* o, void* ws, int32_t* status, cudaStream_t stream);

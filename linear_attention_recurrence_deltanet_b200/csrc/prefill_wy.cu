@@ -81,6 +81,14 @@ struct Rec {
   static constexpr int BYTES = META + 256;
 };
 
+// A window of the packed tiles handled by one conv + prep + chain pass: global tiles [win_lo, win_hi), whose
+// records and v^ images start at entry 0 of the window's buffers and whose per-token parts (q^/k^ rows, gate
+// rows) start at row 0 of theirs (token t_base).
+struct WyWin {
+  int64_t win_lo, win_hi;
+  int64_t t_base;
+};
+
 // v^ image of one (tile, value head): hi then lo, each MN-major K=TILE x N=128
 template <int TILE>
 constexpr int kVImg = TILE * 512;
@@ -97,9 +105,10 @@ __global__ void __launch_bounds__(256)
                    const __nv_bfloat16* __restrict__ hist, int zero_conv, const int4* __restrict__ tile_map,
                    int64_t single_len, __half* __restrict__ qk_hi, __half* __restrict__ qk_lo,
                    unsigned char* __restrict__ vimg, const float* __restrict__ norm_w,
-                   const __nv_bfloat16* __restrict__ z, __half* __restrict__ gate) {
+                   const __nv_bfloat16* __restrict__ z, __half* __restrict__ gate, WyWin win) {
   constexpr int SUB = TILE / 64;
-  const int gt = blockIdx.x / SUB, part = blockIdx.x - gt * SUB;
+  const int part = blockIdx.x % SUB;
+  const int gt = (int)(win.win_lo + blockIdx.x / SUB);
   const int64_t rest = single_len - (int64_t)TILE * gt;
   const int4 cm = tile_map ? tile_map[gt] : make_int4(0, TILE * gt, rest < TILE ? (int)rest : TILE, gt);
   const int slot = blockIdx.y;
@@ -124,12 +133,12 @@ __global__ void __launch_bounds__(256)
         float g[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) g[e] = nw[e] * __fdividef(1.0f, 1.0f + __expf(-zz[e]));
-        st8(reinterpret_cast<unsigned char*>(gate + (cm.y + r0 + i) * HvD + col), g[0], g[1], g[2], g[3]);
+        st8(reinterpret_cast<unsigned char*>(gate + (cm.y + r0 + i - win.t_base) * HvD + col), g[0], g[1], g[2], g[3]);
       }
     }
     return;
   }
-  unsigned char* vrec = slot >= nqk ? vimg + ((int64_t)gt * d.Hv + (slot - nqk)) * kVImg<TILE> : nullptr;
+  unsigned char* vrec = slot >= nqk ? vimg + ((gt - win.win_lo) * d.Hv + (slot - nqk)) * kVImg<TILE> : nullptr;
   if (vrec) {  // rows past the tile's end are zero in both parts
 #pragma unroll
     for (int i = 0; i < kConvRows; ++i)
@@ -198,7 +207,7 @@ __global__ void __launch_bounds__(256)
           hi[e] = __half2float(__float2half_rn(v));
           lo[e] = v - hi[e];
         }
-        const int64_t off = ((int64_t)cm.y + r0 + i) * W2 + c;
+        const int64_t off = ((int64_t)cm.y + r0 + i - win.t_base) * W2 + c;
         st8(reinterpret_cast<unsigned char*>(qk_hi + off), hi[0], hi[1], hi[2], hi[3]);
         st8(reinterpret_cast<unsigned char*>(qk_lo + off), lo[0], lo[1], lo[2], lo[3]);
       }
@@ -304,7 +313,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
                    const __nv_bfloat16* __restrict__ qkv, int zero_conv, __nv_bfloat16* __restrict__ hist,
                    const float* __restrict__ A_log, const float* __restrict__ dt_bias,
                    const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b, int64_t single_len,
-                   int32_t* status) {
+                   WyWin win, int32_t* status) {
   constexpr int TILE = 64;
   using R = Rec<TILE, C>;
   constexpr int NCH = R::NCH;
@@ -317,13 +326,15 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gr = blockIdx.x / d.Hv;  // tiles in reverse order: the first tiles are the freshest in L2 for the chain
   const int h = blockIdx.x - gr * d.Hv;
-  const int g = gridDim.x / d.Hv - 1 - gr;
+  const int g = (int)(win.win_lo + gridDim.x / d.Hv - 1 - gr);
   const int kh = h / d.G;
   const int64_t rest = single_len - (int64_t)TILE * g;
   const int4 cm = tile_map ? tile_map[g] : make_int4(0, TILE * g, rest < TILE ? (int)rest : TILE, g);
   const int64_t t0 = cm.y;
+  const int trow = (int)(t0 - win.t_base);  // the tile's first row in the window's q^/k^ buffers
   const int L = cm.z;
-  unsigned char* rec = records + ((int64_t)g * d.Hv + h) * R::BYTES;
+  const int64_t gw = g - win.win_lo;  // the tile's entry in the window's buffers
+  unsigned char* rec = records + (gw * d.Hv + h) * R::BYTES;
 
   float* misc = reinterpret_cast<float*>(sm + WP_MISC);
   float* s_g = misc;            // g_r, then gamma_r (in-chunk inclusive sum)
@@ -342,12 +353,12 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     const int qx = kh * kD, kx = d.Hk * kD + kh * kD;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-      tma_load_2d(sm + WP_KQH + j * 16384, &tm_hi, kx + 64 * j, (int)t0, &mb_tma);
-      tma_load_2d(sm + WP_KQH + j * 16384 + 8192, &tm_hi, qx + 64 * j, (int)t0, &mb_tma);
-      tma_load_2d(sm + WP_KQL + j * 16384, &tm_lo, kx + 64 * j, (int)t0, &mb_tma);
-      tma_load_2d(sm + WP_KQL + j * 16384 + 8192, &tm_lo, qx + 64 * j, (int)t0, &mb_tma);
+      tma_load_2d(sm + WP_KQH + j * 16384, &tm_hi, kx + 64 * j, trow, &mb_tma);
+      tma_load_2d(sm + WP_KQH + j * 16384 + 8192, &tm_hi, qx + 64 * j, trow, &mb_tma);
+      tma_load_2d(sm + WP_KQL + j * 16384, &tm_lo, kx + 64 * j, trow, &mb_tma);
+      tma_load_2d(sm + WP_KQL + j * 16384 + 8192, &tm_lo, qx + 64 * j, trow, &mb_tma);
     }
-    bulk_load(sm + WP_V, vimg + ((int64_t)g * d.Hv + h) * kVImg<TILE>, 16384, &mb_tma);
+    bulk_load(sm + WP_V, vimg + (gw * d.Hv + h) * kVImg<TILE>, 16384, &mb_tma);
   }
   if (warp == 0) tmem_alloc(&tslot, kPrepTmemCols);
   {  // the block of a sequence's last tile writes the sequence's new conv history for its channels
@@ -471,7 +482,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
   if (tid == 0) {  // v^ lo into the Q halves of KQH (MN-major, LBO 16 KB), behind the generic reads of q^
     fence_async_smem();
     mbar_expect_tx(&mb_vlo, 16384);
-    const unsigned char* vl = vimg + ((int64_t)g * d.Hv + h) * kVImg<TILE> + TILE * 256;
+    const unsigned char* vl = vimg + (gw * d.Hv + h) * kVImg<TILE> + TILE * 256;
     bulk_load(sm + WP_VLO, vl, 8192, &mb_vlo);
     bulk_load(sm + WP_VLO + 16384, vl + 8192, 8192, &mb_vlo);
     bulk_store(rec + R::KT, sm + WP_KT, 16384);  // the K~ image goes to the record as it is
@@ -847,7 +858,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
                       const __nv_bfloat16* __restrict__ qkv, int zero_conv, __nv_bfloat16* __restrict__ hist,
                       const float* __restrict__ A_log, const float* __restrict__ dt_bias,
                       const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b, int64_t single_len,
-                      int32_t* status) {
+                      WyWin win, int32_t* status) {
   constexpr int TILE = 128;
   using R = Rec<128, 128>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -859,14 +870,16 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gr = blockIdx.x / d.Hv;
   const int h = blockIdx.x - gr * d.Hv;
-  const int g = gridDim.x / d.Hv - 1 - gr;
+  const int g = (int)(win.win_lo + gridDim.x / d.Hv - 1 - gr);
   const int kh = h / d.G;
   const int64_t rest = single_len - (int64_t)TILE * g;
   const int4 cm = tile_map ? tile_map[g] : make_int4(0, TILE * g, rest < TILE ? (int)rest : TILE, g);
   const int64_t t0 = cm.y;
+  const int trow = (int)(t0 - win.t_base);  // the tile's first row in the window's q^/k^ buffers
   const int L = cm.z;
-  unsigned char* rec = records + ((int64_t)g * d.Hv + h) * R::BYTES;
-  const unsigned char* vsrc = vimg + ((int64_t)g * d.Hv + h) * kVImg<TILE>;
+  const int64_t gw = g - win.win_lo;  // the tile's entry in the window's buffers
+  unsigned char* rec = records + (gw * d.Hv + h) * R::BYTES;
+  const unsigned char* vsrc = vimg + (gw * d.Hv + h) * kVImg<TILE>;
 
   float* misc = reinterpret_cast<float*>(sm + W8_MISC);
   float* s_g = misc;
@@ -888,7 +901,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
     for (int j = 0; j < 2; ++j)
 #pragma unroll
       for (int rh = 0; rh < 2; ++rh) {  // 64-column block j, 64-row half rh
-        const int y = (int)t0 + 64 * rh, o = j * 16384 + rh * 8192;
+        const int y = trow + 64 * rh, o = j * 16384 + rh * 8192;
         tma_load_2d(sm + W8_KH + o, &tm_hi, kx + 64 * j, y, &mb_tma);
         tma_load_2d(sm + W8_KL + o, &tm_lo, kx + 64 * j, y, &mb_tma);
         tma_load_2d(sm + W8_QH + o, &tm_hi, qx + 64 * j, y, &mb_tma);
@@ -1355,7 +1368,7 @@ template <int TILE, int C>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
     wy_chain_kernel(Dims d, const unsigned char* __restrict__ records,
                     const int32_t* __restrict__ tile_off, const int32_t* __restrict__ order,
-                    const int32_t* __restrict__ cu, int zero_state, const __half* __restrict__ gate,
+                    const int32_t* __restrict__ cu, int zero_state, const __half* __restrict__ gate, WyWin win,
                     float* __restrict__ state, __nv_bfloat16* __restrict__ o, int32_t* status) {
   using R = Rec<TILE, C>;
   using F = ChainCfg<TILE, C>;
@@ -1379,12 +1392,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
   const int pair = blockIdx.x >> 1;
   const int h = pair % d.Hv;
   const int n = order ? order[pair / d.Hv] : pair / d.Hv;
-  const int64_t seq0 = cu[n];
-  const int len = cu[n + 1] - cu[n];
-  if (len <= 0) return;  // both CTAs of the cluster, before any cluster barrier
+  const int len_all = cu[n + 1] - cu[n];
+  if (len_all <= 0) return;  // both CTAs of the cluster, before any cluster barrier
+  // the sequence's tiles inside the window; the state carries in from the previous window (or from zero at
+  // the sequence's first tile) and out to the next
+  const int64_t gfirst = tile_off ? tile_off[n] : 0, win_lo = win.win_lo, t_base = win.t_base;
+  const int64_t ga = max(gfirst, win_lo), gb = min(gfirst + (len_all + TILE - 1) / TILE, (int64_t)win.win_hi);
+  if (ga >= gb) return;  // both CTAs of the cluster, before any cluster barrier
+  const int tile0 = (int)(ga - gfirst);
+  const int64_t seq0 = cu[n] + (int64_t)tile0 * TILE;                   // this window's first token of the sequence
+  const int len = min(len_all - tile0 * TILE, (int)(gb - ga) * TILE);   // and its number of tokens here
   const int ntiles = (len + TILE - 1) / TILE;
   const int nsteps = (len + C - 1) / C;
-  const int64_t g0 = tile_off ? tile_off[n] : 0;
+  const int64_t g0 = ga - win_lo;
+  // with several windows a zero start is written into `state` before the first one, so zero_state is only
+  // set when the whole sequence is in this window
+  const bool zero_here = zero_state;
   const int64_t HvD = (int64_t)d.Hv * kD;
   const bool state_warp = warp < 8, out_warp = warp >= 8 && warp < 12, mma_warp = warp == 12,
              copy_warp = warp == 13, early_warp = warp == 14;
@@ -1436,7 +1459,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
   const int c0 = 64 * vh + 32 * hc;  // first value channel of a state thread's columns
   if (state_warp) {
 #pragma unroll
-    for (int jj = 0; jj < 32; ++jj) S[jj] = zero_state ? 0.f : gst[(int64_t)(c0 + jj) * kD + si];
+    for (int jj = 0; jj < 32; ++jj) S[jj] = zero_here ? 0.f : gst[(int64_t)(c0 + jj) * kD + si];
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       float lo[8];
@@ -1584,10 +1607,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
     // the gate row (128 bytes) of this thread's row of chunk c: prefetched into L2 a few chunks ahead
     // (a plain per-row prefetch: nothing asynchronous outlives the block), loaded one chunk ahead
     constexpr int kGAhead = 3;
+    const __half* gate_r = gate + (seq0 - t_base + r) * HvD + (int64_t)h * kD + 64 * vh;  // row r of tile 0
     auto gate_row = [&](int c) -> const __half* {
       const int t = c / NCH, s = c % NCH;
-      if (c < nsteps && has_row && (r / C) == s && (t * TILE + r) < len)
-        return gate + (seq0 + (int64_t)t * TILE + r) * HvD + (int64_t)h * kD + 64 * vh;
+      if (c < nsteps && has_row && (r / C) == s && (t * TILE + r) < len) return gate_r + (int64_t)t * TILE * HvD;
       return nullptr;
     };
     uint4 gr[8];
@@ -1607,19 +1630,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
       const bool valid = mine && (t * TILE + r) < len;
       if (!mbar_wait(&mb_o[c % kOBufs], (c / kOBufs) & 1, kWaitNs)) bad = true;
       tc::fence_after();
-      float v[32], vl[16], ss = 0.f;
+      // O = its hi column block + its lo block, read 16 columns at a time (warp-collective: every lane)
+      float v[16], vl[16], ss = 0.f;
       const uint32_t ob = tbase + lane_base + CO0 + 128 * (c % kOBufs);
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        tmem_ld32(ob + 32 * hh, v);  // warp-collective: every lane takes part
+      for (int q = 0; q < 4; ++q) {
+        tmem_ld16(ob + 16 * q, v);
+        tmem_ld16(ob + 64 + 16 * q, vl);
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          tmem_ld16(ob + 64 + 32 * hh + 16 * q, vl);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) v[16 * q + j] += vl[j];
+        for (int j = 0; j < 16; ++j) {
+          v[j] += vl[j];
+          ss += v[j] * v[j];
         }
-#pragma unroll
-        for (int j = 0; j < 32; ++j) ss += v[j] * v[j];
       }
       if (mine) st_async_f32(peer_sums + 4 * (TILE * (c & 1) + r), ss, (c & 1) ? peer_x1 : peer_x0);
       if (warp == 8 && lane == 0) mbar_expect_tx(&mb_x[c & 1], C * 4);  // the local arrival of this phase
@@ -1627,23 +1649,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
       const float rinv = valid ? rsqrtf((ss + s_peer[TILE * (c & 1) + r]) * (1.0f / kD) + d.norm_eps) : 0.f;
       __nv_bfloat16* orow = o + tok * HvD + (int64_t)h * kD + 64 * vh;
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        tmem_ld32(ob + 32 * hh, v);
+      for (int q = 0; q < 4; ++q) {
+        tmem_ld16(ob + 16 * q, v);
+        tmem_ld16(ob + 64 + 16 * q, vl);
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          tmem_ld16(ob + 64 + 32 * hh + 16 * q, vl);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) v[16 * q + j] += vl[j];
-        }
-        if (hh == 1) {  // the products of chunk c are read: the buffer takes chunk c+3's
+        for (int j = 0; j < 16; ++j) v[j] += vl[j];
+        if (q == 3) {  // the products of chunk c are read: the buffer takes chunk c+3's
           tc::fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&mb_e[c % kOBufs]);
         }
         if (valid) {
 #pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const uint4 gq = gr[4 * hh + m];
+          for (int m = 0; m < 2; ++m) {
+            const uint4 gq = gr[2 * q + m];
             const __half2* g2 = reinterpret_cast<const __half2*>(&gq);
             uint32_t ow[4];
 #pragma unroll
@@ -1652,7 +1671,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
               __nv_bfloat162 pr = __floats2bfloat162_rn(v[8 * m + 2 * e] * rinv * gf.x, v[8 * m + 2 * e + 1] * rinv * gf.y);
               ow[e] = *reinterpret_cast<uint32_t*>(&pr);
             }
-            *reinterpret_cast<uint4*>(orow + 32 * hh + 8 * m) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+            *reinterpret_cast<uint4*>(orow + 16 * q + 8 * m) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
           }
         }
       }
@@ -1696,61 +1715,91 @@ size_t rec_bytes(int chunk) {
 template <int TILE, int C>
 cudaError_t launch_wy(const Dims& d, const float* conv_w, const float* A_log, const float* dt_bias,
                       const float* norm_w, const void* qkv, const void* z, const void* a, const void* b,
-                      const int32_t* cu, const int32_t* order, const int32_t* tile_off, const int4* tile_map,
-                      int32_t N, int64_t total_tokens, int64_t total_tiles, bool zero_state, bool zero_conv,
-                      const void* conv_state, float* state, void* o, void* ws, int32_t* status,
+                      const int32_t* cu, const int32_t* cu_host, const int32_t* order, const int32_t* tile_off,
+                      const int4* tile_map, int32_t N, int64_t total_tokens, int64_t total_tiles, bool zero_state,
+                      bool zero_conv, const void* conv_state, float* state, void* o, void* ws, int32_t* status,
                       cudaStream_t stream) {
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return cudaErrorNotSupported;
-  const WyLayout Lw = wy_layout(d, total_tokens, total_tiles, C);
+  // The tiles go through conv, prep and the chain one window at a time, so that the intermediates take a
+  // bounded workspace whatever the length; the chain carries each sequence's state from window to window
+  // through `state`.
+  const int64_t W = wy_window_tiles(total_tiles, C);
+  const WyLayout Lw = wy_layout(d, std::min<int64_t>(total_tokens, W * TILE), W, C);
   unsigned char* w = (unsigned char*)ws;
   __half* qk_hi = (__half*)(w + Lw.qk_hi);
   __half* qk_lo = (__half*)(w + Lw.qk_lo);
   unsigned char* vimg = w + Lw.vimg;
   __half* gate = (__half*)(w + Lw.gate);
   unsigned char* records = w + Lw.records;
-  CUtensorMap tm_hi, tm_lo;
   const uint64_t qkw = (uint64_t)2 * d.Hk * kD;
-  if (!encode_2d(enc, &tm_hi, qk_hi, qkw, total_tokens) || !encode_2d(enc, &tm_lo, qk_lo, qkw, total_tokens))
-    return cudaErrorInvalidValue;
+  using F = ChainCfg<TILE, C>;
   cudaError_t e;
-  {
-    LaunchScope scope(GDN_K_WY_CONV, stream);
-    wy_conv_kernel<TILE><<<dim3((unsigned)(total_tiles * (TILE / 64)), (unsigned)(2 * d.Hk + 2 * d.Hv)), 256, 0,
-                           stream>>>(d, conv_w, (const __nv_bfloat16*)qkv, (const __nv_bfloat16*)conv_state,
-                                     zero_conv ? 1 : 0, tile_map, total_tokens, qk_hi, qk_lo, vimg, norm_w,
-                                     (const __nv_bfloat16*)z, gate);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
   if constexpr (TILE == 64) {
     if ((e = cudaFuncSetAttribute(wy_prep_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrepSmem)) !=
         cudaSuccess)
       return e;
-    LaunchScope scope(GDN_K_WY_PREP, stream);
-    wy_prep_kernel<C><<<(unsigned)(total_tiles * d.Hv), kPrepThreads, kPrepSmem, stream>>>(
-        tm_hi, tm_lo, d, tile_map, vimg, records, cu, (const __nv_bfloat16*)qkv, zero_conv ? 1 : 0,
-        (__nv_bfloat16*)const_cast<void*>(conv_state), A_log, dt_bias, (const __nv_bfloat16*)a,
-        (const __nv_bfloat16*)b, total_tokens, status);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
   } else {
     if ((e = cudaFuncSetAttribute(wy_prep128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   kPrep128Smem)) != cudaSuccess)
       return e;
-    LaunchScope scope(GDN_K_WY_PREP, stream);
-    wy_prep128_kernel<<<(unsigned)(total_tiles * d.Hv), kPrepThreads, kPrep128Smem, stream>>>(
-        tm_hi, tm_lo, d, tile_map, vimg, records, cu, (const __nv_bfloat16*)qkv, zero_conv ? 1 : 0,
-        (__nv_bfloat16*)const_cast<void*>(conv_state), A_log, dt_bias, (const __nv_bfloat16*)a,
-        (const __nv_bfloat16*)b, total_tokens, status);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  using F = ChainCfg<TILE, C>;
   if ((e = cudaFuncSetAttribute(wy_chain_kernel<TILE, C>, cudaFuncAttributeMaxDynamicSharedMemorySize, F::SMEM)) !=
       cudaSuccess)
     return e;
-  LaunchScope scope(GDN_K_WY_CHAIN, stream);
-  wy_chain_kernel<TILE, C><<<(unsigned)((int64_t)N * d.Hv * 2), kChainThreads, F::SMEM, stream>>>(
-      d, records, tile_off, order, cu, zero_state ? 1 : 0, gate, state, (__nv_bfloat16*)o, status);
-  return cudaGetLastError();
+  // first token of tile g (tiles are numbered sequence by sequence in id order)
+  int32_t n = 0;
+  int64_t n_first = 0;
+  auto tile_token = [&](int64_t g) -> int64_t {
+    if (N == 1 || !cu_host) return TILE * g;
+    while (n < N) {
+      const int64_t nt = (cu_host[n + 1] - cu_host[n] + TILE - 1) / TILE;
+      if (g < n_first + nt) return cu_host[n] + TILE * (g - n_first);
+      n_first += nt;
+      ++n;
+    }
+    return total_tokens;
+  };
+  if (zero_state && W < total_tiles) {  // a sequence may start in a later window: its zero state comes from here
+    if ((e = cudaMemsetAsync(state, 0, (size_t)N * d.Hv * kD * kD * sizeof(float), stream)) != cudaSuccess) return e;
+    zero_state = false;
+  }
+  for (int64_t g0 = 0; g0 < total_tiles; g0 += W) {
+    const int64_t g1 = std::min<int64_t>(g0 + W, total_tiles);
+    const int64_t t0 = tile_token(g0), t1 = g1 < total_tiles ? tile_token(g1) : total_tokens;
+    const WyWin win{g0, g1, t0};
+    CUtensorMap tm_hi, tm_lo;
+    if (!encode_2d(enc, &tm_hi, qk_hi, qkw, t1 - t0) || !encode_2d(enc, &tm_lo, qk_lo, qkw, t1 - t0))
+      return cudaErrorInvalidValue;
+    {
+      LaunchScope scope(GDN_K_WY_CONV, stream);
+      wy_conv_kernel<TILE><<<dim3((unsigned)((g1 - g0) * (TILE / 64)), (unsigned)(2 * d.Hk + 2 * d.Hv)), 256, 0,
+                             stream>>>(d, conv_w, (const __nv_bfloat16*)qkv, (const __nv_bfloat16*)conv_state,
+                                       zero_conv ? 1 : 0, tile_map, total_tokens, qk_hi, qk_lo, vimg, norm_w,
+                                       (const __nv_bfloat16*)z, gate, win);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if constexpr (TILE == 64) {
+      LaunchScope scope(GDN_K_WY_PREP, stream);
+      wy_prep_kernel<C><<<(unsigned)((g1 - g0) * d.Hv), kPrepThreads, kPrepSmem, stream>>>(
+          tm_hi, tm_lo, d, tile_map, vimg, records, cu, (const __nv_bfloat16*)qkv, zero_conv ? 1 : 0,
+          (__nv_bfloat16*)const_cast<void*>(conv_state), A_log, dt_bias, (const __nv_bfloat16*)a,
+          (const __nv_bfloat16*)b, total_tokens, win, status);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    } else {
+      LaunchScope scope(GDN_K_WY_PREP, stream);
+      wy_prep128_kernel<<<(unsigned)((g1 - g0) * d.Hv), kPrepThreads, kPrep128Smem, stream>>>(
+          tm_hi, tm_lo, d, tile_map, vimg, records, cu, (const __nv_bfloat16*)qkv, zero_conv ? 1 : 0,
+          (__nv_bfloat16*)const_cast<void*>(conv_state), A_log, dt_bias, (const __nv_bfloat16*)a,
+          (const __nv_bfloat16*)b, total_tokens, win, status);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    LaunchScope scope(GDN_K_WY_CHAIN, stream);
+    wy_chain_kernel<TILE, C><<<(unsigned)((int64_t)N * d.Hv * 2), kChainThreads, F::SMEM, stream>>>(
+        d, records, tile_off, order, cu, zero_state ? 1 : 0, gate, win, state, (__nv_bfloat16*)o, status);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -1761,6 +1810,11 @@ bool prefill_wy_supported(const Dims& d, bool bf16, int chunk_size) {
 }
 
 int wy_tile(int chunk_size) { return chunk_size == 128 ? 128 : 64; }
+
+int64_t wy_window_tiles(int64_t total_tiles, int chunk_size) {
+  const int64_t cap = kWyWindowTokens / wy_tile(chunk_size);
+  return total_tiles < cap ? total_tiles : cap;
+}
 
 WyLayout wy_layout(const Dims& d, int64_t total_tokens, int64_t tile_bound, int chunk_size) {
   WyLayout S;
@@ -1777,13 +1831,15 @@ WyLayout wy_layout(const Dims& d, int64_t total_tokens, int64_t tile_bound, int 
 
 cudaError_t launch_prefill_wy(const Dims& d, int chunk_size, const float* conv_w, const float* A_log,
                               const float* dt_bias, const float* norm_w, const void* qkv, const void* z,
-                              const void* a, const void* b, const int32_t* cu, const int32_t* order,
+                              const void* a, const void* b, const int32_t* cu, const int32_t* cu_host,
+                              const int32_t* order,
                               const int32_t* tile_off, const int4* tile_map, int32_t N, int64_t total_tokens,
                               int64_t total_tiles, bool zero_state, bool zero_conv, const void* conv_state,
                               float* state, void* o, void* ws, int32_t* status, cudaStream_t stream) {
   if (N <= 0 || total_tokens <= 0 || total_tiles <= 0) return cudaSuccess;
 #define GDN_WY_ARGS                                                                                               \
-  d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, cu, order, tile_off, tile_map, N, total_tokens, total_tiles, \
+  d, conv_w, A_log, dt_bias, norm_w, qkv, z, a, b, cu, cu_host, order, tile_off, tile_map, N, total_tokens,      \
+      total_tiles,                                                                                                \
       zero_state, zero_conv, conv_state, state, o, ws, status, stream
   switch (chunk_size) {
     case 16: return launch_wy<64, 16>(GDN_WY_ARGS);

@@ -140,11 +140,11 @@ GDN_API gdn_status gdn_conv_step(const gdn_config* cfg, const void* x, const flo
  * num_seqs, chunk_size); 256-byte aligned.  The size covers every path a flag
  * can select.  For the tensor-core paths (bf16, d_k = d_v = 128) it holds the
  * schedule (about 16 bytes per chunk) plus the chunked form's intermediates
- * for one window of at most 16384 tokens: the three kernels run window by
+ * for one window of at most 65536 tokens: the three kernels run window by
  * window, carrying each sequence's state between windows, so beyond the
  * schedule the size does not grow with total_tokens (at 16 key / 48 value
- * heads about 2.0 GB at chunk 64 and 3.4 GB at chunk 16, less for shorter
- * inputs).  With GDN_PREFILL_FUSED the schedule alone suffices.
+ * heads at most about 8.7 GB at chunk 64 and 14.4 GB at chunk 16, less for
+ * shorter inputs).  With GDN_PREFILL_FUSED the schedule alone suffices.
  */
 GDN_API gdn_status gdn_prefill_workspace_size(const gdn_config* cfg, int64_t total_tokens, int32_t num_seqs,
                                       int32_t chunk_size, size_t* bytes);

@@ -77,9 +77,9 @@ struct SplitLayout {
   size_t qk_hi, qk_lo, records, total_bytes;
 };
 SplitLayout split_layout(const Dims& d, int64_t total_tokens, int64_t chunk_bound);
-// the chunks go through conv, prep and chain in windows of at most this many chunks (16384 tokens), so the
+// the chunks go through conv, prep and chain in windows of at most this many chunks (65536 tokens), so the
 // workspace holds the intermediates of one window: split_layout(d, min(T, window * 64), window)
-constexpr int64_t kSplitWindowChunks = 256;
+constexpr int64_t kSplitWindowChunks = 1024;
 int64_t split_window_chunks(int64_t total_chunks);
 cudaError_t launch_prefill_split(const Dims& d, const float* conv_w, const float* A_log, const float* dt_bias,
                                  const float* norm_w, const void* qkv, const void* z, const void* a, const void* b,
@@ -155,7 +155,7 @@ struct WyLayout {
 WyLayout wy_layout(const Dims& d, int64_t total_tokens, int64_t tile_bound, int chunk_size);
 // the tiles go through conv, prep and chain in windows of at most kWyWindowTokens / tile rows, so the
 // workspace holds one window: wy_layout(d, min(T, window * tile), window, chunk)
-constexpr int64_t kWyWindowTokens = 16384;
+constexpr int64_t kWyWindowTokens = 65536;
 int64_t wy_window_tiles(int64_t total_tiles, int chunk_size);
 cudaError_t launch_prefill_wy(const Dims& d, int chunk_size, const float* conv_w, const float* A_log,
                               const float* dt_bias, const float* norm_w, const void* qkv, const void* z,

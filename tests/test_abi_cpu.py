@@ -89,6 +89,18 @@ def test_workspace_size_and_bad_chunk():
     assert e.value.name == "GDN_E_INVAL"
 
 
+def test_workspace_is_bounded_by_one_window():
+    """The chunked paths run conv, prep and chain over windows of at most 65536 tokens, so beyond the
+    schedule (16 bytes per chunk and a few per sequence) the workspace stops growing with the length."""
+    cfg = qwen_cfg()
+    for chunk in (16, 32, 64, 128):
+        w1 = gdn.prefill_workspace_size(cfg, 65536, 1, chunk)
+        w4 = gdn.prefill_workspace_size(cfg, 4 * 65536, 1, chunk)
+        chunks = 3 * 65536 // min(chunk, 64)
+        assert w1 < w4 <= w1 + 16 * chunks + 4096, (chunk, w1, w4)
+        assert gdn.prefill_workspace_size(cfg, 4096, 1, chunk) < w1  # shorter inputs need less
+
+
 class FakeTensor:
     """Host buffer with a data_ptr(), standing in for device memory in calls
     that must fail during validation (nothing may be written)."""

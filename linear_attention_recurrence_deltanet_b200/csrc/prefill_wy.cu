@@ -1262,7 +1262,8 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
     mbar_expect_tx(&mb_p, 32768);
     bulk_load(sm + W8_QH, rec + R::P, 32768, &mb_p);
   }
-  {  // M' -> the record (K-major 128 x 128); U -> the record as hi + lo per value-channel half
+  {  // M' (K-major 128 x 128) staged in KT and U (hi + lo per value-channel half) in KH (half 0) and X
+     // (half 1), all read by the products just completed; they go to the record by bulk stores
     float v[32];
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
@@ -1270,9 +1271,9 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       tmem_ld32(tbase + lane_base + T8_SOLVE + cb, v);
 #pragma unroll
       for (int m = 0; m < 4; ++m)
-        *reinterpret_cast<uint4*>(rec + R::M + kmaj_chunk(128, si, cb + 8 * m)) = pack8h(v + 8 * m);
+        *reinterpret_cast<uint4*>(sm + W8_KT + kmaj_chunk(128, si, cb + 8 * m)) = pack8h(v + 8 * m);
       tmem_ld32(tbase + lane_base + T8_QK + cb, v);
-      unsigned char* uh = rec + R::U + hc * 2 * R::UH;
+      unsigned char* uh = sm + (hc == 0 ? W8_KH : W8_X);
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         float hi[8], lo[8];
@@ -1286,6 +1287,14 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
         *reinterpret_cast<uint4*>(uh + R::UH + off) = pack8h(lo);
       }
     }
+  }
+  fence_async_smem();
+  __syncthreads();
+  if (tid == 0) {
+    bulk_store(rec + R::M, sm + W8_KT, 32768);
+    bulk_store(rec + R::U, sm + W8_KH, 2 * R::UH);
+    bulk_store(rec + R::U + 2 * R::UH, sm + W8_X, 2 * R::UH);
+    bulk_commit();
   }
   // Q' = Qg + P (-W) (columns 384..511)
   if (tid == 0) {
@@ -1302,7 +1311,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
   if (!mbar_wait(&mb_mma, ph, kWaitNs)) bad = true;
   ph ^= 1;
   fence_after();
-  {
+  {  // Q' staged in QL (T' lo, read by U) and written by a bulk store
     float v[32];
     const bool ok = si < L;
 #pragma unroll
@@ -1314,11 +1323,18 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
         float q8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) q8[e] = ok ? v[8 * m + e] : 0.f;
-        *reinterpret_cast<uint4*>(rec + R::Q + kmaj_chunk(TILE, si, cb + 8 * m)) = pack8h(q8);
+        *reinterpret_cast<uint4*>(sm + W8_QL + kmaj_chunk(TILE, si, cb + 8 * m)) = pack8h(q8);
       }
     }
   }
-  if (sync_tc_any(bad) && tid == 0) set_status(status, kTimeoutPrep);
+  fence_async_smem();
+  const bool fail = sync_tc_any(bad);
+  if (tid == 0) {
+    if (fail) set_status(status, kTimeoutPrep);
+    bulk_store(rec + R::Q, sm + W8_QL, TILE * 256);
+    bulk_commit();
+    bulk_wait<0>();  // every record image has left shared memory
+  }
   if (warp == 0) tmem_dealloc(tbase, 512);
 }
 

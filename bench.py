@@ -458,7 +458,9 @@ def run_gdn(args, rank, world, local_rank):
     decode = {"value": round(whole_job_rate(world, N, 1, d_mean), 1), "unit": "tokens/s", "ms_per_step": round(d_mean, 5),
               "median_ms": round(statistics.median(step_ms), 5), "steps": dsteps, "num_seqs": N, "roofline": roof_d,
               "workload": "GDN decode, 64 sequences x 1 token, 16 key / 48 value heads x 128, bf16 inputs, "
-                          "fp32 states ~N(0,0.02), fresh inputs every step"}
+                          "fp32 states ~N(0,0.02), fresh inputs every step",
+              "cpu_baseline": (oracle_decode_sample(gd, seed, N, conv0, st0)
+                               if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None)}
 
     # ---------------- K=2 draft-and-verify rounds on the same sequences: a verify pass over both tokens, then a
     # commit of each sequence's accepted prefix (1 or 2 tokens, seeded); accepted tokens/s is the rate
@@ -542,6 +544,26 @@ def run_gdn(args, rank, world, local_rank):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def oracle_decode_sample(geo, seed, N, conv0, st0, steps=5):
+    """The float64 oracle, as it stands, on the first `steps` decode steps of
+    the decode workload (all sequences and value heads, all host cores): the
+    per-step time beside the GPU's."""
+    import oracle
+    params = gi.make_params(geo, seed)
+    hist, state = conv0, st0
+    times = []
+    for s in range(steps):
+        q, z, a, b = (gi.f32_from_bf16_bits(t) for t in gi.make_decode_step_tokens(geo, N, seed, s))
+        t0 = time.perf_counter()
+        _, state, hist = oracle.decode_step(geo, params, q, z, a, b, hist, state)
+        times.append(time.perf_counter() - t0)
+    med = statistics.median(times)
+    cores = oracle.default_threads()
+    return {"value": round(N / med, 2), "unit": "tokens/s", "ms_per_step": round(1000 * med, 2), "cores": cores,
+            "kind": "oracle", "sample": f"float64 oracle, the first {steps} of the decode workload's steps ({N} "
+                                       f"sequences, all {geo.num_v_heads} value heads), median step, {cores} threads"}
 
 
 def oracle_sample(inp, budget_s=5.0):

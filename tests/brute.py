@@ -3,7 +3,9 @@
 Nothing here is shared with the oracle or the CUDA path.  The conv uses
 ``np.convolve``, the gates ``np.logaddexp``/``scipy.special.expit``, the
 recurrence is expanded into explicit d_k x d_k transition matrices, and the
-chunked twin follows the chunkwise (WY/UT) form of the same recurrence.
+chunked twins follow the chunkwise (WY/UT) form of the same recurrence: its
+factored form, and its affine form (the chunk's terms that multiply the state
+collected into one d_k x d_k map) with (I + A)^-1 by recursive doubling.
 """
 
 from __future__ import annotations
@@ -132,4 +134,67 @@ def chunked_head(S0, q, k, v, g, beta, C):
         O = np.exp(gam)[:, None] * (Q @ S) + (Mm * (Q @ K.T)) @ D
         S = np.exp(gam[-1]) * S + K.T @ (np.exp(gam[-1] - gam)[:, None] * D)
         outs.append(O)
+    return np.concatenate(outs, axis=0), S
+
+
+def doubling_inverse(A, base):
+    """(I + A)^-1 for a strictly lower triangular A by recursive doubling:
+    base x base diagonal blocks by forward substitution, then for b = base,
+    2 base, ... every pair of b-blocks merged by T <- T - T (A_off,b T), where
+    A_off,b keeps the entries of A whose row and column first fall in
+    different halves of a 2b-block.  Padded with zeros to base * 2^k rows."""
+    n = A.shape[0]
+    Np = base
+    while Np < n:
+        Np *= 2
+    Ap = np.zeros((Np, Np))
+    Ap[:n, :n] = A
+    T = np.zeros((Np, Np))
+    for o in range(0, Np, base):
+        blk = Ap[o:o + base, o:o + base]
+        for c in range(base):
+            t = np.zeros(base)
+            for i in range(base):
+                t[i] = (1.0 if i == c else 0.0) - (blk[i, :i] @ t[:i] if i else 0.0)
+                if i < c:
+                    t[i] = 0.0
+            T[o:o + base, o + c] = t
+    b = base
+    while b < Np:
+        Aoff = np.zeros((Np, Np))
+        for o in range(0, Np, 2 * b):
+            Aoff[o + b:o + 2 * b, o:o + b] = Ap[o + b:o + 2 * b, o:o + b]
+        T = T - T @ (Aoff @ T)
+        b *= 2
+    return T[:n, :n]
+
+
+def affine_head(S0, q, k, v, g, beta, C, base=4):
+    """The chunk maps of the gated delta rule collected as affine maps of the
+    state, per chunk (same gamma, A, W, U, P as chunked_head, with T from
+    doubling_inverse):
+      K~ = diag(e^{gamma_L - gamma}) K,   M' = -K~^T W,   Q' = diag(e^gamma) Q - P W,
+      O = Q' S + P U,                      S <- e^{gamma_L} S + M' S + K~^T U.
+    S is [dk, dv].  Returns (o [L, dv] before the output norm, S_final)."""
+    L = q.shape[0]
+    S = S0.copy()
+    outs = []
+    for c0 in range(0, L, C):
+        c1 = min(L, c0 + C)
+        Q, K, V = q[c0:c1], k[c0:c1], v[c0:c1]
+        gam = np.cumsum(g[c0:c1])
+        bt = beta[c0:c1]
+        n = c1 - c0
+        diff = gam[:, None] - gam[None, :]
+        lower = np.tril(np.ones((n, n)), -1)
+        A = (bt[:, None] * np.exp(np.where(lower > 0, diff, 0.0)) * (K @ K.T)) * lower
+        Tm = doubling_inverse(A, base)
+        Wm = Tm @ ((bt * np.exp(gam))[:, None] * K)
+        Um = Tm @ (bt[:, None] * V)
+        P = np.exp(np.where(np.tril(np.ones((n, n))) > 0, diff, -np.inf)) * (Q @ K.T)
+        Kt = np.exp(gam[-1] - gam)[:, None] * K
+        Mp = -(Kt.T @ Wm)
+        Qp = np.exp(gam)[:, None] * Q - P @ Wm
+        outs.append(Qp @ S + P @ Um)
+        S = np.exp(gam[-1]) * S + Mp @ S + Kt.T @ Um
     return np.concatenate(outs, axis=0), S

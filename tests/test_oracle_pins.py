@@ -297,6 +297,34 @@ def test_chunked_form_equals_oracle(C):
         np.testing.assert_allclose(S.T, st_ref[0, h], rtol=1e-11, atol=1e-12)
 
 
+@pytest.mark.parametrize("C,base", [(4, 2), (16, 4), (13, 4), (32, 16)])
+def test_affine_form_equals_oracle(C, base):
+    # the affine chunk maps (M' = -K~^T W, Q' = e^gamma Q - P W) with T by recursive doubling, as the
+    # affine GPU prefill computes them, reproduce the oracle
+    inp = _tiny_problem([37], seed=19, d=6)
+    o_ref, st_ref, _ = oracle.prefill_inputs(inp)
+    geo = inp.geo
+    dv = geo.head_v_dim
+    for h in range(geo.num_v_heads):
+        qh, kh, v = brute.head_inputs(geo, _params(inp), inp.qkv.astype(np.float64), inp.conv_state[0], h)
+        g, _, beta = brute.gates(inp.a[:, h].astype(np.float64), inp.dt_bias[h], inp.A_log[h],
+                                 inp.b[:, h].astype(np.float64))
+        o_pre, S = brute.affine_head(inp.state[0, h].T.astype(np.float64), qh, kh, v, g, beta, C, base)
+        o = np.stack([brute.rmsnorm_gate(o_pre[t], inp.z[t, h * dv:(h + 1) * dv], inp.norm_w, geo.norm_eps)
+                      for t in range(37)])
+        np.testing.assert_allclose(o, o_ref[:, h * dv:(h + 1) * dv], rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(S.T, st_ref[0, h], rtol=1e-11, atol=1e-12)
+
+
+def test_doubling_inverse_is_the_inverse():
+    rng = np.random.default_rng(7)
+    for n, base in ((16, 4), (23, 4), (64, 16), (128, 16)):
+        A = np.tril(rng.normal(0, 0.3, (n, n)), -1)
+        T = brute.doubling_inverse(A, base)
+        np.testing.assert_allclose(T @ (np.eye(n) + A), np.eye(n), atol=1e-10)
+        assert np.array_equal(np.triu(T, 1), np.zeros((n, n)))  # lower triangular, like (I + A)^-1
+
+
 def test_workload_tiny_fp32_runs_and_is_finite():
     inp = gi.workload_inputs("tiny_fp32_t64")
     o, st, hist = oracle.prefill_inputs(inp)

@@ -37,7 +37,16 @@
 // Tiles: the prep and chain kernels work on tiles of 64 rows (chunk sizes 16,
 // 32 and 64: a tile holds 64 / C chunks, and every intra-chunk matrix is block
 // diagonal within the tile) or of 128 rows (chunk size 128).  Tiles restart at
-// every sequence start, so chunk boundaries align with tile boundaries.
+// every sequence start, so chunk boundaries align with tile boundaries.  The
+// three kernels run over windows of at most kWyWindowTokens tokens' tiles, the
+// chain carrying each sequence's state from window to window, so that the
+// intermediates take a bounded workspace.
+//
+// Precision: operands are fp16 with fp32 accumulation; where a rounding would
+// show in the output or the state the operand is carried as hi + lo parts:
+// [K;Q]K^T (hi.hi + hi.lo + lo.hi), T' and v^ in U, U itself, the state in
+// the output products (Q'S loses digits to cancellation when q is nearly
+// orthogonal to the state's columns) and, at chunk 16, Q'.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>

@@ -13,8 +13,8 @@
 //   conv_qkv_kernel   grid (chunk, head slot): causal conv + SiLU of q/k/v
 //                     ("causal depthwise Conv1D", DS4Server issue #88, Scope),
 //                     L2 norm of q and k with epsilon inside the square root;
-//                     q^, k^ as fp16 hi + lo parts, v^ as fp16; and the output
-//                     gate (1 + w) sigmoid(z) of every value head, fp16.
+//                     q^, k^ and v^ as fp16 hi + lo parts; and the output gate
+//                     (1 + w) sigmoid(z) of every value head, fp16.
 //   prep_kernel       grid (chunk, value head): gates, [K;Q]K^T in split
 //                     precision on tcgen05, A and P, T = (I+A)^-1 by recursive
 //                     doubling whose merges are tcgen05 MMAs, then W = T''K
@@ -22,7 +22,8 @@
 //                     value head) whose parts are byte images of the chain
 //                     kernel's shared-memory operands.
 //   chain_kernel      grid (sequence, value head, value-channel half), clusters
-//                     of the two halves: per chunk, [-W;Qg] S on tcgen05, Delta =
+//                     of the two halves: per chunk, [-W;Qg] S on tcgen05 (S as
+//                     fp16 hi + lo; Delta takes the hi products alone), Delta =
 //                     U - W S, then K~^T Delta and [0;P] Delta, then the state
 //                     update, each CTA for 64 of the 128 value channels (the
 //                     columns of the state are independent); the output rows of
@@ -30,6 +31,10 @@
 //                     exchanged through distributed shared memory) are written
 //                     by half of the warps while the other half carries chunk
 //                     c+1 to its second MMA group.
+//
+// The three kernels run over windows of at most kSplitWindowChunks chunks, the
+// chain carrying each sequence's state from window to window, so that the
+// intermediates take a bounded workspace.
 //
 // Record of (chunk, value head), byte images of 128-byte-swizzled operands:
 //   [     0,  32768) [-W ; Qg]  K-major 128 x 128   (Qg = diag(e^gamma) q^)

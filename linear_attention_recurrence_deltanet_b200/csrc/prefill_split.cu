@@ -765,6 +765,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
   unsigned char* sm = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   __shared__ uint64_t mb_a[2], mb_u[2], mb_ld1[2], mb_g[2];  // copies into buffer cc % 2, one phase per use
   __shared__ uint64_t mb_m3, mb_m5;  // completions of [-WS;QgS] and K~^T Delta, one phase per chunk
+  __shared__ uint64_t mb_m3a;        // completion of [-W;Qg] S lo, the last reader of the chunk's A buffer
   __shared__ uint64_t mb_m4[2];      // completion of [0;P] Delta (O of chunk cc complete), cc % 2, one phase per use
   __shared__ uint64_t mb_x[2];       // the peer's row sums of chunk cc arrived, cc % 2, one phase per use
   __shared__ uint32_t tslot;
@@ -813,6 +814,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
       mbar_init(&mb_x[b], 1);  // one local arrival with the expected bytes; the peer's stores complete them
     }
     mbar_init(&mb_m3, 1);
+    mbar_init(&mb_m3a, 1);
     mbar_init(&mb_m5, 1);
     mbar_init_fence();
   }
@@ -963,6 +965,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
 #pragma unroll
           for (int s = 0; s < 8; ++s)
             mma_f16(tbase + colU + 64, desc_kmaj(aa, 128, s), desc_mnmaj(sb + 16384, kD, s), id, s > 0);
+          mma_commit(&mb_m3a);
         }
         if (!mbar_wait(&mb_ld1[c & 1], par, kWaitNs)) bad = true;  // P and K~, long in place
       }
@@ -991,7 +994,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1)
           if (c + 1 < nchunks) issue_ld1(c + 1);
           if (c + 2 < nchunks && vh == 0) prefetch(c + 2);  // behind the copies in the queue
         }
-        if (!mbar_wait(&mb_m3, c & 1, kWaitNs)) bad = true;
+        if (!mbar_wait(&mb_m3a, c & 1, kWaitNs)) bad = true;  // the lo products still read the A buffer after M3
         if (c + 2 < nchunks) issue_a(c + 2);
         if (!mbar_wait(&mb_m5, c & 1, kWaitNs)) bad = true;  // M5 follows the delta warps' reads of U
         if (c + 2 < nchunks && !zero_u) issue_u(c + 2);

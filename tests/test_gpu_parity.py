@@ -121,12 +121,26 @@ def test_varlen_boundaries_are_isolated_bit_exact():
         assert np.array_equal(h1[n], h2[n]) == same, n
 
 
-def test_deterministic():
-    geo = gi.Geometry(num_k_heads=2, num_v_heads=4, head_k_dim=128, head_v_dim=128)
-    inp = gi.make_prefill_inputs(geo, [300, 17], seed=25, zero_init=False)
-    _, o1, st1, _ = run_gpu_prefill(inp, 64)
-    _, o2, st2, _ = run_gpu_prefill(inp, 64)
-    assert np.array_equal(o1, o2) and np.array_equal(st1, st2)
+@pytest.mark.parametrize("chunk,flags", [(64, 0), (64, AFFINE), (16, 0), (32, 0), (128, 0), (64, FUSED)])
+def test_deterministic(chunk, flags):
+    """Repeated prefills give the same bits.  Every head of the 16K/48V geometry runs, so the chain kernels
+    refill their operand buffers while the other clusters load memory: a buffer refilled before its last
+    reader (an MMA still in flight) is done changes output bits from run to run, even when the difference is
+    far inside the oracle tolerance."""
+    inp = gi.make_prefill_inputs(gi.QWEN_GEO, [1, 63, 65, 130, 7, 200, 16, 17, 1000], seed=25, zero_init=False)
+    dp = DeviceProblem(inp, chunk)
+    ref = None
+    for run in range(4):
+        dp.reset_states()
+        dp.o.zero_()
+        dp.prefill(flags)
+        torch.cuda.synchronize()
+        out = (io_numpy(dp.o).copy(), dp.state.cpu().numpy().view(np.int32).copy(), io_numpy(dp.conv_state).copy())
+        if ref is None:
+            ref = out
+            continue
+        diff = [int(np.count_nonzero(x != y)) for x, y in zip(ref, out)]
+        assert diff == [0, 0, 0], f"run {run}: (o, state, history) elements that differ from run 0: {diff}"
 
 
 def test_schedule_matches_host_reference():

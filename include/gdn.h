@@ -184,7 +184,8 @@ GDN_API gdn_status gdn_prefill(const gdn_config* cfg, const gdn_params* params, 
  * GDN_PREFILL_FUSED added to flags: the single-kernel chunked path where it
  * applies (bf16, d = 128, chunk 64), else the token-recurrent kernel; both
  * need only the varlen schedule as scratch, about 16 bytes per chunk plus 8
- * per sequence.  The limit is therefore the workspace gdn_prefill needs with
+ * per sequence.  flags holding GDN_PREFILL_RECURRENT, GDN_PREFILL_FACTORED or
+ * GDN_PREFILL_AFFINE are rejected with GDN_E_INVAL.  The limit is therefore the workspace gdn_prefill needs with
  * GDN_PREFILL_FUSED (not gdn_prefill_workspace_size, which reports the
  * default path's larger need): a problem whose schedule exceeds
  * GDN_NOALLOC_SCRATCH_BYTES, i.e. more than about 250,000 chunks plus

@@ -62,6 +62,17 @@ extern "C" GDN_API gdn_status gdn_prefill_noalloc(const gdn_config* cfg, const g
     gdn::set_error_message("gdn_prefill_noalloc: cu_seqlens_host is NULL");
     return GDN_E_INVAL;
   }
+  // the entry point runs the single-kernel path; another path flag would need a workspace of its own
+  const uint32_t other_paths = flags & (GDN_PREFILL_RECURRENT | GDN_PREFILL_FACTORED | GDN_PREFILL_AFFINE);
+  if (other_paths) {
+    char msg[192];
+    snprintf(msg, sizeof(msg),
+             "gdn_prefill_noalloc: flags 0x%x select another prefill path; this entry point runs the "
+             "single-kernel path (GDN_PREFILL_FUSED) only",
+             other_paths);
+    gdn::set_error_message(msg);
+    return GDN_E_INVAL;
+  }
   // cu_seqlens_host must be valid before its last entry sizes the schedule
   if (cu_seqlens_host[0] != 0) {
     gdn::set_error_message("gdn_prefill_noalloc: cu_seqlens_host[0] is not 0");

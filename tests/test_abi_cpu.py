@@ -181,6 +181,23 @@ def test_prefill_noalloc_validates_cu_seqlens_host_on_the_host():
     assert call(dec.ctypes.data, 2) == -1 and "decreases" in gdn.last_error()
 
 
+def test_prefill_noalloc_rejects_other_path_flags_on_the_host():
+    """The no-scratch prefill runs the single-kernel path only: a flag that
+    selects another path is named in the error, before any device call."""
+    geo = gi.Geometry()
+    cfg = gdn.make_config(geo)
+    params = gdn._params(*(FakeTensor(n) for n in (geo.conv_dim * 16, 192, 192, 512)))
+    t = FakeTensor(1 << 12)
+    cu = np.array([0, 8], np.int32)
+    L = gdn.lib()
+    for f in (gdn.PREFILL_RECURRENT, gdn.PREFILL_FACTORED, gdn.PREFILL_AFFINE,
+              gdn.PREFILL_AFFINE | gdn.ZERO_INIT_STATE):
+        rc = L.gdn_prefill_noalloc(ctypes.byref(cfg), ctypes.byref(params), t.data_ptr(), t.data_ptr(),
+                                   t.data_ptr(), t.data_ptr(), t.data_ptr(), cu.ctypes.data, 1, 64, f, t.data_ptr(),
+                                   t.data_ptr(), t.data_ptr(), None)
+        assert rc == -1 and "another prefill path" in gdn.last_error(), (f, gdn.last_error())
+
+
 def test_decode_multi_validation_rejects_before_launch():
     """Draft counts outside 1..4, an accept array on a verify call and head
     dims other than 128 are refused on the host, with every buffer intact."""

@@ -518,6 +518,7 @@ def run_gdn(args, rank, world, local_rank):
 
     proj = run_projections(gdn, torch, pk, stream, barrier, max_over_ranks, world, args.projection_reps)
     seqpar = run_seqpar(gdn, torch, pk, stream, barrier, max_over_ranks, world)
+    slots = run_slots(gdn, torch, pk, stream, barrier, max_over_ranks, world)
     extra = {} if args.no_workloads else run_workloads(gdn, torch, pk, stream, barrier, max_over_ranks, world, rank,
                                                        clocks)
 
@@ -533,7 +534,7 @@ def run_gdn(args, rank, world, local_rank):
                                    "fp32 state from zero", "global_batch": world, "seq_len": T, "chunk": C,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": f"inputs rotate over {ROTATE} sets (> 4x L2) between steps"},
-            "projections": proj, "seq_parallel": seqpar, "kernels": kernel_share,
+            "projections": proj, "seq_parallel": seqpar, "slots": slots, "kernels": kernel_share,
             "gpu_launches": launches, "clocks": clk, "cpu_baseline": cpu, "e2e": e2e,
             "roofline": roof_p,
             **extra,
@@ -784,6 +785,98 @@ def run_seqpar(gdn, torch, pk, stream, barrier, max_over_ranks, world, reps=5):
     out["workload"] = ("B=1, T=65536, 2 key / 6 value heads x 128 (an eighth of the layer's heads), chunk 64, "
                        "bf16 inputs, fp32 state from zero; time per whole prefill (all kernels)")
     del dp, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_slots(gdn, torch, pk, stream, barrier, max_over_ranks, world, steps=50, reps=10):
+    """Slot-indexed state pools (continuous batching): the states and conv
+    histories of a 256-slot pool, 16 key / 48 value heads x 128, bf16 inputs.
+    (1) Decode of 64 sequences whose states sit at seeded slots of the pool
+    (gdn_decode_step_indexed), fresh inputs every step; (2) one mixed step,
+    4 prefill sequences of 1024 tokens and 60 one-token decode rows packed in
+    one gdn_prefill_indexed call at chunk 64.  The pool (805 MB of state)
+    exceeds L2; CUDA events on the launching stream, and the library profiler
+    for the decode kernel's own time."""
+    from linear_attention_recurrence_deltanet_b200.device import io_tensor
+    geo = gi.QWEN_GEO
+    seed, N, P = 2, 64, 256
+    cfg = gdn.make_config(geo)
+    params = tuple(torch.from_numpy(np.ascontiguousarray(p)).cuda() for p in gi.make_params(geo, seed))
+    conv0, st0 = gi.make_initial_state(geo, P, seed, zero=False)
+    conv = io_tensor(conv0)
+    st = torch.from_numpy(st0).cuda()
+    del conv0, st0
+    rng = np.random.default_rng([seed, 8])
+    dslots = torch.from_numpy(rng.choice(P, size=N, replace=False).astype(np.int32)).cuda()
+    toks = [gi.make_decode_step_tokens(geo, N, seed, s) for s in range(steps)]
+    dq, dz, da, db = (torch.stack([io_tensor(t[i]) for t in toks]) for i in range(4))
+    del toks
+    o = torch.empty((N, geo.value_dim), dtype=torch.bfloat16, device="cuda")
+
+    def dstep(s):
+        gdn.decode_step_indexed(cfg, params, dq[s], dz[s], da[s], db[s], N, dslots, P, conv, st, o, stream=stream)
+
+    for s in range(min(10, steps)):
+        dstep(s)
+    barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gdn.profiler_reset()
+    gdn.profiler_enable(True)
+    a.record(stream)
+    for s in range(steps):
+        dstep(s)
+    b.record(stream)
+    b.synchronize()
+    gdn.profiler_enable(False)
+    d_ms = max_over_ranks(a.elapsed_time(b) / steps)
+    kn, kms = gdn.profiler_read(gdn.K.DECODE)
+    k_ms = max_over_ranks(kms / max(1, kn))
+    dbytes = decode_bytes(geo, N)
+    out = {"decode_indexed": {
+        "value": round(whole_job_rate(world, N, 1, d_ms), 1), "unit": "tokens/s", "ms_per_step": round(d_ms, 5),
+        "steps": steps, "num_seqs": N, "num_slots": P,
+        "roofline": {"bound": "hbm", "achieved": round(dbytes / (k_ms / 1000.0) / 1e9, 1), "peak": pk["hbm"],
+                     "unit": "GB/s", "frac": round(dbytes / (k_ms / 1000.0) / 1e9 / pk["hbm"], 4), "traffic": None,
+                     "kernel": "decode (indexed)", "kernel_ms": round(k_ms, 5), "algorithmic_bytes": dbytes,
+                     "peak_source": pk["src"]}}}
+    del dq, dz, da, db, o
+
+    lens = [1024] * 4 + [1] * 60
+    cu_h = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(cu_h[-1])
+    qkv, z, av, bv = (io_tensor(x) for x in gi.make_tokens(geo, np.random.default_rng([seed, 9]), T))
+    mslots = torch.from_numpy(rng.choice(P, size=len(lens), replace=False).astype(np.int32)).cuda()
+    cu_d = torch.from_numpy(cu_h).cuda()
+    ws = torch.empty(max(256, gdn.prefill_indexed_workspace_size(cfg, T, len(lens), 64)), dtype=torch.uint8,
+                     device="cuda")
+    mo = torch.empty((T, geo.value_dim), dtype=torch.bfloat16, device="cuda")
+
+    def mixed():
+        gdn.prefill_indexed(cfg, params, qkv, z, av, bv, cu_d, cu_h, mslots, P, 64, 0, conv, st, mo, ws,
+                            stream=stream)
+
+    for _ in range(3):
+        mixed()
+    barrier()
+    a.record(stream)
+    for _ in range(reps):
+        mixed()
+    b.record(stream)
+    b.synchronize()
+    m_ms = max_over_ranks(a.elapsed_time(b) / reps)
+    mbytes = prefill_bytes(geo, lens, zero_state=False)
+    gbs = mbytes / (m_ms / 1000.0) / 1e9
+    out["mixed_batch"] = {
+        "value": round(whole_job_rate(world, T, 1, m_ms), 1), "unit": "tokens/s", "ms_per_step": round(m_ms, 5),
+        "tokens": T, "prefill_seqs": 4, "decode_rows": 60, "chunk": 64, "num_slots": P,
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm"], "unit": "GB/s",
+                     "frac": round(gbs / pk["hbm"], 4), "traffic": None, "algorithmic_bytes": mbytes,
+                     "peak_source": pk["src"]}}
+    out["workload"] = ("a pool of 256 state slots, 16 key / 48 value heads x 128, bf16 inputs, fp32 states "
+                       "~N(0,0.02); decode: 64 sequences at seeded slots, 50 steps; mixed: 4 x 1024 prefill tokens "
+                       "and 60 decode rows in one indexed prefill call, chunk 64 (time per call, all kernels)")
+    del qkv, z, av, bv, mo, ws, conv, st
     torch.cuda.empty_cache()
     return out
 
